@@ -1,0 +1,231 @@
+"""Float64 CPU oracle for the CSA/HCA attention-layer core.
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
+benchmark's CPU-baseline leg are the only callers.  The product path never
+imports this package.  It shares no code with the CUDA library; the arithmetic
+lives in ``csa_oracle.c`` (plain C, double precision, OpenMP over query rows)
+and this module only marshals numpy arrays to it.
+
+Functions mirror the method's steps as restated from the page
+"DeepSeek-V4：迈向高效百万 Token 上下文智能", §3.3 (CSA and HCA hybrid
+attention) and the page "DeepSeek V4 完整技术报告", section "混合注意力：CSA +
+HCA".  Each function's docstring names the reading it takes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "csa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+NO_NORM = 1
+NO_ROPE = 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle's C source into ``liboracle.so`` beside it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Fmt(ctypes.Structure):
+    _fields_ = [
+        ("c", ctypes.c_int32),
+        ("rope_dims", ctypes.c_int32),
+        ("rope_base", ctypes.c_double),
+        ("norm_eps", ctypes.c_double),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+@dataclass(frozen=True)
+class Fmt:
+    """Entry format: dim c, RoPE on the last ``rope_dims`` dims."""
+
+    c: int
+    rope_dims: int = 64
+    rope_base: float = 10000.0
+    norm_eps: float = 1e-6
+    flags: int = 0
+
+    def _c(self) -> _Fmt:
+        return _Fmt(self.c, self.rope_dims, self.rope_base, self.norm_eps, self.flags)
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        FP = ctypes.POINTER(_Fmt)
+        _lib.orc_rmsnorm.argtypes = [i32, f64, P, P]
+        _lib.orc_rope.argtypes = [i32, i32, f64, f64, P, P]
+        _lib.orc_visible.argtypes = [i64, i32, i64]
+        _lib.orc_visible.restype = i64
+        _lib.orc_csa_compress.argtypes = [i64, i32, FP, P, P, P, P, i32, i64, P, P]
+        _lib.orc_hca_compress.argtypes = [i64, i32, FP, P, P, i32, i64, P, P]
+        _lib.orc_window_rows.argtypes = [i64, FP, P, i64, P]
+        _lib.orc_indexer_scores.argtypes = [i64, i32, i32, i64, P, P, P, P, i32, P]
+        _lib.orc_topk.argtypes = [i64, i64, P, P, i32, i32, P]
+        _lib.orc_attention.argtypes = [
+            i64, i32, FP, P, P, P, i64, P, i32, i32, P, i64, i64, i32, P, f64, P, P,
+        ]
+        for fn in (
+            "orc_rmsnorm", "orc_rope", "orc_csa_compress", "orc_hca_compress",
+            "orc_window_rows", "orc_indexer_scores", "orc_topk", "orc_attention",
+        ):
+            getattr(_lib, fn).restype = None
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    a = np.asarray(a)
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def rmsnorm(x, eps: float = 1e-6) -> np.ndarray:
+    x = _f64(x)
+    y = np.empty_like(x)
+    _L().orc_rmsnorm(x.shape[-1], eps, _ptr(x), _ptr(y))
+    return y
+
+
+def rope(x, pos: float, rope_dims: int, base: float = 10000.0) -> np.ndarray:
+    x = _f64(x)
+    y = np.empty_like(x)
+    _L().orc_rope(x.shape[-1], rope_dims, base, float(pos), _ptr(x), _ptr(y))
+    return y
+
+
+def visible(pos: int, m: int, n_entries: int) -> int:
+    """Entries visible at query position ``pos`` (an entry is visible once its
+    last token is at or before the query: s < floor((pos+1)/m))."""
+    return int(_L().orc_visible(int(pos), int(m), int(n_entries)))
+
+
+def csa_compress(kv_a, kv_b, z_a, z_b, m: int, fmt: Fmt, pos0: int = 0, want_weights=False):
+    """Overlapped softmax-gated compression, rate exactly 1/m.
+
+    kv_a, kv_b: [T, c]; z_a, z_b: [T, c] or [T, 1].  Returns entries [T//m, c]
+    (and the softmax weights [T//m, 2m, c] when asked; slot order a then b).
+    """
+    kv_a, kv_b, z_a, z_b = map(_f64, (kv_a, kv_b, z_a, z_b))
+    T, c = kv_a.shape
+    assert c == fmt.c and 2 * m <= 512
+    n = T // m
+    ent = np.zeros((n, c))
+    wts = np.zeros((n, 2 * m, c)) if want_weights else None
+    f = fmt._c()
+    _L().orc_csa_compress(T, m, ctypes.byref(f), _ptr(kv_a), _ptr(kv_b), _ptr(z_a), _ptr(z_b),
+                          z_a.shape[1], pos0, _ptr(ent), _ptr(wts))
+    return (ent, wts) if want_weights else ent
+
+
+def hca_compress(kv, z, m_prime: int, fmt: Fmt, pos0: int = 0, want_weights=False):
+    """Non-overlapped softmax-gated compression, rate 1/m'."""
+    kv, z = _f64(kv), _f64(z)
+    T, c = kv.shape
+    assert c == fmt.c
+    n = T // m_prime
+    ent = np.zeros((n, c))
+    wts = np.zeros((n, m_prime, c)) if want_weights else None
+    f = fmt._c()
+    _L().orc_hca_compress(T, m_prime, ctypes.byref(f), _ptr(kv), _ptr(z), z.shape[1], pos0,
+                          _ptr(ent), _ptr(wts))
+    return (ent, wts) if want_weights else ent
+
+
+def window_rows(kv, fmt: Fmt, pos0: int = 0) -> np.ndarray:
+    """Stored window rows: RoPE at pos0+j of RMSNorm(kv[j])."""
+    kv = _f64(kv)
+    out = np.zeros_like(kv)
+    f = fmt._c()
+    _L().orc_window_rows(kv.shape[0], ctypes.byref(f), _ptr(kv), pos0, _ptr(out))
+    return out
+
+
+def _pos(q_pos, Tq):
+    if q_pos is None:
+        q_pos = np.arange(Tq)
+    return np.ascontiguousarray(np.asarray(q_pos, dtype=np.int64).reshape(Tq))
+
+
+def indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:
+    """Lightning-indexer scores [Tq, N]; -inf where the entry is not visible."""
+    q_I, w, k_I = _f64(q_I), _f64(w), _f64(k_I)
+    Tq, HI, dI = q_I.shape
+    N = k_I.shape[0]
+    qp = _pos(q_pos, Tq)
+    sc = np.empty((Tq, N))
+    _L().orc_indexer_scores(Tq, HI, dI, N, _ptr(q_I), _ptr(w), _ptr(k_I), _ptr(qp), m, _ptr(sc))
+    return sc
+
+
+def topk(scores, k: int, m: int, q_pos=None) -> np.ndarray:
+    """Causal top-k of each row: [Tq, k] int32, ascending, -1 padded."""
+    scores = _f64(scores)
+    Tq, N = scores.shape
+    qp = _pos(q_pos, Tq)
+    idx = np.empty((Tq, k), dtype=np.int32)
+    _L().orc_topk(Tq, N, _ptr(scores), _ptr(qp), m, k, _ptr(idx))
+    return idx
+
+
+def attention(q, entries, win, fmt: Fmt, n_win: int, idx=None, m_dense: int = 0, sink=None,
+              q_pos=None, win_pos0: int = 0, scale: float = 0.0, want_lse=False):
+    """Shared-KV MQA over selected (idx) or all visible (m_dense) entries plus the
+    window, with sink.  q: [Tq, H, c]; returns out [Tq, H, c] (and lse [Tq, H])."""
+    q = _f64(q)
+    Tq, H, c = q.shape
+    entries = _f64(entries).reshape(-1, c)
+    win = _f64(win).reshape(-1, c)
+    qp = _pos(q_pos, Tq)
+    if idx is not None:
+        idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32).reshape(Tq, -1))
+        k = idx.shape[1]
+    else:
+        k = 0
+        assert m_dense > 0
+    sk = None if sink is None else _f64(sink).reshape(H)
+    out = np.zeros((Tq, H, c))
+    lse = np.zeros((Tq, H)) if want_lse else None
+    f = fmt._c()
+    _L().orc_attention(Tq, H, ctypes.byref(f), _ptr(q), _ptr(qp), _ptr(entries), entries.shape[0],
+                       _ptr(idx), k, m_dense, _ptr(win), win.shape[0], win_pos0, n_win, _ptr(sk),
+                       float(scale), _ptr(out), _ptr(lse))
+    return (out, lse) if want_lse else out
+
+
+def csa_layer(inp: dict, fmt: Fmt, m: int, k: int, n_win: int, rows=None):
+    """The whole CSA prefill path for one sequence: compress, indexer, top-k,
+    attention.  ``rows`` restricts the attention (and indexer) to those query
+    rows.  Returns dict(entries, win, idx, out)."""
+    ent = csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], m, fmt)
+    win = window_rows(inp["kv_a"], fmt)
+    T = inp["kv_a"].shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    sc = indexer_scores(np.asarray(inp["q_I"])[rows], np.asarray(inp["w"])[rows], inp["k_I"], m,
+                        q_pos=rows)
+    idx = topk(sc, k, m, q_pos=rows)
+    out = attention(np.asarray(inp["q"])[rows], ent, win, fmt, n_win, idx=idx, sink=inp.get("sink"),
+                    q_pos=rows)
+    return dict(entries=ent, win=win, idx=idx, scores=sc, out=out)

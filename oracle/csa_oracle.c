@@ -1,0 +1,358 @@
+/*
+ * CSA / HCA attention-layer core: float64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the parity reference for the CUDA
+ * library and the timed CPU baseline.  Only the test suite, the smoke check of
+ * the package entry module and the CPU-baseline leg of the benchmark may load
+ * it.  It shares no code, header, table or helper with the CUDA path.
+ *
+ * Everything here is a literal, slow restatement of the method in double
+ * precision, one query row at a time (OpenMP spreads rows over host cores).
+ * Sources, by page title and section:
+ *   [P1] "DeepSeek-V4：迈向高效百万 Token 上下文智能" (summary/translation of
+ *        the DeepSeek-V4 report), §3.3 "CSA 与 HCA 混合注意力" -- compression,
+ *        lightning indexer, top-k, shared-KV MQA, HCA, RMSNorm, partial RoPE
+ *        with the output rotated again at position -i, sliding window;
+ *        §3.5 "通用基础设施" -- classical KV blocks and the tail of an
+ *        unfinished block.
+ *   [P2] "DeepSeek V4 完整技术报告", section "混合注意力：CSA + HCA" -- window of
+ *        128 tokens, top-k 512/1024, RoPE on the last 64 dims, learnable sink
+ *        logits that let total attention weight fall below one.
+ *
+ * Readings taken where the pages are silent (each is repeated at its use):
+ *   R1 overlap: entry s pools group a over its own block [m s, m s + m) and
+ *      group b over the previous block [m(s-1), m s); entry 0 has no b slots.
+ *   R2 compression logits are per channel (z_cols == c) or one per token
+ *      (z_cols == 1, broadcast over channels); softmax per channel.
+ *   R4 N = floor(T / m); tail tokens make no entry.
+ *   R5 RMSNorm has unit gain and eps (1e-6 by default), over all c dims;
+ *      it is applied to the query, to compressed entries and to window rows.
+ *   R6 RoPE rotates interleaved pairs (c-r+2i, c-r+2i+1) of the last r dims by
+ *      angle p * base^(-2i/r); an entry sits at position pos0 + m s, window
+ *      row j at pos0 + j, a query at its own position; the output is rotated
+ *      by -pos.
+ *   R7 logit scale 1/sqrt(c) unless given.
+ *   R8 the sink is a per-head logit in the softmax denominator with a zero
+ *      value; absent sink == -inf.
+ *   R9 the window holds the n_win positions pos-n_win+1 .. pos (own token
+ *      included), taken from the per-token rows (group a for CSA).
+ *   R10 one joint softmax over sink, selected entries and window rows.
+ *   R12 top-k order: larger score first, ties to the lower entry index; the
+ *      selected set is emitted in ascending index order, padded with -1.
+ *   R13 entry s is visible to a query at position pos iff its last token
+ *      m(s+1)-1 <= pos, i.e. s < floor((pos+1)/m).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_NO_NORM 1u
+#define ORC_NO_ROPE 2u
+
+typedef struct {
+  int32_t c;          /* entry / head dim */
+  int32_t rope_dims;  /* r: RoPE acts on the last r dims (even) */
+  double rope_base;   /* theta base (10000) */
+  double norm_eps;    /* RMSNorm epsilon */
+  uint32_t flags;     /* ORC_NO_NORM | ORC_NO_ROPE (used only by tests) */
+} orc_fmt;
+
+/* ---- the two per-vector transforms of [P1 §3.3, last paragraph] ---------- */
+
+/* RMSNorm with unit gain (R5): y = x / sqrt(mean(x^2) + eps). */
+static void orc_rmsnorm_inplace(double* x, int c, double eps) {
+  double ss = 0.0;
+  for (int i = 0; i < c; ++i) ss += x[i] * x[i];
+  double inv = 1.0 / sqrt(ss / (double)c + eps);
+  for (int i = 0; i < c; ++i) x[i] *= inv;
+}
+
+/* Partial RoPE on the last r dims at position p (R6). */
+static void orc_rope_inplace(double* x, int c, int r, double base, double p) {
+  int d0 = c - r;
+  for (int i = 0; i < r / 2; ++i) {
+    double theta = pow(base, -2.0 * (double)i / (double)r);
+    double a = p * theta;
+    double cs = cos(a), sn = sin(a);
+    double x0 = x[d0 + 2 * i], x1 = x[d0 + 2 * i + 1];
+    x[d0 + 2 * i] = x0 * cs - x1 * sn;
+    x[d0 + 2 * i + 1] = x0 * sn + x1 * cs;
+  }
+}
+
+/* The transform a stored KV entry (or a query) receives before attention. */
+static void orc_norm_rope(double* x, const orc_fmt* f, double pos) {
+  if (!(f->flags & ORC_NO_NORM)) orc_rmsnorm_inplace(x, f->c, f->norm_eps);
+  if (!(f->flags & ORC_NO_ROPE)) orc_rope_inplace(x, f->c, f->rope_dims, f->rope_base, pos);
+}
+
+/* Exported single-vector forms, so tests can pin each transform by itself. */
+void orc_rmsnorm(int32_t c, double eps, const double* x, double* y) {
+  memcpy(y, x, sizeof(double) * (size_t)c);
+  orc_rmsnorm_inplace(y, c, eps);
+}
+
+void orc_rope(int32_t c, int32_t r, double base, double pos, const double* x, double* y) {
+  memcpy(y, x, sizeof(double) * (size_t)c);
+  orc_rope_inplace(y, c, r, base, pos);
+}
+
+/* R13: number of compressed entries (rate 1/m) visible at query position pos. */
+int64_t orc_visible(int64_t pos, int32_t m, int64_t n_entries) {
+  if (pos < 0) return 0;
+  int64_t v = (pos + 1) / m;
+  return v < n_entries ? v : n_entries;
+}
+
+/* ---- (1) softmax-gated compression [P1 §3.3, CSA and HCA paragraphs] ----- */
+
+/*
+ * Pools one entry: softmax over the listed token slots of the per-channel
+ * compression logits, then the weighted sum of the token rows.
+ * rows/logits: n_slots pointers to a [c] value row and a [z_cols] logit row.
+ * weights_out (optional): [n_slots][c] softmax weights.
+ */
+static void orc_pool(int c, int n_slots, const double* const* rows, const double* const* logits,
+                     int z_cols, double* out, double* weights_out) {
+  for (int ch = 0; ch < c; ++ch) {
+    int zc = (z_cols == 1) ? 0 : ch;
+    double mx = -INFINITY;
+    for (int j = 0; j < n_slots; ++j)
+      if (logits[j][zc] > mx) mx = logits[j][zc];
+    double den = 0.0;
+    for (int j = 0; j < n_slots; ++j) den += exp(logits[j][zc] - mx);
+    double acc = 0.0;
+    for (int j = 0; j < n_slots; ++j) {
+      double wgt = exp(logits[j][zc] - mx) / den;
+      acc += wgt * rows[j][ch];
+      if (weights_out) weights_out[(size_t)j * c + ch] = wgt;
+    }
+    out[ch] = acc;
+  }
+}
+
+/*
+ * CSA compression, rate exactly 1/m with overlapping groups (R1, R2, R4).
+ * ca, cb, za, zb: [T][c] (logits [T][z_cols]); entries: [T/m][c], stored
+ * RMSNorm'd and rotated at position pos0 + m*s.
+ * weights (optional): [T/m][2m][c]; slot order a_0..a_{m-1}, b_0..b_{m-1};
+ * missing b slots of entry 0 get weight 0.
+ */
+void orc_csa_compress(int64_t T, int32_t m, const orc_fmt* f, const double* ca, const double* cb,
+                      const double* za, const double* zb, int32_t z_cols, int64_t pos0,
+                      double* entries, double* weights) {
+  int c = f->c;
+  int64_t n = T / m;
+#pragma omp parallel for schedule(static)
+  for (int64_t s = 0; s < n; ++s) {
+    const double* rows[512];
+    const double* lg[512];
+    int ns = 0;
+    for (int j = 0; j < m; ++j) {
+      int64_t tok = m * s + j;
+      rows[ns] = ca + tok * c;
+      lg[ns] = za + tok * z_cols;
+      ++ns;
+    }
+    if (s >= 1) {
+      for (int j = 0; j < m; ++j) {
+        int64_t tok = m * (s - 1) + j;
+        rows[ns] = cb + tok * c;
+        lg[ns] = zb + tok * z_cols;
+        ++ns;
+      }
+    }
+    double* e = entries + s * c;
+    double* wts = weights ? weights + (size_t)s * 2 * m * c : NULL;
+    if (wts) memset(wts, 0, sizeof(double) * (size_t)2 * m * c);
+    orc_pool(c, ns, rows, lg, z_cols, e, wts);
+    orc_norm_rope(e, f, (double)(pos0 + m * s));
+  }
+}
+
+/*
+ * HCA compression: one group, rate 1/m', no overlap [P1 §3.3, HCA paragraph].
+ * kv, z: [T][c] ([T][z_cols]); entries [T/m'][c] at position pos0 + m' s.
+ * weights (optional): [T/m'][m'][c].
+ */
+void orc_hca_compress(int64_t T, int32_t mp, const orc_fmt* f, const double* kv, const double* z,
+                      int32_t z_cols, int64_t pos0, double* entries, double* weights) {
+  int c = f->c;
+  int64_t n = T / mp;
+#pragma omp parallel for schedule(static)
+  for (int64_t s = 0; s < n; ++s) {
+    const double** rows = (const double**)malloc(sizeof(double*) * (size_t)mp);
+    const double** lg = (const double**)malloc(sizeof(double*) * (size_t)mp);
+    for (int j = 0; j < mp; ++j) {
+      rows[j] = kv + (mp * s + j) * c;
+      lg[j] = z + (mp * s + j) * z_cols;
+    }
+    double* e = entries + s * c;
+    orc_pool(c, mp, rows, lg, z_cols, e, weights ? weights + (size_t)s * mp * c : NULL);
+    orc_norm_rope(e, f, (double)(pos0 + mp * s));
+    free(rows);
+    free(lg);
+  }
+}
+
+/* Window rows: win[j] = RoPE_{pos0+j}(RMSNorm(kv[j])) (R5, R6, R9). */
+void orc_window_rows(int64_t T, const orc_fmt* f, const double* kv, int64_t pos0, double* win) {
+  int c = f->c;
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < T; ++j) {
+    memcpy(win + j * c, kv + j * c, sizeof(double) * (size_t)c);
+    orc_norm_rope(win + j * c, f, (double)(pos0 + j));
+  }
+}
+
+/* ---- (2) lightning indexer and top-k [P1 §3.3, CSA paragraph] ----------- */
+
+/*
+ * I[t,s] = sum_h w[t,h] * ReLU(q_I[t,h] . K_I[s]) for every visible s (R13);
+ * invisible entries get -inf.
+ * q_I: [Tq][H_I][d_I]; w: [Tq][H_I]; k_I: [N][d_I]; q_pos: [Tq];
+ * scores: [Tq][N].
+ */
+void orc_indexer_scores(int64_t Tq, int32_t HI, int32_t dI, int64_t N, const double* qI,
+                        const double* w, const double* kI, const int64_t* q_pos, int32_t m,
+                        double* scores) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < Tq; ++t) {
+    int64_t vis = orc_visible(q_pos[t], m, N);
+    double* row = scores + t * N;
+    for (int64_t s = 0; s < N; ++s) {
+      if (s >= vis) {
+        row[s] = -INFINITY;
+        continue;
+      }
+      double acc = 0.0;
+      for (int h = 0; h < HI; ++h) {
+        const double* q = qI + (t * HI + h) * dI;
+        const double* k = kI + s * dI;
+        double dot = 0.0;
+        for (int d = 0; d < dI; ++d) dot += q[d] * k[d];
+        acc += w[t * HI + h] * (dot > 0.0 ? dot : 0.0);
+      }
+      row[s] = acc;
+    }
+  }
+}
+
+typedef struct {
+  double score;
+  int64_t s;
+} orc_cand;
+
+/* R12: descending score, ties to the lower index -- a strict total order. */
+static int orc_cand_cmp(const void* pa, const void* pb) {
+  const orc_cand* a = (const orc_cand*)pa;
+  const orc_cand* b = (const orc_cand*)pb;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
+  return (a->s < b->s) ? -1 : (a->s > b->s) ? 1 : 0;
+}
+
+static int orc_i32_cmp(const void* pa, const void* pb) {
+  int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+  return (a > b) - (a < b);
+}
+
+/*
+ * Causal per-query top-k over the visible entries; idx: [Tq][k], ascending,
+ * padded with -1 when fewer than k entries are visible.
+ */
+void orc_topk(int64_t Tq, int64_t N, const double* scores, const int64_t* q_pos, int32_t m,
+              int32_t k, int32_t* idx) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < Tq; ++t) {
+    int64_t vis = orc_visible(q_pos[t], m, N);
+    orc_cand* cand = (orc_cand*)malloc(sizeof(orc_cand) * (size_t)(vis > 0 ? vis : 1));
+    for (int64_t s = 0; s < vis; ++s) {
+      cand[s].score = scores[t * N + s];
+      cand[s].s = s;
+    }
+    qsort(cand, (size_t)vis, sizeof(orc_cand), orc_cand_cmp);
+    int64_t keff = vis < k ? vis : k;
+    int32_t* out = idx + t * k;
+    for (int64_t i = 0; i < keff; ++i) out[i] = (int32_t)cand[i].s;
+    qsort(out, (size_t)keff, sizeof(int32_t), orc_i32_cmp);
+    for (int64_t i = keff; i < k; ++i) out[i] = -1;
+    free(cand);
+  }
+}
+
+/* ---- (3) shared-KV MQA with window and sink [P1 §3.3; P2] ---------------- */
+
+/*
+ * One attention layer output for Tq query rows.
+ *   q: [Tq][H][c] raw queries; q_pos: [Tq] absolute positions.
+ *   entries: [N][c] stored (transformed) compressed entries.
+ *   idx: [Tq][k] selected entries (CSA) or NULL for dense HCA, where every
+ *        visible entry s < floor((pos+1)/m_dense) is used.
+ *   win: [Tw][c] stored window rows, row j at position win_pos0 + j.
+ *   sink: [H] logits or NULL (== -inf).
+ *   out: [Tq][H][c]; lse (optional): [Tq][H] natural log of the softmax
+ *        denominator (sink term included).
+ * One joint softmax over {sink} U selected entries U window rows (R8-R10),
+ * logits scale * q^ . key with q^ = RoPE_pos(RMSNorm(q)), then the weighted
+ * sum of the same rows (K = V), then the output rotated by -pos.
+ */
+void orc_attention(int64_t Tq, int32_t H, const orc_fmt* f, const double* q, const int64_t* q_pos,
+                   const double* entries, int64_t N, const int32_t* idx, int32_t k, int32_t m_dense,
+                   const double* win, int64_t Tw, int64_t win_pos0, int32_t n_win,
+                   const double* sink, double scale, double* out, double* lse) {
+  int c = f->c;
+  if (!(scale > 0.0)) scale = 1.0 / sqrt((double)c);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < Tq; ++t) {
+    int64_t pos = q_pos[t];
+    /* key list for this query row */
+    int64_t cap = (idx ? k : (N > 0 ? N : 0)) + n_win + 1;
+    const double** keys = (const double**)malloc(sizeof(double*) * (size_t)cap);
+    int64_t nk = 0;
+    if (idx) {
+      for (int i = 0; i < k; ++i) {
+        int32_t s = idx[t * k + i];
+        if (s >= 0 && s < N) keys[nk++] = entries + (int64_t)s * c;
+      }
+    } else {
+      int64_t vis = orc_visible(pos, m_dense, N);
+      for (int64_t s = 0; s < vis; ++s) keys[nk++] = entries + s * c;
+    }
+    int64_t jlo = pos - n_win + 1;
+    if (jlo < win_pos0) jlo = win_pos0;
+    int64_t jhi = pos;
+    if (jhi > win_pos0 + Tw - 1) jhi = win_pos0 + Tw - 1;
+    for (int64_t j = jlo; j <= jhi; ++j) keys[nk++] = win + (j - win_pos0) * c;
+
+    double* qh = (double*)malloc(sizeof(double) * (size_t)c);
+    double* lg = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1));
+    for (int h = 0; h < H; ++h) {
+      memcpy(qh, q + (t * H + h) * c, sizeof(double) * (size_t)c);
+      orc_norm_rope(qh, f, (double)pos);
+      double zs = sink ? sink[h] : -INFINITY;
+      double mx = zs;
+      for (int64_t i = 0; i < nk; ++i) {
+        double d = 0.0;
+        for (int e = 0; e < c; ++e) d += qh[e] * keys[i][e];
+        lg[i] = scale * d;
+        if (lg[i] > mx) mx = lg[i];
+      }
+      double den = isinf(zs) && zs < 0 ? 0.0 : exp(zs - mx);
+      double* o = out + (t * H + h) * c;
+      for (int e = 0; e < c; ++e) o[e] = 0.0;
+      for (int64_t i = 0; i < nk; ++i) {
+        double p = exp(lg[i] - mx);
+        den += p;
+        for (int e = 0; e < c; ++e) o[e] += p * keys[i][e];
+      }
+      for (int e = 0; e < c; ++e) o[e] = (den > 0.0) ? o[e] / den : 0.0;
+      if (!(f->flags & ORC_NO_ROPE)) orc_rope_inplace(o, c, f->rope_dims, f->rope_base, -(double)pos);
+      if (lse) lse[t * H + h] = log(den) + mx;
+    }
+    free(qh);
+    free(lg);
+    free(keys);
+  }
+}
