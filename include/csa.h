@@ -1,0 +1,212 @@
+/*
+ * csa.h -- C ABI of libcsa.so: the CSA/HCA hybrid attention-layer core on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operations restate the attention layer of DeepSeek-V4 as described on
+ * the page "DeepSeek-V4：迈向高效百万 Token 上下文智能" (a summary/translation of
+ * the DeepSeek-V4 report), §3.3 "CSA 与 HCA 混合注意力", and on the page
+ * "DeepSeek V4 完整技术报告", section "混合注意力：CSA + HCA":
+ *   - csa_compress / hca_compress: softmax-gated compression of per-token KV
+ *     into compressed entries (CSA: two overlapping groups, rate 1/m; HCA: one
+ *     group, rate 1/m'), followed by RMSNorm and partial RoPE;
+ *   - indexer_scores_topk: the lightning-indexer score
+ *     I[t,s] = sum_h w[t,h] ReLU(q_I[t,h] . K_I[s]) and a causal per-query top-k;
+ *   - sparse_mqa_attn / dense_hca_attn: multi-query attention in which each
+ *     compressed entry is both key and value, over the selected entries (CSA)
+ *     or all visible entries (HCA), plus a sliding window of per-token rows and
+ *     a per-head sink logit, with RMSNorm + RoPE on the query and the output
+ *     rotated back by the query position.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers, row-major and contiguous, owned
+ *     by the caller; the library allocates nothing.  Tensors must start on a
+ *     16-byte boundary.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and are stateless and reentrant.
+ *   - Host-side validation runs before any launch and returns CSA_E_ARG or
+ *     CSA_E_UNSUPPORTED without touching device memory.
+ *   - Errors detected by a kernel (a bounded wait that expired, an index out of
+ *     range, a logit beyond the static softmax bound) are written to a status
+ *     word at the start of the workspace; csa_check_status() reads and clears
+ *     it.  Kernels never trap.
+ *   - Positions: token j of a prefill sequence sits at pos0 + j; compressed
+ *     entry s covers tokens [m s, m s + m) counted from the start of the
+ *     sequence and is visible to a query at position p iff s < floor((p+1)/m).
+ *   - Stored entries and window rows are the TRANSFORMED rows (RMSNorm'd and
+ *     rotated at their own positions), as a KV cache holds them; queries are
+ *     raw and are normalised and rotated inside the attention calls.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+typedef int32_t csa_status;
+#define CSA_OK 0
+#define CSA_E_ARG 1          /* null pointer, negative size, misalignment, bad enum */
+#define CSA_E_UNSUPPORTED 2  /* well-formed but outside what the kernels implement */
+#define CSA_E_CUDA 3         /* a CUDA runtime call or kernel launch failed */
+#define CSA_E_DEVICE 4       /* a kernel reported an error in the status word */
+#define CSA_E_WORKSPACE 5    /* workspace missing or smaller than required */
+
+/* device status-word codes (the `detail` of csa_check_status) */
+#define CSA_DEV_OK 0u
+#define CSA_DEV_TIMEOUT 1u     /* a bounded mbarrier wait ran out; results invalid */
+#define CSA_DEV_RANGE 2u       /* a logit exceeded the static softmax bound (un-normalised keys) */
+#define CSA_DEV_BAD_INDEX 3u   /* an index outside [-1, N) was skipped */
+
+/* ---- element types and flags ---------------------------------------- */
+#define CSA_F32 0   /* float32 tensors, float32 arithmetic (CUDA cores) */
+#define CSA_BF16 1  /* bfloat16 tensors, float32 accumulation (tensor cores where dense) */
+
+#define CSA_F_NO_NORM 1u   /* skip RMSNorm (test hook) */
+#define CSA_F_NO_ROPE 2u   /* skip RoPE and the output rotation (test hook) */
+#define CSA_F_PORTABLE 4u  /* use the CUDA-core kernels even where a tensor-core kernel exists */
+
+/* Entry format shared by all calls.  c: entry / head dim (c/vec a power of two,
+ * vec = 8 for bf16, 4 for f32); rope_dims: r, even, <= c, RoPE on dims
+ * [c-r, c) in interleaved pairs (c-r+2i, c-r+2i+1) with angle
+ * pos * rope_base^(-2i/r); norm_eps: RMSNorm epsilon (unit gain). */
+typedef struct csa_fmt {
+  int32_t c;
+  int32_t rope_dims;
+  float rope_base;
+  float norm_eps;
+  uint32_t flags;
+} csa_fmt;
+
+/* Workspace ops for csa_workspace_bytes(). */
+#define CSA_OP_INDEXER 1
+#define CSA_OP_SPARSE_ATTN 2
+#define CSA_OP_DENSE_ATTN 3
+
+/* ---- (1) compression ------------------------------------------------ */
+
+/*
+ * CSA overlapped softmax-gated compression [§3.3 of the summary page: two
+ * groups of KV entries and compression weights, a row softmax over 2m
+ * elements, overlapping index ranges so that the rate is exactly 1/m].
+ *   entry[b,s,ch] = sum_{j<m} sa_j kv_a[b,ms+j,ch] + sum_{j<m} sb_j kv_b[b,m(s-1)+j,ch]
+ * with (sa, sb) = softmax over the 2m logits z_a[b,ms+j,.], z_b[b,m(s-1)+j,.]
+ * taken per channel (z_cols == c) or per token (z_cols == 1); entry 0 has no
+ * b group.  Each entry is then RMSNorm'd and rotated at position pos0 + m s.
+ *   kv_a, kv_b, z_a, z_b: [B, T, c] ([B, T, z_cols] for the logits), `dtype`.
+ *   entries (out): [B, floor(T/m), c].  Tail tokens (T mod m) make no entry.
+ *   win_out (out, optional, may be NULL): [B, T, c] window rows
+ *       RoPE_{pos0+j}(RMSNorm(kv_a[b,j])).
+ * Errors: CSA_E_ARG for null/misaligned pointers or T < 0, m < 1;
+ *         CSA_E_UNSUPPORTED for 2m > 256 or an unsupported c.
+ */
+csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const csa_fmt* fmt,
+                        const void* kv_a, const void* kv_b, const void* z_a, const void* z_b,
+                        int32_t z_cols, int64_t pos0, void* entries, void* win_out,
+                        void* stream);
+
+/*
+ * HCA compression [§3.3 of the summary page: a larger rate m' with no
+ * overlap, otherwise as CSA]:  entry[b,s] = sum_{j<m'} s_j kv[b,m's+j] with s
+ * the per-channel softmax of z over the m' tokens of block s; then RMSNorm and
+ * RoPE at pos0 + m' s.  kv, z: [B, T, c] / [B, T, z_cols]; entries:
+ * [B, floor(T/m'), c]; win_out (optional): [B, T, c] = RoPE_{pos0+j}(RMSNorm(kv[b,j])).
+ * Errors as csa_compress; m' up to 4096.
+ */
+csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, const csa_fmt* fmt,
+                        const void* kv, const void* z, int32_t z_cols, int64_t pos0, void* entries,
+                        void* win_out, void* stream);
+
+/* ---- (2) lightning indexer + top-k ----------------------------------- */
+
+/*
+ * Lightning-indexer scores and causal top-k [§3.3 of the summary page:
+ * I[t,s] = sum_h w[t,h] ReLU(q_I[t,h] . K_I[s]); the top-k entries form the
+ * candidate set].  For each (b, t) with position p = q_pos[b,t] (or t when
+ * q_pos is NULL), the visible entries are s < min(N, floor((p+1)/m)); the
+ * k_eff = min(k, visible) largest scores are selected, ties going to the lower
+ * index, and emitted in ascending index order, padded with -1.
+ *   q_I: [B, Tq, H_I, d_I] (dtype); w: [B, Tq, H_I] float32;
+ *   k_I: [B, N, d_I] (dtype); q_pos: [B, Tq] int64 or NULL;
+ *   idx_out: [B, Tq, k] int32; score_out: [B, Tq, k] float32 or NULL (the
+ *   score of each selected index, -inf for padding).
+ *   ws: workspace of at least csa_workspace_bytes(CSA_OP_INDEXER, ...) bytes,
+ *   zero-filled once before its first use (status word at offset 0).
+ * Arithmetic: bf16 products with float32 accumulation (exact for small
+ * integer inputs); float32 throughout for CSA_F32.
+ */
+csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                               const void* q_I, const float* w, const void* k_I, int64_t N,
+                               const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                               float* score_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- (3) shared-KV MQA ------------------------------------------------ */
+
+/*
+ * Sparse MQA of a CSA layer [§3.3 of the summary page: MQA in which each
+ * compressed entry is both key and value, over the top-k entries; RMSNorm on
+ * the query; partial RoPE on query, entries and output, the output rotated
+ * again at position -i; a sliding-window branch of n_win uncompressed rows.
+ * The page "DeepSeek V4 完整技术报告" adds the learnable per-head sink logit].
+ * For each (b, t, h), with p = q_pos[b,t] (or t):
+ *   q^ = RoPE_p(RMSNorm(q[b,t,h]));
+ *   keys = {entries[b, idx[b,t,i]] : idx >= 0} U {win[b, j - win_pos0[b]] :
+ *           max(p - n_win + 1, win_pos0) <= j <= min(p, win_pos0 + Tw - 1)};
+ *   out[b,t,h] = RoPE_{-p}( sum_key e^{l} key / (e^{sink[h]} + sum_key e^{l}) ),
+ *   l = scale * q^ . key  (scale <= 0 means 1/sqrt(c); sink NULL means -inf).
+ *   q: [B, Tq, H, c]; entries: [B, N, c]; idx: [B, Tq, k] int32 (-1 = none);
+ *   win: [B, Tw, c]; win_pos0: [B] int64 or NULL (0); out: [B, Tq, H, c].
+ * The bf16 tensor-core kernel requires the stored keys to be RMS-normalised
+ * (as the compression calls produce them): it uses the static logit bound
+ * scale*|q^|*sqrt(c) in place of a running maximum and flags CSA_DEV_RANGE
+ * when a logit goes more than 60 (natural log) beyond it.
+ */
+csa_status sparse_mqa_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
+                           const void* q, const int64_t* q_pos, const void* entries, int64_t N,
+                           const int32_t* idx, int32_t k, const void* win, int64_t Tw,
+                           const int64_t* win_pos0, int32_t n_win, const float* sink, float scale,
+                           void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dense MQA of an HCA layer [§3.3 of the summary page: HCA keeps dense
+ * attention, otherwise as CSA]: as sparse_mqa_attn with the key set
+ * {entries[b, s] : s < min(N, floor((p+1)/m_prime))} U window rows.
+ */
+csa_status dense_hca_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
+                          const void* q, const int64_t* q_pos, const void* entries, int64_t N,
+                          int32_t m_prime, const void* win, int64_t Tw, const int64_t* win_pos0,
+                          int32_t n_win, const float* sink, float scale, void* out, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* ---- workspace and status --------------------------------------------- */
+
+/*
+ * Bytes of workspace the op needs for these shapes (always >= 256: the
+ * status word).  op: CSA_OP_*; unused arguments are ignored (k for the dense
+ * op, H and c for the indexer).  Returns 0 for an unknown op.
+ */
+size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int32_t H, int32_t c,
+                           int64_t N, int32_t k, int32_t n_win);
+
+/*
+ * Synchronises `stream`, reads the device status word at the start of `ws`
+ * and clears it.  Returns CSA_OK, CSA_E_DEVICE (with *detail set to a
+ * CSA_DEV_* code when detail != NULL), or CSA_E_CUDA.
+ */
+csa_status csa_check_status(void* ws, void* stream, uint32_t* detail);
+
+/* Human-readable name of a status code (static storage). */
+const char* csa_status_string(csa_status s);
+
+/* Number of kernels this library has launched in this process so far (all
+ * threads, all devices).  For launch accounting in benchmarks. */
+unsigned long long csa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,262 @@
+// extern "C" entry points of libcsa.so: argument validation, workspace
+// layout, kernel selection and the device status word.  See include/csa.h for
+// the contract of each call.
+#include <atomic>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.h"
+
+using namespace csa;
+
+namespace {
+
+std::atomic<unsigned long long> g_launches{0};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+inline cudaStream_t S(void* stream) { return reinterpret_cast<cudaStream_t>(stream); }
+
+inline csa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_E_CUDA; }
+
+// Common checks of the entry format.
+csa_status check_fmt(int32_t dtype, const csa_fmt* fmt, Fmt* out) {
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
+  if (fmt == nullptr) return CSA_E_ARG;
+  if (fmt->c <= 0 || fmt->rope_dims < 0 || fmt->rope_dims > fmt->c || (fmt->rope_dims & 1))
+    return CSA_E_ARG;
+  if (!(fmt->norm_eps >= 0.f) || !(fmt->rope_base > 0.f)) return CSA_E_ARG;
+  if (fmt->flags & ~(CSA_F_NO_NORM | CSA_F_NO_ROPE | CSA_F_PORTABLE)) return CSA_E_ARG;
+  const int vec = dtype == CSA_BF16 ? 8 : 4;
+  if (fmt->c % vec != 0 || !pow2(fmt->c / vec) || fmt->c / vec > 256) return CSA_E_UNSUPPORTED;
+  out->c = fmt->c;
+  out->r = fmt->rope_dims;
+  out->base = fmt->rope_base;
+  out->eps = fmt->norm_eps;
+  out->flags = fmt->flags;
+  return CSA_OK;
+}
+
+csa_status compress_common(int32_t dtype, int64_t B, int64_t T, int32_t m, bool overlap,
+                           const csa_fmt* fmt, const void* kv_a, const void* kv_b,
+                           const void* z_a, const void* z_b, int32_t z_cols, int64_t pos0,
+                           void* entries, void* win_out, void* stream) {
+  Fmt f;
+  csa_status st = check_fmt(dtype, fmt, &f);
+  if (st != CSA_OK) return st;
+  if (B < 0 || T < 0 || m < 1 || B > 65535) return CSA_E_ARG;
+  if (z_cols != 1 && z_cols != f.c) return CSA_E_ARG;
+  if (overlap ? (2 * m > 256) : (m > 4096)) return CSA_E_UNSUPPORTED;
+  const int64_t n = T / m;
+  if (B == 0 || T == 0) return CSA_OK;
+  if (!kv_a || !z_a || (overlap && (!kv_b || !z_b))) return CSA_E_ARG;
+  if (n > 0 && !entries) return CSA_E_ARG;
+  if (!aligned16(kv_a) || (overlap && !aligned16(kv_b)) || (entries && !aligned16(entries)) ||
+      (win_out && !aligned16(win_out)))
+    return CSA_E_ARG;
+  if (z_cols != 1 && (!aligned16(z_a) || (overlap && !aligned16(z_b)))) return CSA_E_ARG;
+  if (n == 0 && !win_out) return CSA_OK;
+  if (n + 1 > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  CompressParams p{};
+  p.kv_a = kv_a;
+  p.kv_b = kv_b;
+  p.z_a = z_a;
+  p.z_b = z_b;
+  p.z_cols = z_cols;
+  p.T = T;
+  p.n_entries = n;
+  p.m = m;
+  p.overlap = overlap ? 1 : 0;
+  p.f = f;
+  p.pos0 = pos0;
+  p.entries = entries;
+  p.win = win_out;
+  g_launches.fetch_add(1);
+  return cuda_status(launch_compress(dtype, p, B, S(stream)));
+}
+
+unsigned* status_word(void* ws) { return static_cast<unsigned*>(ws); }
+
+}  // namespace
+
+extern "C" {
+
+csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const csa_fmt* fmt,
+                        const void* kv_a, const void* kv_b, const void* z_a, const void* z_b,
+                        int32_t z_cols, int64_t pos0, void* entries, void* win_out,
+                        void* stream) {
+  return compress_common(dtype, B, T, m, true, fmt, kv_a, kv_b, z_a, z_b, z_cols, pos0, entries,
+                         win_out, stream);
+}
+
+csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, const csa_fmt* fmt,
+                        const void* kv, const void* z, int32_t z_cols, int64_t pos0, void* entries,
+                        void* win_out, void* stream) {
+  return compress_common(dtype, B, T, m_prime, false, fmt, kv, nullptr, z, nullptr, z_cols, pos0,
+                         entries, win_out, stream);
+}
+
+size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int32_t H, int32_t c,
+                           int64_t N, int32_t k, int32_t n_win) {
+  if (B < 0 || Tq < 0 || N < 0) return 0;
+  switch (op) {
+    case CSA_OP_INDEXER: {
+      size_t a = indexer_portable_scratch(B, Tq, N, k);
+      size_t b = dtype == CSA_BF16 ? indexer_tc_scratch(B, Tq, N, k) : 0;
+      return kWsScratch + (a > b ? a : b);
+    }
+    case CSA_OP_SPARSE_ATTN:
+    case CSA_OP_DENSE_ATTN: {
+      int64_t max_keys = (op == CSA_OP_SPARSE_ATTN ? (int64_t)k : N) + n_win;
+      size_t b = dtype == CSA_BF16 ? attn_tc_scratch(B, Tq, H, c, max_keys) : 0;
+      return kWsScratch + b;
+    }
+    default:
+      return 0;
+  }
+}
+
+csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                               const void* q_I, const float* w, const void* k_I, int64_t N,
+                               const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                               float* score_out, void* ws, size_t ws_bytes, void* stream) {
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
+  if (B < 0 || Tq < 0 || N < 0 || H_I <= 0 || d_I <= 0 || m < 1 || k < 1) return CSA_E_ARG;
+  if (B > 65535 || Tq > 0x7fffffffLL || N > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  if (H_I > 64 || d_I > 1024) return CSA_E_UNSUPPORTED;
+  if (B == 0 || Tq == 0) return CSA_OK;
+  if (!q_I || !w || !idx_out || (N > 0 && !k_I)) return CSA_E_ARG;
+  if (!ws) return CSA_E_WORKSPACE;
+  if (ws_bytes < csa_workspace_bytes(CSA_OP_INDEXER, dtype, B, Tq, 0, 0, N, k, 0))
+    return CSA_E_WORKSPACE;
+  IndexerParams p{};
+  p.B = B;
+  p.Tq = Tq;
+  p.HI = H_I;
+  p.dI = d_I;
+  p.q_I = q_I;
+  p.w = w;
+  p.k_I = k_I;
+  p.N = N;
+  p.q_pos = q_pos;
+  p.m = m;
+  p.k = k;
+  p.idx_out = idx_out;
+  p.score_out = score_out;
+  p.status = status_word(ws);
+  p.scratch = static_cast<char*>(ws) + kWsScratch;
+  p.scratch_bytes = ws_bytes - kWsScratch;
+  if (dtype == CSA_BF16 && indexer_tc_supported(p)) {
+    unsigned long long n_launch = 0;
+    cudaError_t e = launch_indexer_tc(p, S(stream), &n_launch);
+    g_launches.fetch_add(n_launch);
+    return cuda_status(e);
+  }
+  g_launches.fetch_add(2);
+  return cuda_status(launch_indexer_portable(dtype, p, S(stream)));
+}
+
+static csa_status attn_common(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
+                              bool sparse, const void* q, const int64_t* q_pos, const void* entries, int64_t N,
+                              const int32_t* idx, int32_t k, int32_t m_dense, const void* win,
+                              int64_t Tw, const int64_t* win_pos0, int32_t n_win,
+                              const float* sink, float scale, void* out, void* ws,
+                              size_t ws_bytes, void* stream) {
+  Fmt f;
+  csa_status st = check_fmt(dtype, fmt, &f);
+  if (st != CSA_OK) return st;
+  if (B < 0 || Tq < 0 || H <= 0 || N < 0 || Tw < 0 || n_win < 0) return CSA_E_ARG;
+  if (sparse ? k < 0 : m_dense < 1) return CSA_E_ARG;
+  if (B > 65535 || Tq > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  if (f.c % 64 != 0 || f.c > 512) return CSA_E_UNSUPPORTED;
+  if (B == 0 || Tq == 0) return CSA_OK;
+  if (!q || !out || (N > 0 && !entries) || (Tw > 0 && !win)) return CSA_E_ARG;
+  if (!aligned16(q) || !aligned16(out) || (entries && !aligned16(entries)) ||
+      (win && !aligned16(win)))
+    return CSA_E_ARG;
+  if (!ws) return CSA_E_WORKSPACE;
+  const int op = sparse ? CSA_OP_SPARSE_ATTN : CSA_OP_DENSE_ATTN;
+  if (ws_bytes < csa_workspace_bytes(op, dtype, B, Tq, H, f.c, N, k, n_win)) return CSA_E_WORKSPACE;
+  AttnParams p{};
+  p.B = B;
+  p.Tq = Tq;
+  p.H = H;
+  p.f = f;
+  p.q = q;
+  p.q_pos = q_pos;
+  p.entries = entries;
+  p.N = N;
+  p.sparse = sparse ? 1 : 0;
+  p.idx = idx;
+  p.k = sparse ? k : 0;
+  p.m_dense = m_dense;
+  p.win = win;
+  p.Tw = Tw;
+  p.win_pos0 = win_pos0;
+  p.n_win = n_win;
+  p.sink = sink;
+  p.scale = scale;
+  p.out = out;
+  p.status = status_word(ws);
+  p.scratch = static_cast<char*>(ws) + kWsScratch;
+  p.scratch_bytes = ws_bytes - kWsScratch;
+  if (dtype == CSA_BF16 && attn_tc_supported(p)) {
+    unsigned long long n_launch = 0;
+    cudaError_t e = launch_attn_tc(p, S(stream), &n_launch);
+    g_launches.fetch_add(n_launch);
+    return cuda_status(e);
+  }
+  g_launches.fetch_add(1);
+  return cuda_status(launch_attn_portable(dtype, p, S(stream)));
+}
+
+csa_status sparse_mqa_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
+                           const void* q, const int64_t* q_pos, const void* entries, int64_t N,
+                           const int32_t* idx, int32_t k, const void* win, int64_t Tw,
+                           const int64_t* win_pos0, int32_t n_win, const float* sink, float scale,
+                           void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (k < 0 || (!idx && k > 0)) return CSA_E_ARG;
+  return attn_common(dtype, B, Tq, H, fmt, true, q, q_pos, entries, N, idx, k, 1, win, Tw,
+                     win_pos0, n_win, sink, scale, out, ws, ws_bytes, stream);
+}
+
+csa_status dense_hca_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
+                          const void* q, const int64_t* q_pos, const void* entries, int64_t N,
+                          int32_t m_prime, const void* win, int64_t Tw, const int64_t* win_pos0,
+                          int32_t n_win, const float* sink, float scale, void* out, void* ws,
+                          size_t ws_bytes, void* stream) {
+  return attn_common(dtype, B, Tq, H, fmt, false, q, q_pos, entries, N, nullptr, 0, m_prime, win,
+                     Tw, win_pos0, n_win, sink, scale, out, ws, ws_bytes, stream);
+}
+
+csa_status csa_check_status(void* ws, void* stream, uint32_t* detail) {
+  if (!ws) return CSA_E_ARG;
+  cudaError_t e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return CSA_E_CUDA;
+  unsigned word[2] = {0u, 0u};
+  e = cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return CSA_E_CUDA;
+  if (detail) *detail = word[0];
+  if (word[0] == 0u) return CSA_OK;
+  e = cudaMemset(ws, 0, sizeof(word));
+  if (e != cudaSuccess) return CSA_E_CUDA;
+  return CSA_E_DEVICE;
+}
+
+const char* csa_status_string(csa_status s) {
+  switch (s) {
+    case CSA_OK: return "ok";
+    case CSA_E_ARG: return "invalid argument";
+    case CSA_E_UNSUPPORTED: return "unsupported shape or format";
+    case CSA_E_CUDA: return "CUDA error";
+    case CSA_E_DEVICE: return "device-side error (see status word)";
+    case CSA_E_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+unsigned long long csa_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

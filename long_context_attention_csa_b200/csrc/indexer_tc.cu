@@ -1,0 +1,568 @@
+// Lightning indexer with a fused causal top-k on the 5th-generation tensor
+// cores (tcgen05, accumulators in TMEM, operands staged by TMA).
+//
+// Method: page "DeepSeek-V4：迈向高效百万 Token 上下文智能", §3.3 (CSA) --
+// I[t,s] = sum_h w[t,h] ReLU(q_I[t,h] . K_I[s]); the top-k entries of each
+// query are its candidate set.  Readings: entry s is visible iff
+// s < floor((p+1)/m); ties go to the lower index; output ascending, -1 padded.
+//
+// Layout: compressed entries on the MMA's M side (128 per tile, one per TMEM
+// lane) and (token, head) pairs on N (TOK tokens x 64 heads), K = d_I = 128.
+// Every TMEM lane then holds all heads of one entry for TOK tokens, so the
+// epilogue sum_h w ReLU(.) is a per-thread loop with no cross-lane traffic.
+//   warp 0      TMA producer: q_I block once, K_I tiles through a ring;
+//   warp 1      TMEM owner and single-thread MMA issuer (8 MMAs per tile);
+//   warps 2..5  epilogue: TMEM -> registers -> scores in shared memory
+//               (two TMEM accumulators so tile i+1's MMAs overlap tile i's
+//               epilogue); afterwards one warp per token runs an exact radix
+//               select over the scores and an ordered compaction.
+// The score matrix never reaches HBM.  A CTA covers the entries of one chunk
+// (2048 for 4-token groups, 4096 for single tokens); when the entries span
+// several chunks each CTA emits its chunk's top-k as candidates and a merge
+// kernel selects the final k (the union of per-chunk top-k sets contains the
+// global top-k under the same tie rule).
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tc.h"
+#include "tma_host.h"
+
+namespace csa {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;   // entries per tile
+constexpr int kDI = 128;   // indexer dim
+constexpr int kHI = 64;    // indexer heads
+constexpr int kTileBytes = kBM * kDI * 2;     // 32 KB (two 128-byte-swizzled column halves)
+constexpr int kThreads = 192;
+
+template <int TOK> struct Cfg;
+template <> struct Cfg<4> { static constexpr int kStages = 3; static constexpr int kChunk = 2048; };
+template <> struct Cfg<1> { static constexpr int kStages = 4; static constexpr int kChunk = 4096; };
+
+template <int TOK>
+struct Smem {
+  static constexpr int kB = TOK * kHI * kDI * 2;           // q_I block
+  static constexpr int kStages = Cfg<TOK>::kStages;
+  static constexpr int kChunk = Cfg<TOK>::kChunk;
+  static constexpr int off_b = 0;
+  static constexpr int off_a = kB;
+  static constexpr int off_scores = off_a + kStages * kTileBytes;
+  static constexpr int off_w = off_scores + TOK * kChunk * 4;
+  static constexpr int off_hist = off_w + TOK * kHI * 4;
+  static constexpr int off_bar = off_hist + TOK * 256 * 4;
+  static constexpr int kBars = 2 * kStages + 6;
+  static constexpr int off_misc = off_bar + kBars * 8;
+  static constexpr int bytes = off_misc + 64;
+};
+
+struct TcIdxArgs {
+  int64_t Tq, N;
+  int m, k;
+  int n_chunks;
+  const float* w;
+  const int64_t* q_pos;
+  int32_t* idx_out;
+  float* score_out;
+  float* cand_score;   // [B*Tq][n_chunks][k] when n_chunks > 1
+  int32_t* cand_idx;
+  unsigned* status;
+};
+
+__device__ __forceinline__ int64_t vis_count(int64_t pos, int m, int64_t N) {
+  if (pos < 0) return 0;
+  int64_t v = (pos + 1) / m;
+  return v < N ? v : N;
+}
+
+__device__ __forceinline__ unsigned score_key(float f) {
+  unsigned u = __float_as_uint(f + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Warp-level exact top-k of sc[0..n) (ties to the lower index), written in
+// ascending index order as (e0 + j, sc[j]) and padded to k with (-1, -inf).
+__device__ void warp_topk(const float* sc, int n, int k, int64_t e0, unsigned* hist,
+                          int32_t* out_idx, float* out_score) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  unsigned tau = 0u, need_eq = 0u;
+  bool take_all = n <= k;
+  if (!take_all) {
+    unsigned prefix = 0u, mask = 0u;
+    unsigned rem = (unsigned)k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
+      __syncwarp();
+      for (int j = lane; j < n; j += 32) {
+        unsigned key = score_key(sc[j]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      // lane L owns digits 255-8L .. 248-8L (descending)
+      unsigned c[8], sL = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = hist[255 - 8 * lane - i];
+        sL += c[i];
+      }
+      unsigned incl = sL;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      unsigned pre = incl - sL;  // count of digits above this lane's group
+      bool here = pre < rem && rem <= incl;
+      unsigned digit = 0, above = 0;
+      if (here) {
+        unsigned run = pre;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (run + c[i] >= rem) {
+            digit = 255u - 8u * lane - i;
+            above = run;
+            break;
+          }
+          run += c[i];
+        }
+      }
+      unsigned who = __ballot_sync(0xffffffffu, here);
+      int src = __ffs(who) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      prefix |= digit << shift;
+      mask |= 255u << shift;
+      rem -= above;
+      __syncwarp();
+    }
+    tau = prefix;
+    need_eq = rem;
+  }
+  unsigned run_sel = 0, run_eq = 0;
+  for (int base = 0; base < n; base += 32) {
+    int j = base + lane;
+    bool valid = j < n;
+    float s = valid ? sc[j] : 0.f;
+    unsigned key = valid ? score_key(s) : 0u;
+    bool take;
+    if (take_all) {
+      take = valid;
+    } else {
+      bool gt = valid && key > tau;
+      bool eq = valid && key == tau;
+      unsigned beq = __ballot_sync(0xffffffffu, eq);
+      unsigned eq_rank = run_eq + __popc(beq & lt);
+      take = gt || (eq && eq_rank < need_eq);
+      run_eq += __popc(beq);
+    }
+    unsigned bt = __ballot_sync(0xffffffffu, take);
+    unsigned at = run_sel + __popc(bt & lt);
+    if (take) {
+      out_idx[at] = (int32_t)(e0 + j);
+      if (out_score) out_score[at] = s;
+    }
+    run_sel += __popc(bt);
+  }
+  for (int p = (int)run_sel + lane; p < k; p += 32) {
+    out_idx[p] = -1;
+    if (out_score) out_score[p] = -INFINITY;
+  }
+}
+
+template <int TOK>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_k, TcIdxArgs a) {
+  using L = Smem<TOK>;
+  constexpr int kStages = L::kStages;
+  constexpr int kChunk = L::kChunk;
+  constexpr int kN = TOK * kHI;                 // MMA N
+  constexpr uint32_t kCols = 2 * kN;            // two accumulators
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kN, 0, 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sB = sm + L::off_b;
+  uint8_t* sA = sm + L::off_a;
+  float* scores = reinterpret_cast<float*>(sm + L::off_scores);
+  float* sw = reinterpret_cast<float*>(sm + L::off_w);
+  unsigned* hist = reinterpret_cast<unsigned*>(sm + L::off_hist);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::off_bar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* bfull = tempty + 2;
+  uint64_t* drain = bfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::off_misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::off_misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int group = gridDim.y - 1 - blockIdx.y;   // heaviest causal groups first
+  const int b = blockIdx.z;
+  const int64_t t0 = (int64_t)group * TOK;
+  const int64_t e0 = (int64_t)chunk * kChunk;
+
+  // visibility of the TOK tokens and the entry range this CTA scores
+  int64_t vis[TOK];
+  int64_t vmax = 0;
+#pragma unroll
+  for (int i = 0; i < TOK; ++i) {
+    int64_t t = t0 + i;
+    vis[i] = 0;
+    if (t < a.Tq) {
+      int64_t row = (int64_t)b * a.Tq + t;
+      int64_t pos = a.q_pos ? a.q_pos[row] : t;
+      vis[i] = vis_count(pos, a.m, a.N);
+    }
+    vmax = vis[i] > vmax ? vis[i] : vmax;
+  }
+  int64_t e_hi = e0 + kChunk < vmax ? e0 + kChunk : vmax;
+  const int n_tiles = e_hi > e0 ? (int)((e_hi - e0 + kBM - 1) / kBM) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    mbar_init(bfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  for (int i = threadIdx.x; i < TOK * kHI; i += blockDim.x) {
+    int64_t t = t0 + i / kHI;
+    sw[i] = t < a.Tq ? a.w[((int64_t)b * a.Tq + t) * kHI + (i % kHI)] : 0.f;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (n_tiles > 0 && elect_one()) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      mbar_arrive_expect_tx(bfull, L::kB);
+      const int32_t qrow = (int32_t)(t0 * kHI);
+      tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
+      tma_load_3d(sB + L::kB / 2, &map_q, bfull, 64, qrow, b);
+      int issued = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1u)) {
+          *abort_flag = 1;
+          report(a.status, CSA_DEV_TIMEOUT, 1u);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        uint8_t* dst = sA + s * kTileBytes;
+        const int32_t erow = (int32_t)(e0 + (int64_t)i * kBM);
+        tma_load_3d(dst, &map_k, &full[s], 0, erow, b);
+        tma_load_3d(dst + kTileBytes / 2, &map_k, &full[s], 64, erow, b);
+        issued = i + 1;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i)
+        mbar_wait(&full[i % kStages], (uint32_t)(i / kStages) & 1u);
+      mbar_wait(bfull, 0);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (n_tiles > 0 && elect_one()) {
+      if (!mbar_wait(bfull, 0)) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 2u);
+      } else {
+        const uint32_t b_base = smem_u32(sB);
+        const uint32_t a_base = smem_u32(sA);
+        for (int i = 0; i < n_tiles; ++i) {
+          const int s = i % kStages;
+          const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+          const int buf = i & 1;
+          const uint32_t bph = (uint32_t)(i >> 1) & 1u;
+          if (*abort_flag || !mbar_wait(&full[s], ph) || !mbar_wait(&tempty[buf], bph ^ 1u)) {
+            *abort_flag = 1;
+            report(a.status, CSA_DEV_TIMEOUT, 3u);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(buf * kN);
+#pragma unroll
+          for (int kk = 0; kk < kDI / 16; ++kk) {
+            const uint32_t koff = (uint32_t)((kk & 3) * 32);  // 16 bf16 per K step
+            uint64_t ad = smem_desc(a_base + s * kTileBytes + (kk >> 2) * (kTileBytes / 2) + koff,
+                                    16, 1024, 2);
+            uint64_t bd = smem_desc(b_base + (kk >> 2) * (L::kB / 2) + koff, 16, 1024, 2);
+            mma_bf16_ss(d, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[buf]);
+        }
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    // ---------------- epilogue: thread <-> TMEM lane <-> entry
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int buf = i & 1;
+      const uint32_t bph = (uint32_t)(i >> 1) & 1u;
+      if (*abort_flag || !mbar_wait(&tfull[buf], bph)) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 4u);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = tmem_addr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kN));
+#pragma unroll
+      for (int t = 0; t < TOK; ++t) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(base + t * kHI, r0);
+        tmem_ld32(base + t * kHI + 32, r1);
+        tmem_ld_wait();
+        const float* wt = sw + t * kHI;
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) acc = fmaf(wt[h], fmaxf(__uint_as_float(r0[h]), 0.f), acc);
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+          acc = fmaf(wt[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc);
+        scores[t * kChunk + i * kBM + row] = acc;
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  __syncthreads();
+
+  // ---------------- top-k: one warp per token
+  if (warp >= 2 && warp < 2 + TOK && !*abort_flag) {
+    const int t = warp - 2;
+    const int64_t tok = t0 + t;
+    if (tok < a.Tq) {
+      const int64_t row = (int64_t)b * a.Tq + tok;
+      int64_t n64 = vis[t] - e0;
+      n64 = n64 < 0 ? 0 : (n64 > kChunk ? kChunk : n64);
+      const int n = (int)n64;
+      int32_t* oi;
+      float* os;
+      if (a.n_chunks == 1) {
+        oi = a.idx_out + row * a.k;
+        os = a.score_out ? a.score_out + row * a.k : nullptr;
+      } else {
+        const int64_t c = (row * a.n_chunks + chunk) * a.k;
+        oi = a.cand_idx + c;
+        os = a.cand_score + c;
+      }
+      warp_topk(scores + t * kChunk, n, a.k, e0, hist + t * 256, oi, os);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+// Final selection over the per-chunk candidates of one row: exact block radix
+// select, then an ordered compaction (candidates are in ascending entry order:
+// chunk after chunk, ascending within each chunk).
+__global__ void __launch_bounds__(1024)
+    indexer_merge_kernel(TcIdxArgs a) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned tmp[33];
+  __shared__ unsigned s_prefix, s_mask;
+  __shared__ int s_rem;
+  const int64_t row = blockIdx.x;
+  const int64_t n = (int64_t)a.n_chunks * a.k;
+  const float* cs = a.cand_score + row * n;
+  const int32_t* ci = a.cand_idx + row * n;
+  int32_t* out = a.idx_out + row * a.k;
+  float* so = a.score_out ? a.score_out + row * a.k : nullptr;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+
+  // number of valid candidates
+  unsigned cnt = 0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) cnt += ci[j] >= 0;
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) tmp[wid] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned s = 0;
+    for (int i = 0; i < nw; ++i) s += tmp[i];
+    tmp[32] = s;
+    s_prefix = 0u;
+    s_mask = 0u;
+    s_rem = a.k;
+  }
+  __syncthreads();
+  const unsigned n_valid = tmp[32];
+  const bool take_all = n_valid <= (unsigned)a.k;
+  if (!take_all) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
+      __syncthreads();
+      const unsigned prefix = s_prefix, mask = s_mask;
+      for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+        if (ci[j] < 0) continue;
+        unsigned key = score_key(cs[j]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int rem = s_rem;
+        unsigned cum = 0;
+        int d = 255;
+        for (; d > 0; --d) {
+          if (cum + hist[d] >= (unsigned)rem) break;
+          cum += hist[d];
+        }
+        s_prefix = prefix | ((unsigned)d << shift);
+        s_mask = mask | (255u << shift);
+        s_rem = rem - (int)cum;
+      }
+      __syncthreads();
+    }
+  }
+  const unsigned tau = s_prefix, need_eq = (unsigned)s_rem;
+  unsigned run_sel = 0, run_eq = 0;
+  for (int64_t base = 0; base < n; base += blockDim.x) {
+    const int64_t j = base + threadIdx.x;
+    const bool valid = j < n && ci[j] >= 0;
+    const float s = valid ? cs[j] : 0.f;
+    const unsigned key = valid ? score_key(s) : 0u;
+    const bool gt = valid && (take_all || key > tau);
+    const bool eq = valid && !take_all && key == tau;
+    // exclusive counts of eq and take over the block, in thread order
+    unsigned b1 = __ballot_sync(0xffffffffu, eq);
+    __syncthreads();
+    if (lane == 0) tmp[wid] = __popc(b1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned r = 0;
+      for (int i = 0; i < nw; ++i) { unsigned c = tmp[i]; tmp[i] = r; r += c; }
+      tmp[32] = r;
+    }
+    __syncthreads();
+    const unsigned eq_rank = run_eq + tmp[wid] + __popc(b1 & ((1u << lane) - 1u));
+    const unsigned eq_tot = tmp[32];
+    const bool take = gt || (eq && eq_rank < need_eq);
+    unsigned b2 = __ballot_sync(0xffffffffu, take);
+    __syncthreads();
+    if (lane == 0) tmp[wid] = __popc(b2);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned r = 0;
+      for (int i = 0; i < nw; ++i) { unsigned c = tmp[i]; tmp[i] = r; r += c; }
+      tmp[32] = r;
+    }
+    __syncthreads();
+    const unsigned at = run_sel + tmp[wid] + __popc(b2 & ((1u << lane) - 1u));
+    if (take && at < (unsigned)a.k) {
+      out[at] = ci[j];
+      if (so) so[at] = s;
+    }
+    run_sel += tmp[32];
+    run_eq += eq_tot;
+  }
+  for (int64_t p = run_sel + threadIdx.x; p < a.k; p += blockDim.x) {
+    out[p] = -1;
+    if (so) so[p] = -INFINITY;
+  }
+}
+
+inline int tok_for(int64_t Tq) { return Tq >= 4 ? 4 : 1; }
+inline int chunk_for(int tok) { return tok == 4 ? Cfg<4>::kChunk : Cfg<1>::kChunk; }
+inline int n_chunks_for(int64_t N, int tok) {
+  int64_t c = chunk_for(tok);
+  int64_t n = (N + c - 1) / c;
+  return n < 1 ? 1 : (int)n;
+}
+
+template <int TOK>
+cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
+  CUtensorMap mq, mk;
+  if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, TOK * kHI))
+    return cudaErrorInvalidValue;
+  if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64, kBM))
+    return cudaErrorInvalidValue;
+  const int smem = Smem<TOK>::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<TOK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)a.n_chunks, (unsigned)((p.Tq + TOK - 1) / TOK), (unsigned)p.B);
+  indexer_tc_kernel<TOK><<<grid, kThreads, smem, stream>>>(mq, mk, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool indexer_tc_supported(const IndexerParams& p) {
+  auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+  return p.HI == kHI && p.dI == kDI && p.N > 0 && p.N < (1LL << 31) &&
+         p.Tq * kHI < (1LL << 31) && p.B <= 65535 && al(p.q_I) && al(p.k_I) &&
+         (p.Tq + 3) / 4 <= 65535;
+}
+
+size_t indexer_tc_scratch(int64_t B, int64_t Tq, int64_t N, int k) {
+  const int tok = tok_for(Tq);
+  const int nc = n_chunks_for(N, tok);
+  if (nc <= 1) return 0;
+  return (size_t)B * (size_t)Tq * (size_t)nc * (size_t)k * 8;
+}
+
+cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
+                              unsigned long long* n_launch) {
+  *n_launch = 0;
+  if (p.B == 0 || p.Tq == 0) return cudaSuccess;
+  const int tok = tok_for(p.Tq);
+  TcIdxArgs a{};
+  a.Tq = p.Tq;
+  a.N = p.N;
+  a.m = p.m;
+  a.k = p.k;
+  a.n_chunks = n_chunks_for(p.N, tok);
+  a.w = p.w;
+  a.q_pos = p.q_pos;
+  a.idx_out = p.idx_out;
+  a.score_out = p.score_out;
+  a.status = p.status;
+  if (a.n_chunks > 1) {
+    const size_t n = (size_t)p.B * p.Tq * a.n_chunks * p.k;
+    if (p.scratch_bytes < n * 8) return cudaErrorInvalidValue;
+    a.cand_score = static_cast<float*>(p.scratch);
+    a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
+  }
+  cudaError_t e = tok == 4 ? launch_tok<4>(p, a, stream) : launch_tok<1>(p, a, stream);
+  if (e != cudaSuccess) return e;
+  *n_launch = 1;
+  if (a.n_chunks > 1) {
+    indexer_merge_kernel<<<(unsigned)(p.B * p.Tq), 1024, 0, stream>>>(a);
+    e = cudaGetLastError();
+    *n_launch = 2;
+  }
+  return e;
+}
+
+}  // namespace csa

@@ -1,0 +1,76 @@
+// Internal launcher interface between the C ABI (abi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace csa {
+
+// Offsets inside a caller workspace: the status word lives at byte 0; scratch
+// starts at kWsScratch.
+constexpr size_t kWsScratch = 256;
+
+struct CompressParams {
+  const void* kv_a;   // group a (CSA) or the single group (HCA)
+  const void* kv_b;   // group b (CSA only)
+  const void* z_a;
+  const void* z_b;
+  int z_cols;         // c or 1
+  int64_t T;          // tokens per sequence
+  int64_t n_entries;  // floor(T / m)
+  int m;              // rate (m or m')
+  int overlap;        // 1 = CSA two overlapping groups
+  int G;              // slot groups per CTA (set by the launcher)
+  Fmt f;
+  int64_t pos0;
+  void* entries;
+  void* win;          // optional window-row output
+};
+cudaError_t launch_compress(int dtype, CompressParams p, int64_t B, cudaStream_t stream);
+
+struct IndexerParams {
+  int64_t B, Tq;
+  int HI, dI;
+  const void* q_I;       // [B, Tq, HI, dI]
+  const float* w;        // [B, Tq, HI]
+  const void* k_I;       // [B, N, dI]
+  int64_t N;
+  const int64_t* q_pos;  // [B, Tq] or null
+  int m, k;
+  int32_t* idx_out;      // [B, Tq, k]
+  float* score_out;      // [B, Tq, k] or null
+  unsigned* status;      // device status word
+  void* scratch;         // workspace past the status word
+  size_t scratch_bytes;
+};
+size_t indexer_portable_scratch(int64_t B, int64_t Tq, int64_t N, int k);
+cudaError_t launch_indexer_portable(int dtype, const IndexerParams& p, cudaStream_t stream);
+
+struct AttnParams {
+  int64_t B, Tq;
+  int H;
+  Fmt f;
+  const void* q;          // [B, Tq, H, c]
+  const int64_t* q_pos;   // [B, Tq] or null
+  const void* entries;    // [B, N, c]
+  int64_t N;
+  int sparse;             // 1: keys = idx entries; 0: all visible entries
+  const int32_t* idx;     // [B, Tq, k] (sparse; may be null when k == 0)
+  int k;
+  int m_dense;            // dense visibility rate (dense only)
+  const void* win;        // [B, Tw, c]
+  int64_t Tw;
+  const int64_t* win_pos0;  // [B] or null
+  int n_win;
+  const float* sink;      // [H] or null
+  float scale;
+  void* out;              // [B, Tq, H, c]
+  unsigned* status;
+  void* scratch;
+  size_t scratch_bytes;
+};
+cudaError_t launch_attn_portable(int dtype, const AttnParams& p, cudaStream_t stream);
+
+}  // namespace csa

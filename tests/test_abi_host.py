@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every function include/csa.h declares, and rejects bad
+arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*[A-Za-z_][\w \*]*?\b(\w+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_attention_csa_b200 import build, lib
+
+    build.build()
+    return lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert {"csa_compress", "hca_compress", "indexer_scores_topk", "sparse_mqa_attn",
+            "dense_hca_attn"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"libcsa.so does not export {n}"
+
+
+def test_binding_names_match_the_abi():
+    import long_context_attention_csa_b200 as pkg
+
+    for n in ("csa_compress", "hca_compress", "indexer_scores_topk", "sparse_mqa_attn",
+              "dense_hca_attn", "csa_workspace_bytes", "csa_check_status"):
+        assert callable(getattr(pkg, n))
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert len(L.csa_status_string(s)) > 0
+
+
+def test_workspace_sizes(L):
+    from long_context_attention_csa_b200 import CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN
+
+    # at least the status word; scales with the problem
+    a = L.csa_workspace_bytes(CSA_OP_INDEXER, 1, 1, 16, 0, 0, 64, 8, 0)
+    b = L.csa_workspace_bytes(CSA_OP_INDEXER, 1, 1, 1024, 0, 0, 4096, 8, 0)
+    assert 256 <= a < b
+    assert L.csa_workspace_bytes(CSA_OP_SPARSE_ATTN, 1, 1, 8, 64, 512, 2048, 512, 128) >= 256
+    assert L.csa_workspace_bytes(99, 1, 1, 1, 1, 1, 1, 1, 1) == 0
+
+
+def _fmt(c=512, r=64, flags=0):
+    from long_context_attention_csa_b200 import Fmt
+
+    return Fmt(c=c, rope_dims=r, flags=flags)._c()
+
+
+def test_compress_rejects_bad_arguments(L):
+    f = _fmt()
+    dummy = ctypes.c_void_p(4096)   # never dereferenced: validation fails first
+    mis = ctypes.c_void_p(4100)     # not 16-byte aligned
+    # bad dtype, null fmt, bad m, null pointers, misalignment, bad z_cols
+    assert L.csa_compress(7, 1, 64, 4, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0, dummy,
+                          None, None) == 1
+    assert L.csa_compress(1, 1, 64, 4, None, dummy, dummy, dummy, dummy, 512, 0, dummy, None,
+                          None) == 1
+    assert L.csa_compress(1, 1, 64, 0, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0, dummy,
+                          None, None) == 1
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), None, dummy, dummy, dummy, 512, 0, dummy,
+                          None, None) == 1
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), mis, dummy, dummy, dummy, 512, 0, dummy,
+                          None, None) == 1
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), dummy, dummy, dummy, dummy, 7, 0, dummy,
+                          None, None) == 1
+    # odd RoPE dims, RoPE wider than c
+    bad = _fmt(r=63)
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(bad), dummy, dummy, dummy, dummy, 512, 0,
+                          dummy, None, None) == 1
+    bad = _fmt(c=64, r=128)
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(bad), dummy, dummy, dummy, dummy, 64, 0,
+                          dummy, None, None) == 1
+    # unsupported: c not a power-of-two number of vectors, overlap too wide
+    odd = _fmt(c=520, r=64)
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(odd), dummy, dummy, dummy, dummy, 520, 0,
+                          dummy, None, None) == 2
+    assert L.csa_compress(1, 1, 1024, 200, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0,
+                          dummy, None, None) == 2
+    # empty problems are a no-op
+    assert L.csa_compress(1, 0, 64, 4, ctypes.byref(f), None, None, None, None, 512, 0, None, None,
+                          None) == 0
+    assert L.hca_compress(1, 1, 0, 128, ctypes.byref(f), None, None, 512, 0, None, None,
+                          None) == 0
+
+
+def test_indexer_and_attention_reject_bad_arguments(L):
+    d = ctypes.c_void_p(4096)
+    f = _fmt()
+    # indexer: H_I too large, k < 1, missing workspace, workspace too small
+    assert L.indexer_scores_topk(1, 1, 4, 65, 128, d, d, d, 16, None, 4, 2, d, None, d, 1 << 20,
+                                 None) == 2
+    assert L.indexer_scores_topk(1, 1, 4, 64, 128, d, d, d, 16, None, 4, 0, d, None, d, 1 << 20,
+                                 None) == 1
+    assert L.indexer_scores_topk(1, 1, 4, 64, 128, d, d, d, 16, None, 4, 2, d, None, None, 0,
+                                 None) == 5
+    assert L.indexer_scores_topk(1, 1, 4, 64, 128, d, d, d, 16, None, 4, 2, d, None, d, 8,
+                                 None) == 5
+    # attention: idx null with k > 0, negative sizes, c > 512, no workspace
+    assert L.sparse_mqa_attn(1, 1, 1, 64, ctypes.byref(f), d, None, d, 16, None, 4, d, 8, None,
+                             8, None, 0.0, d, d, 1 << 20, None) == 1
+    assert L.sparse_mqa_attn(1, 1, 1, 0, ctypes.byref(f), d, None, d, 16, d, 4, d, 8, None, 8,
+                             None, 0.0, d, d, 1 << 20, None) == 1
+    big = _fmt(c=1024)
+    assert L.dense_hca_attn(1, 1, 1, 64, ctypes.byref(big), d, None, d, 16, 128, d, 8, None, 8,
+                            None, 0.0, d, d, 1 << 20, None) == 2
+    assert L.dense_hca_attn(1, 1, 1, 64, ctypes.byref(f), d, None, d, 16, 128, d, 8, None, 8,
+                            None, 0.0, d, None, 0, None) == 5
+    assert L.dense_hca_attn(1, 1, 1, 64, ctypes.byref(f), d, None, d, 16, 0, d, 8, None, 8, None,
+                            0.0, d, d, 1 << 20, None) == 1

@@ -1,0 +1,302 @@
+"""GPU parity: every C-ABI call against the float64 oracle on the same seeded
+inputs, at small sizes that span several tiles and a ragged tail (compared
+element by element) and at the full workload sizes (compared on sampled rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close, check_topk_rows, f64
+import long_context_attention_csa_b200 as csa
+from long_context_attention_csa_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def ofmt(w, flags=0):
+    return oracle.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base, flags=flags)
+
+
+def gfmt(w, flags=0):
+    return csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base, flags=flags)
+
+
+def sample_rows(T, n=40, seed=0):
+    g = np.random.default_rng(seed)
+    fixed = [0, 1, 2, 3, 4, 5, 126, 127, 128, 129, T // 2, T - 2, T - 1]
+    rnd = g.choice(T, size=min(n, T), replace=False).tolist()
+    return np.array(sorted(set(r for r in fixed + rnd if 0 <= r < T)))
+
+
+# ----------------------------------------------------------------- compression
+
+@pytest.mark.parametrize("wname,T,B,pos0,zc", [
+    ("tiny_csa_fp32", 256, 1, 0, None),
+    ("csa_prefill_8k", 1003, 2, 7, None),
+    ("csa_prefill_8k", 1003, 2, 0, 1),
+    ("csa_prefill_8k", 8192, 1, 0, None),
+])
+def test_csa_compress(wname, T, B, pos0, zc):
+    w = wl.scaled(wl.WORKLOADS[wname], T=T, B=B)
+    inp = wl.csa_prefill_inputs(w, DEV)
+    za, zb = inp["z_a"], inp["z_b"]
+    if zc == 1:
+        za, zb = za[..., :1].contiguous(), zb[..., :1].contiguous()
+    ent, win = csa.csa_compress(inp["kv_a"], inp["kv_b"], za, zb, w.m, gfmt(w), pos0=pos0,
+                                want_win=True)
+    torch.cuda.synchronize()
+    assert ent.shape == (B, T // w.m, w.c)
+    for b in range(B):
+        ref = oracle.csa_compress(f64(inp["kv_a"][b]), f64(inp["kv_b"][b]), f64(za[b]), f64(zb[b]),
+                                  w.m, ofmt(w), pos0=pos0)
+        assert_close(ent[b], ref, w.dtype, f"entries b={b}")
+        refw = oracle.window_rows(f64(inp["kv_a"][b]), ofmt(w), pos0=pos0)
+        assert_close(win[b], refw, w.dtype, f"window b={b}")
+
+
+@pytest.mark.parametrize("T,B,mp", [(1000, 2, 128), (65536, 1, 128), (300, 1, 7)])
+def test_hca_compress(T, B, mp):
+    w = wl.scaled(wl.WORKLOADS["hca_prefill_64k"], T=T, B=B, m_prime=mp)
+    inp = wl.hca_prefill_inputs(w, DEV)
+    del inp["q"]
+    ent, win = csa.hca_compress(inp["kv"], inp["z"], mp, gfmt(w), want_win=True)
+    torch.cuda.synchronize()
+    assert ent.shape == (B, T // mp, w.c)
+    for b in range(B):
+        ref = oracle.hca_compress(f64(inp["kv"][b]), f64(inp["z"][b]), mp, ofmt(w))
+        assert_close(ent[b], ref, w.dtype, f"entries b={b}")
+        rows = sample_rows(T, 200)
+        # window rows at their own positions: the sampled rows one by one
+        refw = np.stack([oracle.window_rows(f64(inp["kv"][b][r:r + 1]), ofmt(w), pos0=int(r))[0]
+                         for r in rows])
+        assert_close(win[b][rows], refw, w.dtype, f"window b={b}")
+
+
+# ----------------------------------------------------------------- indexer
+
+def _indexer_case(w, rows=None, q_pos=None, exact=False):
+    inp = wl.csa_prefill_inputs(w, DEV) if w.kind == "csa_prefill" else wl.csa_decode_inputs(w, DEV)
+    qp = inp.get("q_pos")
+    idx, sc = csa.indexer_scores_topk(inp["q_I"], inp["w"], inp["k_I"], w.m, w.k, q_pos=qp,
+                                      want_scores=True)
+    torch.cuda.synchronize()
+    B, Tq = inp["q_I"].shape[:2]
+    rows = np.arange(Tq) if rows is None else rows
+    differing = 0
+    for b in range(B):
+        pos = rows if qp is None else qp[b].cpu().numpy()[rows]
+        ref_sc = oracle.indexer_scores(f64(inp["q_I"][b][rows]), f64(inp["w"][b][rows]),
+                                       f64(inp["k_I"][b]), w.m, q_pos=pos)
+        ref_idx = oracle.topk(ref_sc, w.k, w.m, q_pos=pos)
+        gi = idx[b][rows].cpu().numpy()
+        differing += check_topk_rows(gi, ref_idx, ref_sc, exact=exact, what=f"b={b}")
+        # scores of the GPU's own selection against the oracle's score of the same entries
+        gs = sc[b][rows].cpu().numpy().astype(np.float64)
+        valid = gi >= 0
+        want = np.take_along_axis(ref_sc, np.where(valid, gi, 0), axis=1)
+        if exact:
+            assert np.array_equal(gs[valid], want[valid])
+        else:
+            err = np.abs(gs[valid] - want[valid]) / np.maximum(1.0, np.abs(want[valid]))
+            assert err.max() <= 1e-4, f"score error {err.max()}"
+        assert np.all(np.isneginf(gs[~valid]))
+    return differing
+
+
+def test_indexer_tiny_fp32():
+    _indexer_case(wl.WORKLOADS["tiny_csa_fp32"])
+
+
+@pytest.mark.parametrize("HI,dI,T,k", [(64, 128, 700, 64), (2, 32, 300, 16), (64, 128, 1000, 256)])
+def test_indexer_integer_inputs_bit_exact(HI, dI, T, k):
+    """Small-integer inputs make every product and sum exact in bf16 x bf16 ->
+    fp32: the selected sets (tie rule included) and scores must be identical."""
+    B, m = 1, 4
+    N = T // m
+    qI = wl.randint_like_float((B, T, HI, dI), 11, -2, 3, DEV, torch.bfloat16)
+    kI = wl.randint_like_float((B, N, dI), 12, -2, 3, DEV, torch.bfloat16)
+    w = wl.randint_like_float((B, T, HI), 13, -2, 3, DEV, torch.float32)
+    idx, sc = csa.indexer_scores_topk(qI, w, kI, m, k, want_scores=True)
+    torch.cuda.synchronize()
+    ref_sc = oracle.indexer_scores(f64(qI[0]), f64(w[0]), f64(kI[0]), m)
+    ref_idx = oracle.topk(ref_sc, k, m)
+    assert np.array_equal(idx[0].cpu().numpy(), ref_idx)
+    gi = idx[0].cpu().numpy()
+    v = gi >= 0
+    assert np.array_equal(sc[0].cpu().numpy().astype(np.float64)[v],
+                          np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v])
+
+
+def test_indexer_csa_prefill_8k_sampled():
+    w = wl.WORKLOADS["csa_prefill_8k"]
+    d = _indexer_case(w, rows=sample_rows(w.T, 48))
+    assert d <= 2
+
+
+@pytest.mark.parametrize("wname", ["csa_decode_b32_128k", "decode_pair_b4_1m"])
+def test_indexer_decode(wname):
+    w = wl.WORKLOADS[wname]
+    d = _indexer_case(w)
+    assert d <= 1
+
+
+def test_indexer_padding_when_few_visible():
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=40, k=16)
+    _indexer_case(w)
+
+
+# ----------------------------------------------------------------- attention
+
+PATHS = [0, csa.CSA_F_PORTABLE]
+
+
+def _attn_inputs_prefill(w, dense=False):
+    g = wl
+    B, T, H, c = w.B, w.T, w.H, w.c
+    N = w.n_hca if dense else w.n_csa
+    inp = dict(
+        q=g._draw(w, "q", (B, T, H, c), DEV, w.q_scale),
+        entries=g._draw(w, "entries", (B, N, c), DEV),
+        win=g._draw(w, "win", (B, T, c), DEV),
+        sink=g.randn((H,), g._seed(w, "sink"), DEV) if w.sink else None,
+    )
+    if not dense:
+        counts = torch.tensor([oracle.visible(t, w.m, N) for t in range(T)])
+        idx = torch.stack([g.random_index_sets(counts, w.k, w.seed * 7 + b) for b in range(B)])
+        inp["idx"] = idx.to(DEV)
+    return inp
+
+
+def _check_attn(w, inp, out, rows, dense, flags=0, q_pos=None, win_pos0=None):
+    B = out.shape[0]
+    for b in range(B):
+        pos = rows if q_pos is None else q_pos[b].cpu().numpy()[rows]
+        wp0 = 0 if win_pos0 is None else int(win_pos0[b])
+        ref = oracle.attention(
+            f64(inp["q"][b][rows]), f64(inp["entries"][b]), f64(inp["win"][b]), ofmt(w, flags),
+            w.n_win, idx=None if dense else inp["idx"][b][rows].cpu().numpy(),
+            m_dense=w.m_prime if dense else 0,
+            sink=None if inp["sink"] is None else f64(inp["sink"]), q_pos=pos, win_pos0=wp0)
+        assert_close(out[b][rows], ref, w.dtype, f"attention b={b}")
+
+
+@pytest.mark.parametrize("flags", PATHS)
+@pytest.mark.parametrize("wname,T,k,sink", [
+    ("tiny_csa_fp32", 256, 16, True),
+    ("csa_prefill_8k", 300, 32, True),
+    ("csa_prefill_8k", 300, 32, False),
+    ("csa_prefill_8k", 261, 0, True),
+])
+def test_sparse_attention_small(wname, T, k, sink, flags):
+    w = wl.scaled(wl.WORKLOADS[wname], T=T, k=k, sink=sink)
+    if w.dtype == torch.float32 and flags == 0:
+        pytest.skip("float32 always runs the portable kernel")
+    inp = _attn_inputs_prefill(w)
+    out = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w, flags),
+                              w.n_win, sink=inp["sink"])
+    torch.cuda.synchronize()
+    _check_attn(w, inp, out, np.arange(T), dense=False, flags=flags)
+
+
+@pytest.mark.parametrize("flags", PATHS)
+@pytest.mark.parametrize("T,mp", [(600, 128), (333, 16)])
+def test_dense_attention_small(T, mp, flags):
+    w = wl.scaled(wl.WORKLOADS["hca_prefill_64k"], T=T, m_prime=mp)
+    inp = _attn_inputs_prefill(w, dense=True)
+    out = csa.dense_hca_attn(inp["q"], inp["entries"], mp, inp["win"], gfmt(w, flags), w.n_win,
+                             sink=inp["sink"])
+    torch.cuda.synchronize()
+    _check_attn(w, inp, out, np.arange(T), dense=True, flags=flags)
+
+
+def test_sparse_attention_csa_prefill_8k_sampled():
+    w = wl.WORKLOADS["csa_prefill_8k"]
+    inp = _attn_inputs_prefill(w)
+    out = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w), w.n_win,
+                              sink=inp["sink"])
+    torch.cuda.synchronize()
+    _check_attn(w, inp, out, sample_rows(w.T, 40), dense=False)
+
+
+def test_dense_attention_hca_prefill_64k_sampled():
+    w = wl.WORKLOADS["hca_prefill_64k"]
+    inp = _attn_inputs_prefill(w, dense=True)
+    out = csa.dense_hca_attn(inp["q"], inp["entries"], w.m_prime, inp["win"], gfmt(w), w.n_win,
+                             sink=inp["sink"])
+    torch.cuda.synchronize()
+    _check_attn(w, inp, out, sample_rows(w.T, 24), dense=True)
+    del out, inp
+    torch.cuda.empty_cache()
+
+
+def _decode_idx(w, inp, seed):
+    B = inp["q"].shape[0]
+    counts = torch.tensor([oracle.visible(w.T - 1, w.m, w.n_csa)])
+    return torch.stack([wl.random_index_sets(counts, w.k, seed + b) for b in range(B)]).to(DEV)
+
+
+@pytest.mark.parametrize("flags", PATHS)
+@pytest.mark.parametrize("wname", ["csa_decode_b32_128k", "decode_pair_b4_1m"])
+def test_decode_attention(wname, flags):
+    w = wl.WORKLOADS[wname]
+    inp = wl.csa_decode_inputs(w, DEV)
+    inp["idx"] = _decode_idx(w, inp, 5)
+    out = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w, flags),
+                              w.n_win, sink=inp["sink"], q_pos=inp["q_pos"],
+                              win_pos0=inp["win_pos0"])
+    torch.cuda.synchronize()
+    _check_attn(w, inp, out, np.arange(1), dense=False, flags=flags, q_pos=inp["q_pos"],
+                win_pos0=inp["win_pos0"].cpu().numpy())
+    if wname == "decode_pair_b4_1m":
+        h = wl.hca_decode_inputs(w, DEV)
+        out = csa.dense_hca_attn(h["q"], h["entries"], w.m_prime, h["win"], gfmt(w, flags),
+                                 w.n_win, sink=h["sink"], q_pos=h["q_pos"], win_pos0=h["win_pos0"])
+        torch.cuda.synchronize()
+        _check_attn(w, h, out, np.arange(1), dense=True, flags=flags, q_pos=h["q_pos"],
+                    win_pos0=h["win_pos0"].cpu().numpy())
+
+
+def test_decode_batch_invariance():
+    """A decode row gives bitwise the same output alone as inside a batch of 32."""
+    w = wl.WORKLOADS["csa_decode_b32_128k"]
+    inp = wl.csa_decode_inputs(w, DEV)
+    inp["idx"] = _decode_idx(w, inp, 5)
+    args = dict(sink=inp["sink"])
+    full = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w), w.n_win,
+                               q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], **args)
+    for b in (0, 13, 31):
+        one = csa.sparse_mqa_attn(inp["q"][b:b + 1].contiguous(), inp["entries"][b:b + 1].contiguous(),
+                                  inp["idx"][b:b + 1].contiguous(), inp["win"][b:b + 1].contiguous(),
+                                  gfmt(w), w.n_win, q_pos=inp["q_pos"][b:b + 1].contiguous(),
+                                  win_pos0=inp["win_pos0"][b:b + 1].contiguous(), **args)
+        torch.cuda.synchronize()
+        assert torch.equal(one[0], full[b])
+    # repeat runs are bitwise identical
+    again = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w),
+                                w.n_win, q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], **args)
+    assert torch.equal(again, full)
+
+
+# ----------------------------------------------------------------- whole layer
+
+@pytest.mark.parametrize("wname,T,k", [("tiny_csa_fp32", 256, 16), ("csa_prefill_8k", 512, 64)])
+def test_csa_layer_end_to_end(wname, T, k):
+    """compress -> indexer -> attention on the GPU against the oracle's own
+    chain from the same raw inputs."""
+    w = wl.scaled(wl.WORKLOADS[wname], T=T, k=k)
+    inp = wl.csa_prefill_inputs(w, DEV)
+    ent, win = csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, gfmt(w),
+                                want_win=True)
+    idx = csa.indexer_scores_topk(inp["q_I"], inp["w"], inp["k_I"], w.m, w.k)
+    out = csa.sparse_mqa_attn(inp["q"], ent, idx, win, gfmt(w), w.n_win, sink=inp["sink"])
+    torch.cuda.synchronize()
+    ref = oracle.csa_layer({kk: (None if v is None else f64(v[0] if v.dim() > 1 else v))
+                            for kk, v in inp.items()}, ofmt(w), w.m, w.k, w.n_win)
+    gi = idx[0].cpu().numpy()
+    check_topk_rows(gi, ref["idx"], ref["scores"], what="layer")
+    same = np.all(gi == ref["idx"], axis=1)
+    assert same.mean() > 0.95
+    assert_close(out[0][same], ref["out"][same], w.dtype, "layer output")
