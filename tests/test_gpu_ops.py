@@ -299,4 +299,6 @@ def test_csa_layer_end_to_end(wname, T, k):
     check_topk_rows(gi, ref["idx"], ref["scores"], what="layer")
     same = np.all(gi == ref["idx"], axis=1)
     assert same.mean() > 0.95
-    assert_close(out[0][same], ref["out"][same], w.dtype, "layer output")
+    # the GPU chain stores the entries and window rows in bf16 before attention
+    # and rounds the output again: two bf16 roundings against the float64 chain
+    assert_close(out[0][same], ref["out"][same], w.dtype, "layer output", roundings=2)
