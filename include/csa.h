@@ -143,6 +143,28 @@ csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I
                                const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
                                float* score_out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * indexer_scores_topk without a workspace.  The pages have no counterpart to
+ * this call: it exists for callers that cannot allocate device memory where
+ * they call the indexer (an engine plug-in whose host owns all device memory
+ * through its own pool, or a decode loop that must not pay for cudaMalloc and
+ * its implicit synchronisation).  Same arguments and results as
+ * indexer_scores_topk minus ws/ws_bytes.  Its scratch lives in a fixed 8 MiB
+ * __device__ array inside libcsa.so that every GPU loading the library holds
+ * until exit; a problem needing more (csa_workspace_bytes of the path taken
+ * minus the 256-byte status word) is rejected with CSA_E_WORKSPACE.  The first
+ * call on each device looks up the array's device address and caches it, so
+ * make that first call before any stream capture.  All calls share the array
+ * and its contents persist between calls: calls that overlap on the GPU race.
+ * Kernel-side status is cleared per call and not reported.  Nothing here calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ */
+csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I,
+                                       int32_t d_I, const void* q_I, const float* w,
+                                       const void* k_I, int64_t N, const int64_t* q_pos,
+                                       int32_t m, int32_t k, int32_t* idx_out, float* score_out,
+                                       void* stream);
+
 /* ---- (3) shared-KV MQA ------------------------------------------------ */
 
 /*
