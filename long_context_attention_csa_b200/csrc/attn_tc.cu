@@ -9,16 +9,17 @@
 // Page "DeepSeek V4 完整技术报告", section "混合注意力：CSA + HCA": a learnable
 // per-head sink logit lets total attention weight fall below one.
 //
-// One CTA takes one query token and 64 heads.  With c = 512 an fp32 output
-// accumulator of 64 heads x 512 dims would not fit next to the scores in TMEM
-// in the usual layout, so the kernel works TRANSPOSED, keys on the MMA's M
-// side:
-//   S^T[key, h] = K_tile . Q^T        (M = 128 keys, N = 64 heads, K = 512)
-//   O^T[c, h]  += V^T . P^T            (M = 128 dims x 4, N = 64, K = 128 keys)
-// which needs 64 + 4 x 64 TMEM columns.  The gathered key tile (one row per
-// selected entry or window row, 1 KB each) is stored once, 128-byte swizzled,
-// and read by both MMAs: K-major as the A operand of S^T and MN-major as the
-// A operand of O^T (K = V).
+// Work item = (query token, group of 64 heads[, key split]).  With c = 512 an
+// fp32 accumulator of 64 heads x 512 dims next to the scores would overflow
+// TMEM in the usual layout, so the kernel works TRANSPOSED, keys on the MMA's
+// M side:
+//   S^T[key, h] = K_tile . Q^T      (M = 64 keys, N = 64 heads, K = 512)
+//   O^T[c, h]  += V^T . P^T          (M = 128 dims x 4, N = 64, K = 64 keys)
+// using 2 x 64 (double-buffered S^T) + 4 x 64 TMEM columns.  A gathered key
+// tile (one 1 KB row per selected entry or window row) is stored once,
+// 128-byte swizzled, and read by both MMAs: K-major as the A operand of S^T,
+// MN-major as the A operand of O^T (K = V).  Two key tiles alternate, so the
+// gather of block b+1 and S^T(b+1) overlap the softmax and O^T of block b.
 //
 // Softmax without a running maximum: q^ and every stored key are RMS-
 // normalised (the method's RMSNorm), so |scale q^ . k| <= scale |q^| sqrt(c)
@@ -27,17 +28,21 @@
 // split partial sums add directly.  A logit more than 60 above the bound (keys
 // far from unit RMS) is reported as CSA_DEV_RANGE.
 //
-// Roles (288 threads): warps 0-3 softmax + epilogue (thread = TMEM lane =
-// key in S^T, = output dim in O^T); warps 4-7 query prologue (RMSNorm, RoPE,
-// bf16, swizzle), index compaction and the key gather (cp.async, 16 B per
-// copy, region by region so the next block's gather overlaps this block's
-// O^T MMAs); warp 8 owns TMEM and issues the MMAs.
-// Decode rows (one query per sequence) split the key list into fixed
-// 256-key pieces whose fp32 partials a combine kernel adds in a fixed order,
-// so a row's result does not depend on the batch it runs in.
+// Persistent CTAs (one per SM) walk their items in turn; roles (288 threads):
+//   warps 4-7  producer: index compaction, RoPE table, the next item's raw q
+//              rows by TMA and their in-place RMSNorm + RoPE, the key gather
+//              (cp.async; each warp-instruction moves four 128-byte row pieces);
+//   warp 8     TMEM owner and single-thread MMA issuer;
+//   warps 0-3  softmax (lanes 0-15: one key each, the M = 64 TMEM layout puts
+//              rows 16w..16w+15 in lanes 0-15 of warp w), then the epilogue
+//              (thread = output dim), which overlaps the next item's first MMAs.
+// Decode rows (one query per sequence) split the key list into fixed 256-key
+// pieces whose fp32 partials a combine kernel adds in a fixed order, so a
+// row's result does not depend on the batch it runs in.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc.h"
+#include "tma_host.h"
 
 namespace csa {
 
@@ -46,30 +51,33 @@ namespace {
 using namespace sm100;
 
 constexpr int kC = 512;                      // entry / head dim
-constexpr int kHG = 64;                      // heads per CTA (MMA N)
-constexpr int kBK = 128;                     // keys per block (MMA M of S^T)
+constexpr int kHG = 64;                      // heads per item (MMA N)
+constexpr int kBK = 64;                      // keys per block (MMA M of S^T)
 constexpr int kRegions = kC / 64;            // 64-element (128-byte) column chunks
-constexpr int kKRegion = kBK * 128;          // 16 KB per key-tile chunk
+constexpr int kKRegion = kBK * 128;          // 8 KB per key-tile chunk
+constexpr int kKTile = kRegions * kKRegion;  // 64 KB
 constexpr int kQRegion = kHG * 128;          // 8 KB per query chunk
+constexpr int kPTile = kBK * 128;            // 8 KB: P^T [64 keys][64 heads] bf16
 constexpr int kSplitKeys = 256;              // decode split size (fixed)
-constexpr int kMaxK = 4096;                  // largest top-k the index list holds
+constexpr int kMaxK = 1024;                  // largest top-k the index list holds
 constexpr int kThreads = 288;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRangeLog2 = 60.f * kLog2e;  // CSA_DEV_RANGE threshold
 
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + kRegions * kQRegion;   // 64 KB
-constexpr int OFF_P = OFF_K + kRegions * kKRegion;   // +128 KB
-constexpr int OFF_LIST = OFF_P + kBK * 128;          // +16 KB
-constexpr int OFF_MB = OFF_LIST + kMaxK * 4;         // +16 KB
-constexpr int OFF_INV = OFF_MB + 256;
-constexpr int OFF_ROPE = OFF_INV + 256;
-constexpr int OFF_BAR = OFF_ROPE + 256;
-constexpr int kNumBars = 8 + 8 + 6;
+constexpr int OFF_K = OFF_Q + kRegions * kQRegion;   // 2 key tiles
+constexpr int OFF_P = OFF_K + 2 * kKTile;            // 2 P tiles
+constexpr int OFF_LIST = OFF_P + 2 * kPTile;         // 2 index lists
+constexpr int OFF_MB = OFF_LIST + 2 * kMaxK * 4;     // [2][64] bounds (log2 units)
+constexpr int OFF_ROPE = OFF_MB + 2 * kHG * 4;       // [2][cos 32 | sin 32]
+constexpr int OFF_RED = OFF_ROPE + 2 * 64 * 4;       // [4][64] partial denominators
+constexpr int OFF_INV = OFF_RED + 4 * kHG * 4;       // [64] 1/denominator
+constexpr int OFF_STERM = OFF_INV + kHG * 4;         // [64] sink term
+constexpr int OFF_NENT = OFF_STERM + kHG * 4;        // [2] entries per item
+constexpr int OFF_BAR = OFF_NENT + 64;
+constexpr int kNumBars = 20;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64;
-constexpr int OFF_RED = OFF_K;                       // epilogue reuse of the key tile
-constexpr int OFF_STAGE = OFF_K + 40960;
 
 static_assert(SMEM_BYTES + 1024 <= 232448, "shared memory budget");
 
@@ -93,6 +101,7 @@ struct TcAttnArgs {
   const float* sink;
   bf16* out;
   int split, n_splits, n_hg;
+  int64_t n_rows, n_items;
   float* o_part;    // [rows][n_hg][n_splits][64][512]
   float* d_part;    // [rows][n_hg][n_splits][64]
   float* mb_part;   // [rows][n_hg][64]
@@ -105,65 +114,187 @@ __device__ __forceinline__ int64_t vis_count(int64_t pos, int m, int64_t N) {
   return v < N ? v : N;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(TcAttnArgs a) {
+// Everything about an item that every role derives the same way.
+struct Item {
+  int64_t row;
+  int hg, split;
+  int64_t bidx, pos, wp0, jlo, n_w;
+};
+
+__device__ __forceinline__ Item decode_item(const TcAttnArgs& a, int64_t it) {
+  Item x;
+  if (a.split) {
+    x.split = (int)(it % a.n_splits);
+    const int64_t rest = it / a.n_splits;
+    x.hg = (int)(rest % a.n_hg);
+    x.row = rest / a.n_hg;
+  } else {
+    x.split = 0;
+    x.hg = (int)(it % a.n_hg);
+    x.row = a.n_rows - 1 - it / a.n_hg;   // late (heavier) rows first
+  }
+  x.bidx = x.row / a.Tq;
+  const int64_t t = x.row % a.Tq;
+  x.pos = a.q_pos ? a.q_pos[x.row] : t;
+  x.wp0 = a.win_pos0 ? a.win_pos0[x.bidx] : 0;
+  int64_t jlo = x.pos - a.n_win + 1;
+  if (jlo < x.wp0) jlo = x.wp0;
+  int64_t jhi = x.pos;
+  if (jhi > x.wp0 + a.Tw - 1) jhi = x.wp0 + a.Tw - 1;
+  x.jlo = jlo;
+  x.n_w = jhi >= jlo ? jhi - jlo + 1 : 0;
+  return x;
+}
+
+// Key range [lo, hi) of an item and its number of 64-key blocks.
+__device__ __forceinline__ int item_blocks(const TcAttnArgs& a, const Item& x, int64_t n_ent,
+                                           int64_t* lo, int64_t* hi) {
+  const int64_t n_keys = n_ent + x.n_w;
+  int64_t l = 0, h = n_keys;
+  if (a.split) {
+    l = (int64_t)x.split * kSplitKeys;
+    h = l + kSplitKeys < n_keys ? l + kSplitKeys : n_keys;
+  }
+  *lo = l;
+  *hi = h;
+  return h > l ? (int)((h - l + kBK - 1) / kBK) : 0;
+}
+
+// In-place query transform by one warp: the raw q rows of heads
+// [16 w, 16 w + 16) sit in the 128-byte-swizzled Q tile (loaded by TMA); each
+// becomes bf16(RoPE_pos(RMSNorm(q))) and mb2[h] = scale |q^| sqrt(c) log2(e)
+// (times 1 + 2^-7), an upper bound of the head's logits against unit-RMS keys.
+// Lane l owns elements [8l, 8l+8) and [256+8l, 256+8l+8); four heads at once.
+__device__ __forceinline__ void query_transform(const TcAttnArgs& a, int w, int lane, float scale,
+                                                uint8_t* sQ, float* mb2, const float* rcs,
+                                                const float* rsn) {
+  float rc[8], rs[8];   // this lane's RoPE factors (identity outside the RoPE dims)
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int el = (k >> 2) * 256 + lane * 8 + (k & 3) * 2;
+    rc[k] = 1.f;
+    rs[k] = 0.f;
+    if (!(a.flags & CSA_F_NO_ROPE) && el >= kC - a.r) {
+      const int pi = (el - (kC - a.r)) >> 1;
+      rc[k] = rcs[pi];
+      rs[k] = rsn[pi];
+    }
+  }
+  const int ch = lane & 7;
+  for (int i0 = 0; i0 < 16; i0 += 4) {
+    uint4 raw[4][2];
+    uint4* ptr[4][2];
+    float x[4][16], ss[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int h = w * 16 + i0 + u;
+      ptr[u][0] = reinterpret_cast<uint4*>(sQ + (lane >> 3) * kQRegion + h * 128 +
+                                           ((ch ^ (h & 7)) << 4));
+      ptr[u][1] = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ptr[u][0]) + 4 * kQRegion);
+      raw[u][0] = *ptr[u][0];
+      raw[u][1] = *ptr[u][1];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t wr[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                              raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+      ss[u] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        x[u][2 * k] = bf16_bits_to_float(wr[k] & 0xffffu);
+        x[u][2 * k + 1] = bf16_bits_to_float(wr[k] >> 16);
+        ss[u] = fmaf(x[u][2 * k], x[u][2 * k], ss[u]);
+        ss[u] = fmaf(x[u][2 * k + 1], x[u][2 * k + 1], ss[u]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float inv = (a.flags & CSA_F_NO_NORM) ? 1.f : rsqrtf(ss[u] / (float)kC + a.eps);
+      uint32_t wd[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float x0 = x[u][2 * k] * inv, x1 = x[u][2 * k + 1] * inv;
+        wd[k] = pack_bf16x2(x0 * rc[k] - x1 * rs[k], x0 * rs[k] + x1 * rc[k]);
+      }
+      *ptr[u][0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      *ptr[u][1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+      if (lane == 0)
+        mb2[w * 16 + i0 + u] =
+            scale * sqrtf(ss[u]) * inv * sqrtf((float)kC) * (1.f + 0.0078125f) * kLog2e;
+    }
+  }
+}
+
+// Sum of v[0..63] over the 32 lanes of a warp by recursive halving: after
+// the five exchange steps lane L holds the totals of entries 2L and 2L+1.
+__device__ __forceinline__ void warp_transpose_sum64(float* v, int lane, float* out2) {
+#pragma unroll
+  for (int o = 16, n = 64; o >= 1; o >>= 1, n >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float lo = v[i], hi = v[i + n / 2];
+      const float send = upper ? lo : hi;
+      const float keep = upper ? hi : lo;
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  out2[0] = v[0];
+  out2[1] = v[1];
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, TcAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = sm + OFF_Q;
-  uint8_t* sK = sm + OFF_K;
-  uint8_t* sP = sm + OFF_P;
-  int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST);
-  float* mb2 = reinterpret_cast<float*>(sm + OFF_MB);
+  float* mb2s = reinterpret_cast<float*>(sm + OFF_MB);
+  float* ropes = reinterpret_cast<float*>(sm + OFF_ROPE);
+  float* red = reinterpret_cast<float*>(sm + OFF_RED);
   float* sinv = reinterpret_cast<float*>(sm + OFF_INV);
-  float* rcs = reinterpret_cast<float*>(sm + OFF_ROPE);        // [32] cos
-  float* rsn = rcs + 32;                                        // [32] sin
+  float* sterm = reinterpret_cast<float*>(sm + OFF_STERM);
+  int* nent = reinterpret_cast<int*>(sm + OFF_NENT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* kfull = bars;
-  uint64_t* kfree = bars + 8;
-  uint64_t* qfull = bars + 16;
-  uint64_t* sfull = bars + 17;
-  uint64_t* pfull = bars + 18;
-  uint64_t* pfree = bars + 19;
-  uint64_t* ofull = bars + 20;
-  uint64_t* drain = bars + 21;
+  uint64_t* kfull = bars;        // [2] key tile landed (128 producer threads)
+  uint64_t* bfree = bars + 2;    // [2] O^T of the block done: key tile and P tile free
+  uint64_t* sfull = bars + 4;    // [2] S^T of the block done
+  uint64_t* pfull = bars + 6;    // [2] P tile written (128 softmax threads)
+  uint64_t* iready = bars + 8;   // [2] item's entry count published
+  uint64_t* qload = bars + 10;   // raw q rows landed (TMA)
+  uint64_t* qfull = bars + 11;   // q^ ready (128 producer threads)
+  uint64_t* qfree = bars + 12;   // last S^T of the item done
+  uint64_t* ofull = bars + 13;   // last O^T of the item done
+  uint64_t* ofree = bars + 14;   // epilogue finished reading O^T (128 threads)
+  uint64_t* drain = bars + 15;
+  uint64_t* ifree = bars + 16;   // [2] MMA and softmax have read the item slot
+  uint64_t* qready = bars + 18;  // [2] the item's q^ and bounds ready (per slot, softmax)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  int* n_ent_slot = reinterpret_cast<int*>(sm + OFF_MISC + 4);
   int* wcnt = reinterpret_cast<int*>(sm + OFF_MISC + 8);        // [4]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 24);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int64_t row;
-  int split_id, hg;
-  if (a.split) {
-    split_id = blockIdx.x;
-    row = blockIdx.y;
-    hg = blockIdx.z;
-  } else {
-    split_id = 0;
-    row = (int64_t)gridDim.x - 1 - blockIdx.x;   // late (heavier) rows first
-    hg = blockIdx.y;
-  }
-  const int64_t bidx = row / a.Tq, t = row % a.Tq;
-  const int64_t pos = a.q_pos ? a.q_pos[row] : t;
-  const int64_t wp0 = a.win_pos0 ? a.win_pos0[bidx] : 0;
-  int64_t jlo = pos - a.n_win + 1;
-  if (jlo < wp0) jlo = wp0;
-  int64_t jhi = pos;
-  if (jhi > wp0 + a.Tw - 1) jhi = wp0 + a.Tw - 1;
-  const int64_t n_w = jhi >= jlo ? jhi - jlo + 1 : 0;
-  const bf16* ent = a.entries + bidx * a.N * kC;
-  const bf16* win = a.win + bidx * a.Tw * kC;
   const float scale = a.scale > 0.f ? a.scale : rsqrtf((float)kC);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&kfull[i], 128);
-      mbar_init(&kfree[i], 1);
+      mbar_init(&bfree[i], 1);
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], 128);
+      mbar_init(&iready[i], 1);
+      mbar_init(&ifree[i], 2);
+      mbar_init(&qready[i], 128);
     }
+    mbar_init(qload, 1);
     mbar_init(qfull, 128);
-    mbar_init(sfull, 1);
-    mbar_init(pfull, 128);
-    mbar_init(pfree, 1);
+    mbar_init(qfree, 1);
     mbar_init(ofull, 1);
+    mbar_init(ofree, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -173,300 +304,414 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(TcAttnArgs a) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-
-  // producer group: RoPE table and the compacted list of selected entries
-  if (warp >= 4 && warp < 8) {
-    const int ptid = threadIdx.x - 128, pw = warp - 4;
-    if (pw == 0 && lane < (a.r >> 1)) {
-      float cs, sn;
-      rope_cos_sin(pos, lane, a.r, a.base, &cs, &sn);
-      rcs[lane] = cs;
-      rsn[lane] = sn;
-    }
-    if (a.sparse) {
-      const int32_t* ir = a.idx + row * (int64_t)a.k;
-      int base = 0;
-      for (int i0 = 0; i0 < a.k; i0 += 128) {
-        const int i = i0 + ptid;
-        const int32_t e = i < a.k ? ir[i] : -1;
-        const bool ok = e >= 0 && e < a.N;
-        if (i < a.k && !ok && e != -1) report(a.status, CSA_DEV_BAD_INDEX, (unsigned)i);
-        const unsigned bal = __ballot_sync(0xffffffffu, ok);
-        if (lane == 0) wcnt[pw] = __popc(bal);
-        named_bar(2, 128);
-        int off = base;
-        for (int w = 0; w < pw; ++w) off += wcnt[w];
-        if (ok) list[off + __popc(bal & ((1u << lane) - 1u))] = e;
-        base += wcnt[0] + wcnt[1] + wcnt[2] + wcnt[3];
-        named_bar(2, 128);
-      }
-      if (ptid == 0) *n_ent_slot = base;
-    } else if (ptid == 0) {
-      *n_ent_slot = (int)vis_count(pos, a.m_dense, a.N);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;          // 64 columns: S^T
-  const uint32_t tO = tmem + 64;     // 4 x 64 columns: O^T
-  const int64_t n_ent = *n_ent_slot;
-  const int64_t n_keys = n_ent + n_w;
-  int64_t k_lo = 0, k_hi = n_keys;
-  if (a.split) {
-    k_lo = (int64_t)split_id * kSplitKeys;
-    k_hi = k_lo + kSplitKeys < n_keys ? k_lo + kSplitKeys : n_keys;
-  }
-  const int n_blocks = k_hi > k_lo ? (int)((k_hi - k_lo + kBK - 1) / kBK) : 0;
+  const uint32_t tS0 = tmem;          // S^T buffers at columns 0 and 64
+  const uint32_t tO = tmem + 128;     // O^T: 4 x 64 columns
 
   if (warp >= 4 && warp < 8) {
-    // ================= query prologue, then the gather
-    const int ptid = threadIdx.x - 128, pw = warp - 4;
-    for (int i = 0; i < 16; ++i) {
-      const int h = pw * 16 + i;
-      const bf16* qr = a.q + (row * a.H + (int64_t)hg * kHG + h) * kC;
-      float x[16];
-      load_vec(qr + lane * 8, x);
-      load_vec(qr + 256 + lane * 8, x + 8);
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) ss += x[e] * x[e];
-      ss = warp_sum(ss);
-      const float inv = (a.flags & CSA_F_NO_NORM) ? 1.f : rsqrtf(ss / (float)kC + a.eps);
-      uint32_t w[8];
-      float nq = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int e0 = half * 256 + lane * 8;
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          float x0 = x[half * 8 + e] * inv, x1 = x[half * 8 + e + 1] * inv;
-          const int el = e0 + e;
-          if (!(a.flags & CSA_F_NO_ROPE) && el >= kC - a.r) {
-            const int pi = (el - (kC - a.r)) >> 1;
-            const float cs = rcs[pi], sn = rsn[pi];
-            const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
-            x0 = y0;
-            x1 = y1;
-          }
-          const uint32_t pk = pack_bf16x2(x0, x1);
-          const float r0 = bf16_bits_to_float(pk & 0xffffu), r1 = bf16_bits_to_float(pk >> 16);
-          nq += r0 * r0 + r1 * r1;
-          w[half * 4 + e / 2] = pk;
+    // ======================= producer
+    // Failure handling: a wait that runs out marks the thread `dead` (made
+    // warp-uniform); dead threads skip waits and work but still pass every
+    // named barrier, so no barrier can be left waiting.
+    const int ptid = threadIdx.x - 128, pw = warp - 4, quad = lane >> 3, g8 = lane & 7;
+    const uint32_t kbase = smem_u32(sm + OFF_K);
+    bool dead = false;
+    auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
+      if (!dead) {
+        if (!mbar_wait(bar, parity)) {
+          *abort_flag = 1;
+          report(a.status, CSA_DEV_TIMEOUT, code);
+          dead = true;
         }
+        dead = dead || *abort_flag;
       }
-      nq = warp_sum(nq);
-      // element lane*8 (+256): chunk region lane/8 (+4), 16-byte chunk lane%8
-      const int ch = lane & 7;
-      uint8_t* d0 = sQ + (lane >> 3) * kQRegion + h * 128 + ((ch ^ (h & 7)) << 4);
-      uint8_t* d1 = sQ + (4 + (lane >> 3)) * kQRegion + h * 128 + ((ch ^ (h & 7)) << 4);
-      *reinterpret_cast<uint4*>(d0) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(d1) = make_uint4(w[4], w[5], w[6], w[7]);
-      if (lane == 0) mb2[h] = scale * sqrtf(nq) * sqrtf((float)kC) * kLog2e;
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(qfull);
+      dead = __any_sync(0xffffffffu, dead);
+    };
+    int64_t gblk = 0;
+    int n = 0;
+    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
+      const int ip = n & 1;
+      const Item x = decode_item(a, it);
+      wait_or_die(&ifree[ip], (uint32_t)((n >> 1) & 1) ^ 1u, 19u);   // item n-2 consumed
+      int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST) + ip * kMaxK;
+      float* rcs = ropes + ip * 64;
+      float* rsn = rcs + 32;
+      const bf16* qrow = a.q + (x.row * a.H + (int64_t)x.hg * kHG) * kC;
+      if (!dead && ptid == 0) {   // warm L2 with this item's q rows ahead of the TMA load
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qrow), "r"(kHG * kC * 2)
+                     : "memory");
+      }
+      if (!dead && pw == 0 && lane < (a.r >> 1)) {
+        float cs, sn;
+        rope_cos_sin(x.pos, lane, a.r, a.base, &cs, &sn);
+        rcs[lane] = cs;
+        rsn[lane] = sn;
+      }
+      int64_t n_ent;
+      if (a.sparse) {
+        // warp pw compacts the contiguous quarter [pw*q4, pw*q4 + q4) of the row
+        const int32_t* ir = a.idx + x.row * (int64_t)a.k;
+        const int q4 = (a.k + 3) / 4;
+        const int lo = pw * q4, hi = lo + q4 < a.k ? lo + q4 : a.k;
+        int32_t ev[kMaxK / 128];
+#pragma unroll
+        for (int u = 0; u < kMaxK / 128; ++u) {
+          const int i = lo + u * 32 + lane;
+          ev[u] = (!dead && u * 32 < q4 && i < hi) ? ir[i] : -1;
+        }
+        int cnt = 0;
+#pragma unroll
+        for (int u = 0; u < kMaxK / 128; ++u) {
+          const bool ok = ev[u] >= 0 && ev[u] < a.N;
+          if (!ok && ev[u] != -1)
+            report(a.status, CSA_DEV_BAD_INDEX, (unsigned)(lo + u * 32 + lane));
+          cnt += __popc(__ballot_sync(0xffffffffu, ok));
+        }
+        named_bar(2, 128);   // previous item's use of wcnt finished
+        if (lane == 0) wcnt[pw] = cnt;
+        named_bar(2, 128);
+        int off = 0;
+        for (int w = 0; w < pw; ++w) off += wcnt[w];
+        n_ent = wcnt[0] + wcnt[1] + wcnt[2] + wcnt[3];
+#pragma unroll
+        for (int u = 0; u < kMaxK / 128; ++u) {
+          const bool ok = ev[u] >= 0 && ev[u] < a.N;
+          const unsigned bal = __ballot_sync(0xffffffffu, ok);
+          if (ok) list[off + __popc(bal & ((1u << lane) - 1u))] = ev[u];
+          off += __popc(bal);
+        }
+      } else {
+        n_ent = vis_count(x.pos, a.m_dense, a.N);
+      }
+      named_bar(2, 128);   // list and RoPE table complete
+      if (!dead && ptid == 0) {
+        nent[ip] = (int)n_ent;
+        mbar_arrive(&iready[ip]);
+      }
+      int64_t k_lo, k_hi;
+      const int nb = dead ? 0 : item_blocks(a, x, n_ent, &k_lo, &k_hi);
 
-    // gather: thread ptid fetches key row ptid of every block
-    const uint32_t kbase = smem_u32(sK);
-    for (int blk = 0; blk < n_blocks && !*abort_flag; ++blk) {
-      const int64_t i = k_lo + (int64_t)blk * kBK + ptid;
-      const bf16* src = nullptr;
-      if (i < k_hi) {
-        if (i < n_ent) src = ent + (int64_t)(a.sparse ? list[i] : i) * kC;
-        else src = win + ((jlo - wp0) + (i - n_ent)) * kC;
+      // the previous item's last S^T is done with Q: load this item's rows
+      if (!dead && ptid == 0) {
+        if (n > 0 && !mbar_wait(qfree, (uint32_t)(n - 1) & 1u)) {
+          *abort_flag = 1;
+          report(a.status, CSA_DEV_TIMEOUT, 20u);
+        } else {
+          mbar_arrive_expect_tx(qload, kRegions * kQRegion);
+          const int32_t qr = (int32_t)(x.row * a.H + (int64_t)x.hg * kHG);
+          for (int r = 0; r < kRegions; ++r)
+            tma_load_3d(sQ + r * kQRegion, &map_q, qload, r * 64, qr, 0);
+        }
       }
-      const uint32_t rowoff = (uint32_t)ptid * 128u;
-      int next_arrive = 0;
-      for (int reg = 0; reg < kRegions; ++reg) {
-        if (blk > 0 && !mbar_try_wait(&kfree[reg], (uint32_t)(blk - 1) & 1u)) {
-          // about to block: publish every region already copied
-          cp_async_wait<0>();
-          fence_proxy_async_smem();
-          for (; next_arrive < reg; ++next_arrive) mbar_arrive(&kfull[next_arrive]);
-          if (!mbar_wait(&kfree[reg], (uint32_t)(blk - 1) & 1u)) {
-            *abort_flag = 1;
-            report(a.status, CSA_DEV_TIMEOUT, 10u);
-            break;
+
+      const bf16* ent = a.entries + x.bidx * a.N * kC;
+      const bf16* win = a.win + x.bidx * a.Tw * kC;
+      for (int b = 0; b < (nb > 0 ? nb : 1); ++b) {
+        const int64_t j = gblk + b;
+        const int s = (int)(j & 1);
+        if (b < nb) {
+          wait_or_die(&bfree[s], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
+          if (!dead) {
+            const uint32_t tile = kbase + s * kKTile;
+            // warp pw fetches rows 16 pw .. 16 pw + 15: four rows per instruction
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = pw * 16 + 4 * i + quad;
+              const int64_t key = k_lo + (int64_t)b * kBK + r;
+              const bf16* src = nullptr;
+              if (key < k_hi) {
+                if (key < n_ent) src = ent + (int64_t)(a.sparse ? list[key] : key) * kC;
+                else src = win + ((x.jlo - x.wp0) + (key - n_ent)) * kC;
+              }
+              const uint32_t dst =
+                  tile + (uint32_t)r * 128u + (((uint32_t)g8 ^ (uint32_t)(r & 7)) << 4);
+#pragma unroll
+              for (int reg = 0; reg < kRegions; ++reg) {
+                const void* sp = src ? (const void*)(src + reg * 64 + g8 * 8) : (const void*)a.q;
+                cp_async16(dst + reg * kKRegion, sp, src ? 16u : 0u);
+              }
+            }
+          }
+          // the barrier counts this thread's arrival once its copies land
+          if (!dead) cp_async_arrive(&kfull[s]);
+        }
+        if (b == 0) {   // transform this item's q while the first block is in flight
+          wait_or_die(qload, (uint32_t)n & 1u, 22u);
+          if (!dead) {
+            query_transform(a, pw, lane, scale, sQ, mb2s + ip * kHG, rcs, rsn);
+            fence_proxy_async_smem();
+            mbar_arrive(qfull);
+            mbar_arrive(&qready[ip]);
           }
         }
-        const uint32_t dst = kbase + reg * kKRegion + rowoff;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const void* s = src ? (const void*)(src + reg * 64 + g * 8) : (const void*)a.q;
-          cp_async16(dst + (((uint32_t)g ^ (uint32_t)(ptid & 7)) << 4), s, src ? 16u : 0u);
-        }
-        cp_async_commit();
-        if (reg - next_arrive >= 2) {   // keep at most three regions in flight
-          cp_async_wait<2>();
-          fence_proxy_async_smem();
-          mbar_arrive(&kfull[next_arrive]);
-          ++next_arrive;
-        }
       }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      for (; next_arrive < kRegions; ++next_arrive) mbar_arrive(&kfull[next_arrive]);
+      gblk += nb;
     }
     cp_async_wait<0>();
   } else if (warp == 8) {
-    // ================= MMA issuer
-    if (n_blocks > 0 && elect_one()) {
+    // ======================= MMA issuer
+    if (elect_one()) {
       constexpr uint32_t idS = idesc_bf16_f32(kBK, kHG, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(128, kHG, 1, 1);
-      const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK), pb = smem_u32(sP);
-      bool ok = mbar_wait(qfull, 0);
-      for (int blk = 0; ok && blk < n_blocks; ++blk) {
-        const uint32_t ph = (uint32_t)blk & 1u;
+      const uint32_t qb = smem_u32(sQ), kb0 = smem_u32(sm + OFF_K), pb0 = smem_u32(sm + OFF_P);
+      int64_t gblk = 0;
+      int n = 0;
+      bool ok = true;
+      auto issue_s = [&](int64_t j) -> bool {
+        const int s = (int)(j & 1);
+        if (*abort_flag || !mbar_wait(&kfull[s], (uint32_t)(j >> 1) & 1u)) return false;
+        fence_proxy_async_smem();   // cp.async (generic proxy) writes -> MMA reads
+        tc_fence_after();
+        const uint32_t kb = kb0 + s * kKTile;
+#pragma unroll
         for (int reg = 0; reg < kRegions; ++reg) {
-          if (*abort_flag || !mbar_wait(&kfull[reg], ph)) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll
           for (int kq = 0; kq < 4; ++kq) {
             const uint64_t ad = smem_desc(kb + reg * kKRegion + kq * 32, 16, 1024, 2);
             const uint64_t bd = smem_desc(qb + reg * kQRegion + kq * 32, 16, 1024, 2);
-            mma_bf16_ss(tS, ad, bd, idS, (reg | kq) != 0 ? 1u : 0u);
+            mma_bf16_ss(tS0 + 64 * s, ad, bd, idS, (reg | kq) != 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&sfull[s]);
+        return true;
+      };
+      for (int64_t it = blockIdx.x; ok && it < a.n_items; it += gridDim.x, ++n) {
+        const Item x = decode_item(a, it);
+        if (!mbar_wait(&iready[n & 1], (uint32_t)(n >> 1) & 1u)) { ok = false; break; }
+        int64_t k_lo, k_hi;
+        const int nb = item_blocks(a, x, nent[n & 1], &k_lo, &k_hi);
+        mbar_arrive(&ifree[n & 1]);
+        if (*abort_flag || !mbar_wait(qfull, (uint32_t)n & 1u)) { ok = false; break; }
+        tc_fence_after();
+        if (nb == 0) {
+          mma_commit(qfree);
+          // keep ofull at most one phase ahead of the epilogue
+          if (n > 0 && !mbar_wait(ofree, (uint32_t)(n - 1) & 1u)) { ok = false; break; }
+          mma_commit(ofull);
+          continue;
+        }
+        // S^T of the item's block bi; the item's last one releases Q
+        auto issue_s_item = [&](int bi) -> bool {
+          if (!issue_s(gblk + bi)) return false;
+          if (bi == nb - 1) mma_commit(qfree);
+          return true;
+        };
+        if (!issue_s_item(0)) { ok = false; break; }
+        int next_s = 1;   // next block whose S^T is still to be issued
+        for (int b = 0; b < nb; ++b) {
+          const int64_t j = gblk + b;
+          const int s = (int)(j & 1);
+          // S^T(j+1) ahead of O^T(j) when its key tile is already here (keeps the
+          // tensor pipe busy through softmax(j+1)); never block O^T(j) on a gather
+          if (next_s == b + 1 && next_s < nb &&
+              mbar_try_wait(&kfull[(j + 1) & 1], (uint32_t)((j + 1) >> 1) & 1u)) {
+            if (!issue_s_item(next_s)) { ok = false; break; }
+            ++next_s;
+          }
+          if (*abort_flag || !mbar_wait(&pfull[s], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
+          if (b == 0 && n > 0 && !mbar_wait(ofree, (uint32_t)(n - 1) & 1u)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kb = kb0 + s * kKTile, pb = pb0 + s * kPTile;
+#pragma unroll 1
+          for (int jt = 0; jt < 4; ++jt) {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = smem_desc(kb + (2 * jt) * kKRegion + kk * 2048, kKRegion, 1024, 2);
+              const uint64_t bd = smem_desc(pb + kk * 2048, kKRegion, 1024, 2);
+              mma_bf16_ss(tO + 64 * jt, ad, bd, idO, (b > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit(&bfree[s]);
+          if (next_s == b + 1 && next_s < nb) {
+            if (!issue_s_item(next_s)) { ok = false; break; }
+            ++next_s;
           }
         }
         if (!ok) break;
-        mma_commit(sfull);
-        if (*abort_flag || !mbar_wait(pfull, ph)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = smem_desc(kb + (2 * j) * kKRegion + kk * 2048, kKRegion, 1024, 2);
-            const uint64_t bd = smem_desc(pb + kk * 2048, kKRegion, 1024, 2);
-            mma_bf16_ss(tO + 64 * j, ad, bd, idO, (blk > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&kfree[2 * j]);
-          mma_commit(&kfree[2 * j + 1]);
-        }
-        mma_commit(pfree);
+        mma_commit(ofull);
+        gblk += nb;
       }
       if (!ok) {
         *abort_flag = 1;
-        report(a.status, CSA_DEV_TIMEOUT, 11u);
+        report(a.status, CSA_DEV_TIMEOUT, 23u);
       }
-      mma_commit(ofull);
       mma_commit(drain);
       mbar_wait(drain, 0);
     }
-  } else {
-    // ================= softmax (warps 0-3): thread = key lane of S^T
+  } else if (warp < 4) {
+    // ======================= softmax + epilogue (same failure handling)
     const int rw = warp * 32 + lane;
+    const bool active = lane < 16;      // M = 64: rows 16w..16w+15 in lanes 0..15
+    const int kb_row = warp * 16 + lane;
     const float c2 = scale * kLog2e;
-    float psum[kHG];
+    bool dead = false;
+    auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
+      if (!dead) {
+        if (!mbar_wait(bar, parity)) {
+          *abort_flag = 1;
+          report(a.status, CSA_DEV_TIMEOUT, code);
+          dead = true;
+        }
+        dead = dead || *abort_flag;
+      }
+      dead = __any_sync(0xffffffffu, dead);
+    };
+    int64_t gblk = 0;
+    int n = 0;
+    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
+      const int ip = n & 1;
+      const Item x = decode_item(a, it);
+      wait_or_die(&iready[ip], (uint32_t)(n >> 1) & 1u, 24u);
+      wait_or_die(&qready[ip], (uint32_t)(n >> 1) & 1u, 24u);
+      const float* mb2 = mb2s + ip * kHG;
+      int64_t k_lo = 0, k_hi = 0;
+      const int nb = dead ? 0 : item_blocks(a, x, nent[ip], &k_lo, &k_hi);
+      // values the epilogue needs, copied now (the producer may refill the
+      // item-parity buffers before the epilogue runs)
+      const int64_t slot = x.row * a.n_hg + x.hg;
+      float my_mb2 = 0.f;
+      if (rw < kHG) {
+        my_mb2 = mb2[rw];
+        sterm[rw] = a.sink ? ex2(fmaf(a.sink[x.hg * kHG + rw], kLog2e, -my_mb2)) : 0.f;
+      }
+      float ecs[4], esn[4];   // RoPE factors of this thread's output pair, per slice
+      {
+        const float* rcs = ropes + ip * 64;
 #pragma unroll
-    for (int h = 0; h < kHG; ++h) psum[h] = 0.f;
-    float xmax = -INFINITY;
-    bool ok = mbar_wait(qfull, 0);   // mb2[] is written by the prologue
-    for (int blk = 0; ok && blk < n_blocks; ++blk) {
-      const uint32_t ph = (uint32_t)blk & 1u;
-      if (*abort_flag || !mbar_wait(sfull, ph)) { ok = false; break; }
+        for (int jt = 0; jt < 4; ++jt) {
+          const int cc = 128 * jt + warp * 32 + (lane & ~1);
+          ecs[jt] = 1.f;
+          esn[jt] = 0.f;
+          if (!(a.flags & CSA_F_NO_ROPE) && cc >= kC - a.r) {
+            const int pi = (cc - (kC - a.r)) >> 1;
+            ecs[jt] = rcs[pi];
+            esn[jt] = rcs[32 + pi];
+          }
+        }
+      }
+      named_bar(1, 128);   // every thread has read the item slot
+      if (rw == 0 && !dead) mbar_arrive(&ifree[ip]);
+      float psum[kHG];
+#pragma unroll
+      for (int h = 0; h < kHG; ++h) psum[h] = 0.f;
+      float xmax = -INFINITY;
+      for (int b = 0; b < nb; ++b) {
+        const int64_t j = gblk + b;
+        const int s = (int)(j & 1);
+        const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+        wait_or_die(&sfull[s], ph, 25u);
+        uint32_t pk[32];
+        if (!dead) {
+          tc_fence_after();
+          const uint32_t ta = tmem_addr(tS0 + 64 * s, (uint32_t)(warp * 32), 0);
+          const bool valid = active && (k_lo + (int64_t)b * kBK + kb_row < k_hi);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {   // 32 heads at a time
+            uint32_t sv[32];
+            tmem_ld32(ta + 32 * half, sv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int h = 32 * half + e;
+              const float x0 = valid ? fmaf(__uint_as_float(sv[e]), c2, -mb2[h]) : -INFINITY;
+              const float x1 =
+                  valid ? fmaf(__uint_as_float(sv[e + 1]), c2, -mb2[h + 1]) : -INFINITY;
+              xmax = fmaxf(xmax, fmaxf(x0, x1));
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              psum[h] += p0;
+              psum[h + 1] += p1;
+              pk[h >> 1] = pack_bf16x2(p0, p1);
+            }
+          }
+        }
+        wait_or_die(&bfree[s], ph ^ 1u, 25u);   // O^T(j-2) has read this P tile
+        if (!dead) {
+          if (active) {
+            uint8_t* prow = sm + OFF_P + s * kPTile + kb_row * 128;
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8)
+              *reinterpret_cast<uint4*>(prow + ((q8 ^ (kb_row & 7)) << 4)) =
+                  make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&pfull[s]);
+        }
+      }
+      if (xmax > kRangeLog2) report(a.status, CSA_DEV_RANGE, (unsigned)x.row);
+      wait_or_die(ofull, (uint32_t)n & 1u, 26u);
       tc_fence_after();
-      uint32_t s0[32], s1[32];
-      const uint32_t ta = tmem_addr(tS, (uint32_t)(warp * 32), 0);
-      tmem_ld32(ta, s0);
-      tmem_ld32(ta + 32, s1);
-      tmem_ld_wait();
-      const bool valid = k_lo + (int64_t)blk * kBK + rw < k_hi;
-      uint32_t pk[32];
-#pragma unroll
-      for (int h = 0; h < kHG; h += 2) {
-        const float l0 = __uint_as_float(h < 32 ? s0[h] : s1[h - 32]);
-        const float l1 = __uint_as_float(h < 32 ? s0[h + 1] : s1[h + 1 - 32]);
-        float x0 = valid ? fmaf(l0, c2, -mb2[h]) : -INFINITY;
-        float x1 = valid ? fmaf(l1, c2, -mb2[h + 1]) : -INFINITY;
-        xmax = fmaxf(xmax, fmaxf(x0, x1));
-        const float p0 = ex2(x0), p1 = ex2(x1);
-        psum[h] += p0;
-        psum[h + 1] += p1;
-        pk[h >> 1] = pack_bf16x2(p0, p1);
-      }
-      if (!mbar_wait(pfree, ph ^ 1u)) { ok = false; break; }
-      uint8_t* prow = sP + rw * 128;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(prow + ((j ^ (rw & 7)) << 4)) =
-            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(pfull);
-    }
-    if (!ok) {
-      *abort_flag = 1;
-      report(a.status, CSA_DEV_TIMEOUT, 12u);
-    }
-    if (xmax > kRangeLog2) report(a.status, CSA_DEV_RANGE, (unsigned)row);
-    bool have_o = n_blocks > 0 && ok && mbar_wait(ofull, 0);
-    tc_fence_after();
+      const bool have_o = nb > 0 && !dead;
 
-    // ---- epilogue: per-head denominators, then O^T -> output
-    float* red = reinterpret_cast<float*>(sm + OFF_RED);   // [128][65]
-#pragma unroll
-    for (int h = 0; h < kHG; ++h) red[rw * 65 + h] = psum[h];
-    named_bar(1, 128);
-    const int64_t slot = (row * a.n_hg + hg);
-    if (rw < kHG) {
-      float tot = 0.f;
-      for (int r = 0; r < 128; ++r) tot += red[r * 65 + rw];
-      if (a.split) {
-        a.d_part[(slot * a.n_splits + split_id) * kHG + rw] = tot;
-        if (split_id == 0) a.mb_part[slot * kHG + rw] = mb2[rw];
-      } else {
-        float den = tot;
-        if (a.sink) {
-          const float z = a.sink[hg * kHG + rw];
-          den += ex2(fmaf(z, kLog2e, -mb2[rw]));
-        }
-        sinv[rw] = den > 0.f ? 1.f / den : 0.f;
-      }
-    }
-    named_bar(1, 128);
-    bf16* stage = reinterpret_cast<bf16*>(sm + OFF_STAGE);   // [64][512]
-    for (int j = 0; j < 4; ++j) {
-      uint32_t o0[32], o1[32];
-      if (have_o) {
-        const uint32_t ta = tmem_addr(tO + 64 * j, (uint32_t)(warp * 32), 0);
-        tmem_ld32(ta, o0);
-        tmem_ld32(ta + 32, o1);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int h = 0; h < 32; ++h) { o0[h] = 0u; o1[h] = 0u; }
-      }
-      const int c = 128 * j + rw;
-      if (a.split) {
-        float* op = a.o_part + ((slot * a.n_splits + split_id) * kHG) * kC + c;
-#pragma unroll
-        for (int h = 0; h < kHG; ++h)
-          op[(int64_t)h * kC] = __uint_as_float(h < 32 ? o0[h] : o1[h - 32]);
-      } else {
-        const bool rot = !(a.flags & CSA_F_NO_ROPE) && c >= kC - a.r;
-        float cs = 1.f, sn = 0.f;
-        if (rot) {
-          const int pi = (c - (kC - a.r)) >> 1;
-          cs = rcs[pi];
-          sn = rsn[pi];
-        }
-#pragma unroll
-        for (int h = 0; h < kHG; ++h) {
-          float v = __uint_as_float(h < 32 ? o0[h] : o1[h - 32]) * sinv[h];
-          const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
-          // rotate by -pos: (x0, x1) -> (x0 cs + x1 sn, -x0 sn + x1 cs)
-          if (rot) v = (lane & 1) ? fmaf(v, cs, -partner * sn) : fmaf(v, cs, partner * sn);
-          stage[h * kC + c] = __float2bfloat16_rn(v);
-        }
-      }
-    }
-    if (!a.split) {
+      // per-head denominators
+      float two[2];
+      warp_transpose_sum64(psum, lane, two);
+      red[warp * kHG + 2 * lane] = two[0];
+      red[warp * kHG + 2 * lane + 1] = two[1];
       named_bar(1, 128);
-      const uint4* s4 = reinterpret_cast<const uint4*>(stage);
-      uint4* o4 = reinterpret_cast<uint4*>(a.out + (row * a.H + (int64_t)hg * kHG) * kC);
-      for (int i = rw; i < kHG * kC / 8; i += 128) o4[i] = s4[i];
+      if (rw < kHG && !dead) {
+        const float tot = red[rw] + red[kHG + rw] + red[2 * kHG + rw] + red[3 * kHG + rw];
+        if (a.split) {
+          a.d_part[(slot * a.n_splits + x.split) * kHG + rw] = tot;
+          if (x.split == 0) a.mb_part[slot * kHG + rw] = my_mb2;
+        } else {
+          const float den = tot + sterm[rw];
+          sinv[rw] = den > 0.f ? 1.f / den : 0.f;
+        }
+      }
+      named_bar(1, 128);
+
+      // O^T -> output: thread = dim 128 jt + 32 warp + lane
+      float iv[kHG];
+#pragma unroll
+      for (int h = 0; h < kHG; ++h) iv[h] = a.split ? 1.f : sinv[h];
+      const int odd = lane & 1;
+#pragma unroll 1
+      for (int jt = 0; jt < 4; ++jt) {
+        const int c = 128 * jt + warp * 32 + lane;
+        const int cc = c - odd;
+        const float cs = ecs[jt], sn = esn[jt];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {   // heads 32 half .. 32 half + 31
+          uint32_t ov[32];
+          if (have_o) {
+            tmem_ld32(tmem_addr(tO + 64 * jt + 32 * half, (uint32_t)(warp * 32), 0), ov);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = 0u;
+          }
+          if (jt == 3 && half == 1 && !dead) {   // every TMEM read of this item is done
+            tc_fence_before();
+            mbar_arrive(ofree);
+          }
+          if (dead) continue;
+          if (a.split) {
+            float* op = a.o_part + ((slot * a.n_splits + x.split) * kHG + 32 * half) * kC + c;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) op[(int64_t)e * kC] = __uint_as_float(ov[e]);
+          } else {
+            bf16* obase = a.out + (x.row * a.H + (int64_t)x.hg * kHG + 32 * half) * kC + cc;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int h = 32 * half + e;
+              const float v0 = __uint_as_float(ov[e]) * iv[h];
+              const float v1 = __uint_as_float(ov[e + 1]) * iv[h + 1];
+              // even lane keeps head h and receives its neighbour's dim; odd lane head h+1
+              const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+              const float x0 = odd ? recv : v0;
+              const float x1 = odd ? v1 : recv;
+              // rotate the pair by -pos: (x0, x1) -> (x0 cs + x1 sn, -x0 sn + x1 cs)
+              const float y0 = fmaf(x0, cs, x1 * sn), y1 = fmaf(x1, cs, -x0 * sn);
+              *reinterpret_cast<uint32_t*>(obase + (int64_t)(e + odd) * kC) = pack_bf16x2(y0, y1);
+            }
+          }
+        }
+      }
+      gblk += nb;
     }
   }
 
@@ -527,6 +772,15 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(TcAttnArgs a) {
   }
 }
 
+// Streaming multiprocessors of the current device (one persistent CTA each).
+inline int64_t num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
+}
+
 inline int n_splits_for(int64_t max_keys) {
   int64_t n = (max_keys + kSplitKeys - 1) / kSplitKeys;
   return n < 1 ? 1 : (int)n;
@@ -537,7 +791,7 @@ inline int n_splits_for(int64_t max_keys) {
 bool attn_tc_supported(const AttnParams& p) {
   auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   if (p.f.c != kC || p.H % kHG != 0 || p.f.r > 64 || (p.f.r & 1)) return false;
-  if (p.sparse && p.k > kMaxK) return false;
+  if (p.sparse && p.k > kMaxK) return false;   // the per-item index list holds kMaxK
   if (p.B * p.Tq >= (1LL << 31)) return false;
   if (p.Tq == 1 && p.B > 65535) return false;
   return al(p.q) && al(p.out) && (p.N == 0 || al(p.entries)) && (p.Tw == 0 || al(p.win));
@@ -581,6 +835,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   const int64_t rows = p.B * p.Tq;
   a.split = p.Tq == 1 ? 1 : 0;
   const int64_t max_keys = (p.sparse ? (int64_t)p.k : p.N) + p.n_win;
+  a.n_rows = rows;
   if (a.split) {
     a.n_splits = n_splits_for(max_keys);
     const size_t need = attn_tc_scratch(p.B, p.Tq, p.H, kC, max_keys);
@@ -592,20 +847,22 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   } else {
     a.n_splits = 1;
   }
+  a.n_items = rows * a.n_hg * a.n_splits;
+  CUtensorMap mq;   // q as [B*Tq*H rows][512] bf16, boxes of 64 rows x 64 dims
+  if (!make_map_bf16_3d(&mq, p.q, kC, (uint64_t)rows * p.H, 1, 64, kHG))
+    return cudaErrorInvalidValue;
   const int smem = SMEM_BYTES + 1024;
   cudaError_t e =
       cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(a.n_items < num_sms() ? a.n_items : num_sms());
+  attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, a);
   if (a.split) {
-    dim3 grid((unsigned)a.n_splits, (unsigned)rows, (unsigned)a.n_hg);
-    attn_tc_kernel<<<grid, kThreads, smem, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_combine_kernel<<<dim3((unsigned)rows, (unsigned)a.n_hg), 256, 0, stream>>>(a);
     *n_launch = 2;
   } else {
-    dim3 grid((unsigned)rows, (unsigned)a.n_hg);
-    attn_tc_kernel<<<grid, kThreads, smem, stream>>>(a);
     *n_launch = 1;
   }
   return cudaGetLastError();
