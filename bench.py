@@ -344,8 +344,49 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One stage of the step alone on the csa_prefill workload at --seq-len
+    tokens (for kernel profiles): warm-up, then --steps timed launches."""
+    torch.cuda.set_device(0)
+    w = wl.scaled(wl.WORKLOADS[WORKLOAD], T=args.seq_len) if args.seq_len else wl.WORKLOADS[WORKLOAD]
+    step = Step(w, torch.device("cuda", 0))
+    inp = step.inp
+    if args.only == "attn":
+        import oracle   # valid index sets only: s < visible entries, ascending
+
+        counts = torch.tensor([oracle.visible(t, w.m, w.n_csa) for t in range(w.T)])
+        step.idx.copy_(wl.random_index_sets(counts, w.k, 5).unsqueeze(0))
+        step.entries.copy_(wl.randn(step.entries.shape, 2, "cuda", dtype=w.dtype))
+        step.win.copy_(wl.randn(step.win.shape, 3, "cuda", dtype=w.dtype))
+
+    def once():
+        if args.only == "compress":
+            csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, step.fmt,
+                             entries=step.entries, win_out=step.win)
+        elif args.only == "indexer":
+            csa.indexer_scores_topk(inp["q_I"], inp["w"], inp["k_I"], w.m, w.k,
+                                    idx_out=step.idx, ws=step.ws_idx)
+        else:
+            csa.sparse_mqa_attn(inp["q"], step.entries, step.idx, step.win, step.fmt, w.n_win,
+                                sink=inp["sink"], out=step.out, ws=step.ws_attn)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"only": args.only, "seq_len": w.T, "ms": e0.elapsed_time(e1) / args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--only", choices=["compress", "indexer", "attn"], default=None,
+                    help="time one stage alone (kernel profiling)")
+    ap.add_argument("--seq-len", type=int, default=0, help="tokens for --only (default 8192)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
@@ -353,6 +394,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.only:
+        run_only(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
