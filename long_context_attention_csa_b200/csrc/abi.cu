@@ -49,6 +49,7 @@ csa_status compress_common(int32_t dtype, int64_t B, int64_t T, int32_t m, bool 
   if (B < 0 || T < 0 || m < 1 || B > 65535) return CSA_E_ARG;
   if (z_cols != 1 && z_cols != f.c) return CSA_E_ARG;
   if (overlap ? (2 * m > 256) : (m > 4096)) return CSA_E_UNSUPPORTED;
+  if (f.c != 64 && f.c != 128 && f.c != 256 && f.c != 512) return CSA_E_UNSUPPORTED;
   const int64_t n = T / m;
   if (B == 0 || T == 0) return CSA_OK;
   if (!kv_a || !z_a || (overlap && (!kv_b || !z_b))) return CSA_E_ARG;

@@ -68,14 +68,14 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + kRegions * kQRegion;   // 2 key tiles
 constexpr int OFF_P = OFF_K + 2 * kKTile;            // 2 P tiles
 constexpr int OFF_LIST = OFF_P + 2 * kPTile;         // 2 index lists
-constexpr int OFF_MB = OFF_LIST + 2 * kMaxK * 4;     // [2][64] bounds (log2 units)
-constexpr int OFF_ROPE = OFF_MB + 2 * kHG * 4;       // [2][cos 32 | sin 32]
-constexpr int OFF_RED = OFF_ROPE + 2 * 64 * 4;       // [4][64] partial denominators
+constexpr int OFF_MB = OFF_LIST + 2 * kMaxK * 4;     // [4][64] bounds (log2 units)
+constexpr int OFF_ROPE = OFF_MB + 4 * kHG * 4;       // [4][cos 32 | sin 32]
+constexpr int OFF_RED = OFF_ROPE + 4 * 64 * 4;       // [4][64] partial denominators
 constexpr int OFF_INV = OFF_RED + 4 * kHG * 4;       // [64] 1/denominator
 constexpr int OFF_STERM = OFF_INV + kHG * 4;         // [64] sink term
 constexpr int OFF_NENT = OFF_STERM + kHG * 4;        // [2] entries per item
 constexpr int OFF_BAR = OFF_NENT + 64;
-constexpr int kNumBars = 20;
+constexpr int kNumBars = 22;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64;
 
@@ -105,6 +105,7 @@ struct TcAttnArgs {
   float* o_part;    // [rows][n_hg][n_splits][64][512]
   float* d_part;    // [rows][n_hg][n_splits][64]
   float* mb_part;   // [rows][n_hg][64]
+  bf16* qhat;       // [grid][2 slots][64 heads][512]: next items' q^, prepared ahead
   unsigned* status;
 };
 
@@ -160,14 +161,16 @@ __device__ __forceinline__ int item_blocks(const TcAttnArgs& a, const Item& x, i
   return h > l ? (int)((h - l + kBK - 1) / kBK) : 0;
 }
 
-// In-place query transform by one warp: the raw q rows of heads
-// [16 w, 16 w + 16) sit in the 128-byte-swizzled Q tile (loaded by TMA); each
-// becomes bf16(RoPE_pos(RMSNorm(q))) and mb2[h] = scale |q^| sqrt(c) log2(e)
-// (times 1 + 2^-7), an upper bound of the head's logits against unit-RMS keys.
-// Lane l owns elements [8l, 8l+8) and [256+8l, 256+8l+8); four heads at once.
-__device__ __forceinline__ void query_transform(const TcAttnArgs& a, int w, int lane, float scale,
-                                                uint8_t* sQ, float* mb2, const float* rcs,
-                                                const float* rsn) {
+// Query preparation by one producer warp, one item ahead of its use: the raw
+// q rows of heads [16 w, 16 w + 16) are read from global memory, replaced by
+// bf16(RoPE_pos(RMSNorm(q))) and written to the CTA's q^ scratch slot (row h,
+// 512 dims), from which a single TMA load brings them into the Q tile when the
+// item starts.  mb2[h] = scale |q^| sqrt(c) log2(e) (times 1 + 2^-7) is an
+// upper bound of the head's logits against unit-RMS keys.  Lane l owns
+// elements [8l, 8l+8) and [256+8l, 256+8l+8); four heads are in flight at once.
+__device__ __forceinline__ void prep_query(const TcAttnArgs& a, const bf16* qsrc, bf16* qdst,
+                                           int w, int lane, float scale, float* mb2,
+                                           const float* rcs, const float* rsn) {
   float rc[8], rs[8];   // this lane's RoPE factors (identity outside the RoPE dims)
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -180,19 +183,14 @@ __device__ __forceinline__ void query_transform(const TcAttnArgs& a, int w, int 
       rs[k] = rsn[pi];
     }
   }
-  const int ch = lane & 7;
   for (int i0 = 0; i0 < 16; i0 += 4) {
     uint4 raw[4][2];
-    uint4* ptr[4][2];
     float x[4][16], ss[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int h = w * 16 + i0 + u;
-      ptr[u][0] = reinterpret_cast<uint4*>(sQ + (lane >> 3) * kQRegion + h * 128 +
-                                           ((ch ^ (h & 7)) << 4));
-      ptr[u][1] = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ptr[u][0]) + 4 * kQRegion);
-      raw[u][0] = *ptr[u][0];
-      raw[u][1] = *ptr[u][1];
+      const bf16* qr = qsrc + (int64_t)(w * 16 + i0 + u) * kC;
+      raw[u][0] = __ldg(reinterpret_cast<const uint4*>(qr + lane * 8));
+      raw[u][1] = __ldg(reinterpret_cast<const uint4*>(qr + 256 + lane * 8));
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -214,6 +212,7 @@ __device__ __forceinline__ void query_transform(const TcAttnArgs& a, int w, int 
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
+      const int h = w * 16 + i0 + u;
       const float inv = (a.flags & CSA_F_NO_NORM) ? 1.f : rsqrtf(ss[u] / (float)kC + a.eps);
       uint32_t wd[8];
 #pragma unroll
@@ -221,11 +220,11 @@ __device__ __forceinline__ void query_transform(const TcAttnArgs& a, int w, int 
         const float x0 = x[u][2 * k] * inv, x1 = x[u][2 * k + 1] * inv;
         wd[k] = pack_bf16x2(x0 * rc[k] - x1 * rs[k], x0 * rs[k] + x1 * rc[k]);
       }
-      *ptr[u][0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      *ptr[u][1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+      bf16* qd = qdst + (int64_t)h * kC;
+      *reinterpret_cast<uint4*>(qd + lane * 8) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      *reinterpret_cast<uint4*>(qd + 256 + lane * 8) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
       if (lane == 0)
-        mb2[w * 16 + i0 + u] =
-            scale * sqrtf(ss[u]) * inv * sqrtf((float)kC) * (1.f + 0.0078125f) * kLog2e;
+        mb2[h] = scale * sqrtf(ss[u]) * inv * sqrtf((float)kC) * (1.f + 0.0078125f) * kLog2e;
     }
   }
 }
@@ -265,14 +264,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* sfull = bars + 4;    // [2] S^T of the block done
   uint64_t* pfull = bars + 6;    // [2] P tile written (128 softmax threads)
   uint64_t* iready = bars + 8;   // [2] item's entry count published
-  uint64_t* qload = bars + 10;   // raw q rows landed (TMA)
-  uint64_t* qfull = bars + 11;   // q^ ready (128 producer threads)
+  uint64_t* qload = bars + 10;   // the item's q^ rows landed in the Q tile (TMA)
   uint64_t* qfree = bars + 12;   // last S^T of the item done
   uint64_t* ofull = bars + 13;   // last O^T of the item done
   uint64_t* ofree = bars + 14;   // epilogue finished reading O^T (128 threads)
   uint64_t* drain = bars + 15;
   uint64_t* ifree = bars + 16;   // [2] MMA and softmax have read the item slot
-  uint64_t* qready = bars + 18;  // [2] the item's q^ and bounds ready (per slot, softmax)
+  uint64_t* qready = bars + 18;  // [4] the item's bounds and RoPE table ready (softmax)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   int* wcnt = reinterpret_cast<int*>(sm + OFF_MISC + 8);        // [4]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 24);
@@ -288,10 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pfull[i], 128);
       mbar_init(&iready[i], 1);
       mbar_init(&ifree[i], 2);
-      mbar_init(&qready[i], 128);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&qready[i], 128);
     mbar_init(qload, 1);
-    mbar_init(qfull, 128);
     mbar_init(qfree, 1);
     mbar_init(ofull, 1);
     mbar_init(ofree, 128);
@@ -318,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // named barrier, so no barrier can be left waiting.
     const int ptid = threadIdx.x - 128, pw = warp - 4, quad = lane >> 3, g8 = lane & 7;
     const uint32_t kbase = smem_u32(sm + OFF_K);
+    bf16* qslots = a.qhat + (int64_t)blockIdx.x * 2 * kHG * kC;
     bool dead = false;
     auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
       if (!dead) {
@@ -330,25 +328,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       dead = __any_sync(0xffffffffu, dead);
     };
-    int64_t gblk = 0;
-    int n = 0;
-    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
-      const int ip = n & 1;
+    // RoPE table, q^ (to scratch slot n&1) and bounds of the CTA's item n
+    auto prepare = [&](int64_t it, int n) {
       const Item x = decode_item(a, it);
-      wait_or_die(&ifree[ip], (uint32_t)((n >> 1) & 1) ^ 1u, 19u);   // item n-2 consumed
-      int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST) + ip * kMaxK;
-      float* rcs = ropes + ip * 64;
+      float* rcs = ropes + (n & 3) * 64;
       float* rsn = rcs + 32;
-      const bf16* qrow = a.q + (x.row * a.H + (int64_t)x.hg * kHG) * kC;
-      if (!dead && ptid == 0) {   // warm L2 with this item's q rows ahead of the TMA load
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qrow), "r"(kHG * kC * 2)
-                     : "memory");
-      }
       if (!dead && pw == 0 && lane < (a.r >> 1)) {
         float cs, sn;
         rope_cos_sin(x.pos, lane, a.r, a.base, &cs, &sn);
         rcs[lane] = cs;
         rsn[lane] = sn;
+      }
+      named_bar(2, 128);   // RoPE table complete
+      if (!dead) {
+        const bf16* qsrc = a.q + (x.row * a.H + (int64_t)x.hg * kHG) * kC;
+        prep_query(a, qsrc, qslots + (n & 1) * kHG * kC, pw, lane, scale, mb2s + (n & 3) * kHG,
+                   rcs, rsn);
+        fence_proxy_async_all();   // q^ stores (generic) -> TMA load (async proxy)
+        mbar_arrive(&qready[n & 3]);
+      }
+      named_bar(2, 128);   // the scratch slot is complete before its TMA load
+    };
+    int64_t gblk = 0;
+    int n = 0;
+    if ((int64_t)blockIdx.x < a.n_items) prepare(blockIdx.x, 0);
+    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
+      const int ip = n & 1;
+      const Item x = decode_item(a, it);
+      wait_or_die(&ifree[ip], (uint32_t)((n >> 1) & 1) ^ 1u, 19u);   // item n-2 consumed
+      int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST) + ip * kMaxK;
+      const int64_t it_next = it + gridDim.x;
+      if (!dead && ptid == 0 && it_next < a.n_items) {   // warm L2 with the next item's q rows
+        const Item y = decode_item(a, it_next);
+        const bf16* qn = a.q + (y.row * a.H + (int64_t)y.hg * kHG) * kC;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qn), "r"(kHG * kC * 2)
+                     : "memory");
       }
       int64_t n_ent;
       if (a.sparse) {
@@ -386,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         n_ent = vis_count(x.pos, a.m_dense, a.N);
       }
-      named_bar(2, 128);   // list and RoPE table complete
+      named_bar(2, 128);   // the index list is complete
       if (!dead && ptid == 0) {
         nent[ip] = (int)n_ent;
         mbar_arrive(&iready[ip]);
@@ -394,14 +408,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t k_lo, k_hi;
       const int nb = dead ? 0 : item_blocks(a, x, n_ent, &k_lo, &k_hi);
 
-      // the previous item's last S^T is done with Q: load this item's rows
+      // the previous item's last S^T is done with Q: bring in this item's q^
       if (!dead && ptid == 0) {
         if (n > 0 && !mbar_wait(qfree, (uint32_t)(n - 1) & 1u)) {
           *abort_flag = 1;
           report(a.status, CSA_DEV_TIMEOUT, 20u);
         } else {
           mbar_arrive_expect_tx(qload, kRegions * kQRegion);
-          const int32_t qr = (int32_t)(x.row * a.H + (int64_t)x.hg * kHG);
+          const int32_t qr = (int32_t)(((int64_t)blockIdx.x * 2 + (n & 1)) * kHG);
           for (int r = 0; r < kRegions; ++r)
             tma_load_3d(sQ + r * kQRegion, &map_q, qload, r * 64, qr, 0);
         }
@@ -438,15 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the barrier counts this thread's arrival once its copies land
           if (!dead) cp_async_arrive(&kfull[s]);
         }
-        if (b == 0) {   // transform this item's q while the first block is in flight
-          wait_or_die(qload, (uint32_t)n & 1u, 22u);
-          if (!dead) {
-            query_transform(a, pw, lane, scale, sQ, mb2s + ip * kHG, rcs, rsn);
-            fence_proxy_async_smem();
-            mbar_arrive(qfull);
-            mbar_arrive(&qready[ip]);
-          }
-        }
+        // the next item's query, once both key tiles are in flight (the
+        // producer would otherwise only wait for a tile to free up)
+        if (b == (nb > 1 ? 1 : 0) && it_next < a.n_items) prepare(it_next, n + 1);
       }
       gblk += nb;
     }
@@ -484,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int64_t k_lo, k_hi;
         const int nb = item_blocks(a, x, nent[n & 1], &k_lo, &k_hi);
         mbar_arrive(&ifree[n & 1]);
-        if (*abort_flag || !mbar_wait(qfull, (uint32_t)n & 1u)) { ok = false; break; }
+        if (*abort_flag || !mbar_wait(qload, (uint32_t)n & 1u)) { ok = false; break; }
         tc_fence_after();
         if (nb == 0) {
           mma_commit(qfree);
@@ -565,8 +573,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ip = n & 1;
       const Item x = decode_item(a, it);
       wait_or_die(&iready[ip], (uint32_t)(n >> 1) & 1u, 24u);
-      wait_or_die(&qready[ip], (uint32_t)(n >> 1) & 1u, 24u);
-      const float* mb2 = mb2s + ip * kHG;
+      wait_or_die(&qready[n & 3], (uint32_t)(n >> 2) & 1u, 24u);
+      const float* mb2 = mb2s + (n & 3) * kHG;
       int64_t k_lo = 0, k_hi = 0;
       const int nb = dead ? 0 : item_blocks(a, x, nent[ip], &k_lo, &k_hi);
       // values the epilogue needs, copied now (the producer may refill the
@@ -579,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float ecs[4], esn[4];   // RoPE factors of this thread's output pair, per slice
       {
-        const float* rcs = ropes + ip * 64;
+        const float* rcs = ropes + (n & 3) * 64;
 #pragma unroll
         for (int jt = 0; jt < 4; ++jt) {
           const int cc = 128 * jt + warp * 32 + (lane & ~1);
@@ -797,12 +805,19 @@ bool attn_tc_supported(const AttnParams& p) {
   return al(p.q) && al(p.out) && (p.N == 0 || al(p.entries)) && (p.Tw == 0 || al(p.win));
 }
 
+// q^ scratch: two 64-head slots per persistent CTA (stays in L2)
+inline size_t qhat_bytes() { return (size_t)num_sms() * 2 * kHG * kC * sizeof(bf16); }
+
 size_t attn_tc_scratch(int64_t B, int64_t Tq, int H, int c, int64_t max_keys) {
-  if (Tq != 1 || c != kC || H % kHG != 0) return 0;
-  const int64_t n_hg = H / kHG;
-  const int64_t ns = n_splits_for(max_keys);
-  const int64_t slots = B * Tq * n_hg;
-  return (size_t)(slots * ns * (kHG * kC + kHG) + slots * kHG) * sizeof(float);
+  if (c != kC || H % kHG != 0) return 0;
+  size_t bytes = qhat_bytes();
+  if (Tq == 1) {
+    const int64_t n_hg = H / kHG;
+    const int64_t ns = n_splits_for(max_keys);
+    const int64_t slots = B * Tq * n_hg;
+    bytes += (size_t)(slots * ns * (kHG * kC + kHG) + slots * kHG) * sizeof(float);
+  }
+  return bytes;
 }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned long long* n_launch) {
@@ -836,26 +851,27 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   a.split = p.Tq == 1 ? 1 : 0;
   const int64_t max_keys = (p.sparse ? (int64_t)p.k : p.N) + p.n_win;
   a.n_rows = rows;
+  const size_t need = attn_tc_scratch(p.B, p.Tq, p.H, kC, max_keys);
+  if (p.scratch_bytes < need) return cudaErrorInvalidValue;
+  a.qhat = static_cast<bf16*>(p.scratch);
   if (a.split) {
     a.n_splits = n_splits_for(max_keys);
-    const size_t need = attn_tc_scratch(p.B, p.Tq, p.H, kC, max_keys);
-    if (p.scratch_bytes < need) return cudaErrorInvalidValue;
     const int64_t slots = rows * a.n_hg;
-    a.o_part = static_cast<float*>(p.scratch);
+    a.o_part = reinterpret_cast<float*>(static_cast<char*>(p.scratch) + qhat_bytes());
     a.d_part = a.o_part + slots * a.n_splits * kHG * kC;
     a.mb_part = a.d_part + slots * a.n_splits * kHG;
   } else {
     a.n_splits = 1;
   }
   a.n_items = rows * a.n_hg * a.n_splits;
-  CUtensorMap mq;   // q as [B*Tq*H rows][512] bf16, boxes of 64 rows x 64 dims
-  if (!make_map_bf16_3d(&mq, p.q, kC, (uint64_t)rows * p.H, 1, 64, kHG))
+  const unsigned grid = (unsigned)(a.n_items < num_sms() ? a.n_items : num_sms());
+  CUtensorMap mq;   // q^ scratch as [grid*2*64 rows][512] bf16, boxes of 64 rows x 64 dims
+  if (!make_map_bf16_3d(&mq, a.qhat, kC, (uint64_t)grid * 2 * kHG, 1, 64, kHG))
     return cudaErrorInvalidValue;
   const int smem = SMEM_BYTES + 1024;
   cudaError_t e =
       cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)(a.n_items < num_sms() ? a.n_items : num_sms());
   attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, a);
   if (a.split) {
     e = cudaGetLastError();
