@@ -21,21 +21,33 @@
 // MN-major as the A operand of O^T (K = V).  Two key tiles alternate, so the
 // gather of block b+1 and S^T(b+1) overlap the softmax and O^T of block b.
 //
+// Query RMSNorm as a per-head scale: the Q tile holds the raw q rows (TMA,
+// dims 0..447) and RoPE(q) for the last 64 dims (written by the producer), so
+// S^T carries |q| instead of |q^| and the softmax multiplies head h's column
+// by scale inv_h log2(e), inv_h = 1/rms(q_h).  RoPE preserves pair norms, so
+// inv_h comes from the raw rows.
+//
 // Softmax without a running maximum: q^ and every stored key are RMS-
 // normalised (the method's RMSNorm), so |scale q^ . k| <= scale |q^| sqrt(c)
 // =: M_h, a per-(token, head) bound known before any key is read.  Weights
 // are exp(l - M_h) in (e^-2M_h, 1]: no rescaling of O, no cross-lane max, and
 // split partial sums add directly.  A logit more than 60 above the bound (keys
-// far from unit RMS) is reported as CSA_DEV_RANGE.
+// far from unit RMS) is reported as CSA_DEV_RANGE.  The per-head sums of the
+// bf16 weights come from the tensor core too (a ones tile times P^T), so the
+// denominators match the numerators' rounding.
 //
-// Persistent CTAs (one per SM) walk their items in turn; roles (288 threads):
-//   warps 4-7  producer: index compaction, RoPE table, the next item's raw q
-//              rows by TMA and their in-place RMSNorm + RoPE, the key gather
-//              (cp.async; each warp-instruction moves four 128-byte row pieces);
-//   warp 8     TMEM owner and single-thread MMA issuer;
-//   warps 0-3  softmax (lanes 0-15: one key each, the M = 64 TMEM layout puts
-//              rows 16w..16w+15 in lanes 0-15 of warp w), then the epilogue
-//              (thread = output dim), which overlaps the next item's first MMAs.
+// Persistent CTAs (one per SM) walk their items in turn; roles (384 threads,
+// the register budget of 288 threads since allocation is per 128 threads):
+//   warps 8-10 producer: index compaction, RoPE table, the item's raw q rows
+//              by TMA, in-place rotation of the RoPE dims and per-head 1/rms,
+//              the key gather (cp.async; each warp-instruction moves four
+//              128-byte row pieces);
+//   warp 11    TMEM owner and single-thread MMA issuer;
+//   warps 0-3  softmax (all 32 lanes: the 16x64b TMEM load gives each lane
+//              one key and the 32 heads of one parity);
+//   warps 4-7  epilogue (thread = output dim), which runs alongside the next
+//              item's softmax; it frees O^T in four 64-column slices, so the
+//              next item's first O^T waits only for the slice it overwrites.
 // Decode rows (one query per sequence) split the key list into fixed 256-key
 // pieces whose fp32 partials a combine kernel adds in a fixed order, so a
 // row's result does not depend on the batch it runs in.
@@ -60,22 +72,28 @@ constexpr int kQRegion = kHG * 128;          // 8 KB per query chunk
 constexpr int kPTile = kBK * 128;            // 8 KB: P^T [64 keys][64 heads] bf16
 constexpr int kSplitKeys = 256;              // decode split size (fixed)
 constexpr int kMaxK = 1024;                  // largest top-k the index list holds
-constexpr int kThreads = 288;
+constexpr int kProdWarp0 = 8;                // warps 8-10 produce, warp 11 issues MMAs
+constexpr int kProdWarps = 3;
+constexpr int kProdThreads = 32 * kProdWarps;
+constexpr int kMmaWarp = kProdWarp0 + kProdWarps;
+constexpr int kGatherIters = (kBK / 4 + kProdWarps - 1) / kProdWarps;   // 4-row groups per warp
+constexpr int kThreads = 32 * (kMmaWarp + 1);  // 384
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRangeLog2 = 60.f * kLog2e;  // CSA_DEV_RANGE threshold
 
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + kRegions * kQRegion;   // 2 key tiles
 constexpr int OFF_P = OFF_K + 2 * kKTile;            // 2 P tiles
-constexpr int OFF_LIST = OFF_P + 2 * kPTile;         // 2 index lists
+constexpr int OFF_ONES = OFF_P + 2 * kPTile;         // 8 rows x 64 bf16 ones (1 KB)
+constexpr int OFF_LIST = OFF_ONES + 1024;            // 2 index lists
 constexpr int OFF_MB = OFF_LIST + 2 * kMaxK * 4;     // [4][64] bounds (log2 units)
 constexpr int OFF_ROPE = OFF_MB + 4 * kHG * 4;       // [4][cos 32 | sin 32]
-constexpr int OFF_RED = OFF_ROPE + 4 * 64 * 4;       // [4][64] partial denominators
-constexpr int OFF_INV = OFF_RED + 4 * kHG * 4;       // [64] 1/denominator
-constexpr int OFF_STERM = OFF_INV + kHG * 4;         // [64] sink term
-constexpr int OFF_NENT = OFF_STERM + kHG * 4;        // [2] entries per item
+constexpr int OFF_C2 = OFF_ROPE + 4 * 64 * 4;        // [4][64] scale inv_h log2(e)
+constexpr int OFF_INV = OFF_C2 + 4 * kHG * 4;        // [64] 1/denominator
+constexpr int OFF_SS7 = OFF_INV + kHG * 4;           // [64] sum of squares of the RoPE dims
+constexpr int OFF_NENT = OFF_SS7 + kHG * 4;          // [2] entries per item
 constexpr int OFF_BAR = OFF_NENT + 64;
-constexpr int kNumBars = 22;
+constexpr int kNumBars = 26;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64;
 
@@ -105,7 +123,6 @@ struct TcAttnArgs {
   float* o_part;    // [rows][n_hg][n_splits][64][512]
   float* d_part;    // [rows][n_hg][n_splits][64]
   float* mb_part;   // [rows][n_hg][64]
-  bf16* qhat;       // [grid][2 slots][64 heads][512]: next items' q^, prepared ahead
   unsigned* status;
 };
 
@@ -161,118 +178,33 @@ __device__ __forceinline__ int item_blocks(const TcAttnArgs& a, const Item& x, i
   return h > l ? (int)((h - l + kBK - 1) / kBK) : 0;
 }
 
-// Query preparation by one producer warp, one item ahead of its use: the raw
-// q rows of heads [16 w, 16 w + 16) are read from global memory, replaced by
-// bf16(RoPE_pos(RMSNorm(q))) and written to the CTA's q^ scratch slot (row h,
-// 512 dims), from which a single TMA load brings them into the Q tile when the
-// item starts.  mb2[h] = scale |q^| sqrt(c) log2(e) (times 1 + 2^-7) is an
-// upper bound of the head's logits against unit-RMS keys.  Lane l owns
-// elements [8l, 8l+8) and [256+8l, 256+8l+8); four heads are in flight at once.
-__device__ __forceinline__ void prep_query(const TcAttnArgs& a, const bf16* qsrc, bf16* qdst,
-                                           int w, int lane, float scale, float* mb2,
-                                           const float* rcs, const float* rsn) {
-  float rc[8], rs[8];   // this lane's RoPE factors (identity outside the RoPE dims)
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int el = (k >> 2) * 256 + lane * 8 + (k & 3) * 2;
-    rc[k] = 1.f;
-    rs[k] = 0.f;
-    if (!(a.flags & CSA_F_NO_ROPE) && el >= kC - a.r) {
-      const int pi = (el - (kC - a.r)) >> 1;
-      rc[k] = rcs[pi];
-      rs[k] = rsn[pi];
-    }
-  }
-  for (int i0 = 0; i0 < 16; i0 += 4) {
-    uint4 raw[4][2];
-    float x[4][16], ss[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bf16* qr = qsrc + (int64_t)(w * 16 + i0 + u) * kC;
-      raw[u][0] = __ldg(reinterpret_cast<const uint4*>(qr + lane * 8));
-      raw[u][1] = __ldg(reinterpret_cast<const uint4*>(qr + 256 + lane * 8));
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t wr[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
-                              raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
-      ss[u] = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        x[u][2 * k] = bf16_bits_to_float(wr[k] & 0xffffu);
-        x[u][2 * k + 1] = bf16_bits_to_float(wr[k] >> 16);
-        ss[u] = fmaf(x[u][2 * k], x[u][2 * k], ss[u]);
-        ss[u] = fmaf(x[u][2 * k + 1], x[u][2 * k + 1], ss[u]);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int h = w * 16 + i0 + u;
-      const float inv = (a.flags & CSA_F_NO_NORM) ? 1.f : rsqrtf(ss[u] / (float)kC + a.eps);
-      uint32_t wd[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float x0 = x[u][2 * k] * inv, x1 = x[u][2 * k + 1] * inv;
-        wd[k] = pack_bf16x2(x0 * rc[k] - x1 * rs[k], x0 * rs[k] + x1 * rc[k]);
-      }
-      bf16* qd = qdst + (int64_t)h * kC;
-      *reinterpret_cast<uint4*>(qd + lane * 8) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      *reinterpret_cast<uint4*>(qd + 256 + lane * 8) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
-      if (lane == 0)
-        mb2[h] = scale * sqrtf(ss[u]) * inv * sqrtf((float)kC) * (1.f + 0.0078125f) * kLog2e;
-    }
-  }
-}
-
-// Sum of v[0..63] over the 32 lanes of a warp by recursive halving: after
-// the five exchange steps lane L holds the totals of entries 2L and 2L+1.
-__device__ __forceinline__ void warp_transpose_sum64(float* v, int lane, float* out2) {
-#pragma unroll
-  for (int o = 16, n = 64; o >= 1; o >>= 1, n >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-      const float lo = v[i], hi = v[i + n / 2];
-      const float send = upper ? lo : hi;
-      const float keep = upper ? hi : lo;
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  out2[0] = v[0];
-  out2[1] = v[1];
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, TcAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = sm + OFF_Q;
   float* mb2s = reinterpret_cast<float*>(sm + OFF_MB);
+  float* c2s = reinterpret_cast<float*>(sm + OFF_C2);
   float* ropes = reinterpret_cast<float*>(sm + OFF_ROPE);
-  float* red = reinterpret_cast<float*>(sm + OFF_RED);
   float* sinv = reinterpret_cast<float*>(sm + OFF_INV);
-  float* sterm = reinterpret_cast<float*>(sm + OFF_STERM);
+  float* ss7 = reinterpret_cast<float*>(sm + OFF_SS7);
   int* nent = reinterpret_cast<int*>(sm + OFF_NENT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* kfull = bars;        // [2] key tile landed (128 producer threads)
+  uint64_t* kfull = bars;        // [2] key tile landed (producer threads)
   uint64_t* bfree = bars + 2;    // [2] O^T of the block done: key tile and P tile free
   uint64_t* sfull = bars + 4;    // [2] S^T of the block done
   uint64_t* pfull = bars + 6;    // [2] P tile written (128 softmax threads)
   uint64_t* iready = bars + 8;   // [2] item's entry count published
-  uint64_t* qload = bars + 10;   // the item's q^ rows landed in the Q tile (TMA)
-  uint64_t* qfree = bars + 12;   // last S^T of the item done
-  uint64_t* ofull = bars + 13;   // last O^T of the item done
-  uint64_t* ofree = bars + 14;   // epilogue finished reading O^T (128 threads)
+  uint64_t* qraw = bars + 10;    // raw q rows landed in the Q tile (TMA)
+  uint64_t* qload = bars + 11;   // Q tile complete: RoPE dims rotated (64 producer threads)
+  uint64_t* qfree = bars + 12;   // last S^T of the item done and its Q rows read (2)
+  uint64_t* ofull = bars + 13;   // last O^T (and row-sum MMA) of the item done
   uint64_t* drain = bars + 15;
-  uint64_t* ifree = bars + 16;   // [2] MMA and softmax have read the item slot
-  uint64_t* qready = bars + 18;  // [4] the item's bounds and RoPE table ready (softmax)
+  uint64_t* ifree = bars + 16;   // [2] MMA, softmax and epilogue have read the item slot
+  uint64_t* qready = bars + 18;  // [4] the item's per-head factors ready (epilogue)
+  uint64_t* ofree = bars + 22;   // [4] epilogue has read O^T columns 64 jt .. 64 jt + 63
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  int* wcnt = reinterpret_cast<int*>(sm + OFF_MISC + 8);        // [4]
+  int* wcnt = reinterpret_cast<int*>(sm + OFF_MISC + 8);        // [3]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 24);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,24 +212,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kfull[i], 128);
+      mbar_init(&kfull[i], kProdThreads);
       mbar_init(&bfree[i], 1);
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);
       mbar_init(&iready[i], 1);
-      mbar_init(&ifree[i], 2);
+      mbar_init(&ifree[i], 3);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&qready[i], 128);
-    mbar_init(qload, 1);
-    mbar_init(qfree, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&qready[i], 1);
+      mbar_init(&ofree[i], 128);
+    }
+    mbar_init(qraw, 1);
+    mbar_init(qload, kHG);
+    mbar_init(qfree, 2);
     mbar_init(ofull, 1);
-    mbar_init(ofree, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 8) {
+  // ones tile of the row-sum MMA: bf16 1.0 everywhere, so the swizzle is moot
+  if (threadIdx.x < 256) {
+    reinterpret_cast<uint32_t*>(sm + OFF_ONES)[threadIdx.x] = 0x3F803F80u;
+    fence_proxy_async_smem();
+  }
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -307,164 +247,215 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS0 = tmem;          // S^T buffers at columns 0 and 64
   const uint32_t tO = tmem + 128;     // O^T: 4 x 64 columns
+  const uint32_t tL = tmem + 384;     // per-head sums of P (64 columns, rows identical)
 
-  if (warp >= 4 && warp < 8) {
-    // ======================= producer
-    // Failure handling: a wait that runs out marks the thread `dead` (made
-    // warp-uniform); dead threads skip waits and work but still pass every
-    // named barrier, so no barrier can be left waiting.
-    const int ptid = threadIdx.x - 128, pw = warp - 4, quad = lane >> 3, g8 = lane & 7;
-    const uint32_t kbase = smem_u32(sm + OFF_K);
-    bf16* qslots = a.qhat + (int64_t)blockIdx.x * 2 * kHG * kC;
-    bool dead = false;
-    auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
-      if (!dead) {
-        if (!mbar_wait(bar, parity)) {
-          *abort_flag = 1;
-          report(a.status, CSA_DEV_TIMEOUT, code);
-          dead = true;
-        }
-        dead = dead || *abort_flag;
+  // Failure handling (every role): a wait that runs out marks the thread
+  // `dead` (made warp-uniform); dead threads skip waits and work but still
+  // pass every named barrier, so no barrier can be left waiting.
+  bool dead = false;
+  auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
+    if (!dead) {
+      if (!mbar_wait(bar, parity)) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, code);
+        dead = true;
       }
-      dead = __any_sync(0xffffffffu, dead);
+      dead = dead || *abort_flag;
+    }
+    dead = __any_sync(0xffffffffu, dead);
+  };
+
+  if (warp >= kProdWarp0 && warp < kMmaWarp) {
+    // ======================= producer (3 warps)
+    // Item n's index list and RoPE table are built while item n-1's keys
+    // stream (its index loads are issued early and consumed a block later),
+    // so an item starts with its Q tile and first key tiles only.
+    const int ptid = threadIdx.x - 32 * kProdWarp0, pw = warp - kProdWarp0;
+    const int quad = lane >> 3, g8 = lane & 7;
+    const uint32_t kbase = smem_u32(sm + OFF_K);
+    constexpr int kEv = (kMaxK / kProdWarps + 31) / 32 + 1;   // index words per lane
+    int32_t ev[kEv];
+    // index loads of item (it, m): warp pw takes the contiguous third of the row
+    auto load_idx = [&](int64_t row) {
+      const int32_t* ir = a.idx + row * (int64_t)a.k;
+      const int q3 = (a.k + 2) / 3;
+      const int lo = pw * q3, hi = lo + q3 < a.k ? lo + q3 : a.k;
+#pragma unroll
+      for (int u = 0; u < kEv; ++u) {
+        const int i = lo + u * 32 + lane;
+        ev[u] = (!dead && a.sparse && u * 32 < q3 && i < hi) ? __ldg(ir + i) : -1;
+      }
     };
-    // RoPE table, q^ (to scratch slot n&1) and bounds of the CTA's item n
-    auto prepare = [&](int64_t it, int n) {
-      const Item x = decode_item(a, it);
-      float* rcs = ropes + (n & 3) * 64;
-      float* rsn = rcs + 32;
+    // builds item m's index list, RoPE table and entry count (slot m & 1)
+    auto compact = [&](const Item& y, int m) -> int64_t {
+      wait_or_die(&ifree[m & 1], (uint32_t)((m >> 1) & 1) ^ 1u, 19u);   // item m-2 consumed
+      float* rcs = ropes + (m & 3) * 64;
       if (!dead && pw == 0 && lane < (a.r >> 1)) {
         float cs, sn;
-        rope_cos_sin(x.pos, lane, a.r, a.base, &cs, &sn);
+        rope_cos_sin(y.pos, lane, a.r, a.base, &cs, &sn);
         rcs[lane] = cs;
-        rsn[lane] = sn;
+        rcs[32 + lane] = sn;
       }
-      named_bar(2, 128);   // RoPE table complete
-      if (!dead) {
-        const bf16* qsrc = a.q + (x.row * a.H + (int64_t)x.hg * kHG) * kC;
-        prep_query(a, qsrc, qslots + (n & 1) * kHG * kC, pw, lane, scale, mb2s + (n & 3) * kHG,
-                   rcs, rsn);
-        fence_proxy_async_all();   // q^ stores (generic) -> TMA load (async proxy)
-        mbar_arrive(&qready[n & 3]);
-      }
-      named_bar(2, 128);   // the scratch slot is complete before its TMA load
-    };
-    int64_t gblk = 0;
-    int n = 0;
-    if ((int64_t)blockIdx.x < a.n_items) prepare(blockIdx.x, 0);
-    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
-      const int ip = n & 1;
-      const Item x = decode_item(a, it);
-      wait_or_die(&ifree[ip], (uint32_t)((n >> 1) & 1) ^ 1u, 19u);   // item n-2 consumed
-      int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST) + ip * kMaxK;
-      const int64_t it_next = it + gridDim.x;
-      if (!dead && ptid == 0 && it_next < a.n_items) {   // warm L2 with the next item's q rows
-        const Item y = decode_item(a, it_next);
-        const bf16* qn = a.q + (y.row * a.H + (int64_t)y.hg * kHG) * kC;
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qn), "r"(kHG * kC * 2)
-                     : "memory");
-      }
-      int64_t n_ent;
+      int64_t ne;
       if (a.sparse) {
-        // warp pw compacts the contiguous quarter [pw*q4, pw*q4 + q4) of the row
-        const int32_t* ir = a.idx + x.row * (int64_t)a.k;
-        const int q4 = (a.k + 3) / 4;
-        const int lo = pw * q4, hi = lo + q4 < a.k ? lo + q4 : a.k;
-        int32_t ev[kMaxK / 128];
-#pragma unroll
-        for (int u = 0; u < kMaxK / 128; ++u) {
-          const int i = lo + u * 32 + lane;
-          ev[u] = (!dead && u * 32 < q4 && i < hi) ? ir[i] : -1;
-        }
+        const int lo = pw * ((a.k + 2) / 3);
+        int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST) + (m & 1) * kMaxK;
         int cnt = 0;
 #pragma unroll
-        for (int u = 0; u < kMaxK / 128; ++u) {
+        for (int u = 0; u < kEv; ++u) {
           const bool ok = ev[u] >= 0 && ev[u] < a.N;
           if (!ok && ev[u] != -1)
             report(a.status, CSA_DEV_BAD_INDEX, (unsigned)(lo + u * 32 + lane));
           cnt += __popc(__ballot_sync(0xffffffffu, ok));
         }
-        named_bar(2, 128);   // previous item's use of wcnt finished
+        named_bar(2, kProdThreads);   // previous use of wcnt finished
         if (lane == 0) wcnt[pw] = cnt;
-        named_bar(2, 128);
+        named_bar(2, kProdThreads);
         int off = 0;
         for (int w = 0; w < pw; ++w) off += wcnt[w];
-        n_ent = wcnt[0] + wcnt[1] + wcnt[2] + wcnt[3];
+        ne = wcnt[0] + wcnt[1] + wcnt[2];
 #pragma unroll
-        for (int u = 0; u < kMaxK / 128; ++u) {
+        for (int u = 0; u < kEv; ++u) {
           const bool ok = ev[u] >= 0 && ev[u] < a.N;
           const unsigned bal = __ballot_sync(0xffffffffu, ok);
           if (ok) list[off + __popc(bal & ((1u << lane) - 1u))] = ev[u];
           off += __popc(bal);
         }
       } else {
-        n_ent = vis_count(x.pos, a.m_dense, a.N);
+        ne = vis_count(y.pos, a.m_dense, a.N);
       }
-      named_bar(2, 128);   // the index list is complete
+      named_bar(2, kProdThreads);   // the index list and the RoPE table are complete
       if (!dead && ptid == 0) {
-        nent[ip] = (int)n_ent;
-        mbar_arrive(&iready[ip]);
+        nent[m & 1] = (int)ne;
+        mbar_arrive(&iready[m & 1]);
       }
-      int64_t k_lo, k_hi;
-      const int nb = dead ? 0 : item_blocks(a, x, n_ent, &k_lo, &k_hi);
+      return ne;
+    };
 
-      // the previous item's last S^T is done with Q: bring in this item's q^
+    int64_t gblk = 0;
+    int n = 0;
+    int64_t cur_ent = 0;
+    if ((int64_t)blockIdx.x < a.n_items) {
+      const Item y = decode_item(a, blockIdx.x);
+      load_idx(y.row);
+      cur_ent = compact(y, 0);
+    }
+    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
+      const Item x = decode_item(a, it);
+      const int32_t* list = reinterpret_cast<const int32_t*>(sm + OFF_LIST) + (n & 1) * kMaxK;
+      const int64_t n_ent = cur_ent;
+      int64_t k_lo = 0, k_hi = 0;
+      const int nb = dead ? 0 : item_blocks(a, x, n_ent, &k_lo, &k_hi);
+      const int nbl = nb > 0 ? nb : 1;
+      const int64_t it_next = it + gridDim.x;
+      const bool has_next = it_next < a.n_items;
+      const Item y = decode_item(a, has_next ? it_next : it);
+      if (!dead && ptid == 0 && has_next) {   // warm L2 with the next item's q rows
+        const bf16* qn = a.q + (y.row * a.H + (int64_t)y.hg * kHG) * kC;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qn), "r"(kHG * kC * 2)
+                     : "memory");
+      }
+      // the previous item's last S^T is done with Q: the raw q rows by TMA
+      if (n > 0) wait_or_die(qfree, (uint32_t)(n - 1) & 1u, 20u);
       if (!dead && ptid == 0) {
-        if (n > 0 && !mbar_wait(qfree, (uint32_t)(n - 1) & 1u)) {
-          *abort_flag = 1;
-          report(a.status, CSA_DEV_TIMEOUT, 20u);
-        } else {
-          mbar_arrive_expect_tx(qload, kRegions * kQRegion);
-          const int32_t qr = (int32_t)(((int64_t)blockIdx.x * 2 + (n & 1)) * kHG);
-          for (int r = 0; r < kRegions; ++r)
-            tma_load_3d(sQ + r * kQRegion, &map_q, qload, r * 64, qr, 0);
-        }
+        mbar_arrive_expect_tx(qraw, kRegions * kQRegion);
+        for (int r = 0; r < kRegions; ++r)
+          tma_load_3d(sQ + r * kQRegion, &map_q, qraw, r * 64, x.hg * kHG, (int32_t)x.row);
       }
 
       const bf16* ent = a.entries + x.bidx * a.N * kC;
       const bf16* win = a.win + x.bidx * a.Tw * kC;
-      for (int b = 0; b < (nb > 0 ? nb : 1); ++b) {
+      const float* rcs = ropes + (n & 3) * 64;
+      for (int b = 0; b < nbl; ++b) {
         const int64_t j = gblk + b;
         const int s = (int)(j & 1);
         if (b < nb) {
           wait_or_die(&bfree[s], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
           if (!dead) {
             const uint32_t tile = kbase + s * kKTile;
-            // warp pw fetches rows 16 pw .. 16 pw + 15: four rows per instruction
+            // groups of four rows (one per 8-lane quad; 128 bytes per lane group
+            // and region) dealt round-robin over the producer warps
+            const bf16* src[kGatherIters];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int r = pw * 16 + 4 * i + quad;
+            for (int u = 0; u < kGatherIters; ++u) {
+              const int r = 4 * (pw + kProdWarps * u) + quad;
               const int64_t key = k_lo + (int64_t)b * kBK + r;
-              const bf16* src = nullptr;
-              if (key < k_hi) {
-                if (key < n_ent) src = ent + (int64_t)(a.sparse ? list[key] : key) * kC;
-                else src = win + ((x.jlo - x.wp0) + (key - n_ent)) * kC;
-              }
+              src[u] = nullptr;
+              if (pw + kProdWarps * u < kBK / 4 && key < k_hi)
+                src[u] = key < n_ent ? ent + (int64_t)(a.sparse ? list[key] : key) * kC
+                                     : win + ((x.jlo - x.wp0) + (key - n_ent)) * kC;
+            }
+#pragma unroll
+            for (int u = 0; u < kGatherIters; ++u) {
+              if (pw + kProdWarps * u >= kBK / 4) break;
+              const int r = 4 * (pw + kProdWarps * u) + quad;
               const uint32_t dst =
                   tile + (uint32_t)r * 128u + (((uint32_t)g8 ^ (uint32_t)(r & 7)) << 4);
 #pragma unroll
               for (int reg = 0; reg < kRegions; ++reg) {
-                const void* sp = src ? (const void*)(src + reg * 64 + g8 * 8) : (const void*)a.q;
-                cp_async16(dst + reg * kKRegion, sp, src ? 16u : 0u);
+                const void* sp =
+                    src[u] ? (const void*)(src[u] + reg * 64 + g8 * 8) : (const void*)a.q;
+                cp_async16(dst + reg * kKRegion, sp, src[u] ? 16u : 0u);
               }
             }
           }
           // the barrier counts this thread's arrival once its copies land
           if (!dead) cp_async_arrive(&kfull[s]);
         }
-        // the next item's query, once both key tiles are in flight (the
-        // producer would otherwise only wait for a tile to free up)
-        if (b == (nb > 1 ? 1 : 0) && it_next < a.n_items) prepare(it_next, n + 1);
+        if (b == 0) {
+          // head ptid < 64: rotate the dims 448..511 of its row in place (their
+          // raw sum of squares kept for the softmax's 1/rms), then let the MMA
+          // read the Q tile
+          if (ptid < kHG) {
+            wait_or_die(qraw, (uint32_t)n & 1u, 22u);
+            if (!dead) {
+              const int h = ptid;
+              float ss = 0.f;   // raw sum of squares of the RoPE-region dims
+              uint8_t* q7row = sQ + (kRegions - 1) * kQRegion + h * 128;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {   // 16-byte chunk k holds dims 448 + 8k .. + 7
+                uint4* cp = reinterpret_cast<uint4*>(q7row + ((k ^ (h & 7)) << 4));
+                const uint4 v = *cp;
+                uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float x0 = bf16_bits_to_float(w4[e] & 0xffffu);
+                  const float x1 = bf16_bits_to_float(w4[e] >> 16);
+                  ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+                  const int d = 448 + 8 * k + 2 * e;   // even dim of the pair
+                  if (!(a.flags & CSA_F_NO_ROPE) && d >= kC - a.r) {
+                    const int pi = (d - (kC - a.r)) >> 1;
+                    w4[e] = pack_bf16x2(x0 * rcs[pi] - x1 * rcs[32 + pi],
+                                        x0 * rcs[32 + pi] + x1 * rcs[pi]);
+                  }
+                }
+                *cp = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
+              ss7[h] = ss;
+              fence_proxy_async_smem();   // generic stores -> the MMA's reads
+              mbar_arrive(qload);
+            }
+          }
+          if (has_next) load_idx(y.row);   // consumed by the compaction below
+        }
+        if (b == (nbl > 2 ? 2 : nbl - 1) && has_next) cur_ent = compact(y, n + 1);
       }
       gblk += nb;
     }
     cp_async_wait<0>();
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     // ======================= MMA issuer
     if (elect_one()) {
       constexpr uint32_t idS = idesc_bf16_f32(kBK, kHG, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(128, kHG, 1, 1);
-      const uint32_t qb = smem_u32(sQ), kb0 = smem_u32(sm + OFF_K), pb0 = smem_u32(sm + OFF_P);
+      constexpr uint32_t idL = idesc_bf16_f32(kBK, kHG, 0, 1);
+      // descriptors built once; an operand at byte offset o adds o >> 4 to the
+      // start-address field (every offset stays inside shared memory)
+      const uint64_t dK = smem_desc(smem_u32(sm + OFF_K), 16, 1024, 2);         // S^T A
+      const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 1024, 2);                 // S^T B
+      const uint64_t dV = smem_desc(smem_u32(sm + OFF_K), kKRegion, 1024, 2);   // O^T A
+      const uint64_t dP = smem_desc(smem_u32(sm + OFF_P), kKRegion, 1024, 2);   // O^T, L B
+      const uint64_t dOnes = smem_desc(smem_u32(sm + OFF_ONES), 16, 0, 2);      // L A
       int64_t gblk = 0;
       int n = 0;
       bool ok = true;
@@ -473,15 +464,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag || !mbar_wait(&kfull[s], (uint32_t)(j >> 1) & 1u)) return false;
         fence_proxy_async_smem();   // cp.async (generic proxy) writes -> MMA reads
         tc_fence_after();
-        const uint32_t kb = kb0 + s * kKTile;
+        const uint64_t dKs = dK + (uint64_t)((s * kKTile) >> 4);
 #pragma unroll
         for (int reg = 0; reg < kRegions; ++reg) {
 #pragma unroll
-          for (int kq = 0; kq < 4; ++kq) {
-            const uint64_t ad = smem_desc(kb + reg * kKRegion + kq * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(qb + reg * kQRegion + kq * 32, 16, 1024, 2);
-            mma_bf16_ss(tS0 + 64 * s, ad, bd, idS, (reg | kq) != 0 ? 1u : 0u);
-          }
+          for (int kq = 0; kq < 4; ++kq)
+            mma_bf16_ss(tS0 + 64 * s, dKs + (uint64_t)((reg * kKRegion + kq * 32) >> 4),
+                        dQ + (uint64_t)((reg * kQRegion + kq * 32) >> 4), idS,
+                        (reg | kq) != 0 ? 1u : 0u);
         }
         mma_commit(&sfull[s]);
         return true;
@@ -497,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nb == 0) {
           mma_commit(qfree);
           // keep ofull at most one phase ahead of the epilogue
-          if (n > 0 && !mbar_wait(ofree, (uint32_t)(n - 1) & 1u)) { ok = false; break; }
+          if (n > 0 && !mbar_wait(&ofree[3], (uint32_t)(n - 1) & 1u)) { ok = false; break; }
           mma_commit(ofull);
           continue;
         }
@@ -520,18 +510,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++next_s;
           }
           if (*abort_flag || !mbar_wait(&pfull[s], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
-          if (b == 0 && n > 0 && !mbar_wait(ofree, (uint32_t)(n - 1) & 1u)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kb = kb0 + s * kKTile, pb = pb0 + s * kPTile;
-#pragma unroll 1
-          for (int jt = 0; jt < 4; ++jt) {
+          const uint64_t dVs = dV + (uint64_t)((s * kKTile) >> 4);
+          const uint64_t dPs = dP + (uint64_t)((s * kPTile) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = smem_desc(kb + (2 * jt) * kKRegion + kk * 2048, kKRegion, 1024, 2);
-              const uint64_t bd = smem_desc(pb + kk * 2048, kKRegion, 1024, 2);
-              mma_bf16_ss(tO + 64 * jt, ad, bd, idO, (b > 0 || kk > 0) ? 1u : 0u);
+          for (int jt = 0; jt < 4; ++jt) {
+            // the item's first block overwrites O^T: wait for the epilogue to
+            // have read the previous item's columns of this slice
+            if (b == 0 && n > 0) {
+              if (!mbar_wait(&ofree[jt], (uint32_t)(n - 1) & 1u)) { ok = false; break; }
+              tc_fence_after();
             }
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              mma_bf16_ss(tO + 64 * jt, dVs + (uint64_t)((2 * jt * kKRegion + kk * 2048) >> 4),
+                          dPs + (uint64_t)((kk * 2048) >> 4), idO, (b > 0 || kk > 0) ? 1u : 0u);
           }
+          if (!ok) break;
+          // L[., h] += sum over the block's keys of P^T[key, h]: A = 64 rows of
+          // ones (stride 0 repeats one 8-row group), B = the P^T tile; the
+          // epilogue reads L before the first O^T slice
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16_ss(tL, dOnes + (uint64_t)((kk * 32) >> 4), dPs + (uint64_t)((kk * 2048) >> 4),
+                        idL, (b > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bfree[s]);
           if (next_s == b + 1 && next_s < nb) {
             if (!issue_s_item(next_s)) { ok = false; break; }
@@ -550,47 +552,146 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0);
     }
   } else if (warp < 4) {
-    // ======================= softmax + epilogue (same failure handling)
+    // ======================= softmax (warps 0-3)
     const int rw = warp * 32 + lane;
-    const bool active = lane < 16;      // M = 64: rows 16w..16w+15 in lanes 0..15
-    const int kb_row = warp * 16 + lane;
-    const float c2 = scale * kLog2e;
-    bool dead = false;
-    auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
-      if (!dead) {
-        if (!mbar_wait(bar, parity)) {
-          *abort_flag = 1;
-          report(a.status, CSA_DEV_TIMEOUT, code);
-          dead = true;
-        }
-        dead = dead || *abort_flag;
-      }
-      dead = __any_sync(0xffffffffu, dead);
-    };
+    // M = 64 scores read with the 16x64b shape: this lane holds key row kb_row
+    // of the block and the heads of parity `par` (head 2 j + par in slot j)
+    const int par = (lane >> 1) & 1;
+    const int kb_row = warp * 16 + (lane >> 2) + 8 * (lane & 1);
     int64_t gblk = 0;
     int n = 0;
     for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
       const int ip = n & 1;
       const Item x = decode_item(a, it);
       wait_or_die(&iready[ip], (uint32_t)(n >> 1) & 1u, 24u);
-      wait_or_die(&qready[n & 3], (uint32_t)(n >> 2) & 1u, 24u);
-      const float* mb2 = mb2s + (n & 3) * kHG;
       int64_t k_lo = 0, k_hi = 0;
       const int nb = dead ? 0 : item_blocks(a, x, nent[ip], &k_lo, &k_hi);
-      // values the epilogue needs, copied now (the producer may refill the
-      // item-parity buffers before the epilogue runs)
-      const int64_t slot = x.row * a.n_hg + x.hg;
-      float my_mb2 = 0.f;
-      if (rw < kHG) {
-        my_mb2 = mb2[rw];
-        sterm[rw] = a.sink ? ex2(fmaf(a.sink[x.hg * kHG + rw], kLog2e, -my_mb2)) : 0.f;
+      // per-head factors while S^T(0) runs: thread rw sums half of head rw/2's
+      // raw dims 0..447 (Q tile regions 0-3 or 4-6, rotated chunk order for the
+      // banks); the RoPE dims' raw sum comes from the producer's rotation
+      wait_or_die(qload, (uint32_t)n & 1u, 24u);
+      if (!dead) {
+        const int h = rw >> 1, hh = rw & 1;
+        float ss = 0.f;
+        for (int r = 4 * hh; r < (hh ? kRegions - 1 : 4); ++r) {
+          const uint8_t* qr = sQ + r * kQRegion + h * 128;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qr + (((g + h) & 7) << 4));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = bf16_bits_to_float(w4[e] & 0xffffu);
+              const float x1 = bf16_bits_to_float(w4[e] >> 16);
+              ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+            }
+          }
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (hh == 0) {
+          ss += ss7[h];
+          const float inv = (a.flags & CSA_F_NO_NORM) ? 1.f : rsqrtf(ss / (float)kC + a.eps);
+          c2s[(n & 3) * kHG + h] = scale * inv * kLog2e;
+          // bound of the head's logits against unit-RMS keys (bf16 slack 2^-7)
+          mb2s[(n & 3) * kHG + h] =
+              scale * sqrtf(ss) * inv * sqrtf((float)kC) * (1.f + 0.0078125f) * kLog2e;
+        }
       }
+      named_bar(1, 128);   // factors complete; the Q rows are no longer read here
+      if (rw == 0 && !dead) {
+        mbar_arrive(qfree);
+        mbar_arrive(&qready[n & 3]);
+      }
+      float mbr[32], c2r[32];   // this lane's heads 2 j + par
+      {
+        const float* mb2 = mb2s + (n & 3) * kHG;
+        const float* c2h = c2s + (n & 3) * kHG;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          mbr[j] = mb2[2 * j + par];
+          c2r[j] = c2h[2 * j + par];
+        }
+      }
+      named_bar(1, 128);   // every thread has read the item slot
+      if (rw == 0 && !dead) mbar_arrive(&ifree[ip]);
+      float xmax = -INFINITY;
+      for (int b = 0; b < nb; ++b) {
+        const int64_t j = gblk + b;
+        const int s = (int)(j & 1);
+        const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+        wait_or_die(&sfull[s], ph, 25u);
+        uint32_t wds[16];   // bf16 pairs of P for this lane's half row
+        if (!dead) {
+          tc_fence_after();
+          uint32_t sv[32];
+          tmem_ld16x64b_x32(tmem_addr(tS0 + 64 * s, (uint32_t)(warp * 32), 0), sv);
+          tmem_ld_wait();
+          const bool valid = k_lo + (int64_t)b * kBK + kb_row < k_hi;
+          uint32_t mine[16];   // my 32 probabilities as bf16, two per word
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = valid ? fmaf(__uint_as_float(sv[e]), c2r[e], -mbr[e]) : -INFINITY;
+            const float x1 =
+                valid ? fmaf(__uint_as_float(sv[e + 1]), c2r[e + 1], -mbr[e + 1]) : -INFINITY;
+            xmax = fmaxf(xmax, fmaxf(x0, x1));
+            mine[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
+          }
+          // the partner lane (lane ^ 2) holds the other parity of the same key:
+          // even-parity lanes assemble heads 0..31, odd-parity lanes 32..63
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t send = par ? mine[q] : mine[8 + q];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 2);
+            // recv holds the partner's slots 2q, 2q+1 (+16 for the odd side)
+            const uint32_t m = par ? mine[8 + q] : mine[q];
+            // word for slot i = 2q+u: low half = even head, high half = odd head
+            const uint32_t ev0 = par ? (recv & 0xffffu) : (m & 0xffffu);
+            const uint32_t od0 = par ? (m & 0xffffu) : (recv & 0xffffu);
+            const uint32_t ev1 = par ? (recv >> 16) : (m >> 16);
+            const uint32_t od1 = par ? (m >> 16) : (recv >> 16);
+            wds[2 * q] = ev0 | (od0 << 16);
+            wds[2 * q + 1] = ev1 | (od1 << 16);
+          }
+        }
+        wait_or_die(&bfree[s], ph ^ 1u, 25u);   // O^T(j-2) has read this P tile
+        if (!dead) {
+          uint8_t* prow = sm + OFF_P + s * kPTile + kb_row * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(prow + (((par * 4 + q) ^ (kb_row & 7)) << 4)) =
+                make_uint4(wds[4 * q], wds[4 * q + 1], wds[4 * q + 2], wds[4 * q + 3]);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&pfull[s]);
+        }
+      }
+      if (xmax > kRangeLog2) report(a.status, CSA_DEV_RANGE, (unsigned)x.row);
+      gblk += nb;
+    }
+  } else if (warp < 8) {
+    // ======================= epilogue (warps 4-7; warp 4 + ew reads TMEM lanes
+    // 32 ew .. 32 ew + 31): thread = output dim, overlapping the next item
+    const int ew = warp - 4, etid = threadIdx.x - 128;
+    int n = 0;
+    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x, ++n) {
+      const int ip = n & 1;
+      const Item x = decode_item(a, it);
+      wait_or_die(&iready[ip], (uint32_t)(n >> 1) & 1u, 27u);
+      wait_or_die(&qready[n & 3], (uint32_t)(n >> 2) & 1u, 27u);
+      int64_t k_lo = 0, k_hi = 0;
+      const int nb = dead ? 0 : item_blocks(a, x, nent[ip], &k_lo, &k_hi);
+      named_bar(3, 128);   // every epilogue thread has read the entry count
+      if (etid == 0 && !dead) mbar_arrive(&ifree[ip]);
+      // the item's factor slot stays intact until this item's epilogue ends:
+      // the producer refills it four items later, after this role's ifree
+      const float* mb2 = mb2s + (n & 3) * kHG;
+      const int64_t slot = x.row * a.n_hg + x.hg;
       float ecs[4], esn[4];   // RoPE factors of this thread's output pair, per slice
       {
         const float* rcs = ropes + (n & 3) * 64;
 #pragma unroll
         for (int jt = 0; jt < 4; ++jt) {
-          const int cc = 128 * jt + warp * 32 + (lane & ~1);
+          const int cc = 128 * jt + ew * 32 + (lane & ~1);
           ecs[jt] = 1.f;
           esn[jt] = 0.f;
           if (!(a.flags & CSA_F_NO_ROPE) && cc >= kC - a.r) {
@@ -600,101 +701,73 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      named_bar(1, 128);   // every thread has read the item slot
-      if (rw == 0 && !dead) mbar_arrive(&ifree[ip]);
-      float psum[kHG];
-#pragma unroll
-      for (int h = 0; h < kHG; ++h) psum[h] = 0.f;
-      float xmax = -INFINITY;
-      for (int b = 0; b < nb; ++b) {
-        const int64_t j = gblk + b;
-        const int s = (int)(j & 1);
-        const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-        wait_or_die(&sfull[s], ph, 25u);
-        uint32_t pk[32];
-        if (!dead) {
-          tc_fence_after();
-          const uint32_t ta = tmem_addr(tS0 + 64 * s, (uint32_t)(warp * 32), 0);
-          const bool valid = active && (k_lo + (int64_t)b * kBK + kb_row < k_hi);
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {   // 32 heads at a time
-            uint32_t sv[32];
-            tmem_ld32(ta + 32 * half, sv);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int h = 32 * half + e;
-              const float x0 = valid ? fmaf(__uint_as_float(sv[e]), c2, -mb2[h]) : -INFINITY;
-              const float x1 =
-                  valid ? fmaf(__uint_as_float(sv[e + 1]), c2, -mb2[h + 1]) : -INFINITY;
-              xmax = fmaxf(xmax, fmaxf(x0, x1));
-              const float p0 = ex2(x0), p1 = ex2(x1);
-              psum[h] += p0;
-              psum[h + 1] += p1;
-              pk[h >> 1] = pack_bf16x2(p0, p1);
-            }
-          }
-        }
-        wait_or_die(&bfree[s], ph ^ 1u, 25u);   // O^T(j-2) has read this P tile
-        if (!dead) {
-          if (active) {
-            uint8_t* prow = sm + OFF_P + s * kPTile + kb_row * 128;
-#pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8)
-              *reinterpret_cast<uint4*>(prow + ((q8 ^ (kb_row & 7)) << 4)) =
-                  make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(&pfull[s]);
-        }
-      }
-      if (xmax > kRangeLog2) report(a.status, CSA_DEV_RANGE, (unsigned)x.row);
       wait_or_die(ofull, (uint32_t)n & 1u, 26u);
       tc_fence_after();
       const bool have_o = nb > 0 && !dead;
+      if (x.split == 0 && a.split && etid < kHG && !dead) a.mb_part[slot * kHG + etid] = mb2[etid];
 
-      // per-head denominators
-      float two[2];
-      warp_transpose_sum64(psum, lane, two);
-      red[warp * kHG + 2 * lane] = two[0];
-      red[warp * kHG + 2 * lane + 1] = two[1];
-      named_bar(1, 128);
-      if (rw < kHG && !dead) {
-        const float tot = red[rw] + red[kHG + rw] + red[2 * kHG + rw] + red[3 * kHG + rw];
-        if (a.split) {
-          a.d_part[(slot * a.n_splits + x.split) * kHG + rw] = tot;
-          if (x.split == 0) a.mb_part[slot * kHG + rw] = my_mb2;
-        } else {
-          const float den = tot + sterm[rw];
-          sinv[rw] = den > 0.f ? 1.f / den : 0.f;
+      // per-head denominators: the row-sum MMA's result, the same in every row;
+      // warp 4 lanes 0..15 read rows 0..15 and publish heads l, l+16, l+32, l+48
+      if (ew == 0) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t lv[32];
+          if (have_o) {
+            tmem_ld32(tmem_addr(tL + 32 * hf, 0u, 0), lv);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) lv[e] = 0u;
+          }
+          // lane l < 16 takes heads 32 hf + l and 32 hf + l + 16 (static selects:
+          // no dynamically indexed registers)
+          float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            t0 = e == lane ? __uint_as_float(lv[e]) : t0;
+            t1 = e == lane ? __uint_as_float(lv[e + 16]) : t1;
+          }
+          if (!dead && lane < 16) {
+            const int h0 = 32 * hf + lane, h1 = h0 + 16;
+            if (a.split) {
+              a.d_part[(slot * a.n_splits + x.split) * kHG + h0] = t0;
+              a.d_part[(slot * a.n_splits + x.split) * kHG + h1] = t1;
+            } else {
+              // sink: exp(z_h - M_h) joins the denominator only
+              const float s0 = a.sink ? ex2(fmaf(a.sink[x.hg * kHG + h0], kLog2e, -mb2[h0])) : 0.f;
+              const float s1 = a.sink ? ex2(fmaf(a.sink[x.hg * kHG + h1], kLog2e, -mb2[h1])) : 0.f;
+              const float d0 = t0 + s0, d1 = t1 + s1;
+              sinv[h0] = d0 > 0.f ? __frcp_rn(d0) : 0.f;
+              sinv[h1] = d1 > 0.f ? __frcp_rn(d1) : 0.f;
+            }
+          }
         }
       }
-      named_bar(1, 128);
+      named_bar(3, 128);
 
-      // O^T -> output: thread = dim 128 jt + 32 warp + lane
+      // O^T -> output: thread = dim 128 jt + 32 ew + lane
       float iv[kHG];
 #pragma unroll
       for (int h = 0; h < kHG; ++h) iv[h] = a.split ? 1.f : sinv[h];
       const int odd = lane & 1;
 #pragma unroll 1
       for (int jt = 0; jt < 4; ++jt) {
-        const int c = 128 * jt + warp * 32 + lane;
+        const int c = 128 * jt + ew * 32 + lane;
         const int cc = c - odd;
         const float cs = ecs[jt], sn = esn[jt];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {   // heads 32 half .. 32 half + 31
           uint32_t ov[32];
           if (have_o) {
-            tmem_ld32(tmem_addr(tO + 64 * jt + 32 * half, (uint32_t)(warp * 32), 0), ov);
+            tmem_ld32(tmem_addr(tO + 64 * jt + 32 * half, (uint32_t)(ew * 32), 0), ov);
             tmem_ld_wait();
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = 0u;
           }
-          if (jt == 3 && half == 1 && !dead) {   // every TMEM read of this item is done
+          if (half == 1 && !dead) {   // this slice's columns are read: O^T may reuse them
             tc_fence_before();
-            mbar_arrive(ofree);
+            mbar_arrive(&ofree[jt]);
           }
           if (dead) continue;
           if (a.split) {
@@ -719,13 +792,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      gblk += nb;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -805,12 +877,9 @@ bool attn_tc_supported(const AttnParams& p) {
   return al(p.q) && al(p.out) && (p.N == 0 || al(p.entries)) && (p.Tw == 0 || al(p.win));
 }
 
-// q^ scratch: two 64-head slots per persistent CTA (stays in L2)
-inline size_t qhat_bytes() { return (size_t)num_sms() * 2 * kHG * kC * sizeof(bf16); }
-
 size_t attn_tc_scratch(int64_t B, int64_t Tq, int H, int c, int64_t max_keys) {
   if (c != kC || H % kHG != 0) return 0;
-  size_t bytes = qhat_bytes();
+  size_t bytes = 0;
   if (Tq == 1) {
     const int64_t n_hg = H / kHG;
     const int64_t ns = n_splits_for(max_keys);
@@ -853,11 +922,10 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   a.n_rows = rows;
   const size_t need = attn_tc_scratch(p.B, p.Tq, p.H, kC, max_keys);
   if (p.scratch_bytes < need) return cudaErrorInvalidValue;
-  a.qhat = static_cast<bf16*>(p.scratch);
   if (a.split) {
     a.n_splits = n_splits_for(max_keys);
     const int64_t slots = rows * a.n_hg;
-    a.o_part = reinterpret_cast<float*>(static_cast<char*>(p.scratch) + qhat_bytes());
+    a.o_part = static_cast<float*>(p.scratch);
     a.d_part = a.o_part + slots * a.n_splits * kHG * kC;
     a.mb_part = a.d_part + slots * a.n_splits * kHG;
   } else {
@@ -865,8 +933,8 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   }
   a.n_items = rows * a.n_hg * a.n_splits;
   const unsigned grid = (unsigned)(a.n_items < num_sms() ? a.n_items : num_sms());
-  CUtensorMap mq;   // q^ scratch as [grid*2*64 rows][512] bf16, boxes of 64 rows x 64 dims
-  if (!make_map_bf16_3d(&mq, a.qhat, kC, (uint64_t)grid * 2 * kHG, 1, 64, kHG))
+  CUtensorMap mq;   // q as [rows][H][512] bf16, boxes of 64 heads x 64 dims
+  if (!make_map_bf16_3d(&mq, a.q, kC, (uint64_t)p.H, (uint64_t)rows, 64, kHG))
     return cudaErrorInvalidValue;
   const int smem = SMEM_BYTES + 1024;
   cudaError_t e =
