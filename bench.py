@@ -17,7 +17,6 @@ from __future__ import annotations
 import argparse
 import json
 import os
-import subprocess
 import sys
 import time
 
@@ -65,52 +64,78 @@ def compress_bytes(w) -> float:
 
 
 class Clocks:
-    """nvidia-smi sampler over the timed region."""
+    """SM clock and clock-event-reason sampler over the timed region.
+
+    NVML is read from a background thread every 2 ms (the timed region of a
+    default run lasts only tens of milliseconds); the device is matched to
+    torch's by UUID.  Samples are also written to gpurun_out/clocks_rank<i>.csv.
+    Only reads the GPU's state."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
     def __init__(self, index: int):
-        self.proc = None
+        import threading
+        self.samples = []
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.stop_evt = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(index).uuid)
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.masks = [(n, getattr(pynvml, c, 0)) for n, c in self.REASONS]
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.time(), float(sm), int(rs)))
+            except Exception:
+                pass
+            self.stop_evt.wait(0.002)
+
+    def start(self):
+        import threading
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+
+    def stop(self, t0: float, t1: float):
+        """Stops sampling; summarises the samples taken in [t0, t1] (the timed
+        region), or the one nearest to it when the region is shorter than the
+        sampling period."""
+        if self.thread is None:
+            return None
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={index}",
-                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
-                 "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-                 "clocks_event_reasons.hw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
-
-    def stop(self):
-        if self.proc is None:
+            with open(self.path, "w") as f:
+                f.write("time,sm_mhz,max_sm_mhz,event_reasons\n")
+                for t, sm, rs in self.samples:
+                    f.write(f"{t:.4f},{sm:.0f},{self.max_mhz:.0f},0x{rs:x}\n")
+        except OSError:
+            pass
+        if not self.samples:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside:
+            inside = [min(self.samples, key=lambda x: min(abs(x[0] - t0), abs(x[0] - t1)))]
+        reasons = sorted({n for _, _, rs in inside for n, m in self.masks if m and rs & m})
+        return {"sm_mhz": float(np.median([sm for _, sm, _ in inside])),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(inside), "source": "NVML sampled every 2 ms over the timed region"}
 
 
 def dist_setup():
@@ -187,6 +212,9 @@ def run_gpu(args):
     w = wl.WORKLOADS[WORKLOAD]
     step = Step(w, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    clocks = Clocks(local) if rank == 0 or ws > 1 else None
+    if clocks:
+        clocks.start()   # running through warm-up, so samples exist when timing starts
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
@@ -197,17 +225,17 @@ def run_gpu(args):
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    clocks = Clocks(local) if rank == 0 or ws > 1 else None
     launches0 = csa.csa_launch_count()
     barrier(ws)
     torch.cuda.synchronize()
+    t_begin = time.time()
     for i in range(K):
         flush.zero_()                       # L2 flushed between timed steps (not timed)
         step.run(ev=evs[i])
     torch.cuda.synchronize()
     barrier(ws)
     launches = csa.csa_launch_count() - launches0
-    ck = clocks.stop() if clocks else None
+    ck = clocks.stop(t_begin, time.time()) if clocks else None
     per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
                      e[0].elapsed_time(e[3])] for e in evs])     # ms
     step_ms = allmax(float(per[:, 3].mean()), ws)

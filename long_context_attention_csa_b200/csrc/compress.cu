@@ -18,6 +18,7 @@
 // registers the pooling loaded them into.  Token rows are read exactly once.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -292,9 +293,360 @@ cudaError_t launch_t(CompressParams p, int64_t B, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---- bf16, c = 512, per-channel logits: streaming fast paths ---------------
+// Rows of every input tensor that one chunk of tokens needs are contiguous, so
+// persistent CTAs stage them through a ring of shared-memory slots with
+// cp.async (16 bytes per thread-instruction, several chunks in flight) and
+// take chunks round-robin; compute reads the staged rows, never global memory.
+constexpr int kFC = 512;                    // channels
+constexpr int kFRowB = kFC * 2;             // bytes per token row
+constexpr int kFThreads = 256;
+constexpr int kFTab = 2048 + 64;            // RoPE cos/sin table: [rows][32 pairs] float2
+constexpr int kFHead = 8192;                // frequencies (256 doubles), reductions, table
+
+// Window row from a staged token row: RoPE_pos(RMSNorm(row)).  Lane l owns the
+// 16-byte chunks l and l + 32 (channels 8l..8l+7 and 256+8l..256+8l+7), so a
+// warp reads and writes the row as two conflict-free 512-byte sweeps.
+__device__ __forceinline__ void window_row_staged(const uint8_t* srow, bf16* dst, int lane,
+                                                  const Fmt& f, const float2* tab) {
+  float v[16];
+  const uint4 u0 = *reinterpret_cast<const uint4*>(srow + lane * 16);
+  const uint4 u1 = *reinterpret_cast<const uint4*>(srow + 512 + lane * 16);
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = bf16_bits_to_float(w[i] & 0xffffu);
+    v[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+  }
+  if (!(f.flags & CSA_F_NO_NORM)) {
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ss = fmaf(v[e], v[e], ss);
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / (float)kFC + f.eps);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] *= inv;
+  }
+  if (!(f.flags & CSA_F_NO_ROPE)) {
+    const int d0 = kFC - f.r;
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const int ch = (e < 8 ? 8 * lane : 256 + 8 * lane) + (e & 7);
+      if (ch >= d0) {
+        const float2 cs = tab[(ch - d0) >> 1];
+        const float x0 = v[e], x1 = v[e + 1];
+        v[e] = x0 * cs.x - x1 * cs.y;
+        v[e + 1] = x0 * cs.y + x1 * cs.x;
+      }
+    }
+  }
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  reinterpret_cast<uint4*>(dst)[lane] = make_uint4(o[0], o[1], o[2], o[3]);
+  reinterpret_cast<uint4*>(dst)[32 + lane] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// One online-softmax step (base 2, one exp2 per element) of a channel.
+__device__ __forceinline__ void osm_step(float z, float v, float& mx, float& den, float& acc) {
+  const float zl = z * kLog2e;
+  const float d = zl - mx;
+  const float t = exp2f(-fabsf(d));
+  const bool gt = d > 0.f;
+  const float so = gt ? t : 1.f;
+  const float sn = gt ? 1.f : t;
+  den = den * so + sn;
+  acc = acc * so + sn * v;
+  mx = fmaxf(mx, zl);
+}
+
+// cos/sin of the RoPE pairs at `rows` positions (row i at position pos(i)) into
+// tab[i][pair]; every thread of the CTA takes a share.
+template <typename PosFn>
+__device__ __forceinline__ void fill_rope_table(float2* tab, int rows, int r, const double* theta,
+                                                PosFn pos) {
+  const int np = r >> 1;
+  for (int q = threadIdx.x; q < rows * 32; q += kFThreads) {
+    const int i = q >> 5, pr = q & 31;
+    if (pr < np) {
+      float cs, sn;
+      rope_angle(pos(i), theta[pr], &cs, &sn);
+      tab[q] = make_float2(cs, sn);
+    }
+  }
+}
+
+// CSA, m = 4: a chunk is 8 tokens (2 entries); slot = C^a, Z^a rows [t0, t0+8)
+// and C^b, Z^b rows [t0-4, t0+4) (group b covers the previous block).
+constexpr int kCR = 8;
+constexpr int kCStage = 4 * kCR * kFRowB;   // 32 KB
+constexpr int kCStages = 3;                 // 96 KB ring: two CTAs per SM
+
+__global__ void __launch_bounds__(kFThreads, 2)
+    csa_compress_fast_kernel(CompressParams p, uint32_t n_chunks, uint32_t total) {
+  extern __shared__ __align__(1024) uint8_t fsm[];
+  double* theta = reinterpret_cast<double*>(fsm);
+  float* red = reinterpret_cast<float*>(fsm + 2048);   // [8]
+  float2* tab = reinterpret_cast<float2*>(fsm + kFTab); // rows 0-7 window, 8-9 entries
+  uint8_t* ring = fsm + kFHead;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  for (int i = t; i < (p.f.r >> 1); i += kFThreads)
+    theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
+  __syncthreads();   // frequencies complete before the first table fill
+  const uint32_t ring_s = sm100::smem_u32(ring);
+  const bf16* kva = static_cast<const bf16*>(p.kv_a);
+  const bf16* kvb = static_cast<const bf16*>(p.kv_b);
+  const bf16* za = static_cast<const bf16*>(p.z_a);
+  const bf16* zb = static_cast<const bf16*>(p.z_b);
+  auto issue = [&](uint32_t u, int slot) {
+    if (u < total) {
+      const int64_t b = u / n_chunks, t0 = (int64_t)(u % n_chunks) * kCR;
+#pragma unroll
+      for (int i = 0; i < 4 * kCR * 64 / kFThreads; ++i) {
+        const int q = t + kFThreads * i;
+        const int tensor = q >> 9, row = (q >> 6) & (kCR - 1), col = q & 63;
+        const int64_t tok = (tensor < 2 ? t0 : t0 - 4) + row;
+        if (tok < 0 || tok >= p.T) continue;
+        const bf16* src = tensor == 0 ? kva : tensor == 1 ? za : tensor == 2 ? kvb : zb;
+        sm100::cp_async16(ring_s + slot * kCStage + (tensor * kCR + row) * kFRowB + col * 16,
+                          src + (b * p.T + tok) * kFC + col * 8, 16u);
+      }
+    }
+    sm100::cp_async_commit();
+  };
+  const int e = t >> 7, cq = t & 127;   // entry of the chunk, channels 4cq .. 4cq+3
+  int k = 0;
+  for (int i = 0; i < kCStages - 1; ++i) issue(blockIdx.x + i * gridDim.x, i);
+  for (uint32_t u = blockIdx.x; u < total; u += gridDim.x, ++k) {
+    issue(u + (kCStages - 1) * gridDim.x, (k + kCStages - 1) % kCStages);
+    const int64_t b = u / n_chunks, t0 = (int64_t)(u % n_chunks) * kCR;
+    if (!(p.f.flags & CSA_F_NO_ROPE))
+      fill_rope_table(tab, kCR + 2, p.f.r, theta,
+                      [&](int i) { return p.pos0 + (i < kCR ? t0 + i : t0 + 4 * (i - kCR)); });
+    sm100::cp_async_wait<kCStages - 1>();
+    __syncthreads();
+    const uint8_t* buf = ring + (k % kCStages) * kCStage;
+    const int64_t s = t0 / 4 + e;
+    const bool have = s < p.n_entries;   // uniform per warp
+    float val[4] = {0.f, 0.f, 0.f, 0.f};
+    if (have) {
+      float mx[4], den[4], acc[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) { mx[c] = -INFINITY; den[c] = 0.f; acc[c] = 0.f; }
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {   // group a (own block), then group b (previous)
+        if (g == 1 && s == 0) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = 4 * e + j;
+          const uint2 cv = *reinterpret_cast<const uint2*>(buf + ((2 * g) * kCR + row) * kFRowB + cq * 8);
+          const uint2 zv = *reinterpret_cast<const uint2*>(buf + ((2 * g + 1) * kCR + row) * kFRowB + cq * 8);
+          const uint32_t cw[2] = {cv.x, cv.y}, zw[2] = {zv.x, zv.y};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t cb = (c & 1) ? cw[c >> 1] >> 16 : cw[c >> 1] & 0xffffu;
+            const uint32_t zbits = (c & 1) ? zw[c >> 1] >> 16 : zw[c >> 1] & 0xffffu;
+            osm_step(bf16_bits_to_float(zbits), bf16_bits_to_float(cb), mx[c], den[c], acc[c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) val[c] = acc[c] / den[c];
+    }
+    // RMSNorm over the entry's 512 channels (128 threads = warps 4e .. 4e+3)
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ss = fmaf(val[c], val[c], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    // window rows: warp w normalises and rotates token row t0 + w
+    if (p.win != nullptr && t0 + warp < p.T)
+      window_row_staged(buf + warp * kFRowB, static_cast<bf16*>(p.win) + (b * p.T + t0 + warp) * kFC,
+                        lane, p.f, tab + warp * 32);
+    __syncthreads();
+    if (have) {
+      const float tot = red[4 * e] + red[4 * e + 1] + red[4 * e + 2] + red[4 * e + 3];
+      if (!(p.f.flags & CSA_F_NO_NORM)) {
+        const float inv = rsqrtf(tot / (float)kFC + p.f.eps);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) val[c] *= inv;
+      }
+      const int d0 = kFC - p.f.r;
+      if (!(p.f.flags & CSA_F_NO_ROPE)) {
+#pragma unroll
+        for (int c = 0; c < 4; c += 2) {
+          const int ch = 4 * cq + c;
+          if (ch >= d0) {
+            const float2 cs = tab[(kCR + e) * 32 + ((ch - d0) >> 1)];
+            const float x0 = val[c], x1 = val[c + 1];
+            val[c] = x0 * cs.x - x1 * cs.y;
+            val[c + 1] = x0 * cs.y + x1 * cs.x;
+          }
+        }
+      }
+      *reinterpret_cast<uint2*>(static_cast<bf16*>(p.entries) + (b * p.n_entries + s) * kFC + 4 * cq) =
+          make_uint2(pack_bf16x2(val[0], val[1]), pack_bf16x2(val[2], val[3]));
+    }
+    __syncthreads();   // table and reductions are rewritten by the next chunk
+  }
+  sm100::cp_async_wait<0>();
+}
+
+// HCA, m' a multiple of 16: a unit is one block of m' tokens (its entry, when
+// complete, plus its window rows) streamed as m'/16 chunks of 16 C and Z rows;
+// thread t keeps the online-softmax state of channels 2t, 2t+1 across chunks.
+constexpr int kHR = 16;
+constexpr int kHStage = 2 * kHR * kFRowB;   // 32 KB
+constexpr int kHStages = 3;                 // 96 KB ring: two CTAs per SM
+
+__global__ void __launch_bounds__(kFThreads, 2)
+    hca_compress_fast_kernel(CompressParams p, uint32_t n_blocks, uint32_t total) {
+  extern __shared__ __align__(1024) uint8_t fsm[];
+  double* theta = reinterpret_cast<double*>(fsm);
+  float* red = reinterpret_cast<float*>(fsm + 2048);   // [8]
+  float2* tab = reinterpret_cast<float2*>(fsm + kFTab); // rows 0-15 window, 16 entry
+  uint8_t* ring = fsm + kFHead;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  for (int i = t; i < (p.f.r >> 1); i += kFThreads)
+    theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
+  __syncthreads();   // frequencies complete before the first table fill
+  const uint32_t ring_s = sm100::smem_u32(ring);
+  const bf16* kv = static_cast<const bf16*>(p.kv_a);
+  const bf16* z = static_cast<const bf16*>(p.z_a);
+  const int cpu = p.m / kHR;                               // chunks per unit
+  const uint32_t n_my = total > blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const uint32_t n_ck = n_my * cpu;                        // this CTA's chunk sequence
+  auto issue = [&](uint32_t kk, int slot) {
+    if (kk < n_ck) {
+      const uint32_t u = blockIdx.x + (kk / cpu) * gridDim.x;
+      const int64_t b = u / n_blocks;
+      const int64_t t0 = (int64_t)(u % n_blocks) * p.m + (int64_t)(kk % cpu) * kHR;
+#pragma unroll
+      for (int i = 0; i < 2 * kHR * 64 / kFThreads; ++i) {
+        const int q = t + kFThreads * i;
+        const int tensor = q >> 10, row = (q >> 6) & (kHR - 1), col = q & 63;
+        const int64_t tok = t0 + row;
+        if (tok >= p.T) continue;
+        sm100::cp_async16(ring_s + slot * kHStage + (tensor * kHR + row) * kFRowB + col * 16,
+                          (tensor ? z : kv) + (b * p.T + tok) * kFC + col * 8, 16u);
+      }
+    }
+    sm100::cp_async_commit();
+  };
+  for (int i = 0; i < kHStages - 1; ++i) issue(i, i);
+  float mx[2], den[2], acc[2];
+  for (uint32_t kk = 0; kk < n_ck; ++kk) {
+    issue(kk + kHStages - 1, (int)((kk + kHStages - 1) % kHStages));
+    const uint32_t u = blockIdx.x + (kk / cpu) * gridDim.x;
+    const int j = (int)(kk % cpu);
+    const int64_t b = u / n_blocks, s = u % n_blocks, t0 = s * p.m + (int64_t)j * kHR;
+    if (!(p.f.flags & CSA_F_NO_ROPE))
+      fill_rope_table(tab, kHR + 1, p.f.r, theta,
+                      [&](int i) { return p.pos0 + (i < kHR ? t0 + i : s * p.m); });
+    sm100::cp_async_wait<kHStages - 1>();
+    __syncthreads();
+    const uint8_t* buf = ring + (kk % kHStages) * kHStage;
+    if (j == 0) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) { mx[c] = -INFINITY; den[c] = 0.f; acc[c] = 0.f; }
+    }
+    const bool have = s < p.n_entries;   // a complete block (CTA-uniform)
+    if (have) {
+#pragma unroll 4
+      for (int r = 0; r < kHR; ++r) {
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(buf + r * kFRowB + t * 4);
+        const uint32_t zw = *reinterpret_cast<const uint32_t*>(buf + (kHR + r) * kFRowB + t * 4);
+        osm_step(bf16_bits_to_float(zw & 0xffffu), bf16_bits_to_float(cw & 0xffffu), mx[0], den[0], acc[0]);
+        osm_step(bf16_bits_to_float(zw >> 16), bf16_bits_to_float(cw >> 16), mx[1], den[1], acc[1]);
+      }
+    }
+    if (p.win != nullptr) {   // window rows: warp w takes rows 2w, 2w+1 of the chunk
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = 2 * warp + h;
+        if (t0 + r < p.T)
+          window_row_staged(buf + r * kFRowB, static_cast<bf16*>(p.win) + (b * p.T + t0 + r) * kFC,
+                            lane, p.f, tab + r * 32);
+      }
+    }
+    if (j == cpu - 1 && have) {   // CTA-uniform: finish the entry
+      float v0 = acc[0] / den[0], v1 = acc[1] / den[1];
+      float ss = warp_sum(fmaf(v0, v0, v1 * v1));
+      if (lane == 0) red[warp] = ss;
+      __syncthreads();
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFThreads / 32; ++w) tot += red[w];
+      if (!(p.f.flags & CSA_F_NO_NORM)) {
+        const float inv = rsqrtf(tot / (float)kFC + p.f.eps);
+        v0 *= inv;
+        v1 *= inv;
+      }
+      const int ch = 2 * t, d0 = kFC - p.f.r;
+      if (!(p.f.flags & CSA_F_NO_ROPE) && ch >= d0) {
+        const float2 cs = tab[kHR * 32 + ((ch - d0) >> 1)];
+        const float x0 = v0, x1 = v1;
+        v0 = x0 * cs.x - x1 * cs.y;
+        v1 = x0 * cs.y + x1 * cs.x;
+      }
+      reinterpret_cast<uint32_t*>(static_cast<bf16*>(p.entries) + (b * p.n_entries + s) * kFC)[t] =
+          pack_bf16x2(v0, v1);
+    }
+    __syncthreads();   // the slot is refilled next iteration; red reused
+  }
+  sm100::cp_async_wait<0>();
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
+}
+
+// Launches a fast path when the shape has one; *taken tells whether it did.
+cudaError_t launch_compress_fast(int dtype, const CompressParams& p, int64_t B, cudaStream_t stream,
+                                 bool* taken) {
+  *taken = false;
+  if (dtype != CSA_BF16 || p.f.c != kFC || p.z_cols != kFC || p.f.r > kFC) return cudaSuccess;
+  if (p.overlap ? p.m != 4 : (p.m % kHR != 0)) return cudaSuccess;
+  *taken = true;
+  const int64_t grid_max = 2 * (int64_t)sm_count();   // two CTAs per SM
+  if (p.overlap) {
+    const int64_t n_chunks = (p.T + kCR - 1) / kCR;
+    const int64_t total = B * n_chunks;
+    if (total == 0) return cudaSuccess;
+    if (total + grid_max * kCStages >= (1LL << 32)) { *taken = false; return cudaSuccess; }
+    const int smem = kFHead + kCStages * kCStage;
+    cudaError_t e = cudaFuncSetAttribute(csa_compress_fast_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(total < grid_max ? total : grid_max);
+    csa_compress_fast_kernel<<<grid, kFThreads, smem, stream>>>(p, (uint32_t)n_chunks,
+                                                                (uint32_t)total);
+  } else {
+    const int64_t n_blocks = (p.T + p.m - 1) / p.m;   // the last may be partial (window only)
+    const int64_t total = B * n_blocks;
+    if (total == 0 || (p.n_entries == 0 && p.win == nullptr)) return cudaSuccess;
+    if ((total + grid_max) * (p.m / kHR) >= (1LL << 32)) { *taken = false; return cudaSuccess; }
+    const int smem = kFHead + kHStages * kHStage;
+    cudaError_t e = cudaFuncSetAttribute(hca_compress_fast_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(total < grid_max ? total : grid_max);
+    hca_compress_fast_kernel<<<grid, kFThreads, smem, stream>>>(p, (uint32_t)n_blocks,
+                                                                (uint32_t)total);
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_compress(int dtype, CompressParams p, int64_t B, cudaStream_t stream) {
+  bool taken = false;
+  cudaError_t e = launch_compress_fast(dtype, p, B, stream, &taken);
+  if (taken) return e;
   const int ns_max = p.overlap ? 2 * p.m : p.m;
   p.G = ns_max >= 32 ? 4 : 1;   // long slot lists are shared by four warps
   const int cpl = p.f.c / 32;
