@@ -37,6 +37,7 @@ constexpr int kDI = 128;   // indexer dim
 constexpr int kHI = 64;    // indexer heads
 constexpr int kTileBytes = kBM * kDI * 2;     // 32 KB (two 128-byte-swizzled column halves)
 constexpr int kThreads = 192;
+constexpr int kBinCap = 64;   // largest boundary bin the value-binned top-k ranks exactly
 
 template <int TOK> struct Cfg;
 template <> struct Cfg<4> { static constexpr int kStages = 3; static constexpr int kChunk = 2048; };
@@ -52,7 +53,8 @@ struct Smem {
   static constexpr int off_scores = off_a + kStages * kTileBytes;
   static constexpr int off_w = off_scores + TOK * kChunk * 4;
   static constexpr int off_hist = off_w + TOK * kHI * 4;
-  static constexpr int off_bar = off_hist + TOK * 256 * 4;
+  static constexpr int off_cand = off_hist + TOK * 256 * 4;   // [TOK][kBinCap] (score, index)
+  static constexpr int off_bar = off_cand + TOK * kBinCap * 8;
   static constexpr int kBars = 2 * kStages + 6;
   static constexpr int off_misc = off_bar + kBars * 8;
   static constexpr int bytes = off_misc + 64;
@@ -173,6 +175,230 @@ __device__ void warp_topk(const float* sc, int n, int k, int64_t e0, unsigned* h
   }
 }
 
+// Bin of a score in 256 equal-width value bins over [lo, hi]: a monotone map
+// (a larger score never lands in a lower bin), evaluated the same way in
+// every pass.
+__device__ __forceinline__ int value_bin(float s, float lo, float scale) {
+  const int b = (int)((s - lo) * scale);
+  return b > 255 ? 255 : b;
+}
+
+// Inclusive warp prefix sum.
+__device__ __forceinline__ unsigned warp_incl_scan(unsigned v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+// Exact warp top-k, the same selection and output as warp_topk: the scores
+// are binned by value, every score in a bin above the one holding the k-th
+// largest is taken, and that boundary bin's members (at most kBinCap) are
+// ranked exactly by (score desc, index asc).  A heavier boundary bin (many
+// equal or clustered scores) or a degenerate range falls back to the radix
+// select.  Lane l reads scores 4l..4l+3 of each 128-score sweep (16-byte
+// loads; sc is 16-byte aligned), so the ordered compactions use a warp
+// prefix sum of per-lane counts.
+__device__ void warp_topk_binned(const float* sc, int n, int k, int64_t e0, unsigned* hist,
+                                 float* cs, int* cj, int32_t* out_idx, float* out_score) {
+  const int lane = threadIdx.x & 31;
+  if (n <= k) {
+    warp_topk(sc, n, k, e0, hist, out_idx, out_score);
+    return;
+  }
+  const float4* sc4 = reinterpret_cast<const float4*>(sc);
+  const int n4 = (n + 3) >> 2;
+  auto get4 = [&](int i, float* v) {   // scores 4i..4i+3, -inf past n
+    const float4 q = sc4[i];
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (4 * i + e >= n) v[e] = -INFINITY;
+  };
+  // every pass takes four independent 32-float4 sweeps per step (latency
+  // overlap); the ordered compactions scan the four sweeps' counts at once
+  constexpr int U = 4;
+  float lo = INFINITY, hi = -INFINITY;
+  for (int base = 0; base < n4; base += 32 * U) {
+    float v[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      if (i < n4) get4(i, v[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (i < n4 && 4 * i + e < n) {
+          lo = fminf(lo, v[u][e]);
+          hi = fmaxf(hi, v[u][e]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const float scale = 255.99f / (hi - lo);
+  if (!(hi > lo) || !(scale < INFINITY)) {
+    warp_topk(sc, n, k, e0, hist, out_idx, out_score);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
+  __syncwarp();
+  for (int base = 0; base < n4; base += 32 * U) {
+    int bins[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      float v[4];
+      if (i < n4) get4(i, v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        bins[u][e] = (i < n4 && 4 * i + e < n) ? value_bin(v[e], lo, scale) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (bins[u][e] >= 0) atomicAdd(&hist[bins[u][e]], 1u);
+  }
+  __syncwarp();
+  // boundary bin: lane L owns bins 255-8L .. 248-8L (descending)
+  unsigned c[8], sL = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = hist[255 - 8 * lane - i];
+    sL += c[i];
+  }
+  const unsigned incl = warp_incl_scan(sL, lane);
+  const unsigned pre = incl - sL, rem = (unsigned)k;
+  const bool here = pre < rem && rem <= incl;
+  unsigned bstar = 0, above = 0, cnt = 0;
+  if (here) {
+    unsigned run = pre;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (run + c[i] >= rem) {
+        bstar = 255u - 8u * lane - i;
+        above = run;
+        cnt = c[i];
+        break;
+      }
+      run += c[i];
+    }
+  }
+  const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+  bstar = __shfl_sync(0xffffffffu, bstar, src);
+  above = __shfl_sync(0xffffffffu, above, src);
+  cnt = __shfl_sync(0xffffffffu, cnt, src);
+  __syncwarp();
+  if (cnt > (unsigned)kBinCap) {
+    warp_topk(sc, n, k, e0, hist, out_idx, out_score);
+    return;
+  }
+  const unsigned need = rem - above;   // members of the boundary bin to take, >= 1
+  // the boundary bin's members, in ascending index order
+  unsigned run = 0;
+  for (int base = 0; base < n4; base += 32 * U) {
+    float v[U][4];
+    unsigned m[U], inc[U];
+    bool in[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      if (i < n4) get4(i, v[u]);
+      m[u] = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        in[u][e] = i < n4 && 4 * i + e < n && value_bin(v[u][e], lo, scale) == (int)bstar;
+        m[u] += in[u][e] ? 1u : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) inc[u] = warp_incl_scan(m[u], lane);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      unsigned at = run + inc[u] - m[u];
+      const int i = base + 32 * u + lane;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (in[u][e]) {
+          cs[at] = v[u][e];
+          cj[at] = 4 * i + e;
+          ++at;
+        }
+      }
+      run += __shfl_sync(0xffffffffu, inc[u], 31);
+    }
+  }
+  __syncwarp();
+  // the need-th member by (score desc, index asc) is the threshold
+  float ts = 0.f;
+  int tj = -1;
+  for (unsigned i = lane; i < cnt; i += 32) {
+    const float si = cs[i];
+    const int ji = cj[i];
+    unsigned rank = 0;
+    for (unsigned q = 0; q < cnt; ++q) {
+      const float sq = cs[q];
+      rank += (sq > si || (sq == si && cj[q] < ji)) ? 1u : 0u;
+    }
+    if (rank == need - 1) {
+      ts = si;
+      tj = ji;
+    }
+  }
+  const int own = __ffs(__ballot_sync(0xffffffffu, tj >= 0)) - 1;
+  ts = __shfl_sync(0xffffffffu, ts, own);
+  tj = __shfl_sync(0xffffffffu, tj, own);
+  // emit in ascending index order
+  unsigned run_sel = 0;
+  for (int base = 0; base < n4; base += 32 * U) {
+    float v[U][4];
+    unsigned m[U], inc[U];
+    bool take[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      if (i < n4) get4(i, v[u]);
+      m[u] = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * i + e;
+        const bool valid = i < n4 && j < n;
+        const int bv = valid ? value_bin(v[u][e], lo, scale) : -1;
+        take[u][e] = valid && (bv > (int)bstar || (bv == (int)bstar &&
+                                                   (v[u][e] > ts || (v[u][e] == ts && j <= tj))));
+        m[u] += take[u][e] ? 1u : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) inc[u] = warp_incl_scan(m[u], lane);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      unsigned at = run_sel + inc[u] - m[u];
+      const int i = base + 32 * u + lane;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (take[u][e]) {
+          out_idx[at] = (int32_t)(e0 + 4 * i + e);
+          if (out_score) out_score[at] = v[u][e];
+          ++at;
+        }
+      }
+      run_sel += __shfl_sync(0xffffffffu, inc[u], 31);
+    }
+  }
+  for (int q = (int)run_sel + lane; q < k; q += 32) {
+    out_idx[q] = -1;
+    if (out_score) out_score[q] = -INFINITY;
+  }
+}
+
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
@@ -239,6 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
+    if (n_tiles > 0) {   // the q_I block first: its latency overlaps the rest of the setup
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      mbar_arrive_expect_tx(bfull, L::kB);
+      const int32_t qrow = (int32_t)(t0 * kHI);
+      tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
+      tma_load_3d(sB + L::kB / 2, &map_q, bfull, 64, qrow, b);
+    }
   }
   for (int i = threadIdx.x; i < TOK * kHI; i += blockDim.x) {
     int64_t t = t0 + i / kHI;
@@ -256,12 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer
     if (n_tiles > 0 && elect_one()) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      mbar_arrive_expect_tx(bfull, L::kB);
-      const int32_t qrow = (int32_t)(t0 * kHI);
-      tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
-      tma_load_3d(sB + L::kB / 2, &map_q, bfull, 64, qrow, b);
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
@@ -374,7 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         oi = a.cand_idx + c;
         os = a.cand_score + c;
       }
-      warp_topk(scores + t * kChunk, n, a.k, e0, hist + t * 256, oi, os);
+      float* cand = reinterpret_cast<float*>(sm + L::off_cand) + t * 2 * kBinCap;
+      warp_topk_binned(scores + t * kChunk, n, a.k, e0, hist + t * 256, cand,
+                       reinterpret_cast<int*>(cand + kBinCap), oi, os);
     }
   }
 
