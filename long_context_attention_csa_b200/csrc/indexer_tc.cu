@@ -615,6 +615,484 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Prefill form (4-token groups): persistent CTAs walk (chunk, group) units,
+// heaviest causal groups first, and the top-k of one unit runs on its own
+// warps while the next unit's tiles stream through the tensor core.
+//   warp 0        TMA producer: the unit's q_I block, K_I tiles (2-slot ring)
+//   warp 1        TMEM owner, single-thread MMA issuer (8 MMAs per tile)
+//   warps 2-5     epilogue: TMEM -> sum_h w ReLU(.) -> the unit's score buffer
+//   warps 6-13    top-k, two warps per token (block_topk), on the previous
+//                 unit's score buffer (two buffers alternate)
+// ---------------------------------------------------------------------------
+constexpr int kPTok = 4;
+constexpr int kPChunk = 2048;
+constexpr int kPN = kPTok * kHI;                  // MMA N = 256
+constexpr int kPStages = 2;
+constexpr int kPTopkWarps = 2;                    // warps per token in the top-k
+constexpr int kPThreads = 32 * (6 + kPTok * kPTopkWarps);   // 448
+
+struct PSmem {
+  static constexpr int kB = kPTok * kHI * kDI * 2;              // q_I block, 64 KB
+  static constexpr int off_b = 0;
+  static constexpr int off_a = kB;                               // K_I tile ring
+  static constexpr int off_scores = off_a + kPStages * kTileBytes;   // [2][4][2048] fp32
+  static constexpr int off_w = off_scores + 2 * kPTok * kPChunk * 4; // [2][4][64] fp32
+  static constexpr int off_hist = off_w + 2 * kPTok * kHI * 4;       // [4][256]
+  static constexpr int off_red = off_hist + kPTok * 256 * 4;         // [4][8] fp32
+  static constexpr int off_wcnt = off_red + kPTok * 8 * 4;           // [4][8]
+  static constexpr int off_cand = off_wcnt + kPTok * 8 * 4;          // [4][kBinCap] (score, index)
+  static constexpr int off_bar = off_cand + kPTok * kBinCap * 8;
+  static constexpr int kBars = 2 * kPStages + 12;
+  static constexpr int off_misc = off_bar + kBars * 8;
+  static constexpr int bytes = off_misc + 64;
+};
+static_assert(PSmem::bytes + 1024 <= 232448, "shared memory budget");
+
+// Cooperative exact top-k of one token's scores by G warps: the same
+// selection and output as warp_topk (larger score first, ties to the lower
+// index, ascending output padded with (-1, -inf)).  Warp w of the group holds
+// scores [w R, (w+1) R), R = kMaxN / G, in registers (lane l: 16-byte groups
+// l, l+32, ...); value bins as in warp_topk_binned, a histogram in shared
+// memory, the boundary bin's members ranked exactly, and an ordered emit with
+// per-warp offsets.  Returns false (nothing written) when the single-warp
+// radix select must run instead: n <= k, a degenerate range, or more than
+// kBinCap members in the boundary bin.
+template <int G, int kMaxN>
+__device__ bool block_topk(const float* sc, int n, int k, int64_t e0, unsigned* hist, float* red,
+                           unsigned* wcnt, float* cs, int* cj, int bar_id, int32_t* out_idx,
+                           float* out_score) {
+  constexpr int R = kMaxN / G;
+  constexpr int V = R / 128;
+  const int lane = threadIdx.x & 31;
+  const int w = (threadIdx.x >> 5) % G;
+  const int gt = threadIdx.x % (32 * G);
+  auto sync = [&]() { named_bar(bar_id, 32 * G); };
+  float v[V][4];
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+    const float4 q = *reinterpret_cast<const float4*>(sc + j0);
+    v[i][0] = q.x; v[i][1] = q.y; v[i][2] = q.z; v[i][3] = q.w;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j0 + e < n) {
+        lo = fminf(lo, v[i][e]);
+        hi = fmaxf(hi, v[i][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  for (int i = gt; i < 256; i += 32 * G) hist[i] = 0u;
+  if (lane == 0) {
+    red[w] = lo;
+    red[G + w] = hi;
+  }
+  sync();
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    lo = fminf(lo, red[i]);
+    hi = fmaxf(hi, red[G + i]);
+  }
+  const float scale = 255.99f / (hi - lo);
+  if (n <= k || !(hi > lo) || !(scale < INFINITY)) return false;
+  int bin[V][4];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      bin[i][e] = j0 + e < n ? value_bin(v[i][e], lo, scale) : -1;
+      if (bin[i][e] >= 0) atomicAdd(&hist[bin[i][e]], 1u);
+    }
+  }
+  sync();
+  if (w == 0) {   // boundary bin: lane L owns bins 255-8L .. 248-8L (descending)
+    unsigned c[8], sL = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = hist[255 - 8 * lane - i];
+      sL += c[i];
+    }
+    const unsigned incl = warp_incl_scan(sL, lane);
+    const unsigned pre = incl - sL, rem = (unsigned)k;
+    if (pre < rem && rem <= incl) {
+      unsigned run = pre;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (run + c[i] >= rem) {
+          wcnt[G] = 255u - 8u * lane - i;   // boundary bin
+          wcnt[G + 1] = run;                // scores above it
+          wcnt[G + 2] = c[i];               // its members
+          break;
+        }
+        run += c[i];
+      }
+    }
+    if (lane == 0) wcnt[G + 3] = 0u;        // member slots used
+  }
+  sync();
+  const int bstar = (int)wcnt[G];
+  const unsigned need = (unsigned)k - wcnt[G + 1], cnt = wcnt[G + 2];
+  if (cnt > (unsigned)kBinCap) return false;
+  // the boundary bin's members, any order (ranked below)
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (bin[i][e] == bstar) {
+        const unsigned at = atomicAdd(&wcnt[G + 3], 1u);
+        cs[at] = v[i][e];
+        cj[at] = j0 + e;
+      }
+    }
+  }
+  sync();
+  // the need-th member by (score desc, index asc) is the threshold
+  for (unsigned i = gt; i < cnt; i += 32 * G) {
+    const float si = cs[i];
+    const int ji = cj[i];
+    unsigned rank = 0;
+    for (unsigned q = 0; q < cnt; ++q) {
+      const float sq = cs[q];
+      rank += (sq > si || (sq == si && cj[q] < ji)) ? 1u : 0u;
+    }
+    if (rank == need - 1) {   // exactly one member
+      red[2 * G] = si;
+      reinterpret_cast<int*>(red)[2 * G + 1] = ji;
+    }
+  }
+  sync();
+  const float ts = red[2 * G];
+  const int tj = reinterpret_cast<const int*>(red)[2 * G + 1];
+  unsigned mine = 0;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + e;
+      const bool take = bin[i][e] > bstar ||
+                        (bin[i][e] == bstar && (v[i][e] > ts || (v[i][e] == ts && j <= tj)));
+      mine += take ? 1u : 0u;
+      bin[i][e] = take ? 1 : 0;   // from here: the take flag
+    }
+  }
+  unsigned wtot = mine;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(0xffffffffu, wtot, o);
+  if (lane == 0) wcnt[w] = wtot;
+  sync();
+  unsigned run = 0;
+#pragma unroll
+  for (int i = 0; i < G; ++i) run += i < w ? wcnt[i] : 0u;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    unsigned m = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m += (unsigned)bin[i][e];
+    const unsigned inc = warp_incl_scan(m, lane);
+    unsigned at = run + inc - m;
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (bin[i][e]) {
+        out_idx[at] = (int32_t)(e0 + j0 + e);
+        if (out_score) out_score[at] = v[i][e];
+        ++at;
+      }
+    }
+    run += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  sync();   // every read of the group's scratch is done before it is reused
+  return true;
+}
+
+struct PUnit {
+  int64_t b, group, chunk, e0;
+  int n_tiles;
+  int64_t vis[kPTok];
+};
+
+// Unit u: heaviest causal groups first (u = (b * n_groups + gi) * n_chunks + c,
+// group = n_groups - 1 - gi).  Every role derives it the same way.
+__device__ __forceinline__ PUnit punit(const TcIdxArgs& a, int64_t u, int64_t n_groups) {
+  PUnit x;
+  x.chunk = u % a.n_chunks;
+  const int64_t r = u / a.n_chunks;
+  x.group = n_groups - 1 - r % n_groups;
+  x.b = r / n_groups;
+  x.e0 = x.chunk * kPChunk;
+  int64_t vmax = 0;
+#pragma unroll
+  for (int i = 0; i < kPTok; ++i) {
+    const int64_t t = x.group * kPTok + i;
+    x.vis[i] = 0;
+    if (t < a.Tq) {
+      const int64_t row = x.b * a.Tq + t;
+      const int64_t pos = a.q_pos ? a.q_pos[row] : t;
+      x.vis[i] = vis_count(pos, a.m, a.N);
+    }
+    vmax = x.vis[i] > vmax ? x.vis[i] : vmax;
+  }
+  const int64_t e_hi = x.e0 + kPChunk < vmax ? x.e0 + kPChunk : vmax;
+  x.n_tiles = e_hi > x.e0 ? (int)((e_hi - x.e0 + kBM - 1) / kBM) : 0;
+  return x;
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    indexer_persist_kernel(const __grid_constant__ CUtensorMap map_q,
+                           const __grid_constant__ CUtensorMap map_k, TcIdxArgs a,
+                           int64_t n_units, int64_t n_groups) {
+  using L = PSmem;
+  constexpr uint32_t kCols = 2 * kPN;   // two accumulators
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kPN, 0, 0);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sB = sm + L::off_b;
+  uint8_t* sA = sm + L::off_a;
+  float* scores = reinterpret_cast<float*>(sm + L::off_scores);
+  float* sw = reinterpret_cast<float*>(sm + L::off_w);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::off_bar);
+  uint64_t* full = bars;                   // [2] K_I tile landed (TMA)
+  uint64_t* empty = bars + kPStages;       // [2] tile consumed (MMA)
+  uint64_t* tfull = bars + 2 * kPStages;   // [2] accumulator ready (MMA)
+  uint64_t* tempty = tfull + 2;            // [2] accumulator read (128 epilogue threads)
+  uint64_t* qfull = tempty + 2;            // the unit's q_I block landed (TMA)
+  uint64_t* qfree = qfull + 1;             // the unit's last MMA done
+  uint64_t* sready = qfree + 1;            // [2] score buffer complete (128 epilogue threads)
+  uint64_t* sfree = sready + 2;            // [2] score buffer consumed (8 top-k warps)
+  uint64_t* drain = sfree + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::off_misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::off_misc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+      mbar_init(&sready[i], 128);
+      mbar_init(&sfree[i], kPTok * kPTopkWarps);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qfree, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&map_q);
+    tma_prefetch_desc(&map_k);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // a timed-out wait marks the thread dead (warp-uniform); dead threads skip
+  // work and waits but pass every named barrier
+  bool dead = false;
+  auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
+    if (!dead) {
+      if (!mbar_wait(bar, parity)) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, code);
+        dead = true;
+      }
+      dead = dead || *abort_flag;
+    }
+    dead = __any_sync(0xffffffffu, dead);
+  };
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (elect_one()) {
+      int64_t tile = 0;   // tiles issued so far
+      int nq = 0;         // q_I blocks loaded so far
+      for (int64_t u = blockIdx.x; u < n_units && !dead; u += gridDim.x) {
+        const PUnit x = punit(a, u, n_groups);
+        if (x.n_tiles == 0) continue;
+        if (nq > 0 && !mbar_wait(qfree, (uint32_t)(nq - 1) & 1u)) { dead = true; break; }
+        mbar_arrive_expect_tx(qfull, L::kB);
+        const int32_t qrow = (int32_t)(x.group * kPTok * kHI);
+        tma_load_3d(sB, &map_q, qfull, 0, qrow, (int32_t)x.b);
+        tma_load_3d(sB + L::kB / 2, &map_q, qfull, 64, qrow, (int32_t)x.b);
+        ++nq;
+        for (int i = 0; i < x.n_tiles; ++i, ++tile) {
+          const int s = (int)(tile % kPStages);
+          if (*abort_flag || !mbar_wait(&empty[s], (uint32_t)((tile / kPStages) & 1) ^ 1u)) {
+            dead = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          uint8_t* dst = sA + s * kTileBytes;
+          const int32_t erow = (int32_t)(x.e0 + (int64_t)i * kBM);
+          tma_load_3d(dst, &map_k, &full[s], 0, erow, (int32_t)x.b);
+          tma_load_3d(dst + kTileBytes / 2, &map_k, &full[s], 64, erow, (int32_t)x.b);
+        }
+      }
+      if (dead) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 1u);
+      }
+      // drain: the last issued copies land before the CTA may exit
+      for (int64_t t = tile - kPStages > 0 ? tile - kPStages : 0; t < tile; ++t)
+        mbar_wait(&full[t % kPStages], (uint32_t)((t / kPStages) & 1));
+      if (nq > 0) mbar_wait(qfull, (uint32_t)(nq - 1) & 1u);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (elect_one()) {
+      const uint64_t dA = smem_desc(smem_u32(sA), 16, 1024, 2);
+      const uint64_t dB = smem_desc(smem_u32(sB), 16, 1024, 2);
+      int64_t tile = 0;
+      int nq = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const PUnit x = punit(a, u, n_groups);
+        if (x.n_tiles == 0) continue;
+        if (*abort_flag || !mbar_wait(qfull, (uint32_t)nq & 1u)) { ok = false; break; }
+        ++nq;
+        for (int i = 0; i < x.n_tiles; ++i, ++tile) {
+          const int s = (int)(tile % kPStages);
+          const int buf = (int)(tile & 1);
+          if (*abort_flag || !mbar_wait(&full[s], (uint32_t)((tile / kPStages) & 1)) ||
+              !mbar_wait(&tempty[buf], (uint32_t)((tile >> 1) & 1) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(buf * kPN);
+          const uint64_t dAs = dA + (uint64_t)((s * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kDI / 16; ++kk)
+            mma_bf16_ss(d, dAs + (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4),
+                        dB + (uint64_t)(((kk >> 2) * (L::kB / 2) + (kk & 3) * 32) >> 4), kIdesc,
+                        kk > 0 ? 1u : 0u);
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[buf]);
+        }
+        if (!ok) break;
+        mma_commit(qfree);   // the q_I block may be replaced once these MMAs are done
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 3u);
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else if (warp < 6) {
+    // ---------------- epilogue: thread <-> TMEM lane <-> entry
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;   // 0..127
+    int64_t tile = 0;
+    int n = 0;
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++n) {
+      const PUnit x = punit(a, u, n_groups);
+      const int sb = n & 1;
+      float* wb = sw + sb * kPTok * kHI;
+      // the unit's head weights (this buffer's previous unit is finished: the
+      // named barrier below ran after its last tile)
+      for (int i = et; i < kPTok * kHI; i += 128) {
+        const int64_t t = x.group * kPTok + i / kHI;
+        wb[i] = (!dead && t < a.Tq) ? a.w[(x.b * a.Tq + t) * kHI + (i % kHI)] : 0.f;
+      }
+      wait_or_die(&sfree[sb], (uint32_t)((n >> 1) & 1) ^ 1u, 5u);   // top-k of unit n-2 done
+      named_bar(5, 128);   // weights visible
+      float* sc = scores + sb * kPTok * kPChunk;
+      for (int i = 0; i < x.n_tiles; ++i, ++tile) {
+        const int buf = (int)(tile & 1);
+        wait_or_die(&tfull[buf], (uint32_t)((tile >> 1) & 1), 4u);
+        if (dead) continue;
+        tc_fence_after();
+        const uint32_t base = tmem_addr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kPN));
+#pragma unroll
+        for (int t = 0; t < kPTok; ++t) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(base + t * kHI, r0);
+          tmem_ld32(base + t * kHI + 32, r1);
+          tmem_ld_wait();
+          const float* wt = wb + t * kHI;
+          float acc = 0.f;
+#pragma unroll
+          for (int h = 0; h < 32; ++h) acc = fmaf(wt[h], fmaxf(__uint_as_float(r0[h]), 0.f), acc);
+#pragma unroll
+          for (int h = 0; h < 32; ++h)
+            acc = fmaf(wt[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc);
+          sc[t * kPChunk + i * kBM + row] = acc;
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+      }
+      named_bar(5, 128);   // every epilogue thread is past this unit's weights
+      if (!dead) mbar_arrive(&sready[sb]);
+    }
+  } else {
+    // ---------------- top-k: two warps per token
+    const int tw = warp - 6;
+    const int t = tw / kPTopkWarps;
+    const bool lead = tw % kPTopkWarps == 0;
+    unsigned* hist = reinterpret_cast<unsigned*>(sm + L::off_hist) + t * 256;
+    float* red = reinterpret_cast<float*>(sm + L::off_red) + t * 8;
+    unsigned* wcnt = reinterpret_cast<unsigned*>(sm + L::off_wcnt) + t * 8;
+    float* cand = reinterpret_cast<float*>(sm + L::off_cand) + t * 2 * kBinCap;
+    int n = 0;
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++n) {
+      const PUnit x = punit(a, u, n_groups);
+      const int sb = n & 1;
+      wait_or_die(&sready[sb], (uint32_t)(n >> 1) & 1u, 6u);
+      const int64_t tok = x.group * kPTok + t;
+      if (tok < a.Tq) {
+        const int64_t row = x.b * a.Tq + tok;
+        int64_t n64 = x.vis[t] - x.e0;
+        n64 = n64 < 0 ? 0 : (n64 > kPChunk ? kPChunk : n64);
+        int32_t* oi;
+        float* os;
+        if (a.n_chunks == 1) {
+          oi = a.idx_out + row * a.k;
+          os = a.score_out ? a.score_out + row * a.k : nullptr;
+        } else {
+          const int64_t c = (row * a.n_chunks + x.chunk) * a.k;
+          oi = a.cand_idx + c;
+          os = a.cand_score + c;
+        }
+        const float* sc = scores + (sb * kPTok + t) * kPChunk;
+        // both warps of the token run the same barrier sequence even after a
+        // timed-out wait (the selection then reads stale scores; the status
+        // word already holds the error)
+        const bool done = block_topk<kPTopkWarps, kPChunk>(
+            sc, (int)n64, a.k, x.e0, hist, red, wcnt, cand,
+            reinterpret_cast<int*>(cand + kBinCap), 1 + t, oi, os);
+        if (!done) {
+          if (lead) warp_topk(sc, (int)n64, a.k, x.e0, hist, oi, os);
+          named_bar(1 + t, 32 * kPTopkWarps);
+        }
+      }
+      if (lane == 0 && !dead) mbar_arrive(&sfree[sb]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
 // Final selection over the per-chunk candidates of one row: exact block radix
 // select, then an ordered compaction (candidates are in ascending entry order:
 // chunk after chunk, ascending within each chunk).
@@ -746,6 +1224,32 @@ cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t 
   return cudaGetLastError();
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
+}
+
+cudaError_t launch_persist(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
+  CUtensorMap mq, mk;
+  if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, kPTok * kHI))
+    return cudaErrorInvalidValue;
+  if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64, kBM))
+    return cudaErrorInvalidValue;
+  const int smem = PSmem::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_persist_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t n_groups = (p.Tq + kPTok - 1) / kPTok;
+  const int64_t n_units = p.B * n_groups * a.n_chunks;
+  const int64_t sms = sm_count();
+  const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);
+  indexer_persist_kernel<<<grid, kPThreads, smem, stream>>>(mq, mk, a, n_units, n_groups);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool indexer_tc_supported(const IndexerParams& p) {
@@ -784,7 +1288,7 @@ cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
     a.cand_score = static_cast<float*>(p.scratch);
     a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
   }
-  cudaError_t e = tok == 4 ? launch_tok<4>(p, a, stream) : launch_tok<1>(p, a, stream);
+  cudaError_t e = tok == 4 ? launch_persist(p, a, stream) : launch_tok<1>(p, a, stream);
   if (e != cudaSuccess) return e;
   *n_launch = 1;
   if (a.n_chunks > 1) {
