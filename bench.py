@@ -372,9 +372,46 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only_hca(args):
+    """HCA compression or dense HCA attention alone on the hca_prefill_64k
+    workload at --seq-len tokens (for kernel profiles)."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w0 = wl.WORKLOADS["hca_prefill_64k"]
+    w = wl.scaled(w0, T=args.seq_len) if args.seq_len else w0
+    inp = wl.hca_prefill_inputs(w, dev)
+    fmt = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
+    entries = torch.empty((w.B, w.n_hca, w.c), dtype=w.dtype, device=dev)
+    win = torch.empty((w.B, w.T, w.c), dtype=w.dtype, device=dev)
+    csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win)
+    out = torch.empty_like(inp["q"])
+    ws = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_DENSE_ATTN, 1, w.B, w.T, w.H, w.c,
+                                               w.n_hca, 0, w.n_win), dev)
+
+    def once():
+        if args.only == "hca_compress":
+            csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win)
+        else:
+            csa.dense_hca_attn(inp["q"], entries, w.m_prime, win, fmt, w.n_win, sink=inp["sink"],
+                               out=out, ws=ws)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"only": args.only, "seq_len": w.T, "ms": e0.elapsed_time(e1) / args.steps}))
+
+
 def run_only(args):
     """One stage of the step alone on the csa_prefill workload at --seq-len
     tokens (for kernel profiles): warm-up, then --steps timed launches."""
+    if args.only.startswith("hca_"):
+        return run_only_hca(args)
     torch.cuda.set_device(0)
     w = wl.scaled(wl.WORKLOADS[WORKLOAD], T=args.seq_len) if args.seq_len else wl.WORKLOADS[WORKLOAD]
     step = Step(w, torch.device("cuda", 0))
@@ -412,7 +449,8 @@ def run_only(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--only", choices=["compress", "indexer", "attn"], default=None,
+    ap.add_argument("--only", choices=["compress", "indexer", "attn", "hca_compress", "hca_attn"],
+                    default=None,
                     help="time one stage alone (kernel profiling)")
     ap.add_argument("--seq-len", type=int, default=0, help="tokens for --only (default 8192)")
     ap.add_argument("--gpus", type=int, default=1)
