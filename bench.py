@@ -417,11 +417,68 @@ def run_only_hca(args):
     print(json.dumps({"only": args.only, "seq_len": w.T, "ms": e0.elapsed_time(e1) / args.steps}))
 
 
+def run_only_decode(args):
+    """The decode step of --decode-workload (indexer + top-k over the cached
+    indexer keys, then sparse MQA; for the 1M layer pair also the HCA layer's
+    dense MQA), each stage timed alone with CUDA events, with its achieved
+    bandwidth over the bytes it must read (HBM-bound stages)."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = wl.WORKLOADS[args.decode_workload]
+    inp = wl.csa_decode_inputs(w, dev)
+    fmt = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
+    idx = torch.empty((w.B, 1, w.k), dtype=torch.int32, device=dev)
+    ws_i = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_INDEXER, 1, w.B, 1, 0, 0, w.n_csa, w.k,
+                                                 0), dev)
+    ws_a = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_SPARSE_ATTN, 1, w.B, 1, w.H, w.c,
+                                                 w.n_csa, w.k, w.n_win), dev)
+    out = torch.empty_like(inp["q"])
+    stages = {
+        "indexer_scores_topk": (lambda: csa.indexer_scores_topk(
+            inp["q_I"], inp["w"], inp["k_I"], w.m, w.k, q_pos=inp["q_pos"], idx_out=idx, ws=ws_i),
+            w.B * w.n_csa * w.dI * 2),
+        "sparse_mqa_attn": (lambda: csa.sparse_mqa_attn(
+            inp["q"], inp["entries"], idx, inp["win"], fmt, w.n_win, sink=inp["sink"],
+            q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], out=out, ws=ws_a),
+            w.B * (min(w.k, w.n_csa) + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2),
+    }
+    if w.kind == "decode_pair":
+        h = wl.hca_decode_inputs(w, dev)
+        n_h = h["entries"].shape[1]
+        ws_h = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_DENSE_ATTN, 1, w.B, 1, w.H, w.c, n_h,
+                                                     0, w.n_win), dev)
+        out_h = torch.empty_like(h["q"])
+        stages["dense_hca_attn"] = (lambda: csa.dense_hca_attn(
+            h["q"], h["entries"], w.m_prime, h["win"], fmt, w.n_win, sink=h["sink"],
+            q_pos=h["q_pos"], win_pos0=h["win_pos0"], out=out_h, ws=ws_h),
+            w.B * (n_h + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for name, (fn, nbytes) in stages.items():
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(args.steps):
+            flush.zero_()   # L2 flushed before every timed launch
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        ms = tot / args.steps
+        res[name] = {"ms": ms, "bytes": nbytes, "GBps": nbytes / ms / 1e6}
+    print(json.dumps({"only": "decode", "workload": w.name, "stages": res}))
+
+
 def run_only(args):
     """One stage of the step alone on the csa_prefill workload at --seq-len
     tokens (for kernel profiles): warm-up, then --steps timed launches."""
     if args.only.startswith("hca_"):
         return run_only_hca(args)
+    if args.only == "decode":
+        return run_only_decode(args)
     torch.cuda.set_device(0)
     w = wl.scaled(wl.WORKLOADS[WORKLOAD], T=args.seq_len) if args.seq_len else wl.WORKLOADS[WORKLOAD]
     step = Step(w, torch.device("cuda", 0))
@@ -459,10 +516,13 @@ def run_only(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--only", choices=["compress", "indexer", "attn", "hca_compress", "hca_attn"],
+    ap.add_argument("--only", choices=["compress", "indexer", "attn", "hca_compress", "hca_attn",
+                                       "decode"],
                     default=None,
                     help="time one stage alone (kernel profiling)")
     ap.add_argument("--seq-len", type=int, default=0, help="tokens for --only (default 8192)")
+    ap.add_argument("--decode-workload", default="csa_decode_b32_128k",
+                    choices=["csa_decode_b32_128k", "decode_pair_b4_1m"], help="for --only decode")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)

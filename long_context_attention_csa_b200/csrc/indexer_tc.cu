@@ -38,10 +38,11 @@ constexpr int kHI = 64;    // indexer heads
 constexpr int kTileBytes = kBM * kDI * 2;     // 32 KB (two 128-byte-swizzled column halves)
 constexpr int kThreads = 192;
 constexpr int kBinCap = 64;   // largest boundary bin the value-binned top-k ranks exactly
+constexpr int kMergeCap = 2048;   // the same for the chunk-candidate merge
 
 template <int TOK> struct Cfg;
 template <> struct Cfg<4> { static constexpr int kStages = 3; static constexpr int kChunk = 2048; };
-template <> struct Cfg<1> { static constexpr int kStages = 4; static constexpr int kChunk = 4096; };
+template <> struct Cfg<1> { static constexpr int kStages = 2; static constexpr int kChunk = 4096; };
 
 template <int TOK>
 struct Smem {
@@ -54,7 +55,9 @@ struct Smem {
   static constexpr int off_w = off_scores + TOK * kChunk * 4;
   static constexpr int off_hist = off_w + TOK * kHI * 4;
   static constexpr int off_cand = off_hist + TOK * 256 * 4;   // [TOK][kBinCap] (score, index)
-  static constexpr int off_bar = off_cand + TOK * kBinCap * 8;
+  static constexpr int off_red = off_cand + TOK * kBinCap * 8;  // [16] cooperative top-k
+  static constexpr int off_wcnt = off_red + 64;                 // [16]
+  static constexpr int off_bar = off_wcnt + 64;
   static constexpr int kBars = 2 * kStages + 6;
   static constexpr int off_misc = off_bar + kBars * 8;
   static constexpr int bytes = off_misc + 64;
@@ -399,8 +402,173 @@ __device__ void warp_topk_binned(const float* sc, int n, int k, int64_t e0, unsi
   }
 }
 
+// Cooperative exact top-k of one token's scores by G warps: the same
+// selection and output as warp_topk (larger score first, ties to the lower
+// index, ascending output padded with (-1, -inf)).  Warp w of the group holds
+// scores [w R, (w+1) R), R = kMaxN / G, in registers (lane l: 16-byte groups
+// l, l+32, ...); value bins as in warp_topk_binned, a histogram in shared
+// memory, the boundary bin's members ranked exactly, and an ordered emit with
+// per-warp offsets.  Returns false (nothing written) when the single-warp
+// radix select must run instead: n <= k, a degenerate range, or more than
+// kBinCap members in the boundary bin.
+template <int G, int kMaxN>
+__device__ bool block_topk(const float* sc, int n, int k, int64_t e0, unsigned* hist, float* red,
+                           unsigned* wcnt, float* cs, int* cj, int bar_id, int32_t* out_idx,
+                           float* out_score) {
+  constexpr int R = kMaxN / G;
+  constexpr int V = R / 128;
+  const int lane = threadIdx.x & 31;
+  const int w = (threadIdx.x >> 5) % G;
+  const int gt = threadIdx.x % (32 * G);
+  auto sync = [&]() { named_bar(bar_id, 32 * G); };
+  float v[V][4];
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+    const float4 q = *reinterpret_cast<const float4*>(sc + j0);
+    v[i][0] = q.x; v[i][1] = q.y; v[i][2] = q.z; v[i][3] = q.w;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j0 + e < n) {
+        lo = fminf(lo, v[i][e]);
+        hi = fmaxf(hi, v[i][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  for (int i = gt; i < 256; i += 32 * G) hist[i] = 0u;
+  if (lane == 0) {
+    red[w] = lo;
+    red[G + w] = hi;
+  }
+  sync();
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    lo = fminf(lo, red[i]);
+    hi = fmaxf(hi, red[G + i]);
+  }
+  const float scale = 255.99f / (hi - lo);
+  if (n <= k || !(hi > lo) || !(scale < INFINITY)) return false;
+  int bin[V][4];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      bin[i][e] = j0 + e < n ? value_bin(v[i][e], lo, scale) : -1;
+      if (bin[i][e] >= 0) atomicAdd(&hist[bin[i][e]], 1u);
+    }
+  }
+  sync();
+  if (w == 0) {   // boundary bin: lane L owns bins 255-8L .. 248-8L (descending)
+    unsigned c[8], sL = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = hist[255 - 8 * lane - i];
+      sL += c[i];
+    }
+    const unsigned incl = warp_incl_scan(sL, lane);
+    const unsigned pre = incl - sL, rem = (unsigned)k;
+    if (pre < rem && rem <= incl) {
+      unsigned run = pre;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (run + c[i] >= rem) {
+          wcnt[G] = 255u - 8u * lane - i;   // boundary bin
+          wcnt[G + 1] = run;                // scores above it
+          wcnt[G + 2] = c[i];               // its members
+          break;
+        }
+        run += c[i];
+      }
+    }
+    if (lane == 0) wcnt[G + 3] = 0u;        // member slots used
+  }
+  sync();
+  const int bstar = (int)wcnt[G];
+  const unsigned need = (unsigned)k - wcnt[G + 1], cnt = wcnt[G + 2];
+  if (cnt > (unsigned)kBinCap) return false;
+  // the boundary bin's members, any order (ranked below)
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (bin[i][e] == bstar) {
+        const unsigned at = atomicAdd(&wcnt[G + 3], 1u);
+        cs[at] = v[i][e];
+        cj[at] = j0 + e;
+      }
+    }
+  }
+  sync();
+  // the need-th member by (score desc, index asc) is the threshold
+  for (unsigned i = gt; i < cnt; i += 32 * G) {
+    const float si = cs[i];
+    const int ji = cj[i];
+    unsigned rank = 0;
+    for (unsigned q = 0; q < cnt; ++q) {
+      const float sq = cs[q];
+      rank += (sq > si || (sq == si && cj[q] < ji)) ? 1u : 0u;
+    }
+    if (rank == need - 1) {   // exactly one member
+      red[2 * G] = si;
+      reinterpret_cast<int*>(red)[2 * G + 1] = ji;
+    }
+  }
+  sync();
+  const float ts = red[2 * G];
+  const int tj = reinterpret_cast<const int*>(red)[2 * G + 1];
+  unsigned mine = 0;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + e;
+      const bool take = bin[i][e] > bstar ||
+                        (bin[i][e] == bstar && (v[i][e] > ts || (v[i][e] == ts && j <= tj)));
+      mine += take ? 1u : 0u;
+      bin[i][e] = take ? 1 : 0;   // from here: the take flag
+    }
+  }
+  unsigned wtot = mine;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(0xffffffffu, wtot, o);
+  if (lane == 0) wcnt[w] = wtot;
+  sync();
+  unsigned run = 0;
+#pragma unroll
+  for (int i = 0; i < G; ++i) run += i < w ? wcnt[i] : 0u;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    unsigned m = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m += (unsigned)bin[i][e];
+    const unsigned inc = warp_incl_scan(m, lane);
+    unsigned at = run + inc - m;
+    const int j0 = w * R + 4 * (32 * i + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (bin[i][e]) {
+        out_idx[at] = (int32_t)(e0 + j0 + e);
+        if (out_score) out_score[at] = v[i][e];
+        ++at;
+      }
+    }
+    run += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  sync();   // every read of the group's scratch is done before it is reused
+  return true;
+}
+
 template <int TOK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k, TcIdxArgs a) {
   using L = Smem<TOK>;
@@ -584,7 +752,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   // ---------------- top-k: one warp per token
-  if (warp >= 2 && warp < 2 + TOK && !*abort_flag) {
+  if (TOK == 1 && warp >= 2 && !*abort_flag) {
+    // one token: the four epilogue warps select together (named barrier 1)
+    const int64_t tok = t0;
+    if (tok < a.Tq) {
+      const int64_t row = (int64_t)b * a.Tq + tok;
+      int64_t n64 = vis[0] - e0;
+      n64 = n64 < 0 ? 0 : (n64 > kChunk ? kChunk : n64);
+      int32_t* oi;
+      float* os;
+      if (a.n_chunks == 1) {
+        oi = a.idx_out + row * a.k;
+        os = a.score_out ? a.score_out + row * a.k : nullptr;
+      } else {
+        const int64_t c = (row * a.n_chunks + chunk) * a.k;
+        oi = a.cand_idx + c;
+        os = a.cand_score + c;
+      }
+      float* cand = reinterpret_cast<float*>(sm + L::off_cand);
+      const bool done = block_topk<4, kChunk>(
+          scores, (int)n64, a.k, e0, hist, reinterpret_cast<float*>(sm + L::off_red),
+          reinterpret_cast<unsigned*>(sm + L::off_wcnt), cand,
+          reinterpret_cast<int*>(cand + kBinCap), 1, oi, os);
+      if (!done) {
+        if (warp == 2) warp_topk(scores, (int)n64, a.k, e0, hist, oi, os);
+        named_bar(1, 128);
+      }
+    }
+  } else if (TOK > 1 && warp >= 2 && warp < 2 + TOK && !*abort_flag) {
     const int t = warp - 2;
     const int64_t tok = t0 + t;
     if (tok < a.Tq) {
@@ -649,170 +844,6 @@ struct PSmem {
 };
 static_assert(PSmem::bytes + 1024 <= 232448, "shared memory budget");
 
-// Cooperative exact top-k of one token's scores by G warps: the same
-// selection and output as warp_topk (larger score first, ties to the lower
-// index, ascending output padded with (-1, -inf)).  Warp w of the group holds
-// scores [w R, (w+1) R), R = kMaxN / G, in registers (lane l: 16-byte groups
-// l, l+32, ...); value bins as in warp_topk_binned, a histogram in shared
-// memory, the boundary bin's members ranked exactly, and an ordered emit with
-// per-warp offsets.  Returns false (nothing written) when the single-warp
-// radix select must run instead: n <= k, a degenerate range, or more than
-// kBinCap members in the boundary bin.
-template <int G, int kMaxN>
-__device__ bool block_topk(const float* sc, int n, int k, int64_t e0, unsigned* hist, float* red,
-                           unsigned* wcnt, float* cs, int* cj, int bar_id, int32_t* out_idx,
-                           float* out_score) {
-  constexpr int R = kMaxN / G;
-  constexpr int V = R / 128;
-  const int lane = threadIdx.x & 31;
-  const int w = (threadIdx.x >> 5) % G;
-  const int gt = threadIdx.x % (32 * G);
-  auto sync = [&]() { named_bar(bar_id, 32 * G); };
-  float v[V][4];
-  float lo = INFINITY, hi = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int j0 = w * R + 4 * (32 * i + lane);
-    const float4 q = *reinterpret_cast<const float4*>(sc + j0);
-    v[i][0] = q.x; v[i][1] = q.y; v[i][2] = q.z; v[i][3] = q.w;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (j0 + e < n) {
-        lo = fminf(lo, v[i][e]);
-        hi = fmaxf(hi, v[i][e]);
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  for (int i = gt; i < 256; i += 32 * G) hist[i] = 0u;
-  if (lane == 0) {
-    red[w] = lo;
-    red[G + w] = hi;
-  }
-  sync();
-#pragma unroll
-  for (int i = 0; i < G; ++i) {
-    lo = fminf(lo, red[i]);
-    hi = fmaxf(hi, red[G + i]);
-  }
-  const float scale = 255.99f / (hi - lo);
-  if (n <= k || !(hi > lo) || !(scale < INFINITY)) return false;
-  int bin[V][4];
-#pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int j0 = w * R + 4 * (32 * i + lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      bin[i][e] = j0 + e < n ? value_bin(v[i][e], lo, scale) : -1;
-      if (bin[i][e] >= 0) atomicAdd(&hist[bin[i][e]], 1u);
-    }
-  }
-  sync();
-  if (w == 0) {   // boundary bin: lane L owns bins 255-8L .. 248-8L (descending)
-    unsigned c[8], sL = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c[i] = hist[255 - 8 * lane - i];
-      sL += c[i];
-    }
-    const unsigned incl = warp_incl_scan(sL, lane);
-    const unsigned pre = incl - sL, rem = (unsigned)k;
-    if (pre < rem && rem <= incl) {
-      unsigned run = pre;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (run + c[i] >= rem) {
-          wcnt[G] = 255u - 8u * lane - i;   // boundary bin
-          wcnt[G + 1] = run;                // scores above it
-          wcnt[G + 2] = c[i];               // its members
-          break;
-        }
-        run += c[i];
-      }
-    }
-    if (lane == 0) wcnt[G + 3] = 0u;        // member slots used
-  }
-  sync();
-  const int bstar = (int)wcnt[G];
-  const unsigned need = (unsigned)k - wcnt[G + 1], cnt = wcnt[G + 2];
-  if (cnt > (unsigned)kBinCap) return false;
-  // the boundary bin's members, any order (ranked below)
-#pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int j0 = w * R + 4 * (32 * i + lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (bin[i][e] == bstar) {
-        const unsigned at = atomicAdd(&wcnt[G + 3], 1u);
-        cs[at] = v[i][e];
-        cj[at] = j0 + e;
-      }
-    }
-  }
-  sync();
-  // the need-th member by (score desc, index asc) is the threshold
-  for (unsigned i = gt; i < cnt; i += 32 * G) {
-    const float si = cs[i];
-    const int ji = cj[i];
-    unsigned rank = 0;
-    for (unsigned q = 0; q < cnt; ++q) {
-      const float sq = cs[q];
-      rank += (sq > si || (sq == si && cj[q] < ji)) ? 1u : 0u;
-    }
-    if (rank == need - 1) {   // exactly one member
-      red[2 * G] = si;
-      reinterpret_cast<int*>(red)[2 * G + 1] = ji;
-    }
-  }
-  sync();
-  const float ts = red[2 * G];
-  const int tj = reinterpret_cast<const int*>(red)[2 * G + 1];
-  unsigned mine = 0;
-#pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int j0 = w * R + 4 * (32 * i + lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = j0 + e;
-      const bool take = bin[i][e] > bstar ||
-                        (bin[i][e] == bstar && (v[i][e] > ts || (v[i][e] == ts && j <= tj)));
-      mine += take ? 1u : 0u;
-      bin[i][e] = take ? 1 : 0;   // from here: the take flag
-    }
-  }
-  unsigned wtot = mine;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(0xffffffffu, wtot, o);
-  if (lane == 0) wcnt[w] = wtot;
-  sync();
-  unsigned run = 0;
-#pragma unroll
-  for (int i = 0; i < G; ++i) run += i < w ? wcnt[i] : 0u;
-#pragma unroll
-  for (int i = 0; i < V; ++i) {
-    unsigned m = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) m += (unsigned)bin[i][e];
-    const unsigned inc = warp_incl_scan(m, lane);
-    unsigned at = run + inc - m;
-    const int j0 = w * R + 4 * (32 * i + lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (bin[i][e]) {
-        out_idx[at] = (int32_t)(e0 + j0 + e);
-        if (out_score) out_score[at] = v[i][e];
-        ++at;
-      }
-    }
-    run += __shfl_sync(0xffffffffu, inc, 31);
-  }
-  sync();   // every read of the group's scratch is done before it is reused
-  return true;
-}
 
 struct PUnit {
   int64_t b, group, chunk, e0;
@@ -1093,16 +1124,29 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-// Final selection over the per-chunk candidates of one row: exact block radix
-// select, then an ordered compaction (candidates are in ascending entry order:
-// chunk after chunk, ascending within each chunk).
-__global__ void __launch_bounds__(1024)
-    indexer_merge_kernel(TcIdxArgs a) {
-  __shared__ unsigned hist[256];
-  __shared__ unsigned tmp[33];
-  __shared__ unsigned s_prefix, s_mask;
-  __shared__ int s_rem;
-  const int64_t row = blockIdx.x;
+struct MergeShared {
+  unsigned hist[256];
+  unsigned tmp[33];
+  unsigned s_prefix, s_mask;
+  int s_rem;
+  float red[64];          // per-warp min / max
+  unsigned info[4];       // boundary bin, scores above it, its members, slots used
+  float ts;
+  int tj;
+  float cs[kMergeCap];    // the boundary bin's members
+  int cj[kMergeCap];
+};
+
+// Final selection over the per-chunk candidates of one row by exact block
+// radix select, then an ordered compaction (candidates are in ascending entry
+// order: chunk after chunk, ascending within each chunk).  The fallback of the
+// value-binned merge below; the same selection.
+__device__ void merge_radix(const TcIdxArgs& a, int64_t row, MergeShared& sh) {
+  unsigned* hist = sh.hist;
+  unsigned* tmp = sh.tmp;
+  unsigned& s_prefix = sh.s_prefix;
+  unsigned& s_mask = sh.s_mask;
+  int& s_rem = sh.s_rem;
   const int64_t n = (int64_t)a.n_chunks * a.k;
   const float* cs = a.cand_score + row * n;
   const int32_t* ci = a.cand_idx + row * n;
@@ -1197,6 +1241,159 @@ __global__ void __launch_bounds__(1024)
   for (int64_t p = run_sel + threadIdx.x; p < a.k; p += blockDim.x) {
     out[p] = -1;
     if (so) so[p] = -INFINITY;
+  }
+}
+
+
+// Block-wide exclusive prefix sum of one value per thread (1024 threads).
+__device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* tmp, unsigned* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned incl = warp_incl_scan(v, lane);
+  __syncthreads();
+  if (lane == 31) tmp[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    const unsigned wv = lane < (int)(blockDim.x >> 5) ? tmp[lane] : 0u;
+    const unsigned wi = warp_incl_scan(wv, lane);
+    tmp[lane] = wi - wv;
+    if (lane == 31) tmp[32] = wi;
+  }
+  __syncthreads();
+  *total = tmp[32];
+  return tmp[wid] + incl - v;
+}
+
+// Final selection over one row's per-chunk candidates (in ascending entry
+// order), the same selection as merge_radix: value bins over the valid
+// candidates' range, every candidate above the boundary bin taken, the
+// boundary bin's members (at most kMergeCap) ranked exactly by (score desc,
+// entry asc), and an ordered emit.  The unordered passes stride over the
+// candidates (coalesced); the ordered emit gives warp w the contiguous
+// segment [w seg, (w+1) seg), compacted with ballots and offset by a block
+// scan of the warps' counts.
+__global__ void __launch_bounds__(1024)
+    indexer_merge_kernel(TcIdxArgs a) {
+  __shared__ MergeShared sh;
+  const int64_t row = blockIdx.x;
+  const int64_t n = (int64_t)a.n_chunks * a.k;
+  const float* cs = a.cand_score + row * n;
+  const int32_t* ci = a.cand_idx + row * n;
+  int32_t* out = a.idx_out + row * a.k;
+  float* so = a.score_out ? a.score_out + row * a.k : nullptr;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  unsigned cnt = 0;
+  float lo = INFINITY, hi = -INFINITY;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    if (ci[j] < 0) continue;
+    const float v = cs[j];
+    ++cnt;
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sh.red[wid] = lo;
+    sh.red[32 + wid] = hi;
+  }
+  unsigned n_valid;
+  block_excl_scan(cnt, sh.tmp, &n_valid);   // (its barriers also publish red)
+  for (int i = 0; i < nw; ++i) {
+    lo = fminf(lo, sh.red[i]);
+    hi = fmaxf(hi, sh.red[32 + i]);
+  }
+  const float scale = 255.99f / (hi - lo);
+  if (n_valid <= (unsigned)a.k || !(hi > lo) || !(scale < INFINITY)) {
+    merge_radix(a, row, sh);
+    return;
+  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0u;
+  __syncthreads();
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x)
+    if (ci[j] >= 0) atomicAdd(&sh.hist[value_bin(cs[j], lo, scale)], 1u);
+  __syncthreads();
+  if (wid == 0) {   // boundary bin: lane L owns bins 255-8L .. 248-8L (descending)
+    unsigned c[8], sL = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = sh.hist[255 - 8 * lane - i];
+      sL += c[i];
+    }
+    const unsigned incl = warp_incl_scan(sL, lane);
+    const unsigned pre = incl - sL, rem = (unsigned)a.k;
+    if (pre < rem && rem <= incl) {
+      unsigned run = pre;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (run + c[i] >= rem) {
+          sh.info[0] = 255u - 8u * lane - i;
+          sh.info[1] = run;
+          sh.info[2] = c[i];
+          break;
+        }
+        run += c[i];
+      }
+    }
+    if (lane == 0) sh.info[3] = 0u;
+  }
+  __syncthreads();
+  const int bstar = (int)sh.info[0];
+  const unsigned need = (unsigned)a.k - sh.info[1], members = sh.info[2];
+  if (members > (unsigned)kMergeCap) {
+    merge_radix(a, row, sh);
+    return;
+  }
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    if (ci[j] >= 0 && value_bin(cs[j], lo, scale) == bstar) {
+      const unsigned at = atomicAdd(&sh.info[3], 1u);
+      sh.cs[at] = cs[j];
+      sh.cj[at] = ci[j];
+    }
+  }
+  __syncthreads();
+  for (unsigned i = threadIdx.x; i < members; i += blockDim.x) {
+    const float si = sh.cs[i];
+    const int ji = sh.cj[i];
+    unsigned rank = 0;
+    for (unsigned q = 0; q < members; ++q) {
+      const float sq = sh.cs[q];
+      rank += (sq > si || (sq == si && sh.cj[q] < ji)) ? 1u : 0u;
+    }
+    if (rank == need - 1) {   // exactly one member
+      sh.ts = si;
+      sh.tj = ji;
+    }
+  }
+  __syncthreads();
+  const float ts = sh.ts;
+  const int tj = sh.tj;
+  auto take = [&](int64_t j) {
+    if (j >= n || ci[j] < 0) return false;
+    const float v = cs[j];
+    const int bv = value_bin(v, lo, scale);
+    return bv > bstar || (bv == bstar && (v > ts || (v == ts && ci[j] <= tj)));
+  };
+  const int64_t seg = ((n + nw - 1) / nw + 31) / 32 * 32;
+  const int64_t s0 = (int64_t)wid * seg, s1 = s0 + seg;
+  unsigned mine = 0;
+  for (int64_t base = s0; base < s1; base += 32) mine += __popc(__ballot_sync(0xffffffffu, take(base + lane)));
+  unsigned total;
+  unsigned run = block_excl_scan(lane == 0 ? mine : 0u, sh.tmp, &total);
+  run = __shfl_sync(0xffffffffu, run, 0);
+  for (int64_t base = s0; base < s1; base += 32) {
+    const int64_t j = base + lane;
+    const bool t = take(j);
+    const unsigned bal = __ballot_sync(0xffffffffu, t);
+    if (t) {
+      const unsigned at = run + __popc(bal & lt);
+      out[at] = ci[j];
+      if (so) so[at] = cs[j];
+    }
+    run += __popc(bal);
   }
 }
 
