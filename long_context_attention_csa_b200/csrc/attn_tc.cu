@@ -48,7 +48,7 @@
 //   warps 4-7  epilogue (thread = output dim), which runs alongside the next
 //              item's softmax; it frees O^T in four 64-column slices, so the
 //              next item's first O^T waits only for the slice it overwrites.
-// Decode rows (one query per sequence) split the key list into fixed 256-key
+// Decode rows (one query per sequence) split the key list into fixed 320-key
 // pieces whose fp32 partials a combine kernel adds in a fixed order, so a
 // row's result does not depend on the batch it runs in.
 #include "common.cuh"
@@ -70,7 +70,7 @@ constexpr int kKRegion = kBK * 128;          // 8 KB per key-tile chunk
 constexpr int kKTile = kRegions * kKRegion;  // 64 KB
 constexpr int kQRegion = kHG * 128;          // 8 KB per query chunk
 constexpr int kPTile = kBK * 128;            // 8 KB: P^T [64 keys][64 heads] bf16
-constexpr int kSplitKeys = 256;              // decode split size (fixed)
+constexpr int kSplitKeys = 320;              // decode split size (fixed: five 64-key blocks)
 constexpr int kMaxK = 1024;                  // largest top-k the index list holds
 constexpr int kProdWarp0 = 8;                // warps 8-10 produce, warp 11 issues MMAs
 constexpr int kProdWarps = 3;
@@ -805,50 +805,65 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Sums the fixed-order split partials of one (row, head group), divides by
 // the denominator (sink included) and rotates the output back by -pos.
+constexpr int kCombHeads = 8;   // heads per combine CTA
+
 __global__ void __launch_bounds__(256) attn_combine_kernel(TcAttnArgs a) {
-  __shared__ float inv[kHG];
+  __shared__ float inv[kCombHeads];
   __shared__ float cs_t[32], sn_t[32];
   const int64_t row = blockIdx.x;
   const int hg = blockIdx.y;
+  const int h0 = blockIdx.z * kCombHeads;   // this CTA's heads within the group
   const int64_t slot = row * a.n_hg + hg;
   const int64_t t = row % a.Tq;
   const int64_t pos = a.q_pos ? a.q_pos[row] : t;
-  if (threadIdx.x < kHG) {
+  if (threadIdx.x < kCombHeads) {
+    const int h = h0 + threadIdx.x;
     float tot = 0.f;
-    for (int s = 0; s < a.n_splits; ++s)
-      tot += a.d_part[(slot * a.n_splits + s) * kHG + threadIdx.x];
+    for (int s = 0; s < a.n_splits; ++s)   // fixed order: bits independent of the batch
+      tot += a.d_part[(slot * a.n_splits + s) * kHG + h];
     if (a.sink) {
-      const float z = a.sink[hg * kHG + threadIdx.x];
-      tot += ex2(fmaf(z, kLog2e, -a.mb_part[slot * kHG + threadIdx.x]));
+      const float z = a.sink[hg * kHG + h];
+      tot += ex2(fmaf(z, kLog2e, -a.mb_part[slot * kHG + h]));
     }
     inv[threadIdx.x] = tot > 0.f ? 1.f / tot : 0.f;
-  } else if (threadIdx.x >= 64 && threadIdx.x < 64 + (a.r >> 1)) {
+  } else if (threadIdx.x >= 32 && threadIdx.x < 32 + (a.r >> 1)) {
     float cs, sn;
-    rope_cos_sin(-pos, threadIdx.x - 64, a.r, a.base, &cs, &sn);
-    cs_t[threadIdx.x - 64] = cs;
-    sn_t[threadIdx.x - 64] = sn;
+    rope_cos_sin(-pos, threadIdx.x - 32, a.r, a.base, &cs, &sn);
+    cs_t[threadIdx.x - 32] = cs;
+    sn_t[threadIdx.x - 32] = sn;
   }
   __syncthreads();
-  for (int pi = threadIdx.x; pi < kHG * kC / 2; pi += blockDim.x) {
-    const int h = pi / (kC / 2);
-    const int c = (pi % (kC / 2)) * 2;
-    float o0 = 0.f, o1 = 0.f;
+  // thread: 4 consecutive dims of one head, 4 times (16-byte loads)
+  constexpr int kQuads = kCombHeads * kC / 4;   // 1024
+#pragma unroll
+  for (int r = 0; r < kQuads / 256; ++r) {
+    const int q = threadIdx.x + 256 * r;
+    const int hl = q / (kC / 4), c = (q % (kC / 4)) * 4;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
     for (int s = 0; s < a.n_splits; ++s) {
-      const float* op = a.o_part + ((slot * a.n_splits + s) * kHG + h) * kC + c;
-      const float2 v = *reinterpret_cast<const float2*>(op);
-      o0 += v.x;
-      o1 += v.y;
+      const float4 v = *reinterpret_cast<const float4*>(
+          a.o_part + ((slot * a.n_splits + s) * kHG + h0 + hl) * kC + c);
+      o[0] += v.x;
+      o[1] += v.y;
+      o[2] += v.z;
+      o[3] += v.w;
     }
-    o0 *= inv[h];
-    o1 *= inv[h];
-    if (!(a.flags & CSA_F_NO_ROPE) && c >= kC - a.r) {
-      const int i = (c - (kC - a.r)) >> 1;
-      const float y0 = o0 * cs_t[i] - o1 * sn_t[i], y1 = o0 * sn_t[i] + o1 * cs_t[i];
-      o0 = y0;
-      o1 = y1;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] *= inv[hl];
+    if (!(a.flags & CSA_F_NO_ROPE)) {
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        if (c + e >= kC - a.r) {
+          const int i = (c + e - (kC - a.r)) >> 1;
+          const float y0 = o[e] * cs_t[i] - o[e + 1] * sn_t[i];
+          const float y1 = o[e] * sn_t[i] + o[e + 1] * cs_t[i];
+          o[e] = y0;
+          o[e + 1] = y1;
+        }
+      }
     }
-    *reinterpret_cast<uint32_t*>(a.out + (row * a.H + (int64_t)hg * kHG + h) * kC + c) =
-        pack_bf16x2(o0, o1);
+    *reinterpret_cast<uint2*>(a.out + (row * a.H + (int64_t)hg * kHG + h0 + hl) * kC + c) =
+        make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
   }
 }
 
@@ -944,7 +959,8 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   if (a.split) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<dim3((unsigned)rows, (unsigned)a.n_hg), 256, 0, stream>>>(a);
+    attn_combine_kernel<<<dim3((unsigned)rows, (unsigned)a.n_hg, kHG / kCombHeads), 256, 0,
+                          stream>>>(a);
     *n_launch = 2;
   } else {
     *n_launch = 1;
