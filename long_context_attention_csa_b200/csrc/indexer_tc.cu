@@ -44,6 +44,29 @@ template <int TOK> struct Cfg;
 template <> struct Cfg<4> { static constexpr int kStages = 3; static constexpr int kChunk = 2048; };
 template <> struct Cfg<1> { static constexpr int kStages = 2; static constexpr int kChunk = 4096; };
 
+// sum_h w[h] ReLU(s[h]) over 64 heads (s: two 32-column TMEM loads) with
+// packed fp32 FMAs (two heads per instruction; even and odd heads accumulate
+// separately and are added at the end).
+__device__ __forceinline__ float relu_weighted_sum64(const float* wt, const uint32_t* r0,
+                                                     const uint32_t* r1) {
+  unsigned long long acc = 0ull;
+  const float2* w2 = reinterpret_cast<const float2*>(wt);
+#pragma unroll
+  for (int h = 0; h < 64; h += 2) {
+    const uint32_t* r = h < 32 ? r0 : r1;
+    const float s0 = fmaxf(__uint_as_float(r[h & 31]), 0.f);
+    const float s1 = fmaxf(__uint_as_float(r[(h & 31) + 1]), 0.f);
+    const float2 wv = w2[h >> 1];
+    unsigned long long sp, wp;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(sp) : "f"(s0), "f"(s1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(wp) : "f"(wv.x), "f"(wv.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(wp), "l"(sp));
+  }
+  float a0, a1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+  return a0 + a1;
+}
+
 template <int TOK>
 struct Smem {
   static constexpr int kB = TOK * kHI * kDI * 2;           // q_I block
@@ -735,14 +758,7 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
         tmem_ld32(base + t * kHI, r0);
         tmem_ld32(base + t * kHI + 32, r1);
         tmem_ld_wait();
-        const float* wt = sw + t * kHI;
-        float acc = 0.f;
-#pragma unroll
-        for (int h = 0; h < 32; ++h) acc = fmaf(wt[h], fmaxf(__uint_as_float(r0[h]), 0.f), acc);
-#pragma unroll
-        for (int h = 0; h < 32; ++h)
-          acc = fmaf(wt[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc);
-        scores[t * kChunk + i * kBM + row] = acc;
+        scores[t * kChunk + i * kBM + row] = relu_weighted_sum64(sw + t * kHI, r0, r1);
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
@@ -1056,14 +1072,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tmem_ld32(base + t * kHI, r0);
           tmem_ld32(base + t * kHI + 32, r1);
           tmem_ld_wait();
-          const float* wt = wb + t * kHI;
-          float acc = 0.f;
-#pragma unroll
-          for (int h = 0; h < 32; ++h) acc = fmaf(wt[h], fmaxf(__uint_as_float(r0[h]), 0.f), acc);
-#pragma unroll
-          for (int h = 0; h < 32; ++h)
-            acc = fmaf(wt[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc);
-          sc[t * kPChunk + i * kBM + row] = acc;
+          sc[t * kPChunk + i * kBM + row] = relu_weighted_sum64(wb + t * kHI, r0, r1);
         }
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
