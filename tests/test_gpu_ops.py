@@ -136,6 +136,49 @@ def test_indexer_csa_prefill_8k_sampled():
     assert d <= 2
 
 
+def test_indexer_prefill_multichunk_sampled():
+    """More than 2048 entries: the prefill kernel emits per-chunk candidates
+    (three chunks here) that the merge kernel reduces; two sequences."""
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], B=2, T=20000)
+    d = _indexer_case(w, rows=np.unique(np.concatenate([sample_rows(w.T, 24),
+                                                        np.arange(w.T - 8, w.T)])))
+    assert d <= 2
+
+
+def test_indexer_multichunk_integer_bit_exact():
+    """Integer inputs (exact sums, many ties) across three 2048-entry chunks:
+    candidates and the merge must reproduce the oracle's sets and scores."""
+    B, T, HI, dI, m, k = 1, 9000, 64, 128, 4, 256
+    N = T // m
+    qI = wl.randint_like_float((B, T, HI, dI), 31, -2, 3, DEV, torch.bfloat16)
+    kI = wl.randint_like_float((B, N, dI), 32, -2, 3, DEV, torch.bfloat16)
+    w = wl.randint_like_float((B, T, HI), 33, -2, 3, DEV, torch.float32)
+    idx, sc = csa.indexer_scores_topk(qI, w, kI, m, k, want_scores=True)
+    torch.cuda.synchronize()
+    rows = sample_rows(T, 12)
+    ref_sc = oracle.indexer_scores(f64(qI[0][rows]), f64(w[0][rows]), f64(kI[0]), m, q_pos=rows)
+    ref_idx = oracle.topk(ref_sc, k, m, q_pos=rows)
+    assert np.array_equal(idx[0][rows].cpu().numpy(), ref_idx)
+
+
+def test_indexer_prefill_positions():
+    """Prefill with explicit positions (a chunk continuing a longer context):
+    visibility follows q_pos, not the row index."""
+    B, T, HI, dI, m, k = 1, 600, 64, 128, 4, 128
+    pos = torch.arange(T, dtype=torch.int64).unsqueeze(0) + 3000
+    N = (3000 + T) // m
+    qI = wl.randn((B, T, HI, dI), 21, DEV, dtype=torch.bfloat16)
+    kI = wl.randn((B, N, dI), 22, DEV, dtype=torch.bfloat16)
+    w = wl.randn((B, T, HI), 23, DEV) / 8
+    idx, sc = csa.indexer_scores_topk(qI, w, kI, m, k, q_pos=pos.to(DEV), want_scores=True)
+    torch.cuda.synchronize()
+    rows = sample_rows(T, 16)
+    p = pos[0].numpy()[rows]
+    ref_sc = oracle.indexer_scores(f64(qI[0][rows]), f64(w[0][rows]), f64(kI[0]), m, q_pos=p)
+    ref_idx = oracle.topk(ref_sc, k, m, q_pos=p)
+    assert check_topk_rows(idx[0][rows].cpu().numpy(), ref_idx, ref_sc, what="q_pos") <= 1
+
+
 @pytest.mark.parametrize("wname", ["csa_decode_b32_128k", "decode_pair_b4_1m"])
 def test_indexer_decode(wname):
     w = wl.WORKLOADS[wname]
