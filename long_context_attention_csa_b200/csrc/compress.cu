@@ -347,11 +347,13 @@ __device__ __forceinline__ void window_row_staged(const uint8_t* srow, bf16* dst
   reinterpret_cast<uint4*>(dst)[32 + lane] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// One online-softmax step (base 2, one exp2 per element) of a channel.
+// One online-softmax step (base 2, one exp2 per element) of a channel.  The
+// exponent is never positive, so the hardware ex2 (relative error ~2^-22,
+// results below 2^-126 flushed to 0) replaces the libm call.
 __device__ __forceinline__ void osm_step(float z, float v, float& mx, float& den, float& acc) {
   const float zl = z * kLog2e;
   const float d = zl - mx;
-  const float t = exp2f(-fabsf(d));
+  const float t = sm100::ex2(-fabsf(d));
   const bool gt = d > 0.f;
   const float so = gt ? t : 1.f;
   const float sn = gt ? 1.f : t;
