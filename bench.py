@@ -279,6 +279,12 @@ def run_gpu(args):
     if st:
         raise RuntimeError(f"device status after timing: {st}/{d}")
 
+    del step, dev_in, host
+    torch.cuda.empty_cache()
+    decode = {} if args.no_decode else {
+        n: measure_decode(n, dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
+        for n in DECODE_WORKLOADS}
+
     hbm, bf16, src = peaks()
     tokens = w.B * w.T
     fl_attn = attn_useful_flops(w)
@@ -327,6 +333,8 @@ def run_gpu(args):
             "gpu_launches": int(launches),
             "clocks": ck,
         }
+        if decode:
+            line["decode"] = decode
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
         print(json.dumps(line), flush=True)
@@ -417,59 +425,183 @@ def run_only_hca(args):
     print(json.dumps({"only": args.only, "seq_len": w.T, "ms": e0.elapsed_time(e1) / args.steps}))
 
 
+DECODE_WORKLOADS = ("csa_decode_b32_128k", "decode_pair_b4_1m")
+
+
+def decode_bytes(w) -> float:
+    """Bytes one decode step must move: the indexer keys of every visible entry
+    (all of them: the query sits at the end of its context), q_I and w, the
+    selected entries and the window rows gathered once, the queries read and
+    the outputs written; for the layer pair also the HCA layer's entries,
+    window, queries and outputs."""
+    e = 2
+    nb = w.B * w.n_csa * w.dI * e + w.B * w.HI * (w.dI * e + 4)
+    nb += w.B * (min(w.k, w.n_csa) + w.n_win) * w.c * e + 2 * w.B * w.H * w.c * e
+    if w.kind == "decode_pair":
+        nb += w.B * (w.n_hca + w.n_win) * w.c * e + 2 * w.B * w.H * w.c * e
+    return float(nb)
+
+
+class DecodeStep:
+    """One decode step of a decode workload through the public API, into
+    preallocated outputs: indexer + top-k over the cached indexer keys, then
+    sparse MQA over the selected entries and the window; for the 1M layer
+    pair also the HCA layer's dense MQA."""
+
+    def __init__(self, w, dev):
+        self.w = w
+        inp = wl.csa_decode_inputs(w, dev)
+        fmt = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
+        self.idx = torch.empty((w.B, 1, w.k), dtype=torch.int32, device=dev)
+        self.ws = [csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_INDEXER, 1, w.B, 1, 0, 0,
+                                                         w.n_csa, w.k, 0), dev),
+                   csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_SPARSE_ATTN, 1, w.B, 1, w.H,
+                                                         w.c, w.n_csa, w.k, w.n_win), dev)]
+        self.out = torch.empty_like(inp["q"])
+        ws_i, ws_a = self.ws
+        self.stages = [
+            ("indexer_scores_topk", lambda: csa.indexer_scores_topk(
+                inp["q_I"], inp["w"], inp["k_I"], w.m, w.k, q_pos=inp["q_pos"], idx_out=self.idx,
+                ws=ws_i), w.B * w.n_csa * w.dI * 2),
+            ("sparse_mqa_attn", lambda: csa.sparse_mqa_attn(
+                inp["q"], inp["entries"], self.idx, inp["win"], fmt, w.n_win, sink=inp["sink"],
+                q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], out=self.out, ws=ws_a),
+                w.B * (min(w.k, w.n_csa) + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2),
+        ]
+        if w.kind == "decode_pair":
+            h = wl.hca_decode_inputs(w, dev)
+            n_h = h["entries"].shape[1]
+            ws_h = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_DENSE_ATTN, 1, w.B, 1, w.H,
+                                                         w.c, n_h, 0, w.n_win), dev)
+            self.ws.append(ws_h)
+            self.out_h = torch.empty_like(h["q"])
+            self.stages.append(("dense_hca_attn", lambda: csa.dense_hca_attn(
+                h["q"], h["entries"], w.m_prime, h["win"], fmt, w.n_win, sink=h["sink"],
+                q_pos=h["q_pos"], win_pos0=h["win_pos0"], out=self.out_h, ws=ws_h),
+                w.B * (n_h + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2))
+        self.inp = inp
+
+    def run(self):
+        for _, fn, _ in self.stages:
+            fn()
+
+    def check(self):
+        for ws in self.ws:
+            st, d = csa.csa_check_status(ws)
+            if st:
+                raise RuntimeError(f"{self.w.name}: device status {st}/{d}")
+
+
+def graph_ms(fn, steps: int, flush) -> float:
+    """Mean device time of `fn` captured once in a CUDA graph and replayed
+    `steps` times, with the L2 flushed before each replay (outside the events),
+    as a decode server replays its step."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    del g
+    return ms
+
+
+def decode_cpu_baseline(w, queries: int):
+    """The float64 oracle on `queries` decode queries of the workload (indexer
+    scores over the whole cache, top-k, sparse MQA; for the layer pair also the
+    HCA layer's dense MQA), in queries per second."""
+    import oracle
+
+    inp = wl.csa_decode_inputs(w, "cpu")
+    fmt = oracle.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
+    h = wl.hca_decode_inputs(w, "cpu") if w.kind == "decode_pair" else None
+    sink = None if inp["sink"] is None else inp["sink"].double().numpy()
+    t0 = time.perf_counter()
+    for b in range(queries):
+        pos = inp["q_pos"][b].numpy()
+        sc = oracle.indexer_scores(inp["q_I"][b].double().numpy(), inp["w"][b].double().numpy(),
+                                   inp["k_I"][b].double().numpy(), w.m, q_pos=pos)
+        idx = oracle.topk(sc, w.k, w.m, q_pos=pos)
+        oracle.attention(inp["q"][b].double().numpy(), inp["entries"][b].double().numpy(),
+                         inp["win"][b].double().numpy(), fmt, w.n_win, idx=idx, sink=sink,
+                         q_pos=pos, win_pos0=int(inp["win_pos0"][b]))
+        if h is not None:
+            oracle.attention(h["q"][b].double().numpy(), h["entries"][b].double().numpy(),
+                             h["win"][b].double().numpy(), fmt, w.n_win, m_dense=w.m_prime,
+                             sink=h["sink"].double().numpy(), q_pos=pos,
+                             win_pos0=int(h["win_pos0"][b]))
+    dt = time.perf_counter() - t0
+    return {"value": queries / dt, "unit": "queries/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{queries} of {w.B} queries (the whole decode step for each), float64, "
+                      f"{dt:.1f} s"}
+
+
+def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cpu: bool):
+    """Decode queries/s of one decode workload: the whole step as one CUDA-graph
+    replay (max over ranks), each stage also alone, and the step's HBM
+    roofline over the bytes it must move."""
+    w = wl.WORKLOADS[name]
+    d = DecodeStep(w, dev)
+    for _ in range(warmup):
+        d.run()
+    torch.cuda.synchronize()
+    d.check()
+    step_ms = allmax(graph_ms(d.run, steps, flush), ws_n)
+    stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.stages}
+    d.check()
+    hbm, _, src = peaks()
+    nb = decode_bytes(w)
+    achieved = nb / (step_ms * 1e-3) / 1e9
+    res = {
+        "value": w.B * ws_n / (step_ms * 1e-3), "unit": "queries/s", "ms_per_step": step_ms,
+        "config": {"workload": w.name, "batch": w.B, "context": w.T, "heads": w.H,
+                   "entries": w.n_csa, "top_k": w.k, "n_win": w.n_win, "sink": True,
+                   **({"hca_entries": w.n_hca} if w.kind == "decode_pair" else {}),
+                   "l2": "flushed before every replay (outside the events)",
+                   "timing": "whole step captured once in a CUDA graph, replayed"},
+        "stages_ms": stages,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "algorithmic_bytes_per_step": nb,
+                     "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json)"
+                     if src == "measured" else "fallback 6.65 TB/s"},
+    }
+    if cpu:
+        res["cpu_baseline"] = decode_cpu_baseline(w, 1)
+    del d
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_only_decode(args):
-    """The decode step of --decode-workload (indexer + top-k over the cached
-    indexer keys, then sparse MQA; for the 1M layer pair also the HCA layer's
-    dense MQA), each stage timed alone with CUDA events, with its achieved
-    bandwidth over the bytes it must read (HBM-bound stages)."""
+    """The decode step of --decode-workload, each stage replayed alone from a
+    CUDA graph, with its bandwidth over the bytes it must read."""
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = wl.WORKLOADS[args.decode_workload]
-    inp = wl.csa_decode_inputs(w, dev)
-    fmt = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
-    idx = torch.empty((w.B, 1, w.k), dtype=torch.int32, device=dev)
-    ws_i = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_INDEXER, 1, w.B, 1, 0, 0, w.n_csa, w.k,
-                                                 0), dev)
-    ws_a = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_SPARSE_ATTN, 1, w.B, 1, w.H, w.c,
-                                                 w.n_csa, w.k, w.n_win), dev)
-    out = torch.empty_like(inp["q"])
-    stages = {
-        "indexer_scores_topk": (lambda: csa.indexer_scores_topk(
-            inp["q_I"], inp["w"], inp["k_I"], w.m, w.k, q_pos=inp["q_pos"], idx_out=idx, ws=ws_i),
-            w.B * w.n_csa * w.dI * 2),
-        "sparse_mqa_attn": (lambda: csa.sparse_mqa_attn(
-            inp["q"], inp["entries"], idx, inp["win"], fmt, w.n_win, sink=inp["sink"],
-            q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], out=out, ws=ws_a),
-            w.B * (min(w.k, w.n_csa) + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2),
-    }
-    if w.kind == "decode_pair":
-        h = wl.hca_decode_inputs(w, dev)
-        n_h = h["entries"].shape[1]
-        ws_h = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_DENSE_ATTN, 1, w.B, 1, w.H, w.c, n_h,
-                                                     0, w.n_win), dev)
-        out_h = torch.empty_like(h["q"])
-        stages["dense_hca_attn"] = (lambda: csa.dense_hca_attn(
-            h["q"], h["entries"], w.m_prime, h["win"], fmt, w.n_win, sink=h["sink"],
-            q_pos=h["q_pos"], win_pos0=h["win_pos0"], out=out_h, ws=ws_h),
-            w.B * (n_h + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2)
+    d = DecodeStep(w, dev)
+    for _ in range(args.warmup):
+        d.run()
+    torch.cuda.synchronize()
+    d.check()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     res = {}
-    for name, (fn, nbytes) in stages.items():
-        for _ in range(args.warmup):
-            fn()
-        torch.cuda.synchronize()
-        tot = 0.0
-        for _ in range(args.steps):
-            flush.zero_()   # L2 flushed before every timed launch
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            tot += e0.elapsed_time(e1)
-        ms = tot / args.steps
+    for name, fn, nbytes in d.stages:
+        ms = graph_ms(fn, args.steps, flush)
         res[name] = {"ms": ms, "bytes": nbytes, "GBps": nbytes / ms / 1e6}
-    print(json.dumps({"only": "decode", "workload": w.name, "stages": res}))
+    step = graph_ms(d.run, args.steps, flush)
+    d.check()
+    print(json.dumps({"only": "decode", "workload": w.name, "stages": res, "step_ms": step,
+                      "queries_per_s": w.B / (step * 1e-3),
+                      "step_GBps": decode_bytes(w) / step / 1e6}))
 
 
 def run_only(args):
@@ -529,6 +661,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode workloads")
     args = ap.parse_args()
     if args.only:
         run_only(args)

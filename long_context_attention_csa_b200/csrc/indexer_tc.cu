@@ -590,6 +590,237 @@ __device__ bool block_topk(const float* sc, int n, int k, int64_t e0, unsigned* 
   return true;
 }
 
+// Block-wide exclusive prefix sum of one value per thread (up to 1024 threads).
+__device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* tmp, unsigned* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned incl = warp_incl_scan(v, lane);
+  __syncthreads();
+  if (lane == 31) tmp[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    const unsigned wv = lane < (int)(blockDim.x >> 5) ? tmp[lane] : 0u;
+    const unsigned wi = warp_incl_scan(wv, lane);
+    tmp[lane] = wi - wv;
+    if (lane == 31) tmp[32] = wi;
+  }
+  __syncthreads();
+  *total = tmp[32];
+  return tmp[wid] + incl - v;
+}
+
+// ---------------------------------------------------------------------------
+// Cluster top-k: exact selection of the k largest of a list split over the
+// CTAs of a cluster, in order (CTA rank, then thread, then element), each
+// thread holding R of them in registers (id < 0: not a candidate).  The keys
+// are the scores' order-preserving 32-bit images; a radix select on them
+// starts below the bits that every valid key shares (the cluster-wide key
+// minimum and maximum fix those) and takes at most 11 bits a pass (at most
+// three passes), so a pass spreads its keys over up to 2048 bins.  Each CTA
+// counts its own keys; every CTA sums the cluster's counts through
+// distributed shared memory and so takes the same decisions, and a pass ends
+// the select early once the boundary bucket is taken whole.  A candidate is
+// then taken if its key prefix is above the boundary, or equal to it and
+// among the first `rem` such candidates in list order (ties to the lower
+// index, since the list is in ascending index order); one exchange of per-CTA
+// (above, equal) counts gives every CTA its output offset, and the output is
+// ascending, padded with (-1, -inf).  Every CTA of the cluster runs this with
+// all of its threads, which all take the same barriers.
+// ---------------------------------------------------------------------------
+constexpr int kSelBins = 2048;
+constexpr int kSelMaxCluster = 8;   // portable cluster size
+
+struct SelShared {
+  unsigned hist[3][kSelBins];   // this CTA's counts, one buffer per pass (read remotely)
+  unsigned red[3][32];          // per-warp count / key min / key max (read remotely)
+  unsigned tot;                 // packed (above | equal << 16) counts (read remotely)
+  unsigned tmp[33];
+  unsigned glob[3];
+  unsigned dec[3];              // boundary digit, count above it, its bucket size
+  unsigned base[2];             // equal-key members before this CTA, output offset
+};
+
+template <int R, int NT>
+__device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], int k,
+                                  SelShared& sh, int32_t* out, float* so) {
+  static_assert(R * NT < 65536, "per-CTA counts are packed in 16 bits");
+  static_assert(NT * 4 == kSelBins, "four bins per thread in the bucket search");
+  const uint32_t CL = cluster_nctarank(), rank = cluster_ctarank();
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  constexpr int NW = NT / 32;
+  if (k <= 0) return;   // uniform over the cluster
+
+  for (int i = tid; i < 3 * kSelBins; i += NT) (&sh.hist[0][0])[i] = 0u;
+  unsigned cnt = 0, kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int e = 0; e < R; ++e) {
+    if (id[e] >= 0) {
+      const unsigned key = score_key(v[e]);
+      ++cnt;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sh.red[0][wid] = cnt;
+    sh.red[1][wid] = kmin;
+    sh.red[2][wid] = kmax;
+  }
+  cluster_sync();
+  if (wid == 0) {
+    unsigned c = 0, lo = 0xffffffffu, hi = 0u;
+    for (int i = lane; i < (int)CL * NW; i += 32) {
+      const uint32_t r = (uint32_t)(i / NW);
+      const int w = i % NW;
+      c += dsmem_ld_u32(&sh.red[0][w], r);
+      lo = min(lo, dsmem_ld_u32(&sh.red[1][w], r));
+      hi = max(hi, dsmem_ld_u32(&sh.red[2][w], r));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c += __shfl_xor_sync(0xffffffffu, c, o);
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      sh.glob[0] = c;
+      sh.glob[1] = lo;
+      sh.glob[2] = hi;
+    }
+  }
+  __syncthreads();
+  const unsigned n_valid = sh.glob[0];
+  const bool take_all = n_valid <= (unsigned)k;
+
+  // after the select the taken candidates are those whose key prefix
+  // (key & M) is above P, and the first `rem` (in list order) equal to it
+  unsigned P = 0u, M = 0u, rem = (unsigned)k;
+  if (!take_all) {
+    const unsigned gmin = sh.glob[1], gmax = sh.glob[2];
+    const unsigned diff = gmin ^ gmax;
+    int hb = diff ? 31 - __clz((int)diff) : -1;   // highest bit where valid keys differ
+    M = hb < 0 ? 0xffffffffu : (hb == 31 ? 0u : ~((2u << hb) - 1u));
+    P = gmin & M;
+    for (int pass = 0; hb >= 0; ++pass) {   // uniform over the cluster; at most 3 passes
+      const int shift = hb + 1 > 11 ? hb + 1 - 11 : 0;
+      const unsigned dmask = (1u << (hb + 1 - shift)) - 1u;
+      unsigned* h = sh.hist[pass];
+#pragma unroll
+      for (int e = 0; e < R; ++e) {
+        if (id[e] >= 0) {
+          const unsigned key = score_key(v[e]);
+          if ((key & M) == P) atomicAdd(&h[(key >> shift) & dmask], 1u);
+        }
+      }
+      cluster_sync();
+      // bucket search: thread t owns bins 2047-4t .. 2044-4t (descending),
+      // summed over the cluster (every rank's load issued before any is used)
+      uint4 x[kSelMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kSelMaxCluster; ++r)
+        if ((uint32_t)r < CL) x[r] = dsmem_ld_u32x4(&h[kSelBins - 4 * (tid + 1)], (uint32_t)r);
+      unsigned c[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int r = 0; r < kSelMaxCluster; ++r) {
+        if ((uint32_t)r < CL) {
+          c[0] += x[r].w;
+          c[1] += x[r].z;
+          c[2] += x[r].y;
+          c[3] += x[r].x;
+        }
+      }
+      const unsigned sT = c[0] + c[1] + c[2] + c[3];
+      unsigned total;
+      const unsigned above = block_excl_scan(sT, sh.tmp, &total);
+      if (above < rem && rem <= above + sT) {
+        unsigned run = above;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (run + c[i] >= rem) {
+            sh.dec[0] = (unsigned)(kSelBins - 1 - 4 * tid - i);
+            sh.dec[1] = run;
+            sh.dec[2] = c[i];
+            break;
+          }
+          run += c[i];
+        }
+      }
+      __syncthreads();
+      const unsigned d = sh.dec[0], bucket = sh.dec[2];
+      rem -= sh.dec[1];
+      P |= d << shift;
+      M |= dmask << shift;
+      if (bucket == rem) break;   // the whole bucket is taken
+      hb = shift - 1;
+    }
+  }
+
+  // ordered emit
+  unsigned gt = 0, eq = 0;
+#pragma unroll
+  for (int e = 0; e < R; ++e) {
+    if (id[e] >= 0) {
+      const unsigned km = score_key(v[e]) & M;
+      gt += km > P ? 1u : 0u;
+      eq += km == P ? 1u : 0u;
+    }
+  }
+  unsigned tot;
+  const unsigned excl = block_excl_scan(gt | (eq << 16), sh.tmp, &tot);
+  if (tid == 0) sh.tot = tot;
+  cluster_sync();
+  if (wid == 0) {   // output offset: the lower-ranked CTAs' taken counts, in order
+    const unsigned t = (uint32_t)lane < rank ? dsmem_ld_u32(&sh.tot, lane) : 0u;
+    unsigned eq_before = 0u, out_before = 0u;
+    for (uint32_t r = 0; r < rank; ++r) {
+      const unsigned tr = __shfl_sync(0xffffffffu, t, (int)r);
+      const unsigned q = tr >> 16;
+      const unsigned left = rem > eq_before ? rem - eq_before : 0u;
+      out_before += (tr & 0xffffu) + min(left, q);
+      eq_before += q;
+    }
+    if (lane == 0) {
+      sh.base[0] = eq_before;
+      sh.base[1] = out_before;
+    }
+  }
+  __syncthreads();
+  cluster_arrive();   // this CTA's remote reads are done
+  const unsigned eq_base = sh.base[0];
+  const unsigned left = rem > eq_base ? rem - eq_base : 0u;
+  unsigned at = sh.base[1] + (excl & 0xffffu) + min(left, excl >> 16);
+  unsigned eq_rank = eq_base + (excl >> 16);
+#pragma unroll
+  for (int e = 0; e < R; ++e) {
+    if (id[e] >= 0) {
+      const unsigned km = score_key(v[e]) & M;
+      bool take = km > P;
+      if (km == P) {
+        take = eq_rank < rem;
+        ++eq_rank;
+      }
+      if (take) {
+        out[at] = id[e];
+        if (so) so[at] = v[e];
+        ++at;
+      }
+    }
+  }
+  if (rank == 0) {   // padding after the taken ones
+    const unsigned taken = take_all ? n_valid : (unsigned)k;
+    for (int p = (int)taken + tid; p < k; p += NT) {
+      out[p] = -1;
+      if (so) so[p] = -INFINITY;
+    }
+  }
+  cluster_wait();   // no CTA leaves while another may still read its shared memory
+}
+
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
@@ -1254,23 +1485,6 @@ __device__ void merge_radix(const TcIdxArgs& a, int64_t row, MergeShared& sh) {
 }
 
 
-// Block-wide exclusive prefix sum of one value per thread (1024 threads).
-__device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* tmp, unsigned* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const unsigned incl = warp_incl_scan(v, lane);
-  __syncthreads();
-  if (lane == 31) tmp[wid] = incl;
-  __syncthreads();
-  if (wid == 0) {
-    const unsigned wv = lane < (int)(blockDim.x >> 5) ? tmp[lane] : 0u;
-    const unsigned wi = warp_incl_scan(wv, lane);
-    tmp[lane] = wi - wv;
-    if (lane == 31) tmp[32] = wi;
-  }
-  __syncthreads();
-  *total = tmp[32];
-  return tmp[wid] + incl - v;
-}
 
 // Final selection over one row's per-chunk candidates (in ascending entry
 // order), the same selection as merge_radix: value bins over the valid
@@ -1406,6 +1620,48 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// Cluster merge of the per-chunk candidates: one row's candidates split over
+// a cluster of up to kSelMaxCluster CTAs, 16 contiguous ones per thread.
+constexpr int kMThreads = 512;
+constexpr int kMRun = 16;
+constexpr int kMSlice = kMThreads * kMRun;      // per CTA: 8192
+
+__global__ void __launch_bounds__(kMThreads)
+    indexer_merge_cluster_kernel(TcIdxArgs a) {
+  __shared__ __align__(16) SelShared sh;
+  const uint32_t CL = cluster_nctarank(), rank = cluster_ctarank();
+  const int64_t row = blockIdx.x / CL;
+  const int64_t n = (int64_t)a.n_chunks * a.k;
+  const float* cs = a.cand_score + row * n;
+  const int32_t* ci = a.cand_idx + row * n;
+  const int64_t j0 = (int64_t)rank * kMSlice + (int64_t)threadIdx.x * kMRun;
+  float v[kMRun];
+  int32_t id[kMRun];
+  if ((n & 3) == 0) {   // 16-byte aligned rows: j0 and n are multiples of 4
+#pragma unroll
+    for (int q = 0; q < kMRun / 4; ++q) {
+      const int64_t j = j0 + 4 * q;
+      float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      int4 i4 = make_int4(-1, -1, -1, -1);
+      if (j < n) {
+        s4 = *reinterpret_cast<const float4*>(cs + j);
+        i4 = *reinterpret_cast<const int4*>(ci + j);
+      }
+      v[4 * q] = s4.x; v[4 * q + 1] = s4.y; v[4 * q + 2] = s4.z; v[4 * q + 3] = s4.w;
+      id[4 * q] = i4.x; id[4 * q + 1] = i4.y; id[4 * q + 2] = i4.z; id[4 * q + 3] = i4.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kMRun; ++e) {
+      const int64_t j = j0 + e;
+      id[e] = j < n ? ci[j] : -1;
+      v[e] = j < n ? cs[j] : 0.f;
+    }
+  }
+  cluster_topk_emit<kMRun, kMThreads>(v, id, a.k, sh, a.idx_out + row * a.k,
+                                      a.score_out ? a.score_out + row * a.k : nullptr);
+}
+
 inline int tok_for(int64_t Tq) { return Tq >= 4 ? 4 : 1; }
 inline int chunk_for(int tok) { return tok == 4 ? Cfg<4>::kChunk : Cfg<1>::kChunk; }
 inline int n_chunks_for(int64_t N, int tok) {
@@ -1436,6 +1692,30 @@ int sm_count() {
       cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     n = 148;
   return n;
+}
+
+// The candidate merge: the cluster kernel when one row's candidates fit a
+// cluster of at most kSelMaxCluster CTAs, else one CTA per row.
+cudaError_t launch_merge(const TcIdxArgs& a, int64_t rows, cudaStream_t stream) {
+  const int64_t n = (int64_t)a.n_chunks * a.k;
+  const int64_t cl = (n + kMSlice - 1) / kMSlice;
+  if (cl > kSelMaxCluster || rows * cl > (int64_t)0x7fffffff) {
+    indexer_merge_kernel<<<(unsigned)rows, 1024, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
+  cfg.blockDim = dim3(kMThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)cl;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, indexer_merge_cluster_kernel, a);
 }
 
 cudaError_t launch_persist(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
@@ -1498,8 +1778,7 @@ cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
   if (e != cudaSuccess) return e;
   *n_launch = 1;
   if (a.n_chunks > 1) {
-    indexer_merge_kernel<<<(unsigned)(p.B * p.Tq), 1024, 0, stream>>>(a);
-    e = cudaGetLastError();
+    e = launch_merge(a, p.B * p.Tq, stream);
     *n_launch = 2;
   }
   return e;

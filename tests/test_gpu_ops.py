@@ -186,6 +186,36 @@ def test_indexer_decode(wname):
     assert d <= 1
 
 
+@pytest.mark.parametrize("N", [40000, 30000])
+@pytest.mark.parametrize("k,zero", [(1023, False), (1024, False), (1024, True)])
+def test_indexer_decode_select_integer_bit_exact(N, k, zero):
+    """Single-token queries over N entries in 4096-entry chunks: 40000 (ten
+    chunks: per-chunk candidates, merged by a cluster of two CTAs) and 30000
+    (eight chunks: the row's CTAs select as one cluster).  Integer inputs give
+    exact sums and many ties across CTA boundaries; an odd k takes the
+    unaligned loads; the third context is short (most chunks empty, fewer
+    visible than k); zero q_I makes every score equal (the lowest k indices
+    win)."""
+    B, HI, dI, m = 3, 64, 128, 4
+    pos = torch.tensor([[m * N - 1], [m * (N // 2) + 5], [m * 300]], dtype=torch.int64)
+    qI = wl.randint_like_float((B, 1, HI, dI), 41, -2, 3, DEV, torch.bfloat16)
+    if zero:
+        qI.zero_()
+    kI = wl.randint_like_float((B, N, dI), 42, -2, 3, DEV, torch.bfloat16)
+    w = wl.randint_like_float((B, 1, HI), 43, -2, 3, DEV, torch.float32)
+    idx, sc = csa.indexer_scores_topk(qI, w, kI, m, k, q_pos=pos.to(DEV), want_scores=True)
+    torch.cuda.synchronize()
+    for b in range(B):
+        p = pos[b].numpy()
+        ref_sc = oracle.indexer_scores(f64(qI[b]), f64(w[b]), f64(kI[b]), m, q_pos=p)
+        ref_idx = oracle.topk(ref_sc, k, m, q_pos=p)
+        gi = idx[b].cpu().numpy()
+        assert np.array_equal(gi, ref_idx), f"row {b}"
+        v = gi >= 0
+        assert np.array_equal(sc[b].cpu().numpy().astype(np.float64)[v],
+                              np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v])
+
+
 def test_indexer_padding_when_few_visible():
     w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=40, k=16)
     _indexer_case(w)
