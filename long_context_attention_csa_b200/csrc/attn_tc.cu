@@ -275,6 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t kbase = smem_u32(sm + OFF_K);
     constexpr int kEv = (kMaxK / kProdWarps + 31) / 32 + 1;   // index words per lane
     int32_t ev[kEv];
+    // RoPE frequency of pair `lane` (warp 0 builds the per-item cos/sin table)
+    const double theta = rope_theta(lane, a.r > 0 ? a.r : 2, a.base);
     // index loads of item (it, m): warp pw takes the contiguous third of the row
     auto load_idx = [&](int64_t row) {
       const int32_t* ir = a.idx + row * (int64_t)a.k;
@@ -283,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < kEv; ++u) {
         const int i = lo + u * 32 + lane;
-        ev[u] = (!dead && a.sparse && u * 32 < q3 && i < hi) ? __ldg(ir + i) : -1;
+        // volatile loads: issued here, a block before their use, not sunk to it
+        ev[u] = (!dead && a.sparse && u * 32 < q3 && i < hi) ? ldg_nc_volatile(ir + i) : -1;
       }
     };
     // builds item m's index list, RoPE table and entry count (slot m & 1)
@@ -292,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* rcs = ropes + (m & 3) * 64;
       if (!dead && pw == 0 && lane < (a.r >> 1)) {
         float cs, sn;
-        rope_cos_sin(y.pos, lane, a.r, a.base, &cs, &sn);
+        rope_cos_sin_theta(y.pos, theta, &cs, &sn);
         rcs[lane] = cs;
         rcs[32 + lane] = sn;
       }
@@ -828,7 +831,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(TcAttnArgs a) {
     inv[threadIdx.x] = tot > 0.f ? 1.f / tot : 0.f;
   } else if (threadIdx.x >= 32 && threadIdx.x < 32 + (a.r >> 1)) {
     float cs, sn;
-    rope_cos_sin(-pos, threadIdx.x - 32, a.r, a.base, &cs, &sn);
+    rope_cos_sin_theta(-pos, rope_theta(threadIdx.x - 32, a.r, a.base), &cs, &sn);
     cs_t[threadIdx.x - 32] = cs;
     sn_t[threadIdx.x - 32] = sn;
   }

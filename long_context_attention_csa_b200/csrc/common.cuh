@@ -35,6 +35,14 @@ template <typename T> struct VecOf;
 template <> struct VecOf<float> { static constexpr int N = 4; };
 template <> struct VecOf<bf16> { static constexpr int N = 8; };
 
+// A read-only global load the compiler keeps in program order (volatile asm):
+// for loads issued well ahead of their first use.
+__device__ __forceinline__ int32_t ldg_nc_volatile(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
   return __uint_as_float(bits16 << 16);
 }
@@ -98,6 +106,25 @@ __device__ __forceinline__ void rope_cos_sin(int64_t pos, int i, int r, float ba
   sincos(a, &s, &c);
   *cs = (float)c;
   *sn = (float)s;
+}
+
+// theta_i = base^(-2i/r) of RoPE pair i, in double: the angle pos * theta_i
+// needs more than single precision once pos is large.
+__device__ __forceinline__ double rope_theta(int i, int r, float base) {
+  return pow((double)base, -2.0 * (double)i / (double)r);
+}
+
+// cos and sin of pos * theta for a precomputed theta: the angle is formed and
+// reduced by a multiple of 2 pi in double (the reduced angle is accurate to
+// about 1e-10 rad for |pos| < 2^32), then its sine and cosine are taken in
+// single precision.
+__device__ __forceinline__ void rope_cos_sin_theta(int64_t pos, double theta, float* cs,
+                                                   float* sn) {
+  constexpr double kTwoPi = 6.283185307179586;
+  const double ang = (double)pos * theta;
+  const double turns = rint(ang * (1.0 / kTwoPi));
+  const float red = (float)fma(-turns, kTwoPi, ang);
+  sincosf(red, sn, cs);
 }
 
 // Rotate the pairs of a VEC-wide slice [ch0, ch0+VEC) that fall in the RoPE
