@@ -22,7 +22,7 @@
 // gather of block b+1 and S^T(b+1) overlap the softmax and O^T of block b.
 //
 // Query RMSNorm as a per-head scale: the Q tile holds the raw q rows (TMA,
-// dims 0..447) and RoPE(q) for the last 64 dims (written by the producer), so
+// dims 0..447) and RoPE(q) for the last 64 dims (rotated in place), so
 // S^T carries |q| instead of |q^| and the softmax multiplies head h's column
 // by scale inv_h log2(e), inv_h = 1/rms(q_h).  RoPE preserves pair norms, so
 // inv_h comes from the raw rows.
@@ -39,12 +39,13 @@
 // Persistent CTAs (one per SM) walk their items in turn; roles (384 threads,
 // the register budget of 288 threads since allocation is per 128 threads):
 //   warps 8-10 producer: index compaction, RoPE table, the item's raw q rows
-//              by TMA, in-place rotation of the RoPE dims and per-head 1/rms,
-//              the key gather (cp.async; each warp-instruction moves four
-//              128-byte row pieces);
+//              by TMA, the key gather (cp.async; each warp-instruction moves
+//              four 128-byte row pieces);
 //   warp 11    TMEM owner and single-thread MMA issuer;
 //   warps 0-3  softmax (all 32 lanes: the 16x64b TMEM load gives each lane
-//              one key and the 32 heads of one parity);
+//              one key and the 32 heads of one parity); at an item's start
+//              they rotate the Q tile's RoPE dims in place as soon as the raw
+//              rows land, then derive the per-head 1/rms while S^T(0) runs;
 //   warps 4-7  epilogue (thread = output dim), which runs alongside the next
 //              item's softmax; it frees O^T in four 64-column slices, so the
 //              next item's first O^T waits only for the slice it overwrites.
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pfull = bars + 6;    // [2] P tile written (128 softmax threads)
   uint64_t* iready = bars + 8;   // [2] item's entry count published
   uint64_t* qraw = bars + 10;    // raw q rows landed in the Q tile (TMA)
-  uint64_t* qload = bars + 11;   // Q tile complete: RoPE dims rotated (64 producer threads)
+  uint64_t* qload = bars + 11;   // Q tile complete: RoPE dims rotated (128 softmax threads)
   uint64_t* qfree = bars + 12;   // last S^T of the item done and its Q rows read (2)
   uint64_t* ofull = bars + 13;   // last O^T (and row-sum MMA) of the item done
   uint64_t* drain = bars + 15;
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ofree[i], 128);
     }
     mbar_init(qraw, 1);
-    mbar_init(qload, kHG);
+    mbar_init(qload, 128);
     mbar_init(qfree, 2);
     mbar_init(ofull, 1);
     mbar_init(drain, 1);
@@ -406,39 +407,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!dead) cp_async_arrive(&kfull[s]);
         }
         if (b == 0) {
-          // head ptid < 64: rotate the dims 448..511 of its row in place (their
-          // raw sum of squares kept for the softmax's 1/rms), then let the MMA
-          // read the Q tile
-          if (ptid < kHG) {
-            wait_or_die(qraw, (uint32_t)n & 1u, 22u);
-            if (!dead) {
-              const int h = ptid;
-              float ss = 0.f;   // raw sum of squares of the RoPE-region dims
-              uint8_t* q7row = sQ + (kRegions - 1) * kQRegion + h * 128;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {   // 16-byte chunk k holds dims 448 + 8k .. + 7
-                uint4* cp = reinterpret_cast<uint4*>(q7row + ((k ^ (h & 7)) << 4));
-                const uint4 v = *cp;
-                uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float x0 = bf16_bits_to_float(w4[e] & 0xffffu);
-                  const float x1 = bf16_bits_to_float(w4[e] >> 16);
-                  ss = fmaf(x0, x0, fmaf(x1, x1, ss));
-                  const int d = 448 + 8 * k + 2 * e;   // even dim of the pair
-                  if (!(a.flags & CSA_F_NO_ROPE) && d >= kC - a.r) {
-                    const int pi = (d - (kC - a.r)) >> 1;
-                    w4[e] = pack_bf16x2(x0 * rcs[pi] - x1 * rcs[32 + pi],
-                                        x0 * rcs[32 + pi] + x1 * rcs[pi]);
-                  }
-                }
-                *cp = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-              }
-              ss7[h] = ss;
-              fence_proxy_async_smem();   // generic stores -> the MMA's reads
-              mbar_arrive(qload);
-            }
-          }
           if (has_next) load_idx(y.row);   // consumed by the compaction below
         }
         if (b == (nbl > 2 ? 2 : nbl - 1) && has_next) cur_ent = compact(y, n + 1);
@@ -505,14 +473,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < nb; ++b) {
           const int64_t j = gblk + b;
           const int s = (int)(j & 1);
-          // S^T(j+1) ahead of O^T(j) when its key tile is already here (keeps the
-          // tensor pipe busy through softmax(j+1)); never block O^T(j) on a gather
-          if (next_s == b + 1 && next_s < nb &&
-              mbar_try_wait(&kfull[(j + 1) & 1], (uint32_t)((j + 1) >> 1) & 1u)) {
-            if (!issue_s_item(next_s)) { ok = false; break; }
-            ++next_s;
+          // wait for P(j); S^T(j+1) goes first if its key tile lands before
+          // (keeps the tensor pipe busy through softmax(j+1)); never block
+          // O^T(j) on a gather
+          {
+            const uint64_t t0 = globaltimer_ns();
+            for (;;) {
+              if (next_s == b + 1 && next_s < nb &&
+                  mbar_test_wait(&kfull[(j + 1) & 1], (uint32_t)((j + 1) >> 1) & 1u)) {
+                if (!issue_s_item(next_s)) { ok = false; break; }
+                ++next_s;
+              }
+              if (mbar_try_wait_sleep(&pfull[s], (uint32_t)(j >> 1) & 1u, 256u)) break;
+              if (*abort_flag || globaltimer_ns() - t0 > 2000000000ull) { ok = false; break; }
+            }
+            if (!ok) break;
           }
-          if (*abort_flag || !mbar_wait(&pfull[s], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
           tc_fence_after();
           const uint64_t dVs = dV + (uint64_t)((s * kKTile) >> 4);
           const uint64_t dPs = dP + (uint64_t)((s * kPTile) >> 4);
@@ -569,9 +545,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_or_die(&iready[ip], (uint32_t)(n >> 1) & 1u, 24u);
       int64_t k_lo = 0, k_hi = 0;
       const int nb = dead ? 0 : item_blocks(a, x, nent[ip], &k_lo, &k_hi);
+      // as soon as the raw q rows land, the Q tile's dims 448..511 (region
+      // 7): lane `lane` rotates pair `lane` (dims 448 + 2 lane, + 1) of heads
+      // warp, warp + 4, ... in place, all of its loads in flight at once (the
+      // lanes cover one 128-byte row: no bank conflicts), keeping the raw
+      // squares; a transposing butterfly leaves head warp + 4 l's raw sum of
+      // squares in lane l < 16.  Then the MMA may read the Q tile.
+      wait_or_die(qraw, (uint32_t)n & 1u, 24u);
+      if (!dead) {
+        const float* rcs = ropes + (n & 3) * 64;
+        const int d = (kRegions - 1) * 64 + 2 * lane;   // even dim of the pair
+        const bool rot = !(a.flags & CSA_F_NO_ROPE) && d >= kC - a.r;
+        const int pi = rot ? (d - (kC - a.r)) >> 1 : 0;
+        const float cs = rot ? rcs[pi] : 1.f, sn = rot ? rcs[32 + pi] : 0.f;
+        uint8_t* q7 = sQ + (kRegions - 1) * kQRegion + (lane & 3) * 4;
+        uint32_t wv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int h = warp + 4 * i;
+          wv[i] = *reinterpret_cast<const uint32_t*>(q7 + h * 128 + (((lane >> 2) ^ (h & 7)) << 4));
+        }
+        float sq[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int h = warp + 4 * i;
+          const float x0 = bf16_bits_to_float(wv[i] & 0xffffu);
+          const float x1 = bf16_bits_to_float(wv[i] >> 16);
+          sq[i] = fmaf(x0, x0, x1 * x1);
+          if (rot)
+            *reinterpret_cast<uint32_t*>(q7 + h * 128 + (((lane >> 2) ^ (h & 7)) << 4)) =
+                pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], 16);
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) {
+          const bool up = (lane & off) != 0;
+#pragma unroll
+          for (int i = 0; i < off; ++i) {
+            const float send = up ? sq[i] : sq[i + off];
+            const float keep = up ? sq[i + off] : sq[i];
+            sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+          }
+        }
+        if (lane < 16) ss7[warp + 4 * lane] = sq[0];
+        fence_proxy_async_smem();   // generic stores -> the MMA's reads
+        mbar_arrive(qload);
+      }
       // per-head factors while S^T(0) runs: thread rw sums half of head rw/2's
       // raw dims 0..447 (Q tile regions 0-3 or 4-6, rotated chunk order for the
-      // banks); the RoPE dims' raw sum comes from the producer's rotation
+      // banks) and adds region 7's raw sum from above
       wait_or_die(qload, (uint32_t)n & 1u, 24u);
       if (!dead) {
         const int h = rw >> 1, hh = rw & 1;
