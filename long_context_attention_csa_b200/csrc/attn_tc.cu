@@ -49,8 +49,9 @@
 //   warps 4-7  epilogue (thread = output dim), which runs alongside the next
 //              item's softmax; it frees O^T in four 64-column slices, so the
 //              next item's first O^T waits only for the slice it overwrites.
-// Decode rows (one query per sequence) split the key list into fixed 320-key
-// pieces whose fp32 partials a combine kernel adds in a fixed order, so a
+// Decode rows (one query per sequence) split the key list into pieces of a
+// size fixed by the row's own key count (at least 320 keys, at most 16
+// pieces) whose fp32 partials a combine kernel adds in a fixed order, so a
 // row's result does not depend on the batch it runs in.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -71,7 +72,8 @@ constexpr int kKRegion = kBK * 128;          // 8 KB per key-tile chunk
 constexpr int kKTile = kRegions * kKRegion;  // 64 KB
 constexpr int kQRegion = kHG * 128;          // 8 KB per query chunk
 constexpr int kPTile = kBK * 128;            // 8 KB: P^T [64 keys][64 heads] bf16
-constexpr int kSplitKeys = 320;              // decode split size (fixed: five 64-key blocks)
+constexpr int kSplitKeys = 320;              // smallest decode split (five 64-key blocks)
+constexpr int kMaxSplits = 16;               // most splits of one decode row
 constexpr int kMaxK = 1024;                  // largest top-k the index list holds
 constexpr int kProdWarp0 = 8;                // warps 8-10 produce, warp 11 issues MMAs
 constexpr int kProdWarps = 3;
@@ -165,14 +167,25 @@ __device__ __forceinline__ Item decode_item(const TcAttnArgs& a, int64_t it) {
   return x;
 }
 
+// Decode split size of a row with n_keys keys: at least kSplitKeys, and large
+// enough (whole 64-key blocks) for at most kMaxSplits splits.  It depends on
+// the row's own key count only, so a row's result does not depend on the
+// batch it runs in.
+__host__ __device__ __forceinline__ int64_t split_keys_for(int64_t n_keys) {
+  const int64_t per = (n_keys + kMaxSplits - 1) / kMaxSplits;
+  const int64_t blk = (per + kBK - 1) / kBK * kBK;
+  return blk > kSplitKeys ? blk : kSplitKeys;
+}
+
 // Key range [lo, hi) of an item and its number of 64-key blocks.
 __device__ __forceinline__ int item_blocks(const TcAttnArgs& a, const Item& x, int64_t n_ent,
                                            int64_t* lo, int64_t* hi) {
   const int64_t n_keys = n_ent + x.n_w;
   int64_t l = 0, h = n_keys;
   if (a.split) {
-    l = (int64_t)x.split * kSplitKeys;
-    h = l + kSplitKeys < n_keys ? l + kSplitKeys : n_keys;
+    const int64_t sk = split_keys_for(n_keys);
+    l = (int64_t)x.split * sk;
+    h = l + sk < n_keys ? l + sk : n_keys;
   }
   *lo = l;
   *hi = h;
@@ -902,8 +915,11 @@ inline int64_t num_sms() {
   return n;
 }
 
+// Splits per decode row: enough for the row with the most keys (a row with
+// fewer keys leaves its last splits empty; their zero partials add exactly).
 inline int n_splits_for(int64_t max_keys) {
   int64_t n = (max_keys + kSplitKeys - 1) / kSplitKeys;
+  n = n < kMaxSplits ? n : kMaxSplits;
   return n < 1 ? 1 : (int)n;
 }
 
