@@ -63,11 +63,11 @@ def compress_bytes(w) -> float:
     return float(w.B * (4 * w.T * w.c + w.n_csa * w.c + w.T * w.c) * e)
 
 
-# DRAM bytes per attention launch at 8192 query rows: the counters of the
-# 2048-row capture summarised in profiles/attn_tc_kernel_csa_prefill_2k.md
-# (141.2 MB read + 90.8 MB written) scaled by the rows processed.  Refresh it
-# whenever the attention kernel changes.
-ATTN_DRAM_BYTES_8K = 4 * (141.185536e6 + 90.788352e6)
+# DRAM bytes per attention launch at 8192 query rows: dram__bytes_read.sum +
+# dram__bytes_write.sum of the full-size launch list summarised in
+# profiles/csa_prefill_8k_launch_list.md (564.6 MB read + 489.2 MB written).
+# Refresh it whenever the attention kernel changes.
+ATTN_DRAM_BYTES_8K = 564.6e6 + 489.2e6
 
 
 class Clocks:
@@ -322,9 +322,9 @@ def run_gpu(args):
             "roofline": {"bound": "tensor", "kernel": "sparse_mqa_attn",
                          "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
                          "frac": achieved / bf16, "traffic": ATTN_DRAM_BYTES_8K,
-                         "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of a "
-                                           "2048-token ncu capture x 4 (query rows), "
-                                           "profiles/attn_tc_kernel_csa_prefill_2k.md",
+                         "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of the "
+                                           "full-size ncu launch list, "
+                                           "profiles/csa_prefill_8k_launch_list.md",
                          "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)"
                          if src == "measured" else "fallback 1.59 PFLOP/s",
                          "algorithmic_flops_per_launch": fl_attn},
