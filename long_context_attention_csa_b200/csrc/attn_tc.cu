@@ -75,12 +75,22 @@ constexpr int kPTile = kBK * 128;            // 8 KB: P^T [64 keys][64 heads] bf
 constexpr int kSplitKeys = 320;              // smallest decode split (five 64-key blocks)
 constexpr int kMaxSplits = 16;               // most splits of one decode row
 constexpr int kMaxK = 1024;                  // largest top-k the index list holds
-constexpr int kProdWarp0 = 8;                // warps 8-10 produce, warp 11 issues MMAs
-constexpr int kProdWarps = 3;
+// 16 warps in four warpgroups: softmax (0-3), epilogue (4-7), producers
+// 8-10 and 12-14, the S^T issuer and TMEM owner (11), the O^T issuer (15).
+constexpr int kProdWarps = 6;
 constexpr int kProdThreads = 32 * kProdWarps;
-constexpr int kMmaWarp = kProdWarp0 + kProdWarps;
+constexpr int kMmaWarp = 11;
+constexpr int kMmaWarpO = 15;
 constexpr int kGatherIters = (kBK / 4 + kProdWarps - 1) / kProdWarps;   // 4-row groups per warp
-constexpr int kThreads = 32 * (kMmaWarp + 1);  // 384
+constexpr int kThreads = 512;
+// registers per thread: launched with 128; softmax and epilogue warpgroups
+// raise theirs, the producer / issuer warpgroups lower theirs, and the sum
+// stays at the launch total (128 threads per warpgroup):
+constexpr int kRegHeavy = 136, kRegLight = 120;
+static_assert(2 * kRegHeavy + 2 * kRegLight <= 4 * 128, "register split exceeds the launch budget");
+__device__ __forceinline__ int prod_index(int warp) {   // producer warp -> 0..5, else -1
+  return (warp >= 8 && warp <= 10) ? warp - 8 : (warp >= 12 && warp <= 14) ? warp - 9 : -1;
+}
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRangeLog2 = 60.f * kLog2e;  // CSA_DEV_RANGE threshold
 
@@ -96,7 +106,7 @@ constexpr int OFF_INV = OFF_C2 + 4 * kHG * 4;        // [64] 1/denominator
 constexpr int OFF_SS7 = OFF_INV + kHG * 4;           // [64] sum of squares of the RoPE dims
 constexpr int OFF_NENT = OFF_SS7 + kHG * 4;          // [2] entries per item
 constexpr int OFF_BAR = OFF_NENT + 64;
-constexpr int kNumBars = 26;
+constexpr int kNumBars = 38;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64;
 
@@ -204,34 +214,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* ss7 = reinterpret_cast<float*>(sm + OFF_SS7);
   int* nent = reinterpret_cast<int*>(sm + OFF_NENT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* kfull = bars;        // [2] key tile landed (producer threads)
-  uint64_t* bfree = bars + 2;    // [2] O^T of the block done: key tile and P tile free
-  uint64_t* sfull = bars + 4;    // [2] S^T of the block done
-  uint64_t* pfull = bars + 6;    // [2] P tile written (128 softmax threads)
-  uint64_t* iready = bars + 8;   // [2] item's entry count published
-  uint64_t* qraw = bars + 10;    // raw q rows landed in the Q tile (TMA)
-  uint64_t* qload = bars + 11;   // Q tile complete: RoPE dims rotated (128 softmax threads)
-  uint64_t* qfree = bars + 12;   // last S^T of the item done and its Q rows read (2)
-  uint64_t* ofull = bars + 13;   // last O^T (and row-sum MMA) of the item done
-  uint64_t* drain = bars + 15;
-  uint64_t* ifree = bars + 16;   // [2] MMA, softmax and epilogue have read the item slot
-  uint64_t* qready = bars + 18;  // [4] the item's per-head factors ready (epilogue)
-  uint64_t* ofree = bars + 22;   // [4] epilogue has read O^T columns 64 jt .. 64 jt + 63
+  // key tiles move in four region pairs (dims 128 h .. 128 h + 127, regions
+  // 2h and 2h+1), the columns one O^T slice reads: barrier [4 s + h]
+  uint64_t* kfull = bars;        // [2][4] region pair landed (producer threads)
+  uint64_t* bfree = bars + 8;    // [2][4] O^T slice h of the block done: its regions free;
+                                 //        [4 s + 3] also frees P tile s (row sums go first)
+  uint64_t* sfull = bars + 16;   // [2] S^T of the block done
+  uint64_t* pfull = bars + 18;   // [2] P tile written (128 softmax threads)
+  uint64_t* iready = bars + 20;  // [2] item's entry count published
+  uint64_t* qraw = bars + 22;    // raw q rows landed in the Q tile (TMA)
+  uint64_t* qload = bars + 23;   // Q tile complete: RoPE dims rotated (128 softmax threads)
+  uint64_t* qfree = bars + 24;   // last S^T of the item done and its Q rows read (2)
+  uint64_t* ofull = bars + 25;   // last O^T (and row-sum MMA) of the item done
+  uint64_t* drain = bars + 26;
+  uint64_t* ifree = bars + 27;   // [2] both issuers, softmax and epilogue have read the item slot
+  uint64_t* qready = bars + 29;  // [4] the item's per-head factors ready (epilogue)
+  uint64_t* ofree = bars + 33;   // [4] epilogue has read O^T columns 64 jt .. 64 jt + 63
+  uint64_t* drain_o = bars + 37;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  int* wcnt = reinterpret_cast<int*>(sm + OFF_MISC + 8);        // [3]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 24);
+  int* wcnt = reinterpret_cast<int*>(sm + OFF_MISC + 8);        // [kProdWarps]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 40);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float scale = a.scale > 0.f ? a.scale : rsqrtf((float)kC);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 8; ++i) {
       mbar_init(&kfull[i], kProdThreads);
       mbar_init(&bfree[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);
       mbar_init(&iready[i], 1);
-      mbar_init(&ifree[i], 3);
+      mbar_init(&ifree[i], 4);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&qready[i], 1);
@@ -242,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(qfree, 2);
     mbar_init(ofull, 1);
     mbar_init(drain, 1);
+    mbar_init(drain_o, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -263,6 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tO = tmem + 128;     // O^T: 4 x 64 columns
   const uint32_t tL = tmem + 384;     // per-head sums of P (64 columns, rows identical)
 
+  // register budgets per warpgroup (every warp of a warpgroup takes the same)
+  if (warp < 8)
+    setmaxnreg_inc<kRegHeavy>();
+  else
+    setmaxnreg_dec<kRegLight>();
+
   // Failure handling (every role): a wait that runs out marks the thread
   // `dead` (made warp-uniform); dead threads skip waits and work but still
   // pass every named barrier, so no barrier can be left waiting.
@@ -279,22 +302,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     dead = __any_sync(0xffffffffu, dead);
   };
 
-  if (warp >= kProdWarp0 && warp < kMmaWarp) {
-    // ======================= producer (3 warps)
+  if (prod_index(warp) >= 0) {
+    // ======================= producer (6 warps)
     // Item n's index list and RoPE table are built while item n-1's keys
     // stream (its index loads are issued early and consumed a block later),
     // so an item starts with its Q tile and first key tiles only.
-    const int ptid = threadIdx.x - 32 * kProdWarp0, pw = warp - kProdWarp0;
+    const int pw = prod_index(warp), ptid = pw * 32 + lane;
     const int quad = lane >> 3, g8 = lane & 7;
     const uint32_t kbase = smem_u32(sm + OFF_K);
     constexpr int kEv = (kMaxK / kProdWarps + 31) / 32 + 1;   // index words per lane
     int32_t ev[kEv];
     // RoPE frequency of pair `lane` (warp 0 builds the per-item cos/sin table)
     const double theta = rope_theta(lane, a.r > 0 ? a.r : 2, a.base);
-    // index loads of item (it, m): warp pw takes the contiguous third of the row
+    // index loads of item (it, m): warp pw takes the contiguous pw-th share of the row
     auto load_idx = [&](int64_t row) {
       const int32_t* ir = a.idx + row * (int64_t)a.k;
-      const int q3 = (a.k + 2) / 3;
+      const int q3 = (a.k + kProdWarps - 1) / kProdWarps;   // this warp's share
       const int lo = pw * q3, hi = lo + q3 < a.k ? lo + q3 : a.k;
 #pragma unroll
       for (int u = 0; u < kEv; ++u) {
@@ -315,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int64_t ne;
       if (a.sparse) {
-        const int lo = pw * ((a.k + 2) / 3);
+        const int lo = pw * ((a.k + kProdWarps - 1) / kProdWarps);
         int32_t* list = reinterpret_cast<int32_t*>(sm + OFF_LIST) + (m & 1) * kMaxK;
         int cnt = 0;
 #pragma unroll
@@ -330,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar(2, kProdThreads);
         int off = 0;
         for (int w = 0; w < pw; ++w) off += wcnt[w];
-        ne = wcnt[0] + wcnt[1] + wcnt[2];
+        ne = 0;
+        for (int w = 0; w < kProdWarps; ++w) ne += wcnt[w];
 #pragma unroll
         for (int u = 0; u < kEv; ++u) {
           const bool ok = ev[u] >= 0 && ev[u] < a.N;
@@ -387,37 +411,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t j = gblk + b;
         const int s = (int)(j & 1);
         if (b < nb) {
-          wait_or_die(&bfree[s], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
-          if (!dead) {
-            const uint32_t tile = kbase + s * kKTile;
-            // groups of four rows (one per 8-lane quad; 128 bytes per lane group
-            // and region) dealt round-robin over the producer warps
-            const bf16* src[kGatherIters];
+          const uint32_t tile = kbase + s * kKTile;
+          // groups of four rows (one per 8-lane quad; 128 bytes per lane group
+          // and region) dealt round-robin over the producer warps
+          const bf16* src[kGatherIters];
 #pragma unroll
-            for (int u = 0; u < kGatherIters; ++u) {
-              const int r = 4 * (pw + kProdWarps * u) + quad;
-              const int64_t key = k_lo + (int64_t)b * kBK + r;
-              src[u] = nullptr;
-              if (pw + kProdWarps * u < kBK / 4 && key < k_hi)
-                src[u] = key < n_ent ? ent + (int64_t)(a.sparse ? list[key] : key) * kC
-                                     : win + ((x.jlo - x.wp0) + (key - n_ent)) * kC;
-            }
+          for (int u = 0; u < kGatherIters; ++u) {
+            const int r = 4 * (pw + kProdWarps * u) + quad;
+            const int64_t key = k_lo + (int64_t)b * kBK + r;
+            src[u] = nullptr;
+            if (!dead && pw + kProdWarps * u < kBK / 4 && key < k_hi)
+              src[u] = key < n_ent ? ent + (int64_t)(a.sparse ? list[key] : key) * kC
+                                   : win + ((x.jlo - x.wp0) + (key - n_ent)) * kC;
+          }
+          // region pair h as soon as O^T slice h of the tile's previous block
+          // has read it
+#pragma unroll 1
+          for (int h = 0; h < 4; ++h) {
+            wait_or_die(&bfree[4 * s + h], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
+            if (!dead) {
 #pragma unroll
-            for (int u = 0; u < kGatherIters; ++u) {
-              if (pw + kProdWarps * u >= kBK / 4) break;
-              const int r = 4 * (pw + kProdWarps * u) + quad;
-              const uint32_t dst =
-                  tile + (uint32_t)r * 128u + (((uint32_t)g8 ^ (uint32_t)(r & 7)) << 4);
+              for (int u = 0; u < kGatherIters; ++u) {
+                if (pw + kProdWarps * u >= kBK / 4) continue;
+                const int r = 4 * (pw + kProdWarps * u) + quad;
+                const uint32_t dst =
+                    tile + (uint32_t)r * 128u + (((uint32_t)g8 ^ (uint32_t)(r & 7)) << 4);
 #pragma unroll
-              for (int reg = 0; reg < kRegions; ++reg) {
-                const void* sp =
-                    src[u] ? (const void*)(src[u] + reg * 64 + g8 * 8) : (const void*)a.q;
-                cp_async16(dst + reg * kKRegion, sp, src[u] ? 16u : 0u);
+                for (int rr = 0; rr < 2; ++rr) {
+                  const int reg = 2 * h + rr;
+                  const void* sp =
+                      src[u] ? (const void*)(src[u] + reg * 64 + g8 * 8) : (const void*)a.q;
+                  cp_async16(dst + reg * kKRegion, sp, src[u] ? 16u : 0u);
+                }
               }
+              // the barrier counts this thread's arrival once its copies land
+              cp_async_arrive(&kfull[4 * s + h]);
             }
           }
-          // the barrier counts this thread's arrival once its copies land
-          if (!dead) cp_async_arrive(&kfull[s]);
         }
         if (b == 0) {
           if (has_next) load_idx(y.row);   // consumed by the compaction below
@@ -428,38 +458,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_wait<0>();
   } else if (warp == kMmaWarp) {
-    // ======================= MMA issuer
+    // ======================= S^T issuer (TMEM owner)
     if (elect_one()) {
       constexpr uint32_t idS = idesc_bf16_f32(kBK, kHG, 0, 0);
-      constexpr uint32_t idO = idesc_bf16_f32(128, kHG, 1, 1);
-      constexpr uint32_t idL = idesc_bf16_f32(kBK, kHG, 0, 1);
       // descriptors built once; an operand at byte offset o adds o >> 4 to the
       // start-address field (every offset stays inside shared memory)
-      const uint64_t dK = smem_desc(smem_u32(sm + OFF_K), 16, 1024, 2);         // S^T A
-      const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 1024, 2);                 // S^T B
-      const uint64_t dV = smem_desc(smem_u32(sm + OFF_K), kKRegion, 1024, 2);   // O^T A
-      const uint64_t dP = smem_desc(smem_u32(sm + OFF_P), kKRegion, 1024, 2);   // O^T, L B
-      const uint64_t dOnes = smem_desc(smem_u32(sm + OFF_ONES), 16, 0, 2);      // L A
+      const uint64_t dK = smem_desc(smem_u32(sm + OFF_K), 16, 1024, 2);   // A: key tile
+      const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 1024, 2);           // B: Q tile
       int64_t gblk = 0;
       int n = 0;
       bool ok = true;
-      auto issue_s = [&](int64_t j) -> bool {
-        const int s = (int)(j & 1);
-        if (*abort_flag || !mbar_wait(&kfull[s], (uint32_t)(j >> 1) & 1u)) return false;
-        fence_proxy_async_smem();   // cp.async (generic proxy) writes -> MMA reads
-        tc_fence_after();
-        const uint64_t dKs = dK + (uint64_t)((s * kKTile) >> 4);
-#pragma unroll
-        for (int reg = 0; reg < kRegions; ++reg) {
-#pragma unroll
-          for (int kq = 0; kq < 4; ++kq)
-            mma_bf16_ss(tS0 + 64 * s, dKs + (uint64_t)((reg * kKRegion + kq * 32) >> 4),
-                        dQ + (uint64_t)((reg * kQRegion + kq * 32) >> 4), idS,
-                        (reg | kq) != 0 ? 1u : 0u);
-        }
-        mma_commit(&sfull[s]);
-        return true;
-      };
       for (int64_t it = blockIdx.x; ok && it < a.n_items; it += gridDim.x, ++n) {
         const Item x = decode_item(a, it);
         if (!mbar_wait(&iready[n & 1], (uint32_t)(n >> 1) & 1u)) { ok = false; break; }
@@ -468,44 +476,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ifree[n & 1]);
         if (*abort_flag || !mbar_wait(qload, (uint32_t)n & 1u)) { ok = false; break; }
         tc_fence_after();
+        for (int b = 0; b < nb; ++b) {
+          const int64_t j = gblk + b;
+          const int s = (int)(j & 1);
+          // S^T buffer s is free once the softmax has turned S^T(j-2) into P
+          if ((j >= 2 && !mbar_wait(&pfull[s], (uint32_t)((j - 2) >> 1) & 1u)) || *abort_flag) {
+            ok = false;
+            break;
+          }
+          const uint64_t dKs = dK + (uint64_t)((s * kKTile) >> 4);
+          // each region pair as soon as its gather landed
+#pragma unroll 1
+          for (int h = 0; h < 4 && ok; ++h) {
+            if (*abort_flag || !mbar_wait(&kfull[4 * s + h], (uint32_t)(j >> 1) & 1u)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_smem();   // cp.async (generic proxy) writes -> MMA reads
+            tc_fence_after();
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const int reg = 2 * h + rr;
+#pragma unroll
+              for (int kq = 0; kq < 4; ++kq)
+                mma_bf16_ss(tS0 + 64 * s, dKs + (uint64_t)((reg * kKRegion + kq * 32) >> 4),
+                            dQ + (uint64_t)((reg * kQRegion + kq * 32) >> 4), idS,
+                            (reg | kq) != 0 ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&sfull[s]);
+        }
+        if (!ok) break;
+        mma_commit(qfree);   // the item's S^T MMAs are the Q tile's only readers
+        gblk += nb;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 23u);
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else if (warp == kMmaWarpO) {
+    // ======================= O^T and row-sum issuer
+    if (elect_one()) {
+      constexpr uint32_t idO = idesc_bf16_f32(128, kHG, 1, 1);
+      constexpr uint32_t idL = idesc_bf16_f32(kBK, kHG, 0, 1);
+      const uint64_t dV = smem_desc(smem_u32(sm + OFF_K), kKRegion, 1024, 2);   // O^T A
+      const uint64_t dP = smem_desc(smem_u32(sm + OFF_P), kKRegion, 1024, 2);   // O^T, L B
+      const uint64_t dOnes = smem_desc(smem_u32(sm + OFF_ONES), 16, 0, 2);      // L A
+      int64_t gblk = 0;
+      int n = 0;
+      bool ok = true;
+      for (int64_t it = blockIdx.x; ok && it < a.n_items; it += gridDim.x, ++n) {
+        const Item x = decode_item(a, it);
+        if (!mbar_wait(&iready[n & 1], (uint32_t)(n >> 1) & 1u)) { ok = false; break; }
+        int64_t k_lo, k_hi;
+        const int nb = item_blocks(a, x, nent[n & 1], &k_lo, &k_hi);
+        mbar_arrive(&ifree[n & 1]);
         if (nb == 0) {
-          mma_commit(qfree);
           // keep ofull at most one phase ahead of the epilogue
           if (n > 0 && !mbar_wait(&ofree[3], (uint32_t)(n - 1) & 1u)) { ok = false; break; }
           mma_commit(ofull);
           continue;
         }
-        // S^T of the item's block bi; the item's last one releases Q
-        auto issue_s_item = [&](int bi) -> bool {
-          if (!issue_s(gblk + bi)) return false;
-          if (bi == nb - 1) mma_commit(qfree);
-          return true;
-        };
-        if (!issue_s_item(0)) { ok = false; break; }
-        int next_s = 1;   // next block whose S^T is still to be issued
         for (int b = 0; b < nb; ++b) {
           const int64_t j = gblk + b;
           const int s = (int)(j & 1);
-          // wait for P(j); S^T(j+1) goes first if its key tile lands before
-          // (keeps the tensor pipe busy through softmax(j+1)); never block
-          // O^T(j) on a gather
-          {
-            const uint64_t t0 = globaltimer_ns();
-            for (;;) {
-              if (next_s == b + 1 && next_s < nb &&
-                  mbar_test_wait(&kfull[(j + 1) & 1], (uint32_t)((j + 1) >> 1) & 1u)) {
-                if (!issue_s_item(next_s)) { ok = false; break; }
-                ++next_s;
-              }
-              if (mbar_try_wait_sleep(&pfull[s], (uint32_t)(j >> 1) & 1u, 256u)) break;
-              if (*abort_flag || globaltimer_ns() - t0 > 2000000000ull) { ok = false; break; }
-            }
-            if (!ok) break;
-          }
+          if (*abort_flag || !mbar_wait(&pfull[s], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
           tc_fence_after();
           const uint64_t dVs = dV + (uint64_t)((s * kKTile) >> 4);
           const uint64_t dPs = dP + (uint64_t)((s * kPTile) >> 4);
+          // L[., h] += sum over the block's keys of P^T[key, h]: A = 64 rows of
+          // ones (stride 0 repeats one 8-row group), B = the P^T tile.  Issued
+          // first, so the last slice's commit covers every reader of P tile s
 #pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16_ss(tL, dOnes + (uint64_t)((kk * 32) >> 4), dPs + (uint64_t)((kk * 2048) >> 4),
+                        idL, (b > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll 1
           for (int jt = 0; jt < 4; ++jt) {
             // the item's first block overwrites O^T: wait for the epilogue to
             // have read the previous item's columns of this slice
@@ -517,20 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kBK / 16; ++kk)
               mma_bf16_ss(tO + 64 * jt, dVs + (uint64_t)((2 * jt * kKRegion + kk * 2048) >> 4),
                           dPs + (uint64_t)((kk * 2048) >> 4), idO, (b > 0 || kk > 0) ? 1u : 0u);
+            // regions 2 jt, 2 jt + 1 of key tile s read (S^T(j) finished before P(j))
+            mma_commit(&bfree[4 * s + jt]);
           }
           if (!ok) break;
-          // L[., h] += sum over the block's keys of P^T[key, h]: A = 64 rows of
-          // ones (stride 0 repeats one 8-row group), B = the P^T tile; the
-          // epilogue reads L before the first O^T slice
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ss(tL, dOnes + (uint64_t)((kk * 32) >> 4), dPs + (uint64_t)((kk * 2048) >> 4),
-                        idL, (b > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bfree[s]);
-          if (next_s == b + 1 && next_s < nb) {
-            if (!issue_s_item(next_s)) { ok = false; break; }
-            ++next_s;
-          }
         }
         if (!ok) break;
         mma_commit(ofull);
@@ -538,10 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         *abort_flag = 1;
-        report(a.status, CSA_DEV_TIMEOUT, 23u);
+        report(a.status, CSA_DEV_TIMEOUT, 28u);
       }
-      mma_commit(drain);
-      mbar_wait(drain, 0);
+      mma_commit(drain_o);
+      mbar_wait(drain_o, 0);
     }
   } else if (warp < 4) {
     // ======================= softmax (warps 0-3)
@@ -692,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             wds[2 * q + 1] = ev1 | (od1 << 16);
           }
         }
-        wait_or_die(&bfree[s], ph ^ 1u, 25u);   // O^T(j-2) has read this P tile
+        wait_or_die(&bfree[4 * s + 3], ph ^ 1u, 25u);   // O^T(j-2) has read this P tile
         if (!dead) {
           uint8_t* prow = sm + OFF_P + s * kPTile + kb_row * 128;
 #pragma unroll

@@ -161,6 +161,19 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Per-warpgroup register budget changes (every warp of a warpgroup executes
+// the same one).  An increase waits until decreases elsewhere in the CTA have
+// returned enough registers: the budgets after all changes must add up to no
+// more than the CTA was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
