@@ -825,9 +825,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(3, 128);
 
       // O^T -> output: thread = dim 128 jt + 32 ew + lane
-      float iv[kHG];
-#pragma unroll
-      for (int h = 0; h < kHG; ++h) iv[h] = a.split ? 1.f : sinv[h];
       const int odd = lane & 1;
 #pragma unroll 1
       for (int jt = 0; jt < 4; ++jt) {
@@ -858,8 +855,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
               const int h = 32 * half + e;
-              const float v0 = __uint_as_float(ov[e]) * iv[h];
-              const float v1 = __uint_as_float(ov[e + 1]) * iv[h + 1];
+              const float v0 = __uint_as_float(ov[e]) * sinv[h];   // broadcast reads
+              const float v1 = __uint_as_float(ov[e + 1]) * sinv[h + 1];
               // even lane keeps head h and receives its neighbour's dim; odd lane head h+1
               const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
               const float x0 = odd ? recv : v0;
