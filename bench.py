@@ -284,6 +284,7 @@ def run_gpu(args):
     decode = {} if args.no_decode else {
         n: measure_decode(n, dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
         for n in DECODE_WORKLOADS}
+    comp_1m = None if args.no_decode else measure_compress_1m(dev, min(K, 10), args.warmup)
 
     hbm, bf16, src = peaks()
     tokens = w.B * w.T
@@ -335,6 +336,8 @@ def run_gpu(args):
         }
         if decode:
             line["decode"] = decode
+        if comp_1m:
+            line["compress_1m_tokens"] = comp_1m
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
         print(json.dumps(line), flush=True)
@@ -513,6 +516,48 @@ def graph_ms(fn, steps: int, flush) -> float:
     ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     del g
     return ms
+
+
+def measure_compress_1m(dev, steps: int, warmup: int):
+    """CSA (m = 4) and HCA (m' = 128) compression alone at 2^20 tokens, c = 512
+    bf16, window rows written: inputs of 2-4 GiB (far larger than L2), so
+    the kernels' HBM bandwidth shows without launch overhead (the 8192-token
+    workload moves only 42 MB).  Algorithmic bytes: every input read once,
+    entries and window rows written once."""
+    T, c = 1 << 20, 512
+    fmt = csa.Fmt(c=c, rope_dims=64)
+    hbm, _, src = peaks()
+    res = {}
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    x = [wl.randn((1, T, c), 100 + i, dev, dtype=torch.bfloat16) for i in range(4)]
+    ent = torch.empty((1, T // 4, c), dtype=torch.bfloat16, device=dev)
+    win = torch.empty((1, T, c), dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: csa.csa_compress(x[0], x[1], x[2], x[3], 4, fmt, entries=ent, win_out=win))
+    nb = (4 * T + T // 4 + T) * c * 2
+    res["csa_compress"] = {"ms": ms, "bytes": nb, "GBps": nb / ms / 1e6, "frac": nb / ms / 1e6 / hbm}
+    del x, ent
+    x = [wl.randn((1, T, c), 110 + i, dev, dtype=torch.bfloat16) for i in range(2)]
+    ent = torch.empty((1, T // 128, c), dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: csa.hca_compress(x[0], x[1], 128, fmt, entries=ent, win_out=win))
+    nb = (2 * T + T // 128 + T) * c * 2
+    res["hca_compress"] = {"ms": ms, "bytes": nb, "GBps": nb / ms / 1e6, "frac": nb / ms / 1e6 / hbm}
+    del x, ent, win
+    torch.cuda.empty_cache()
+    res["config"] = {"tokens": T, "entry_dim": c, "dtype": "bf16", "window_rows": True,
+                     "peak": f"{src} HBM copy {hbm} GB/s"}
+    return res
 
 
 def decode_cpu_baseline(w, queries: int):
