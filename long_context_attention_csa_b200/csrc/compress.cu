@@ -25,17 +25,8 @@ namespace csa {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr double kTwoPi = 6.283185307179586476925286766559;
 constexpr int kWarps = 8;   // warps per CTA
 
-// cos/sin of pos * theta: the angle is formed and reduced modulo 2*pi in
-// double precision (positions up to 2^20 keep full accuracy), then evaluated
-// in single precision on [-pi, pi].
-__device__ __forceinline__ void rope_angle(int64_t pos, double theta, float* cs, float* sn) {
-  double ang = (double)pos * theta;
-  ang -= kTwoPi * rint(ang * (1.0 / kTwoPi));
-  sincosf((float)ang, sn, cs);
-}
 
 // Load CPL consecutive elements as float (CPL * sizeof(T) bytes, aligned).
 template <typename T, int CPL>
@@ -127,7 +118,7 @@ __device__ __forceinline__ void norm_rope_row(float* v, int lane, const Fmt& f, 
         const int ch = ch0 + e;
         if (ch >= d0) {
           float cs, sn;
-          rope_angle(pos, theta[(ch - d0) >> 1], &cs, &sn);
+          rope_cos_sin_theta(pos, theta[(ch - d0) >> 1], &cs, &sn);
           const float x0 = v[e], x1 = v[e + 1];
           v[e] = x0 * cs - x1 * sn;
           v[e + 1] = x0 * sn + x1 * cs;
@@ -372,7 +363,7 @@ __device__ __forceinline__ void fill_rope_table(float2* tab, int rows, int r, co
     const int i = q >> 5, pr = q & 31;
     if (pr < np) {
       float cs, sn;
-      rope_angle(pos(i), theta[pr], &cs, &sn);
+      rope_cos_sin_theta(pos(i), theta[pr], &cs, &sn);
       tab[q] = make_float2(cs, sn);
     }
   }
