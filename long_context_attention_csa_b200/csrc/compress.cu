@@ -293,7 +293,10 @@ constexpr int kFC = 512;                    // channels
 constexpr int kFRowB = kFC * 2;             // bytes per token row
 constexpr int kFThreads = 256;
 constexpr int kFTab = 2048 + 64;            // RoPE cos/sin table: [rows][32 pairs] float2
-constexpr int kFHead = 8192;                // frequencies (256 doubles), reductions, table
+constexpr int kFDelta = 8192;               // (cos, sin) of i * theta, i < 16: [16][32] float2
+constexpr int kFBase = kFDelta + 16 * 32 * 8;   // a chunk's row-0 (cos, sin): [32] float2
+constexpr int kFHead = 13312;               // frequencies, reductions, tables
+static_assert(kFTab + 17 * 32 * 8 <= kFDelta && kFBase + 32 * 8 <= kFHead, "head layout");
 
 // Window row from a staged token row: RoPE_pos(RMSNorm(row)).  Lane l owns the
 // 16-byte chunks l and l + 32 (channels 8l..8l+7 and 256+8l..256+8l+7), so a
@@ -353,18 +356,37 @@ __device__ __forceinline__ void osm_step(float z, float v, float& mx, float& den
   mx = fmaxf(mx, zl);
 }
 
-// cos/sin of the RoPE pairs at `rows` positions (row i at position pos(i)) into
-// tab[i][pair]; every thread of the CTA takes a share.
-template <typename PosFn>
-__device__ __forceinline__ void fill_rope_table(float2* tab, int rows, int r, const double* theta,
-                                                PosFn pos) {
+// Per-CTA table of (cos, sin) of i * theta_pr, i < 16: a chunk's table rows are
+// positions p0 + i, so each is the row-0 angle rotated by one of these.
+__device__ __forceinline__ void fill_delta_table(float2* dtab, int r, const double* theta) {
+  for (int q = threadIdx.x; q < 16 * 32; q += kFThreads) {
+    const int i = q >> 5, pr = q & 31;
+    float cs = 1.f, sn = 0.f;
+    if (pr < (r >> 1)) rope_cos_sin_theta(i, theta[pr], &cs, &sn);
+    dtab[q] = make_float2(cs, sn);
+  }
+}
+
+// tab[i][pr] = (cos, sin) of (p0 + delta(i)) theta_pr for i < rows, with
+// delta(i) < 16: warp 0 forms the row-0 angles (double-reduced), then every
+// thread takes a share of the complex products with the delta table.  Every
+// thread of the CTA calls this (it holds a barrier).
+template <typename DeltaFn>
+__device__ __forceinline__ void fill_rope_rows(float2* tab, float2* base, const float2* dtab,
+                                               int rows, int r, const double* theta, int64_t p0,
+                                               DeltaFn delta) {
   const int np = r >> 1;
+  if (threadIdx.x < np) {
+    float cs, sn;
+    rope_cos_sin_theta(p0, theta[threadIdx.x], &cs, &sn);
+    base[threadIdx.x] = make_float2(cs, sn);
+  }
+  __syncthreads();
   for (int q = threadIdx.x; q < rows * 32; q += kFThreads) {
     const int i = q >> 5, pr = q & 31;
     if (pr < np) {
-      float cs, sn;
-      rope_cos_sin_theta(pos(i), theta[pr], &cs, &sn);
-      tab[q] = make_float2(cs, sn);
+      const float2 b = base[pr], d = dtab[delta(i) * 32 + pr];
+      tab[q] = make_float2(b.x * d.x - b.y * d.y, b.x * d.y + b.y * d.x);
     }
   }
 }
@@ -381,11 +403,15 @@ __global__ void __launch_bounds__(kFThreads, 2)
   double* theta = reinterpret_cast<double*>(fsm);
   float* red = reinterpret_cast<float*>(fsm + 2048);   // [8]
   float2* tab = reinterpret_cast<float2*>(fsm + kFTab); // rows 0-7 window, 8-9 entries
+  float2* dtab = reinterpret_cast<float2*>(fsm + kFDelta);
+  float2* rbase = reinterpret_cast<float2*>(fsm + kFBase);
   uint8_t* ring = fsm + kFHead;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int i = t; i < (p.f.r >> 1); i += kFThreads)
     theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
-  __syncthreads();   // frequencies complete before the first table fill
+  __syncthreads();   // frequencies complete before the tables
+  if (!(p.f.flags & CSA_F_NO_ROPE)) fill_delta_table(dtab, p.f.r, theta);
+  __syncthreads();
   const uint32_t ring_s = sm100::smem_u32(ring);
   const bf16* kva = static_cast<const bf16*>(p.kv_a);
   const bf16* kvb = static_cast<const bf16*>(p.kv_b);
@@ -413,9 +439,10 @@ __global__ void __launch_bounds__(kFThreads, 2)
   for (uint32_t u = blockIdx.x; u < total; u += gridDim.x, ++k) {
     issue(u + (kCStages - 1) * gridDim.x, (k + kCStages - 1) % kCStages);
     const int64_t b = u / n_chunks, t0 = (int64_t)(u % n_chunks) * kCR;
+    // rows 0-7: the chunk's tokens; rows 8-9: its two entries (at t0, t0 + 4)
     if (!(p.f.flags & CSA_F_NO_ROPE))
-      fill_rope_table(tab, kCR + 2, p.f.r, theta,
-                      [&](int i) { return p.pos0 + (i < kCR ? t0 + i : t0 + 4 * (i - kCR)); });
+      fill_rope_rows(tab, rbase, dtab, kCR + 2, p.f.r, theta, p.pos0 + t0,
+                     [](int i) { return i < kCR ? i : 4 * (i - kCR); });
     sm100::cp_async_wait<kCStages - 1>();
     __syncthreads();
     const uint8_t* buf = ring + (k % kCStages) * kCStage;
@@ -498,11 +525,15 @@ __global__ void __launch_bounds__(kFThreads, 2)
   double* theta = reinterpret_cast<double*>(fsm);
   float* red = reinterpret_cast<float*>(fsm + 2048);   // [8]
   float2* tab = reinterpret_cast<float2*>(fsm + kFTab); // rows 0-15 window, 16 entry
+  float2* dtab = reinterpret_cast<float2*>(fsm + kFDelta);
+  float2* rbase = reinterpret_cast<float2*>(fsm + kFBase);
   uint8_t* ring = fsm + kFHead;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int i = t; i < (p.f.r >> 1); i += kFThreads)
     theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
-  __syncthreads();   // frequencies complete before the first table fill
+  __syncthreads();   // frequencies complete before the tables
+  if (!(p.f.flags & CSA_F_NO_ROPE)) fill_delta_table(dtab, p.f.r, theta);
+  __syncthreads();
   const uint32_t ring_s = sm100::smem_u32(ring);
   const bf16* kv = static_cast<const bf16*>(p.kv_a);
   const bf16* z = static_cast<const bf16*>(p.z_a);
@@ -533,9 +564,16 @@ __global__ void __launch_bounds__(kFThreads, 2)
     const uint32_t u = blockIdx.x + (kk / cpu) * gridDim.x;
     const int j = (int)(kk % cpu);
     const int64_t b = u / n_blocks, s = u % n_blocks, t0 = s * p.m + (int64_t)j * kHR;
-    if (!(p.f.flags & CSA_F_NO_ROPE))
-      fill_rope_table(tab, kHR + 1, p.f.r, theta,
-                      [&](int i) { return p.pos0 + (i < kHR ? t0 + i : s * p.m); });
+    // rows 0-15: the chunk's tokens; row 16: the block's entry (at s m'), on
+    // the block's last chunk only, where the entry is finished
+    if (!(p.f.flags & CSA_F_NO_ROPE)) {
+      fill_rope_rows(tab, rbase, dtab, kHR, p.f.r, theta, p.pos0 + t0, [](int i) { return i; });
+      if (j == cpu - 1 && t < (p.f.r >> 1)) {
+        float cs, sn;
+        rope_cos_sin_theta(p.pos0 + s * p.m, theta[t], &cs, &sn);
+        tab[kHR * 32 + t] = make_float2(cs, sn);
+      }
+    }
     sm100::cp_async_wait<kHStages - 1>();
     __syncthreads();
     const uint8_t* buf = ring + (kk % kHStages) * kHStage;
