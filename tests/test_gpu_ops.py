@@ -353,6 +353,73 @@ def test_decode_batch_invariance():
     assert torch.equal(again, full)
 
 
+def test_decode_mixed_contexts_and_invariance():
+    """Decode rows of very different context lengths in one batch (the split
+    size follows each row's own key count, so short rows leave splits empty
+    and the index lists padded): parity with the oracle for the CSA layer
+    (sparse) and the HCA layer (dense), and each row bitwise equal alone."""
+    w = wl.WORKLOADS["decode_pair_b4_1m"]
+    H, c, n_win = w.H, w.c, w.n_win
+    L = [131072, 9000, 1300, 50]
+    B = len(L)
+    N, NH = 32768, 8192
+    q = wl.randn((B, 1, H, c), 61, DEV, dtype=torch.bfloat16)
+    ent = wl.randn((B, N, c), 62, DEV, dtype=torch.bfloat16)
+    hent = wl.randn((B, NH, c), 63, DEV, dtype=torch.bfloat16)
+    win = wl.randn((B, n_win, c), 64, DEV, dtype=torch.bfloat16)
+    sink = wl.randn((H,), 65, DEV)
+    q_pos = torch.tensor([[x - 1] for x in L], dtype=torch.int64, device=DEV)
+    wp0 = torch.tensor([max(x - n_win, 0) for x in L], dtype=torch.int64, device=DEV)
+    idx = torch.stack([wl.random_index_sets(torch.tensor([oracle.visible(x - 1, w.m, N)]), w.k,
+                                            70 + b) for b, x in enumerate(L)]).to(DEV)
+    fmt = gfmt(w)
+    outs = csa.sparse_mqa_attn(q, ent, idx, win, fmt, n_win, sink=sink, q_pos=q_pos, win_pos0=wp0)
+    outd = csa.dense_hca_attn(q, hent, w.m_prime, win, fmt, n_win, sink=sink, q_pos=q_pos,
+                              win_pos0=wp0)
+    torch.cuda.synchronize()
+    for b in range(B):
+        pos = q_pos[b].cpu().numpy()
+        refs = oracle.attention(f64(q[b]), f64(ent[b]), f64(win[b]), ofmt(w), n_win,
+                                idx=idx[b].cpu().numpy(), sink=f64(sink), q_pos=pos,
+                                win_pos0=int(wp0[b]))
+        assert_close(outs[b], refs, w.dtype, f"sparse decode L={L[b]}")
+        refd = oracle.attention(f64(q[b]), f64(hent[b]), f64(win[b]), ofmt(w), n_win,
+                                m_dense=w.m_prime, sink=f64(sink), q_pos=pos, win_pos0=int(wp0[b]))
+        assert_close(outd[b], refd, w.dtype, f"dense decode L={L[b]}")
+        sl = slice(b, b + 1)
+        one_s = csa.sparse_mqa_attn(q[sl].contiguous(), ent[sl].contiguous(), idx[sl].contiguous(),
+                                    win[sl].contiguous(), fmt, n_win, sink=sink,
+                                    q_pos=q_pos[sl].contiguous(), win_pos0=wp0[sl].contiguous())
+        one_d = csa.dense_hca_attn(q[sl].contiguous(), hent[sl].contiguous(), w.m_prime,
+                                   win[sl].contiguous(), fmt, n_win, sink=sink,
+                                   q_pos=q_pos[sl].contiguous(), win_pos0=wp0[sl].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(one_s[0], outs[b]), f"sparse row {b} differs alone"
+        assert torch.equal(one_d[0], outd[b]), f"dense row {b} differs alone"
+
+
+def test_sparse_with_every_visible_entry_equals_dense():
+    """k >= vis(t) with the index list of every visible entry: sparse MQA over
+    the selection equals dense MQA with m' = m over the same entries (the
+    method's own reduction, here through the two GPU entry points)."""
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=600)
+    B, T, H, c, m = 1, w.T, w.H, w.c, w.m
+    N = T // m
+    q = wl.randn((B, T, H, c), 81, DEV, dtype=torch.bfloat16)
+    ent = wl.randn((B, N, c), 82, DEV, dtype=torch.bfloat16)
+    win = wl.randn((B, T, c), 83, DEV, dtype=torch.bfloat16)
+    sink = wl.randn((H,), 84, DEV)
+    idx = torch.full((B, T, N), -1, dtype=torch.int32)
+    for t in range(T):
+        v = oracle.visible(t, m, N)
+        idx[0, t, :v] = torch.arange(v, dtype=torch.int32)
+    idx = idx.to(DEV)
+    outs = csa.sparse_mqa_attn(q, ent, idx, win, gfmt(w), w.n_win, sink=sink)
+    outd = csa.dense_hca_attn(q, ent, m, win, gfmt(w), w.n_win, sink=sink)
+    torch.cuda.synchronize()
+    assert_close(outs[0], f64(outd[0]), w.dtype, "sparse(all visible) vs dense", roundings=2)
+
+
 # ----------------------------------------------------------------- whole layer
 
 @pytest.mark.parametrize("wname,T,k", [("tiny_csa_fp32", 256, 16), ("csa_prefill_8k", 512, 64)])
