@@ -909,20 +909,28 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(TcAttnArgs a) {
     sn_t[threadIdx.x - 32] = sn;
   }
   __syncthreads();
-  // thread: 4 consecutive dims of one head, 4 times (16-byte loads)
+  // thread: 4 consecutive dims of one head, 4 times (16-byte loads); every
+  // split's load is issued before the first is added (fixed order kept)
   constexpr int kQuads = kCombHeads * kC / 4;   // 1024
-#pragma unroll
+#pragma unroll 1
   for (int r = 0; r < kQuads / 256; ++r) {
     const int q = threadIdx.x + 256 * r;
     const int hl = q / (kC / 4), c = (q % (kC / 4)) * 4;
+    float4 pv[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+      if (s < a.n_splits)
+        pv[s] = *reinterpret_cast<const float4*>(
+            a.o_part + ((slot * a.n_splits + s) * kHG + h0 + hl) * kC + c);
     float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < a.n_splits; ++s) {
-      const float4 v = *reinterpret_cast<const float4*>(
-          a.o_part + ((slot * a.n_splits + s) * kHG + h0 + hl) * kC + c);
-      o[0] += v.x;
-      o[1] += v.y;
-      o[2] += v.z;
-      o[3] += v.w;
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      if (s < a.n_splits) {
+        o[0] += pv[s].x;
+        o[1] += pv[s].y;
+        o[2] += pv[s].z;
+        o[3] += pv[s].w;
+      }
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[e] *= inv[hl];
