@@ -36,12 +36,16 @@
 // bf16 weights come from the tensor core too (a ones tile times P^T), so the
 // denominators match the numerators' rounding.
 //
-// Persistent CTAs (one per SM) walk their items in turn; roles (384 threads,
-// the register budget of 288 threads since allocation is per 128 threads):
-//   warps 8-10 producer: index compaction, RoPE table, the item's raw q rows
-//              by TMA, the key gather (cp.async; each warp-instruction moves
-//              four 128-byte row pieces);
-//   warp 11    TMEM owner and single-thread MMA issuer;
+// Persistent CTAs (one per SM) walk their items in turn; 512 threads in four
+// warpgroups, whose register budgets are rebalanced at the start (softmax and
+// epilogue up, producers and issuers down):
+//   warps 8-10, 12-14 producer: index compaction, RoPE table, the item's raw
+//              q rows by TMA, the key gather (cp.async; each warp-instruction
+//              moves four 128-byte row pieces), 128-dim region pair by region
+//              pair as the tile's previous block releases them;
+//   warp 11    TMEM owner and S^T issuer (each region pair as it lands);
+//   warp 15    O^T and row-sum issuer (a commit per 128-dim O^T slice frees
+//              that region pair of the key tile);
 //   warps 0-3  softmax (all 32 lanes: the 16x64b TMEM load gives each lane
 //              one key and the 32 heads of one parity); at an item's start
 //              they rotate the Q tile's RoPE dims in place as soon as the raw
