@@ -191,8 +191,9 @@ class Step:
         self.ws_attn = csa.workspace(csa.csa_workspace_bytes(
             csa.CSA_OP_SPARSE_ATTN, w.dtype, B, T, w.H, c, w.n_csa, w.k, w.n_win), device)
 
-    def run(self, inp=None, ev=None):
+    def run(self, inp=None, ev=None, out=None):
         inp = inp or self.inp
+        out = self.out if out is None else out
         w = self.w
         s = torch.cuda.current_stream()
         if ev:
@@ -206,10 +207,10 @@ class Step:
         if ev:
             ev[2].record(s)
         csa.sparse_mqa_attn(inp["q"], self.entries, self.idx, self.win, self.fmt, w.n_win,
-                            sink=inp["sink"], out=self.out, ws=self.ws_attn)
+                            sink=inp["sink"], out=out, ws=self.ws_attn)
         if ev:
             ev[3].record(s)
-        return self.out
+        return out
 
 
 def run_gpu(args):
@@ -248,38 +249,63 @@ def run_gpu(args):
     step_ms = allmax(float(per[:, 3].mean()), ws)
     t_compress, t_index, t_attn = (float(per[:, i].mean()) for i in range(3))
 
-    # e2e through the public API: pinned host inputs -> device, step, result -> host
+    # e2e through the public API: every step copies its inputs from pinned host
+    # memory to the device, runs, and copies its output back to pinned host
+    # memory.  Steps are pipelined over three streams with two sets of device
+    # inputs and outputs: step i+1's inputs upload while step i computes and
+    # step i-1's output downloads (the copy engines of the two directions
+    # work at once); every buffer is reused only after the event of its last
+    # user.  Timed from the first upload to the last download.
     host = {k: (v.to("cpu").pin_memory() if v is not None else None) for k, v in step.inp.items()}
-    dev_in = {k: (torch.empty_like(v, device=dev) if v is not None else None)
-              for k, v in host.items()}
-    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    dev_in = [{k: (torch.empty_like(v, device=dev) if v is not None else None)
+               for k, v in host.items()} for _ in range(2)]
+    dev_out = [step.out, torch.empty_like(step.out)]
+    out_host = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = out_host.numel() * out_host.element_size()
-    e2e_steps = max(1, min(K, 5))
-    for _ in range(2):
-        for kk, v in host.items():
-            if v is not None:
-                dev_in[kk].copy_(v, non_blocking=True)
-        step.run(dev_in)
-        out_host.copy_(step.out, non_blocking=True)
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    e2e_steps = max(2, min(K, 6))
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def pipelined(n):
+        ev_up = [torch.cuda.Event() for _ in range(n)]
+        ev_comp = [torch.cuda.Event() for _ in range(n)]
+        ev_down = [torch.cuda.Event() for _ in range(n)]
+        for i in range(n):
+            j = i & 1
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(ev_comp[i - 2])      # dev_in[j] no longer read
+                for kk, v in host.items():
+                    if v is not None:
+                        dev_in[j][kk].copy_(v, non_blocking=True)
+                ev_up[i].record(up)
+            comp.wait_event(ev_up[i])
+            if i >= 2:
+                comp.wait_event(ev_down[i - 2])        # dev_out[j] downloaded
+            step.run(dev_in[j], out=dev_out[j])
+            ev_comp[i].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_comp[i])
+                out_host[j].copy_(dev_out[j], non_blocking=True)
+                ev_down[i].record(down)
+        return ev_down[n - 1]
+
+    pipelined(2)
     torch.cuda.synchronize()
     barrier(ws)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        for kk, v in host.items():
-            if v is not None:
-                dev_in[kk].copy_(v, non_blocking=True)
-        step.run(dev_in)
-        out_host.copy_(step.out, non_blocking=True)
-    e1.record()
+    e0.record(up)
+    last = pipelined(e2e_steps)
+    down.wait_event(last)
+    e1.record(down)
     torch.cuda.synchronize()
     e2e_ms = allmax(e0.elapsed_time(e1) / e2e_steps, ws)
     st, d = csa.csa_check_status(step.ws_attn)
     if st:
         raise RuntimeError(f"device status after timing: {st}/{d}")
 
-    del step, dev_in, host
+    del step, dev_in, dev_out, host, out_host
     torch.cuda.empty_cache()
     decode = {} if args.no_decode else {
         n: measure_decode(n, dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
@@ -330,7 +356,11 @@ def run_gpu(args):
                          if src == "measured" else "fallback 1.59 PFLOP/s",
                          "algorithmic_flops_per_launch": fl_attn},
             "e2e": {"value": tokens * ws / (e2e_ms * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps,
+                    "schedule": "pinned host <-> device copies every step, pipelined over three "
+                                "streams (uploads of step i+1 and the download of step i-1 "
+                                "overlap step i)"},
             "gpu_launches": int(launches),
             "clocks": ck,
         }
