@@ -159,9 +159,11 @@ def dist_setup():
 
 
 def allmax(x: float, ws: int) -> float:
+    """Max over ranks (every rank calls it, in the same order)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
