@@ -220,6 +220,18 @@ size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int
  */
 csa_status csa_check_status(void* ws, void* stream, uint32_t* detail);
 
+/*
+ * Failure-path self test: one CTA waits on an mbarrier that nothing
+ * arrives on, with the same bounded wait every kernel here uses but a limit of
+ * limit_ns nanoseconds (1e3 .. 1e10).  The wait runs out; the kernel
+ * records CSA_DEV_TIMEOUT in the status word of `ws` (at least 256 bytes) and
+ * returns, and the context stays usable.  csa_check_status() then reports
+ * CSA_E_DEVICE with detail CSA_DEV_TIMEOUT.  Asynchronous on `stream`.
+ * Errors: CSA_E_ARG (null ws, ws_bytes < 256, limit out of range),
+ * CSA_E_CUDA.
+ */
+csa_status csa_selftest_wait(int64_t limit_ns, void* ws, size_t ws_bytes, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* csa_status_string(csa_status s);
 

@@ -30,6 +30,7 @@ CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX = 1, 2, 3
 EXPORTED = (
     "csa_compress", "hca_compress", "indexer_scores_topk", "sparse_mqa_attn", "dense_hca_attn",
     "csa_workspace_bytes", "csa_check_status", "csa_status_string", "csa_launch_count",
+    "csa_selftest_wait",
 )
 
 
@@ -95,10 +96,11 @@ def lib():
     L.csa_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     L.csa_status_string.argtypes = [i32]
     L.csa_status_string.restype = ctypes.c_char_p
+    L.csa_selftest_wait.argtypes = [i64, P, sz, P]
     L.csa_launch_count.argtypes = []
     L.csa_launch_count.restype = ctypes.c_ulonglong
     for fn in ("csa_compress", "hca_compress", "indexer_scores_topk", "sparse_mqa_attn",
-               "dense_hca_attn", "csa_check_status"):
+               "dense_hca_attn", "csa_check_status", "csa_selftest_wait"):
         getattr(L, fn).restype = i32
     _lib = L
     return L
@@ -148,6 +150,14 @@ def csa_check_status(ws: torch.Tensor, stream=None) -> tuple[int, int]:
     d = ctypes.c_uint32(0)
     st = lib().csa_check_status(_p(ws), _s(stream), ctypes.byref(d))
     return int(st), int(d.value)
+
+
+def csa_selftest_wait(limit_ns: int, ws: torch.Tensor, stream=None) -> None:
+    """Failure-path self test: a device wait that nothing satisfies runs out
+    after limit_ns and records CSA_DEV_TIMEOUT in ws's status word."""
+    st = lib().csa_selftest_wait(int(limit_ns), _p(ws), ws.numel() * ws.element_size(), _s(stream))
+    if st != CSA_OK:
+        raise CSAError(st, "csa_selftest_wait")
 
 
 def csa_launch_count() -> int:

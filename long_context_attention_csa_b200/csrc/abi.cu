@@ -4,6 +4,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "sm100.cuh"
 #include "internal.h"
 #include "tc.h"
 
@@ -230,6 +231,28 @@ csa_status dense_hca_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const
                           size_t ws_bytes, void* stream) {
   return attn_common(dtype, B, Tq, H, fmt, false, q, q_pos, entries, N, nullptr, 0, m_prime, win,
                      Tw, win_pos0, n_win, sink, scale, out, ws, ws_bytes, stream);
+}
+
+namespace {
+// One thread waits, bounded, on a barrier that no thread ever arrives on.
+__global__ void selftest_wait_kernel(unsigned* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !sm100::mbar_wait(&bar, 0u, limit_ns))
+    report(status, CSA_DEV_TIMEOUT, 0x5e1fu);
+}
+}  // namespace
+
+csa_status csa_selftest_wait(int64_t limit_ns, void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsScratch || limit_ns < 1000 || limit_ns > 10000000000LL)
+    return CSA_E_ARG;
+  selftest_wait_kernel<<<1, 32, 0, S(stream)>>>(status_word(ws), (uint64_t)limit_ns);
+  g_launches.fetch_add(1);
+  return cuda_status(cudaGetLastError());
 }
 
 csa_status csa_check_status(void* ws, void* stream, uint32_t* detail) {

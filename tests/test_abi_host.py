@@ -128,3 +128,13 @@ def test_indexer_and_attention_reject_bad_arguments(L):
                             None, 0.0, d, None, 0, None) == 5
     assert L.dense_hca_attn(1, 1, 1, 64, ctypes.byref(f), d, None, d, 16, 0, d, 8, None, 8, None,
                             0.0, d, d, 1 << 20, None) == 1
+
+
+def test_selftest_wait_rejects_bad_arguments(L):
+    """The failure-path self test checks its arguments before any CUDA call."""
+    import ctypes
+    buf = (ctypes.c_uint8 * 256)()
+    assert L.csa_selftest_wait(10 ** 6, None, 256, None) == 1             # null workspace
+    assert L.csa_selftest_wait(10 ** 6, ctypes.addressof(buf), 128, None) == 1   # too small
+    assert L.csa_selftest_wait(10, ctypes.addressof(buf), 256, None) == 1        # limit too short
+    assert L.csa_selftest_wait(10 ** 11, ctypes.addressof(buf), 256, None) == 1  # too long

@@ -420,6 +420,25 @@ def test_sparse_with_every_visible_entry_equals_dense():
     assert_close(outs[0], f64(outd[0]), w.dtype, "sparse(all visible) vs dense", roundings=2)
 
 
+def test_device_wait_timeout_is_reported_and_the_context_survives():
+    """A bounded device wait that nothing satisfies runs out (50 ms), the
+    kernel records CSA_DEV_TIMEOUT and returns; the host reads and clears the
+    status, and the next calls run and are correct."""
+    ws = csa.workspace(256)
+    csa.csa_selftest_wait(50_000_000, ws)
+    st, d = csa.csa_check_status(ws)
+    assert st == csa.CSA_E_DEVICE and d == csa.CSA_DEV_TIMEOUT
+    st, d = csa.csa_check_status(ws)
+    assert st == csa.CSA_OK and d == 0
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=64)
+    inp = wl.csa_prefill_inputs(w, DEV)
+    ent = csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, gfmt(w))
+    torch.cuda.synchronize()
+    ref = oracle.csa_compress(f64(inp["kv_a"][0]), f64(inp["kv_b"][0]), f64(inp["z_a"][0]),
+                              f64(inp["z_b"][0]), w.m, ofmt(w))
+    assert_close(ent[0], ref, w.dtype, "entries after the timeout")
+
+
 # ----------------------------------------------------------------- whole layer
 
 @pytest.mark.parametrize("wname,T,k", [("tiny_csa_fp32", 256, 16), ("csa_prefill_8k", 512, 64)])
