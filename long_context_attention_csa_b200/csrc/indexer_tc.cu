@@ -648,6 +648,14 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   constexpr int NW = NT / 32;
   if (k <= 0) return;   // uniform over the cluster
+  // a cluster of one CTA: CTA barriers and local loads do
+  const bool solo = CL == 1;
+  auto csync = [&]() {
+    if (solo) __syncthreads(); else cluster_sync();
+  };
+  auto rd = [&](const unsigned* local, uint32_t r) -> unsigned {
+    return solo ? *reinterpret_cast<const volatile unsigned*>(local) : dsmem_ld_u32(local, r);
+  };
 
   for (int i = tid; i < 3 * kSelBins; i += NT) (&sh.hist[0][0])[i] = 0u;
   unsigned cnt = 0, kmin = 0xffffffffu, kmax = 0u;
@@ -671,15 +679,15 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
     sh.red[1][wid] = kmin;
     sh.red[2][wid] = kmax;
   }
-  cluster_sync();
+  csync();
   if (wid == 0) {
     unsigned c = 0, lo = 0xffffffffu, hi = 0u;
     for (int i = lane; i < (int)CL * NW; i += 32) {
       const uint32_t r = (uint32_t)(i / NW);
       const int w = i % NW;
-      c += dsmem_ld_u32(&sh.red[0][w], r);
-      lo = min(lo, dsmem_ld_u32(&sh.red[1][w], r));
-      hi = max(hi, dsmem_ld_u32(&sh.red[2][w], r));
+      c += rd(&sh.red[0][w], r);
+      lo = min(lo, rd(&sh.red[1][w], r));
+      hi = max(hi, rd(&sh.red[2][w], r));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -717,13 +725,17 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
           if ((key & M) == P) atomicAdd(&h[(key >> shift) & dmask], 1u);
         }
       }
-      cluster_sync();
+      csync();
       // bucket search: thread t owns bins 2047-4t .. 2044-4t (descending),
       // summed over the cluster (every rank's load issued before any is used)
       uint4 x[kSelMaxCluster];
+      if (solo) {
+        x[0] = *reinterpret_cast<const uint4*>(&h[kSelBins - 4 * (tid + 1)]);
+      } else {
 #pragma unroll
-      for (int r = 0; r < kSelMaxCluster; ++r)
-        if ((uint32_t)r < CL) x[r] = dsmem_ld_u32x4(&h[kSelBins - 4 * (tid + 1)], (uint32_t)r);
+        for (int r = 0; r < kSelMaxCluster; ++r)
+          if ((uint32_t)r < CL) x[r] = dsmem_ld_u32x4(&h[kSelBins - 4 * (tid + 1)], (uint32_t)r);
+      }
       unsigned c[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int r = 0; r < kSelMaxCluster; ++r) {
@@ -773,9 +785,9 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
   unsigned tot;
   const unsigned excl = block_excl_scan(gt | (eq << 16), sh.tmp, &tot);
   if (tid == 0) sh.tot = tot;
-  cluster_sync();
+  csync();
   if (wid == 0) {   // output offset: the lower-ranked CTAs' taken counts, in order
-    const unsigned t = (uint32_t)lane < rank ? dsmem_ld_u32(&sh.tot, lane) : 0u;
+    const unsigned t = (uint32_t)lane < rank ? rd(&sh.tot, lane) : 0u;
     unsigned eq_before = 0u, out_before = 0u;
     for (uint32_t r = 0; r < rank; ++r) {
       const unsigned tr = __shfl_sync(0xffffffffu, t, (int)r);
@@ -790,7 +802,7 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
     }
   }
   __syncthreads();
-  cluster_arrive();   // this CTA's remote reads are done
+  if (!solo) cluster_arrive();   // this CTA's remote reads are done
   const unsigned eq_base = sh.base[0];
   const unsigned left = rem > eq_base ? rem - eq_base : 0u;
   unsigned at = sh.base[1] + (excl & 0xffffu) + min(left, excl >> 16);
@@ -818,7 +830,7 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
       if (so) so[p] = -INFINITY;
     }
   }
-  cluster_wait();   // no CTA leaves while another may still read its shared memory
+  if (!solo) cluster_wait();   // no CTA leaves while another may still read its shared memory
 }
 
 template <int TOK>
