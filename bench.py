@@ -192,6 +192,8 @@ class Step:
             csa.CSA_OP_INDEXER, w.dtype, B, T, 0, 0, w.n_csa, w.k, 0), device)
         self.ws_attn = csa.workspace(csa.csa_workspace_bytes(
             csa.CSA_OP_SPARSE_ATTN, w.dtype, B, T, w.H, c, w.n_csa, w.k, w.n_win), device)
+        self.ws_comp = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_COMPRESS, w.dtype, B, T),
+                                     device)
 
     def run(self, inp=None, ev=None, out=None):
         inp = inp or self.inp
@@ -201,7 +203,7 @@ class Step:
         if ev:
             ev[0].record(s)
         csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, self.fmt,
-                         entries=self.entries, win_out=self.win)
+                         entries=self.entries, win_out=self.win, ws=self.ws_comp)
         if ev:
             ev[1].record(s)
         csa.indexer_scores_topk(inp["q_I"], inp["w"], inp["k_I"], w.m, w.k, idx_out=self.idx,
@@ -436,14 +438,16 @@ def run_only_hca(args):
     fmt = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
     entries = torch.empty((w.B, w.n_hca, w.c), dtype=w.dtype, device=dev)
     win = torch.empty((w.B, w.T, w.c), dtype=w.dtype, device=dev)
-    csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win)
+    ws_c = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_COMPRESS, 1, w.B, w.T), dev)
+    csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win, ws=ws_c)
     out = torch.empty_like(inp["q"])
     ws = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_DENSE_ATTN, 1, w.B, w.T, w.H, w.c,
                                                w.n_hca, 0, w.n_win), dev)
 
     def once():
         if args.only == "hca_compress":
-            csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win)
+            csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win,
+                             ws=ws_c)
         else:
             csa.dense_hca_attn(inp["q"], entries, w.m_prime, win, fmt, w.n_win, sink=inp["sink"],
                                out=out, ws=ws)
@@ -576,13 +580,16 @@ def measure_compress_1m(dev, steps: int, warmup: int):
     x = [wl.randn((1, T, c), 100 + i, dev, dtype=torch.bfloat16) for i in range(4)]
     ent = torch.empty((1, T // 4, c), dtype=torch.bfloat16, device=dev)
     win = torch.empty((1, T, c), dtype=torch.bfloat16, device=dev)
-    ms = timed(lambda: csa.csa_compress(x[0], x[1], x[2], x[3], 4, fmt, entries=ent, win_out=win))
+    ws_c = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_COMPRESS, 1, 1, T), dev)
+    ms = timed(lambda: csa.csa_compress(x[0], x[1], x[2], x[3], 4, fmt, entries=ent, win_out=win,
+                                        ws=ws_c))
     nb = (4 * T + T // 4 + T) * c * 2
     res["csa_compress"] = {"ms": ms, "bytes": nb, "GBps": nb / ms / 1e6, "frac": nb / ms / 1e6 / hbm}
     del x, ent
     x = [wl.randn((1, T, c), 110 + i, dev, dtype=torch.bfloat16) for i in range(2)]
     ent = torch.empty((1, T // 128, c), dtype=torch.bfloat16, device=dev)
-    ms = timed(lambda: csa.hca_compress(x[0], x[1], 128, fmt, entries=ent, win_out=win))
+    ms = timed(lambda: csa.hca_compress(x[0], x[1], 128, fmt, entries=ent, win_out=win,
+                                        ws=ws_c))
     nb = (2 * T + T // 128 + T) * c * 2
     res["hca_compress"] = {"ms": ms, "bytes": nb, "GBps": nb / ms / 1e6, "frac": nb / ms / 1e6 / hbm}
     del x, ent, win
@@ -703,7 +710,7 @@ def run_only(args):
     def once():
         if args.only == "compress":
             csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, step.fmt,
-                             entries=step.entries, win_out=step.win)
+                             entries=step.entries, win_out=step.win, ws=step.ws_comp)
         elif args.only == "indexer":
             csa.indexer_scores_topk(inp["q_I"], inp["w"], inp["k_I"], w.m, w.k,
                                     idx_out=step.idx, ws=step.ws_idx)

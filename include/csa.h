@@ -85,6 +85,7 @@ typedef struct csa_fmt {
 #define CSA_OP_INDEXER 1
 #define CSA_OP_SPARSE_ATTN 2
 #define CSA_OP_DENSE_ATTN 3
+#define CSA_OP_COMPRESS 4
 
 /* ---- (1) compression ------------------------------------------------ */
 
@@ -100,13 +101,18 @@ typedef struct csa_fmt {
  *   entries (out): [B, floor(T/m), c].  Tail tokens (T mod m) make no entry.
  *   win_out (out, optional, may be NULL): [B, T, c] window rows
  *       RoPE_{pos0+j}(RMSNorm(kv_a[b,j])).
+ *   ws: workspace of at least csa_workspace_bytes(CSA_OP_COMPRESS, ...) bytes
+ *       (256: the status word), zeroed before first use; the streaming path
+ *       records a copy wait that runs out there (CSA_DEV_TIMEOUT).
  * Errors: CSA_E_ARG for null/misaligned pointers or T < 0, m < 1;
- *         CSA_E_UNSUPPORTED for 2m > 256 or an unsupported c.
+ *         CSA_E_UNSUPPORTED for 2m > 256 or an unsupported c;
+ *         CSA_E_WORKSPACE for a null or short ws (checked after the others,
+ *         and only when there is work to launch).
  */
 csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const csa_fmt* fmt,
                         const void* kv_a, const void* kv_b, const void* z_a, const void* z_b,
-                        int32_t z_cols, int64_t pos0, void* entries, void* win_out,
-                        void* stream);
+                        int32_t z_cols, int64_t pos0, void* entries, void* win_out, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /*
  * HCA compression [§3.3 of the summary page: a larger rate m' with no
@@ -114,11 +120,11 @@ csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const cs
  * the per-channel softmax of z over the m' tokens of block s; then RMSNorm and
  * RoPE at pos0 + m' s.  kv, z: [B, T, c] / [B, T, z_cols]; entries:
  * [B, floor(T/m'), c]; win_out (optional): [B, T, c] = RoPE_{pos0+j}(RMSNorm(kv[b,j])).
- * Errors as csa_compress; m' up to 4096.
+ * ws as csa_compress.  Errors as csa_compress; m' up to 4096.
  */
 csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, const csa_fmt* fmt,
                         const void* kv, const void* z, int32_t z_cols, int64_t pos0, void* entries,
-                        void* win_out, void* stream);
+                        void* win_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- (2) lightning indexer + top-k ----------------------------------- */
 

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libcsa.so")
 CSA_OK, CSA_E_ARG, CSA_E_UNSUPPORTED, CSA_E_CUDA, CSA_E_DEVICE, CSA_E_WORKSPACE = range(6)
 CSA_F32, CSA_BF16 = 0, 1
 CSA_F_NO_NORM, CSA_F_NO_ROPE, CSA_F_PORTABLE = 1, 2, 4
-CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN = 1, 2, 3
+CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS = 1, 2, 3, 4
 CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX = 1, 2, 3
 
 EXPORTED = (
@@ -83,8 +83,8 @@ def lib():
     P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     sz = ctypes.c_size_t
     FP = ctypes.POINTER(_CFmt)
-    L.csa_compress.argtypes = [i32, i64, i64, i32, FP, P, P, P, P, i32, i64, P, P, P]
-    L.hca_compress.argtypes = [i32, i64, i64, i32, FP, P, P, i32, i64, P, P, P]
+    L.csa_compress.argtypes = [i32, i64, i64, i32, FP, P, P, P, P, i32, i64, P, P, P, sz, P]
+    L.hca_compress.argtypes = [i32, i64, i64, i32, FP, P, P, i32, i64, P, P, P, sz, P]
     L.indexer_scores_topk.argtypes = [i32, i64, i64, i32, i32, P, P, P, i64, P, i32, i32, P, P,
                                       P, sz, P]
     L.sparse_mqa_attn.argtypes = [i32, i64, i64, i32, FP, P, P, P, i64, P, i32, P, i64, P, i32,
@@ -165,7 +165,7 @@ def csa_launch_count() -> int:
 
 
 def csa_compress(kv_a, kv_b, z_a, z_b, m: int, fmt: Fmt, pos0: int = 0, entries=None,
-                 win_out=None, want_win=False, stream=None):
+                 win_out=None, want_win=False, ws=None, stream=None):
     """CSA compression of [B, T, c] token groups -> entries [B, T//m, c]
     (and window rows [B, T, c] when ``want_win``)."""
     B, T, c = kv_a.shape
@@ -173,24 +173,29 @@ def csa_compress(kv_a, kv_b, z_a, z_b, m: int, fmt: Fmt, pos0: int = 0, entries=
         entries = torch.empty((B, T // m, c), dtype=kv_a.dtype, device=kv_a.device)
     if want_win and win_out is None:
         win_out = torch.empty_like(kv_a)
+    if ws is None:
+        ws = workspace(csa_workspace_bytes(CSA_OP_COMPRESS, _dt(kv_a), B, T), kv_a.device)
     f = fmt._c()
     st = lib().csa_compress(_dt(kv_a), B, T, m, ctypes.byref(f), _p(kv_a), _p(kv_b), _p(z_a),
-                            _p(z_b), z_a.shape[-1], pos0, _p(entries), _p(win_out), _s(stream))
+                            _p(z_b), z_a.shape[-1], pos0, _p(entries), _p(win_out), _p(ws),
+                            ws.numel(), _s(stream))
     _check(st, "csa_compress")
     return (entries, win_out) if win_out is not None else entries
 
 
 def hca_compress(kv, z, m_prime: int, fmt: Fmt, pos0: int = 0, entries=None, win_out=None,
-                 want_win=False, stream=None):
+                 want_win=False, ws=None, stream=None):
     """HCA compression of [B, T, c] tokens -> entries [B, T//m', c] (+ window rows)."""
     B, T, c = kv.shape
     if entries is None:
         entries = torch.empty((B, T // m_prime, c), dtype=kv.dtype, device=kv.device)
     if want_win and win_out is None:
         win_out = torch.empty_like(kv)
+    if ws is None:
+        ws = workspace(csa_workspace_bytes(CSA_OP_COMPRESS, _dt(kv), B, T), kv.device)
     f = fmt._c()
     st = lib().hca_compress(_dt(kv), B, T, m_prime, ctypes.byref(f), _p(kv), _p(z), z.shape[-1],
-                            pos0, _p(entries), _p(win_out), _s(stream))
+                            pos0, _p(entries), _p(win_out), _p(ws), ws.numel(), _s(stream))
     _check(st, "hca_compress")
     return (entries, win_out) if win_out is not None else entries
 

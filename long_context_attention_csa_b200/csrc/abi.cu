@@ -40,10 +40,13 @@ csa_status check_fmt(int32_t dtype, const csa_fmt* fmt, Fmt* out) {
   return CSA_OK;
 }
 
+unsigned* status_word(void* ws) { return static_cast<unsigned*>(ws); }
+
 csa_status compress_common(int32_t dtype, int64_t B, int64_t T, int32_t m, bool overlap,
                            const csa_fmt* fmt, const void* kv_a, const void* kv_b,
                            const void* z_a, const void* z_b, int32_t z_cols, int64_t pos0,
-                           void* entries, void* win_out, void* stream) {
+                           void* entries, void* win_out, void* ws, size_t ws_bytes,
+                           void* stream) {
   Fmt f;
   csa_status st = check_fmt(dtype, fmt, &f);
   if (st != CSA_OK) return st;
@@ -61,6 +64,7 @@ csa_status compress_common(int32_t dtype, int64_t B, int64_t T, int32_t m, bool 
   if (z_cols != 1 && (!aligned16(z_a) || (overlap && !aligned16(z_b)))) return CSA_E_ARG;
   if (n == 0 && !win_out) return CSA_OK;
   if (n + 1 > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  if (!ws || ws_bytes < kWsScratch) return CSA_E_WORKSPACE;
   CompressParams p{};
   p.kv_a = kv_a;
   p.kv_b = kv_b;
@@ -75,11 +79,10 @@ csa_status compress_common(int32_t dtype, int64_t B, int64_t T, int32_t m, bool 
   p.pos0 = pos0;
   p.entries = entries;
   p.win = win_out;
+  p.status = status_word(ws);
   g_launches.fetch_add(1);
   return cuda_status(launch_compress(dtype, p, B, S(stream)));
 }
-
-unsigned* status_word(void* ws) { return static_cast<unsigned*>(ws); }
 
 }  // namespace
 
@@ -87,23 +90,25 @@ extern "C" {
 
 csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const csa_fmt* fmt,
                         const void* kv_a, const void* kv_b, const void* z_a, const void* z_b,
-                        int32_t z_cols, int64_t pos0, void* entries, void* win_out,
-                        void* stream) {
+                        int32_t z_cols, int64_t pos0, void* entries, void* win_out, void* ws,
+                        size_t ws_bytes, void* stream) {
   return compress_common(dtype, B, T, m, true, fmt, kv_a, kv_b, z_a, z_b, z_cols, pos0, entries,
-                         win_out, stream);
+                         win_out, ws, ws_bytes, stream);
 }
 
 csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, const csa_fmt* fmt,
                         const void* kv, const void* z, int32_t z_cols, int64_t pos0, void* entries,
-                        void* win_out, void* stream) {
+                        void* win_out, void* ws, size_t ws_bytes, void* stream) {
   return compress_common(dtype, B, T, m_prime, false, fmt, kv, nullptr, z, nullptr, z_cols, pos0,
-                         entries, win_out, stream);
+                         entries, win_out, ws, ws_bytes, stream);
 }
 
 size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int32_t H, int32_t c,
                            int64_t N, int32_t k, int32_t n_win) {
   if (B < 0 || Tq < 0 || N < 0) return 0;
   switch (op) {
+    case CSA_OP_COMPRESS:
+      return kWsScratch;
     case CSA_OP_INDEXER: {
       size_t a = indexer_portable_scratch(B, Tq, N, k);
       size_t b = dtype == CSA_BF16 ? indexer_tc_scratch(B, Tq, N, k) : 0;

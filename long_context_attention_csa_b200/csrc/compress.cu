@@ -286,8 +286,9 @@ cudaError_t launch_t(CompressParams p, int64_t B, cudaStream_t stream) {
 
 // ---- bf16, c = 512, per-channel logits: streaming fast paths ---------------
 // Rows of every input tensor that one chunk of tokens needs are contiguous, so
-// persistent CTAs stage them through a ring of shared-memory slots with
-// cp.async (16 bytes per thread-instruction, several chunks in flight) and
+// persistent CTAs stage them through a ring of shared-memory slots, one bulk
+// asynchronous copy per tensor and chunk (several chunks in flight; the copy
+// engine, not per-thread 16-byte requests, keeps the bytes in flight), and
 // take chunks round-robin; compute reads the staged rows, never global memory.
 constexpr int kFC = 512;                    // channels
 constexpr int kFRowB = kFC * 2;             // bytes per token row
@@ -295,8 +296,44 @@ constexpr int kFThreads = 256;
 constexpr int kFTab = 2048 + 64;            // RoPE cos/sin table: [rows][32 pairs] float2
 constexpr int kFDelta = 8192;               // (cos, sin) of i * theta, i < 16: [16][32] float2
 constexpr int kFBase = kFDelta + 16 * 32 * 8;   // a chunk's row-0 (cos, sin): [32] float2
-constexpr int kFHead = 13312;               // frequencies, reductions, tables
-static_assert(kFTab + 17 * 32 * 8 <= kFDelta && kFBase + 32 * 8 <= kFHead, "head layout");
+constexpr int kFBar = kFBase + 32 * 8;      // ring-slot mbarriers: [stages] u64
+constexpr int kFHead = 13312;               // frequencies, reductions, tables, barriers
+static_assert(kFTab + 17 * 32 * 8 <= kFDelta && kFBar + 4 * 8 <= kFHead, "head layout");
+
+// Fills ring slot `slot_s` with token rows [st, st + rows) of one [B, T, 512]
+// tensor of sequence b, clipped to [0, T) (rows outside stay stale and are
+// never read); returns the bytes requested.  count_only: no copy is issued.
+__device__ __forceinline__ uint32_t stage_rows(uint32_t slot_s, const bf16* src, int64_t b,
+                                               int64_t T, int64_t st, int rows, uint64_t* bar,
+                                               bool count_only) {
+  const int64_t lo = st > 0 ? st : 0, hi = st + rows < T ? st + rows : T;
+  if (hi <= lo) return 0u;
+  const uint32_t bytes = (uint32_t)(hi - lo) * kFRowB;
+  if (!count_only)
+    sm100::bulk_load(slot_s + (uint32_t)(lo - st) * kFRowB, src + (b * T + lo) * kFC, bytes, bar);
+  return bytes;
+}
+
+// Waits for ring phase k (slot k % S); false once a wait ran out on any
+// thread of the CTA (the status word then holds the error).
+template <int S>
+__device__ __forceinline__ bool ring_ready(uint64_t* full, uint32_t k, unsigned* status,
+                                           unsigned detail) {
+  const bool ok = sm100::mbar_wait(&full[k % S], (k / S) & 1u);
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) report(status, CSA_DEV_TIMEOUT, detail);
+    return false;
+  }
+  return true;
+}
+
+// Before the CTA exits: the copies of the phases issued past the last one
+// consumed (k, k + 1, ...) have landed (bounded waits; thread 0).
+template <int S>
+__device__ __forceinline__ void ring_drain(uint64_t* full, uint32_t k) {
+  if (threadIdx.x == 0)
+    for (int i = 0; i < S - 1; ++i) sm100::mbar_wait(&full[(k + i) % S], ((k + i) / S) & 1u);
+}
 
 // Window row from a staged token row: RoPE_pos(RMSNorm(row)).  Lane l owns the
 // 16-byte chunks l and l + 32 (channels 8l..8l+7 and 256+8l..256+8l+7), so a
@@ -405,33 +442,40 @@ __global__ void __launch_bounds__(kFThreads, 2)
   float2* tab = reinterpret_cast<float2*>(fsm + kFTab); // rows 0-7 window, 8-9 entries
   float2* dtab = reinterpret_cast<float2*>(fsm + kFDelta);
   float2* rbase = reinterpret_cast<float2*>(fsm + kFBase);
+  uint64_t* full = reinterpret_cast<uint64_t*>(fsm + kFBar);   // [kCStages] slot landed
   uint8_t* ring = fsm + kFHead;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  if (t == 0) {
+    for (int i = 0; i < kCStages; ++i) sm100::mbar_init(&full[i], 1);
+    sm100::fence_barrier_init();
+  }
   for (int i = t; i < (p.f.r >> 1); i += kFThreads)
     theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
-  __syncthreads();   // frequencies complete before the tables
+  __syncthreads();   // frequencies and barriers complete before the tables
   if (!(p.f.flags & CSA_F_NO_ROPE)) fill_delta_table(dtab, p.f.r, theta);
   __syncthreads();
   const uint32_t ring_s = sm100::smem_u32(ring);
-  const bf16* kva = static_cast<const bf16*>(p.kv_a);
-  const bf16* kvb = static_cast<const bf16*>(p.kv_b);
-  const bf16* za = static_cast<const bf16*>(p.z_a);
-  const bf16* zb = static_cast<const bf16*>(p.z_b);
+  // slot layout: [kv_a, z_a rows t0..t0+7][kv_b, z_b rows t0-4..t0+3]
+  const bf16* src4[4] = {static_cast<const bf16*>(p.kv_a), static_cast<const bf16*>(p.z_a),
+                         static_cast<const bf16*>(p.kv_b), static_cast<const bf16*>(p.z_b)};
+  // thread 0 fills `slot` with chunk u (past the end: an arrival with no
+  // bytes, so the slot's phases stay in step).  The slot was last read in the
+  // iteration before, which ended with a CTA barrier.
   auto issue = [&](uint32_t u, int slot) {
-    if (u < total) {
-      const int64_t b = u / n_chunks, t0 = (int64_t)(u % n_chunks) * kCR;
-#pragma unroll
-      for (int i = 0; i < 4 * kCR * 64 / kFThreads; ++i) {
-        const int q = t + kFThreads * i;
-        const int tensor = q >> 9, row = (q >> 6) & (kCR - 1), col = q & 63;
-        const int64_t tok = (tensor < 2 ? t0 : t0 - 4) + row;
-        if (tok < 0 || tok >= p.T) continue;
-        const bf16* src = tensor == 0 ? kva : tensor == 1 ? za : tensor == 2 ? kvb : zb;
-        sm100::cp_async16(ring_s + slot * kCStage + (tensor * kCR + row) * kFRowB + col * 16,
-                          src + (b * p.T + tok) * kFC + col * 8, 16u);
-      }
-    }
-    sm100::cp_async_commit();
+    if (t != 0) return;
+    const uint32_t s0 = ring_s + slot * kCStage;
+    const int64_t b = u < total ? u / n_chunks : 0;
+    const int64_t t0 = u < total ? (int64_t)(u % n_chunks) * kCR : 0;
+    uint32_t bytes = 0;
+    if (u < total)
+      for (int i = 0; i < 4; ++i)
+        bytes += stage_rows(0, src4[i], b, p.T, i < 2 ? t0 : t0 - 4, kCR, nullptr, true);
+    sm100::fence_proxy_async_smem();
+    sm100::mbar_arrive_expect_tx(&full[slot], bytes);
+    if (u < total)
+      for (int i = 0; i < 4; ++i)
+        stage_rows(s0 + i * kCR * kFRowB, src4[i], b, p.T, i < 2 ? t0 : t0 - 4, kCR, &full[slot],
+                   false);
   };
   const int e = t >> 7, cq = t & 127;   // entry of the chunk, channels 4cq .. 4cq+3
   int k = 0;
@@ -443,8 +487,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
     if (!(p.f.flags & CSA_F_NO_ROPE))
       fill_rope_rows(tab, rbase, dtab, kCR + 2, p.f.r, theta, p.pos0 + t0,
                      [](int i) { return i < kCR ? i : 4 * (i - kCR); });
-    sm100::cp_async_wait<kCStages - 1>();
-    __syncthreads();
+    if (!ring_ready<kCStages>(full, (uint32_t)k, p.status, 40u)) break;
     const uint8_t* buf = ring + (k % kCStages) * kCStage;
     const int64_t s = t0 / 4 + e;
     const bool have = s < p.n_entries;   // uniform per warp
@@ -507,9 +550,9 @@ __global__ void __launch_bounds__(kFThreads, 2)
       *reinterpret_cast<uint2*>(static_cast<bf16*>(p.entries) + (b * p.n_entries + s) * kFC + 4 * cq) =
           make_uint2(pack_bf16x2(val[0], val[1]), pack_bf16x2(val[2], val[3]));
     }
-    __syncthreads();   // table and reductions are rewritten by the next chunk
+    __syncthreads();   // table, reductions and this slot are rewritten next
   }
-  sm100::cp_async_wait<0>();
+  ring_drain<kCStages>(full, (uint32_t)k);
 }
 
 // HCA, m' a multiple of 16: a unit is one block of m' tokens (its entry, when
@@ -527,11 +570,16 @@ __global__ void __launch_bounds__(kFThreads, 2)
   float2* tab = reinterpret_cast<float2*>(fsm + kFTab); // rows 0-15 window, 16 entry
   float2* dtab = reinterpret_cast<float2*>(fsm + kFDelta);
   float2* rbase = reinterpret_cast<float2*>(fsm + kFBase);
+  uint64_t* full = reinterpret_cast<uint64_t*>(fsm + kFBar);   // [kHStages] slot landed
   uint8_t* ring = fsm + kFHead;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  if (t == 0) {
+    for (int i = 0; i < kHStages; ++i) sm100::mbar_init(&full[i], 1);
+    sm100::fence_barrier_init();
+  }
   for (int i = t; i < (p.f.r >> 1); i += kFThreads)
     theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
-  __syncthreads();   // frequencies complete before the tables
+  __syncthreads();   // frequencies and barriers complete before the tables
   if (!(p.f.flags & CSA_F_NO_ROPE)) fill_delta_table(dtab, p.f.r, theta);
   __syncthreads();
   const uint32_t ring_s = sm100::smem_u32(ring);
@@ -540,24 +588,29 @@ __global__ void __launch_bounds__(kFThreads, 2)
   const int cpu = p.m / kHR;                               // chunks per unit
   const uint32_t n_my = total > blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const uint32_t n_ck = n_my * cpu;                        // this CTA's chunk sequence
+  // thread 0 fills `slot` with chunk kk of this CTA's sequence ([kv rows]
+  // [z rows], 16 each; past the end: an arrival with no bytes).  The slot was
+  // last read in the iteration before, which ended with a CTA barrier.
   auto issue = [&](uint32_t kk, int slot) {
+    if (t != 0) return;
+    const uint32_t s0 = ring_s + slot * kHStage;
+    int64_t b = 0, t0 = 0;
+    uint32_t bytes = 0;
     if (kk < n_ck) {
       const uint32_t u = blockIdx.x + (kk / cpu) * gridDim.x;
-      const int64_t b = u / n_blocks;
-      const int64_t t0 = (int64_t)(u % n_blocks) * p.m + (int64_t)(kk % cpu) * kHR;
-#pragma unroll
-      for (int i = 0; i < 2 * kHR * 64 / kFThreads; ++i) {
-        const int q = t + kFThreads * i;
-        const int tensor = q >> 10, row = (q >> 6) & (kHR - 1), col = q & 63;
-        const int64_t tok = t0 + row;
-        if (tok >= p.T) continue;
-        sm100::cp_async16(ring_s + slot * kHStage + (tensor * kHR + row) * kFRowB + col * 16,
-                          (tensor ? z : kv) + (b * p.T + tok) * kFC + col * 8, 16u);
-      }
+      b = u / n_blocks;
+      t0 = (int64_t)(u % n_blocks) * p.m + (int64_t)(kk % cpu) * kHR;
+      bytes = 2 * stage_rows(0, kv, b, p.T, t0, kHR, nullptr, true);
     }
-    sm100::cp_async_commit();
+    sm100::fence_proxy_async_smem();
+    sm100::mbar_arrive_expect_tx(&full[slot], bytes);
+    if (kk < n_ck) {
+      stage_rows(s0, kv, b, p.T, t0, kHR, &full[slot], false);
+      stage_rows(s0 + kHR * kFRowB, z, b, p.T, t0, kHR, &full[slot], false);
+    }
   };
   for (int i = 0; i < kHStages - 1; ++i) issue(i, i);
+  uint32_t n_done = n_ck;   // phases consumed (the loop's count unless a wait ran out)
   float mx[2], den[2], acc[2];
   for (uint32_t kk = 0; kk < n_ck; ++kk) {
     issue(kk + kHStages - 1, (int)((kk + kHStages - 1) % kHStages));
@@ -574,8 +627,10 @@ __global__ void __launch_bounds__(kFThreads, 2)
         tab[kHR * 32 + t] = make_float2(cs, sn);
       }
     }
-    sm100::cp_async_wait<kHStages - 1>();
-    __syncthreads();
+    if (!ring_ready<kHStages>(full, kk, p.status, 41u)) {
+      n_done = kk;
+      break;
+    }
     const uint8_t* buf = ring + (kk % kHStages) * kHStage;
     if (j == 0) {
 #pragma unroll
@@ -625,7 +680,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
     }
     __syncthreads();   // the slot is refilled next iteration; red reused
   }
-  sm100::cp_async_wait<0>();
+  ring_drain<kHStages>(full, n_done);
 }
 
 int sm_count() {

@@ -27,6 +27,7 @@ struct CompressParams {
   int64_t pos0;
   void* entries;
   void* win;          // optional window-row output
+  unsigned* status;   // device status word (timed-out copy waits)
 };
 cudaError_t launch_compress(int dtype, CompressParams p, int64_t B, cudaStream_t stream);
 

@@ -73,35 +73,41 @@ def test_compress_rejects_bad_arguments(L):
     mis = ctypes.c_void_p(4100)     # not 16-byte aligned
     # bad dtype, null fmt, bad m, null pointers, misalignment, bad z_cols
     assert L.csa_compress(7, 1, 64, 4, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0, dummy,
-                          None, None) == 1
+                          None, None, 0, None) == 1
     assert L.csa_compress(1, 1, 64, 4, None, dummy, dummy, dummy, dummy, 512, 0, dummy, None,
-                          None) == 1
+                          None, 0, None) == 1
     assert L.csa_compress(1, 1, 64, 0, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0, dummy,
-                          None, None) == 1
+                          None, None, 0, None) == 1
     assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), None, dummy, dummy, dummy, 512, 0, dummy,
-                          None, None) == 1
+                          None, None, 0, None) == 1
     assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), mis, dummy, dummy, dummy, 512, 0, dummy,
-                          None, None) == 1
+                          None, None, 0, None) == 1
     assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), dummy, dummy, dummy, dummy, 7, 0, dummy,
-                          None, None) == 1
+                          None, None, 0, None) == 1
     # odd RoPE dims, RoPE wider than c
     bad = _fmt(r=63)
     assert L.csa_compress(1, 1, 64, 4, ctypes.byref(bad), dummy, dummy, dummy, dummy, 512, 0,
-                          dummy, None, None) == 1
+                          dummy, None, None, 0, None) == 1
     bad = _fmt(c=64, r=128)
     assert L.csa_compress(1, 1, 64, 4, ctypes.byref(bad), dummy, dummy, dummy, dummy, 64, 0,
-                          dummy, None, None) == 1
+                          dummy, None, None, 0, None) == 1
     # unsupported: c not a power-of-two number of vectors, overlap too wide
     odd = _fmt(c=520, r=64)
     assert L.csa_compress(1, 1, 64, 4, ctypes.byref(odd), dummy, dummy, dummy, dummy, 520, 0,
-                          dummy, None, None) == 2
+                          dummy, None, None, 0, None) == 2
     assert L.csa_compress(1, 1, 1024, 200, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0,
-                          dummy, None, None) == 2
+                          dummy, None, None, 0, None) == 2
     # empty problems are a no-op
     assert L.csa_compress(1, 0, 64, 4, ctypes.byref(f), None, None, None, None, 512, 0, None, None,
-                          None) == 0
+                          None, 0, None) == 0
     assert L.hca_compress(1, 1, 0, 128, ctypes.byref(f), None, None, 512, 0, None, None,
-                          None) == 0
+                          None, 0, None) == 0
+    # a launchable problem without (or with too small) a workspace
+    assert L.csa_compress(1, 1, 64, 4, ctypes.byref(f), dummy, dummy, dummy, dummy, 512, 0, dummy,
+                          None, None, 0, None) == 5
+    assert L.hca_compress(1, 1, 256, 128, ctypes.byref(f), dummy, dummy, 512, 0, dummy, None,
+                          dummy, 255, None) == 5
+    assert L.csa_workspace_bytes(4, 1, 1, 64, 0, 0, 0, 0, 0) == 256
 
 
 def test_indexer_and_attention_reject_bad_arguments(L):

@@ -75,6 +75,28 @@ def test_hca_compress(T, B, mp):
         assert_close(win[b][rows], refw, w.dtype, f"window b={b}")
 
 
+def test_compress_streaming_path_leaves_the_status_word_clear():
+    """The bulk-copy ring of the streaming compression kernels: short and
+    ragged sequences (chunks that run past T, the first chunk's previous block
+    before token 0) land every copy; the status word stays clear."""
+    ws = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_COMPRESS, 1, 3, 77))
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=77, B=3)
+    inp = wl.csa_prefill_inputs(w, DEV)
+    ent, win = csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, gfmt(w),
+                                want_win=True, ws=ws)
+    wh = wl.scaled(wl.WORKLOADS["hca_prefill_64k"], T=77, B=3, m_prime=32)
+    hin = wl.hca_prefill_inputs(wh, DEV)
+    hent, hwin = csa.hca_compress(hin["kv"], hin["z"], 32, gfmt(wh), want_win=True, ws=ws)
+    assert csa.csa_check_status(ws) == (csa.CSA_OK, 0)
+    for b in range(3):
+        ref = oracle.csa_compress(f64(inp["kv_a"][b]), f64(inp["kv_b"][b]), f64(inp["z_a"][b]),
+                                  f64(inp["z_b"][b]), w.m, ofmt(w))
+        assert_close(ent[b], ref, w.dtype, f"csa entries b={b}")
+        assert_close(win[b], oracle.window_rows(f64(inp["kv_a"][b]), ofmt(w)), w.dtype, "window")
+        href = oracle.hca_compress(f64(hin["kv"][b]), f64(hin["z"][b]), 32, ofmt(wh))
+        assert_close(hent[b], href, wh.dtype, f"hca entries b={b}")
+
+
 # ----------------------------------------------------------------- indexer
 
 def _indexer_case(w, rows=None, q_pos=None, exact=False):
