@@ -378,19 +378,18 @@ __device__ __forceinline__ void window_row_staged(const uint8_t* srow, bf16* dst
   reinterpret_cast<uint4*>(dst)[32 + lane] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// One online-softmax step (base 2, one exp2 per element) of a channel.  The
-// exponent is never positive, so the hardware ex2 (relative error ~2^-22,
-// results below 2^-126 flushed to 0) replaces the libm call.
-__device__ __forceinline__ void osm_step(float z, float v, float& mx, float& den, float& acc) {
-  const float zl = z * kLog2e;
-  const float d = zl - mx;
-  const float t = sm100::ex2(-fabsf(d));
-  const bool gt = d > 0.f;
-  const float so = gt ? t : 1.f;
-  const float sn = gt ? 1.f : t;
-  den = den * so + sn;
-  acc = acc * so + sn * v;
-  mx = fmaxf(mx, zl);
+// The two bf16 values packed in a 32-bit word, widened exactly.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// One softmax-weighted term in base 2 against a running maximum mxl (in log2
+// units, at least z log2(e) up to rounding): e = 2^(z log2 e - mxl).  The
+// exponent is never meaningfully positive, so the hardware ex2 (relative
+// error ~2^-22, results below 2^-126 flushed to 0) replaces the libm call.
+__device__ __forceinline__ void sm_term(float z, float v, float mxl, float& den, float& acc) {
+  const float e = sm100::ex2(fmaf(z, kLog2e, -mxl));
+  den += e;
+  acc = fmaf(e, v, acc);
 }
 
 // Per-CTA table of (cos, sin) of i * theta_pr, i < 16: a chunk's table rows are
@@ -493,24 +492,39 @@ __global__ void __launch_bounds__(kFThreads, 2)
     const bool have = s < p.n_entries;   // uniform per warp
     float val[4] = {0.f, 0.f, 0.f, 0.f};
     if (have) {
-      float mx[4], den[4], acc[4];
+      // the entry's 2m = 8 slots (group a: its own block; group b: the
+      // previous block, absent for entry 0) for channels 4cq .. 4cq+3: the
+      // logits' maximum first, then one exp2 per slot
+      const int ns = s == 0 ? 4 : 8;   // uniform per warp
+      uint2 cv[8], zv[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) { mx[c] = -INFINITY; den[c] = 0.f; acc[c] = 0.f; }
+      for (int i = 0; i < 8; ++i) {
+        const int g = i >> 2, row = 4 * e + (i & 3);
+        if (i < ns) {
+          cv[i] = *reinterpret_cast<const uint2*>(buf + ((2 * g) * kCR + row) * kFRowB + cq * 8);
+          zv[i] = *reinterpret_cast<const uint2*>(buf + ((2 * g + 1) * kCR + row) * kFRowB + cq * 8);
+        }
+      }
+      float mxl[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {   // group a (own block), then group b (previous)
-        if (g == 1 && s == 0) break;
+      for (int i = 0; i < 8; ++i) {
+        if (i < ns) {
+          mxl[0] = fmaxf(mxl[0], bf16_lo(zv[i].x));
+          mxl[1] = fmaxf(mxl[1], bf16_hi(zv[i].x));
+          mxl[2] = fmaxf(mxl[2], bf16_lo(zv[i].y));
+          mxl[3] = fmaxf(mxl[3], bf16_hi(zv[i].y));
+        }
+      }
+      float den[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = 4 * e + j;
-          const uint2 cv = *reinterpret_cast<const uint2*>(buf + ((2 * g) * kCR + row) * kFRowB + cq * 8);
-          const uint2 zv = *reinterpret_cast<const uint2*>(buf + ((2 * g + 1) * kCR + row) * kFRowB + cq * 8);
-          const uint32_t cw[2] = {cv.x, cv.y}, zw[2] = {zv.x, zv.y};
+      for (int c = 0; c < 4; ++c) mxl[c] *= kLog2e;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t cb = (c & 1) ? cw[c >> 1] >> 16 : cw[c >> 1] & 0xffffu;
-            const uint32_t zbits = (c & 1) ? zw[c >> 1] >> 16 : zw[c >> 1] & 0xffffu;
-            osm_step(bf16_bits_to_float(zbits), bf16_bits_to_float(cb), mx[c], den[c], acc[c]);
-          }
+      for (int i = 0; i < 8; ++i) {
+        if (i < ns) {
+          sm_term(bf16_lo(zv[i].x), bf16_lo(cv[i].x), mxl[0], den[0], acc[0]);
+          sm_term(bf16_hi(zv[i].x), bf16_hi(cv[i].x), mxl[1], den[1], acc[1]);
+          sm_term(bf16_lo(zv[i].y), bf16_lo(cv[i].y), mxl[2], den[2], acc[2]);
+          sm_term(bf16_hi(zv[i].y), bf16_hi(cv[i].y), mxl[3], den[3], acc[3]);
         }
       }
 #pragma unroll
@@ -638,12 +652,31 @@ __global__ void __launch_bounds__(kFThreads, 2)
     }
     const bool have = s < p.n_entries;   // a complete block (CTA-uniform)
     if (have) {
-#pragma unroll 4
+      // the chunk's 16 rows of channels 2t, 2t+1: their logits' maximum
+      // updates the running one (one rescale of the state per chunk), then
+      // one exp2 per row
+      uint32_t cw[kHR], zw[kHR];
+      float cm0 = -INFINITY, cm1 = -INFINITY;
+#pragma unroll
       for (int r = 0; r < kHR; ++r) {
-        const uint32_t cw = *reinterpret_cast<const uint32_t*>(buf + r * kFRowB + t * 4);
-        const uint32_t zw = *reinterpret_cast<const uint32_t*>(buf + (kHR + r) * kFRowB + t * 4);
-        osm_step(bf16_bits_to_float(zw & 0xffffu), bf16_bits_to_float(cw & 0xffffu), mx[0], den[0], acc[0]);
-        osm_step(bf16_bits_to_float(zw >> 16), bf16_bits_to_float(cw >> 16), mx[1], den[1], acc[1]);
+        cw[r] = *reinterpret_cast<const uint32_t*>(buf + r * kFRowB + t * 4);
+        zw[r] = *reinterpret_cast<const uint32_t*>(buf + (kHR + r) * kFRowB + t * 4);
+        cm0 = fmaxf(cm0, bf16_lo(zw[r]));
+        cm1 = fmaxf(cm1, bf16_hi(zw[r]));
+      }
+      const float cm[2] = {cm0 * kLog2e, cm1 * kLog2e};
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float mn = fmaxf(mx[c], cm[c]);
+        const float sc = sm100::ex2(mx[c] - mn);   // 0 on the block's first chunk
+        den[c] *= sc;
+        acc[c] *= sc;
+        mx[c] = mn;
+      }
+#pragma unroll
+      for (int r = 0; r < kHR; ++r) {
+        sm_term(bf16_lo(zw[r]), bf16_lo(cw[r]), mx[0], den[0], acc[0]);
+        sm_term(bf16_hi(zw[r]), bf16_hi(cw[r]), mx[1], den[1], acc[1]);
       }
     }
     if (p.win != nullptr) {   // window rows: warp w takes rows 2w, 2w+1 of the chunk
