@@ -554,13 +554,13 @@ def graph_ms(fn, steps: int, flush) -> float:
     return ms
 
 
-def measure_compress_1m(dev, steps: int, warmup: int):
+def measure_compress_1m(dev, steps: int, warmup: int, T: int = 1 << 20):
     """CSA (m = 4) and HCA (m' = 128) compression alone at 2^20 tokens, c = 512
     bf16, window rows written: inputs of 2-4 GiB (far larger than L2), so
     the kernels' HBM bandwidth shows without launch overhead (the 8192-token
     workload moves only 42 MB).  Algorithmic bytes: every input read once,
     entries and window rows written once."""
-    T, c = 1 << 20, 512
+    c = 512
     fmt = csa.Fmt(c=c, rope_dims=64)
     hbm, _, src = peaks()
     res = {}
@@ -691,6 +691,12 @@ def run_only_decode(args):
 def run_only(args):
     """One stage of the step alone on the csa_prefill workload at --seq-len
     tokens (for kernel profiles): warm-up, then --steps timed launches."""
+    if args.only == "compress_stream":   # CSA then HCA compression alone, inputs only
+        torch.cuda.set_device(0)
+        res = measure_compress_1m(torch.device("cuda", 0), args.steps, args.warmup,
+                                  T=args.seq_len or (1 << 20))
+        print(json.dumps({"only": args.only, **res}))
+        return
     if args.only.startswith("hca_"):
         return run_only_hca(args)
     if args.only == "decode":
@@ -732,7 +738,8 @@ def run_only(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--only", choices=["compress", "indexer", "attn", "hca_compress", "hca_attn",
+    ap.add_argument("--only", choices=["compress", "compress_stream", "indexer", "attn",
+                                       "hca_compress", "hca_attn",
                                        "decode"],
                     default=None,
                     help="time one stage alone (kernel profiling)")
