@@ -327,12 +327,13 @@ __device__ __forceinline__ bool ring_ready(uint64_t* full, uint32_t k, unsigned*
   return true;
 }
 
-// Before the CTA exits: the copies of the phases issued past the last one
-// consumed (k, k + 1, ...) have landed (bounded waits; thread 0).
+// Before the CTA exits: the copies of every phase issued but not consumed
+// ([consumed, issued), at most S of them) have landed (bounded waits;
+// thread 0).
 template <int S>
-__device__ __forceinline__ void ring_drain(uint64_t* full, uint32_t k) {
+__device__ __forceinline__ void ring_drain(uint64_t* full, uint32_t consumed, uint32_t issued) {
   if (threadIdx.x == 0)
-    for (int i = 0; i < S - 1; ++i) sm100::mbar_wait(&full[(k + i) % S], ((k + i) / S) & 1u);
+    for (uint32_t k = consumed; k < issued; ++k) sm100::mbar_wait(&full[k % S], (k / S) & 1u);
 }
 
 // Window row from a staged token row: RoPE_pos(RMSNorm(row)).  Lane l owns the
@@ -460,7 +461,9 @@ __global__ void __launch_bounds__(kFThreads, 2)
   // thread 0 fills `slot` with chunk u (past the end: an arrival with no
   // bytes, so the slot's phases stay in step).  The slot was last read in the
   // iteration before, which ended with a CTA barrier.
+  uint32_t n_issued = 0;   // ring phases issued (the same count on every thread)
   auto issue = [&](uint32_t u, int slot) {
+    ++n_issued;
     if (t != 0) return;
     const uint32_t s0 = ring_s + slot * kCStage;
     const int64_t b = u < total ? u / n_chunks : 0;
@@ -566,7 +569,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
     }
     __syncthreads();   // table, reductions and this slot are rewritten next
   }
-  ring_drain<kCStages>(full, (uint32_t)k);
+  ring_drain<kCStages>(full, (uint32_t)k, n_issued);
 }
 
 // HCA, m' a multiple of 16: a unit is one block of m' tokens (its entry, when
@@ -605,7 +608,9 @@ __global__ void __launch_bounds__(kFThreads, 2)
   // thread 0 fills `slot` with chunk kk of this CTA's sequence ([kv rows]
   // [z rows], 16 each; past the end: an arrival with no bytes).  The slot was
   // last read in the iteration before, which ended with a CTA barrier.
+  uint32_t n_issued = 0;   // ring phases issued (the same count on every thread)
   auto issue = [&](uint32_t kk, int slot) {
+    ++n_issued;
     if (t != 0) return;
     const uint32_t s0 = ring_s + slot * kHStage;
     int64_t b = 0, t0 = 0;
@@ -713,7 +718,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
     }
     __syncthreads();   // the slot is refilled next iteration; red reused
   }
-  ring_drain<kHStages>(full, n_done);
+  ring_drain<kHStages>(full, n_done, n_issued);
 }
 
 int sm_count() {
