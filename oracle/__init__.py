@@ -69,7 +69,9 @@ _lib = None
 def _L():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        # CSA_ORACLE_LIB: a build of a modified copy of csa_oracle.c, used by
+        # the test that plants mistakes in the oracle to show the pins catch them
+        _lib = ctypes.CDLL(os.environ.get("CSA_ORACLE_LIB") or build())
         P = ctypes.c_void_p
         i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         FP = ctypes.POINTER(_Fmt)
