@@ -87,9 +87,16 @@ def _L():
         _lib.orc_attention.argtypes = [
             i64, i32, FP, P, P, P, i64, P, i32, i32, P, i64, i64, i32, P, f64, P, P,
         ]
+        _lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        _lib.orc_e4m3_value.restype = f64
+        _lib.orc_e4m3_encode.argtypes = [f64]
+        _lib.orc_e4m3_encode.restype = ctypes.c_uint8
+        _lib.orc_mxfp8_quantize.argtypes = [i64, P, P, P]
+        _lib.orc_mxfp8_dequantize.argtypes = [i64, P, P, P]
         for fn in (
             "orc_rmsnorm", "orc_rope", "orc_csa_compress", "orc_hca_compress",
             "orc_window_rows", "orc_indexer_scores", "orc_topk", "orc_attention",
+            "orc_mxfp8_quantize", "orc_mxfp8_dequantize",
         ):
             getattr(_lib, fn).restype = None
     return _lib
@@ -231,3 +238,42 @@ def csa_layer(inp: dict, fmt: Fmt, m: int, k: int, n_win: int, rows=None):
     out = attention(np.asarray(inp["q"])[rows], ent, win, fmt, n_win, idx=idx, sink=inp.get("sink"),
                     q_pos=rows)
     return dict(entries=ent, win=win, idx=idx, scores=sc, out=out)
+
+
+# ---- (next) block-scaled FP8 indexer inputs --------------------------------
+
+def e4m3_value(code: int) -> float:
+    """Value of an FP8 E4M3 (FN) code."""
+    return float(_L().orc_e4m3_value(int(code)))
+
+
+def e4m3_encode(x: float) -> int:
+    """Nearest E4M3 code (ties to the even code, saturating at +-448)."""
+    return int(_L().orc_e4m3_encode(float(x)))
+
+
+def mxfp8_quantize(x):
+    """OCP MX quantization along the last axis (a multiple of 32): returns
+    (codes uint8 with x's shape, scale exponents int32 [..., n/32])."""
+    x = _f64(x)
+    assert x.shape[-1] % 32 == 0
+    codes = np.empty(x.shape, dtype=np.uint8)
+    exps = np.empty(x.shape[:-1] + (x.shape[-1] // 32,), dtype=np.int32)
+    _L().orc_mxfp8_quantize(x.size, _ptr(x), _ptr(codes), _ptr(exps))
+    return codes, exps
+
+
+def mxfp8_dequantize(codes, exps) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    exps = np.ascontiguousarray(exps, dtype=np.int32)
+    y = np.empty(codes.shape)
+    _L().orc_mxfp8_dequantize(codes.size, _ptr(codes), _ptr(exps), _ptr(y))
+    return y
+
+
+def mxfp8_indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:
+    """Indexer scores with q_I and K_I passed through MX-FP8 (blocks of 32
+    along the indexer dim); the products and sums stay in float64."""
+    qd = mxfp8_dequantize(*mxfp8_quantize(q_I))
+    kd = mxfp8_dequantize(*mxfp8_quantize(k_I))
+    return indexer_scores(qd, w, kd, m, q_pos=q_pos)

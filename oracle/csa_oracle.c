@@ -356,3 +356,65 @@ void orc_attention(int64_t Tq, int32_t H, const orc_fmt* f, const double* q, con
     free(keys);
   }
 }
+
+/* ---- (next) block-scaled FP8 indexer inputs ------------------------------ */
+/*
+ * The pages run the indexer's QK product in low precision ([P1] §3.3, last
+ * paragraph: an FP4 lightning indexer that keeps almost all of the bf16
+ * top-k).  These functions restate the OCP Microscaling (MX) format for that
+ * path with FP8 E4M3 elements (the FN variant: no infinities; 0x7f and 0xff
+ * are NaN; largest finite 448): blocks of 32 consecutive elements share one
+ * power-of-two scale X = 2^(floor(log2(amax)) - 8), 8 being E4M3's largest
+ * exponent; each element is the E4M3 value nearest to v / X (ties to the code
+ * with an even mantissa), saturated to +-448.
+ */
+
+/* Value of an E4M3 code. */
+double orc_e4m3_value(uint8_t code) {
+  int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  double mag = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
+/* Nearest E4M3 code to x by search over every finite magnitude code; ties go
+ * to the even code; |x| beyond 448 saturates; NaN maps to 0x7f. */
+uint8_t orc_e4m3_encode(double x) {
+  if (isnan(x)) return 0x7f;
+  double a = fabs(x);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c < 0x7f; ++c) {   /* 0x00 .. 0x7e: every finite magnitude */
+    double err = fabs(orc_e4m3_value((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = c;
+      best_err = err;
+    }
+  }
+  if (best == 0) return 0x00;   /* +0 for both signs: the sign of zero is not kept */
+  return (uint8_t)(x < 0 ? (best | 0x80) : best);
+}
+
+/* MX quantization of n elements (n a multiple of 32): codes[n], exps[n/32]
+ * (the scale exponent; an all-zero block gets -127). */
+void orc_mxfp8_quantize(int64_t n, const double* x, uint8_t* codes, int32_t* exps) {
+  for (int64_t b = 0; b < n / 32; ++b) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) {
+      double a = fabs(x[b * 32 + i]);
+      if (a > amax) amax = a;
+    }
+    int e = -127;
+    if (amax > 0.0) {
+      e = (int)floor(log2(amax)) - 8;
+      if (e < -127) e = -127;
+      if (e > 127) e = 127;
+    }
+    exps[b] = e;
+    for (int i = 0; i < 32; ++i) codes[b * 32 + i] = orc_e4m3_encode(ldexp(x[b * 32 + i], -e));
+  }
+}
+
+void orc_mxfp8_dequantize(int64_t n, const uint8_t* codes, const int32_t* exps, double* y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = ldexp(orc_e4m3_value(codes[i]), exps[i / 32]);
+}

@@ -2,7 +2,8 @@
 
 Each case plants one mistake in a copy of ``oracle/csa_oracle.c`` (a text
 substitution that must match the source exactly once), builds it, and runs
-``test_oracle_pins.py`` against that build in a child process.  The planted
+``test_oracle_pins.py`` and ``test_oracle_mxfp8.py`` against that build in a
+child process.  The planted
 build must fail at least two pins.  The real oracle is never modified; the
 mutants live in a temporary directory.
 """
@@ -53,6 +54,12 @@ MUTANTS = [
      "orc_rope_inplace(o, c, f->rope_dims, f->rope_base, (double)pos);"),
     ("logit scale 1/c",
      "scale = 1.0 / sqrt((double)c);", "scale = 1.0 / (double)c;"),
+    ("E4M3 exponent bias 8",
+     "ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
+    ("E4M3 ties to the odd code",
+     "(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+    ("MX scale without E4M3's largest exponent",
+     "e = (int)floor(log2(amax)) - 8;", "e = (int)floor(log2(amax));"),
 ]
 
 
@@ -70,10 +77,11 @@ def _build(tmp, i, old, new):
 
 def _failed_pins(lib):
     env = dict(os.environ, CSA_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
-    p = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests",
-                        "test_oracle_pins.py"), "-q", "-p", "no:cacheprovider", "--maxfail=2",
-                        "-m", "not gpu"], env=env, capture_output=True, text=True, timeout=600,
-                       cwd=ROOT)
+    p = subprocess.run([sys.executable, "-m", "pytest",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_mxfp8.py"), "-q", "-p",
+                        "no:cacheprovider", "--maxfail=2", "-m", "not gpu"], env=env,
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
     m = re.search(r"(\d+) failed", p.stdout)
     return int(m.group(1)) if m else 0, p.stdout[-2000:]
 
