@@ -93,10 +93,17 @@ def _L():
         _lib.orc_e4m3_encode.restype = ctypes.c_uint8
         _lib.orc_mxfp8_quantize.argtypes = [i64, P, P, P]
         _lib.orc_mxfp8_dequantize.argtypes = [i64, P, P, P]
+        _lib.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        _lib.orc_e2m1_value.restype = f64
+        _lib.orc_e2m1_encode.argtypes = [f64]
+        _lib.orc_e2m1_encode.restype = ctypes.c_uint8
+        _lib.orc_mxfp4_quantize.argtypes = [i64, P, P, P]
+        _lib.orc_mxfp4_dequantize.argtypes = [i64, P, P, P]
         for fn in (
             "orc_rmsnorm", "orc_rope", "orc_csa_compress", "orc_hca_compress",
             "orc_window_rows", "orc_indexer_scores", "orc_topk", "orc_attention",
-            "orc_mxfp8_quantize", "orc_mxfp8_dequantize",
+            "orc_mxfp8_quantize", "orc_mxfp8_dequantize", "orc_mxfp4_quantize",
+            "orc_mxfp4_dequantize",
         ):
             getattr(_lib, fn).restype = None
     return _lib
@@ -276,4 +283,41 @@ def mxfp8_indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:
     along the indexer dim); the products and sums stay in float64."""
     qd = mxfp8_dequantize(*mxfp8_quantize(q_I))
     kd = mxfp8_dequantize(*mxfp8_quantize(k_I))
+    return indexer_scores(qd, w, kd, m, q_pos=q_pos)
+
+
+def e2m1_value(code: int) -> float:
+    """Value of an FP4 E2M1 code (4 bits)."""
+    return float(_L().orc_e2m1_value(int(code)))
+
+
+def e2m1_encode(x: float) -> int:
+    """Nearest E2M1 code (ties to the even code, saturating at +-6)."""
+    return int(_L().orc_e2m1_encode(float(x)))
+
+
+def mxfp4_quantize(x):
+    """OCP MX quantization with E2M1 elements along the last axis (a multiple
+    of 32): (codes uint8 holding 4-bit codes, scale exponents int32)."""
+    x = _f64(x)
+    assert x.shape[-1] % 32 == 0
+    codes = np.empty(x.shape, dtype=np.uint8)
+    exps = np.empty(x.shape[:-1] + (x.shape[-1] // 32,), dtype=np.int32)
+    _L().orc_mxfp4_quantize(x.size, _ptr(x), _ptr(codes), _ptr(exps))
+    return codes, exps
+
+
+def mxfp4_dequantize(codes, exps) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    exps = np.ascontiguousarray(exps, dtype=np.int32)
+    y = np.empty(codes.shape)
+    _L().orc_mxfp4_dequantize(codes.size, _ptr(codes), _ptr(exps), _ptr(y))
+    return y
+
+
+def mxfp4_indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:
+    """Indexer scores with q_I and K_I passed through MX-FP4 (blocks of 32
+    along the indexer dim); the products and sums stay in float64."""
+    qd = mxfp4_dequantize(*mxfp4_quantize(q_I))
+    kd = mxfp4_dequantize(*mxfp4_quantize(k_I))
     return indexer_scores(qd, w, kd, m, q_pos=q_pos)

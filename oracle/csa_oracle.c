@@ -418,3 +418,53 @@ void orc_mxfp8_quantize(int64_t n, const double* x, uint8_t* codes, int32_t* exp
 void orc_mxfp8_dequantize(int64_t n, const uint8_t* codes, const int32_t* exps, double* y) {
   for (int64_t i = 0; i < n; ++i) y[i] = ldexp(orc_e4m3_value(codes[i]), exps[i / 32]);
 }
+
+/*
+ * The same MX scheme with FP4 E2M1 elements (the pages' indexer precision):
+ * 4-bit codes, sign bit 3, a 2-bit exponent with bias 1 and one mantissa bit,
+ * so the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6; blocks of 32 share the
+ * scale 2^(floor(log2(amax)) - 2), 2 being E2M1's largest exponent.
+ */
+double orc_e2m1_value(uint8_t code) {
+  int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  double mag = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, e - 1);
+  return sign ? -mag : mag;
+}
+
+/* Nearest E2M1 code (ties to the even code), saturating at +-6. */
+uint8_t orc_e2m1_encode(double x) {
+  double a = fabs(x);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c < 8; ++c) {
+    double err = fabs(orc_e2m1_value((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = c;
+      best_err = err;
+    }
+  }
+  if (best == 0) return 0;
+  return (uint8_t)(x < 0 ? (best | 8) : best);
+}
+
+void orc_mxfp4_quantize(int64_t n, const double* x, uint8_t* codes, int32_t* exps) {
+  for (int64_t b = 0; b < n / 32; ++b) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) {
+      double a = fabs(x[b * 32 + i]);
+      if (a > amax) amax = a;
+    }
+    int e = -127;
+    if (amax > 0.0) {
+      e = (int)floor(log2(amax)) - 2;
+      if (e < -127) e = -127;
+      if (e > 127) e = 127;
+    }
+    exps[b] = e;
+    for (int i = 0; i < 32; ++i) codes[b * 32 + i] = orc_e2m1_encode(ldexp(x[b * 32 + i], -e));
+  }
+}
+
+void orc_mxfp4_dequantize(int64_t n, const uint8_t* codes, const int32_t* exps, double* y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = ldexp(orc_e2m1_value(codes[i]), exps[i / 32]);
+}

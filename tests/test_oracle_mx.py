@@ -117,3 +117,58 @@ def test_mx_indexer_top_k_recall_on_the_workload_distribution():
     rec = [len(set(a[t][a[t] >= 0]) & set(b[t][b[t] >= 0])) / max(1, (a[t] >= 0).sum())
            for t in range(T) if (a[t] >= 0).any()]
     assert np.mean(rec) >= 0.95
+
+
+# ---------------------------------------------------------------- FP4 (E2M1)
+
+def test_e2m1_format_values():
+    mags = [oracle.e2m1_value(c) for c in range(8)]
+    assert mags == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert [oracle.e2m1_value(8 + c) for c in range(1, 8)] == [-x for x in mags[1:]]
+
+
+def test_e2m1_round_trip_ties_and_saturation():
+    for c in list(range(8)) + list(range(9, 16)):
+        assert oracle.e2m1_encode(oracle.e2m1_value(c)) == c
+    # midpoints go to the code with an even mantissa bit
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for x, want in ties.items():
+        assert oracle.e2m1_value(oracle.e2m1_encode(x)) == want, x
+        assert oracle.e2m1_value(oracle.e2m1_encode(-x)) == -want, x
+    for x in (6.5, 7.0, 100.0):
+        assert oracle.e2m1_value(oracle.e2m1_encode(x)) == 6.0
+        assert oracle.e2m1_value(oracle.e2m1_encode(-x)) == -6.0
+    sweep = np.linspace(-8, 8, 4001)
+    vals = [oracle.e2m1_value(oracle.e2m1_encode(x)) for x in sweep]
+    assert all(a <= b for a, b in zip(vals, vals[1:]))
+    for x in sweep:   # nearest: no magnitude is closer than the chosen one
+        y = oracle.e2m1_value(oracle.e2m1_encode(x))
+        best = min(abs(abs(x) - v) for v in [0, 0.5, 1, 1.5, 2, 3, 4, 6])
+        assert abs(abs(y) - min(abs(x), 6.0)) <= best + 1e-12 or abs(x) > 6
+
+
+@pytest.mark.parametrize("amax,exp", [(1.0, -2), (6.0, 0), (0.3, -4), (2.0 ** 10, 8)])
+def test_mxfp4_block_scale(amax, exp):
+    x = np.zeros(32)
+    x[9] = amax
+    codes, exps = oracle.mxfp4_quantize(x)
+    assert exps.tolist() == [exp]
+    y = oracle.mxfp4_dequantize(codes, exps)
+    # amax / X lies in [4, 8): it is exact when it is a code (4 or 6), else it
+    # rounds to the nearest code or clips to 6
+    r = amax / 2.0 ** exp
+    want = min((4.0, 6.0), key=lambda v: abs(v - r)) if r < 7 else 6.0
+    assert y[9] == want * 2.0 ** exp
+
+
+def test_mx_fp4_indexer_top_k_recall_on_the_workload_distribution():
+    rng = np.random.default_rng(0)
+    T, HI, dI, N, m, k = 256, 64, 128, 64, 4, 16
+    q = rng.standard_normal((T, HI, dI)) / np.sqrt(dI)
+    kk = rng.standard_normal((N, dI)) / np.sqrt(dI)
+    w = rng.standard_normal((T, HI)) / 8
+    a = oracle.topk(oracle.indexer_scores(q, w, kk, m), k, m)
+    b = oracle.topk(oracle.mxfp4_indexer_scores(q, w, kk, m), k, m)
+    rec = [len(set(a[t][a[t] >= 0]) & set(b[t][b[t] >= 0])) / max(1, (a[t] >= 0).sum())
+           for t in range(T) if (a[t] >= 0).any()]
+    assert np.mean(rec) >= 0.90
