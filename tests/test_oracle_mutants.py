@@ -57,7 +57,15 @@ MUTANTS = [
     ("E4M3 exponent bias 8",
      "ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
     ("E4M3 ties to the odd code",
-     "(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+     "double err = fabs(orc_e4m3_value((uint8_t)c) - a);\n"
+     "    if (err < best_err || (err == best_err && (c & 1) == 0)) {",
+     "double err = fabs(orc_e4m3_value((uint8_t)c) - a);\n"
+     "    if (err < best_err || (err == best_err && (c & 1) == 1)) {"),
+    ("E2M1 ties to the odd code",
+     "double err = fabs(orc_e2m1_value((uint8_t)c) - a);\n"
+     "    if (err < best_err || (err == best_err && (c & 1) == 0)) {",
+     "double err = fabs(orc_e2m1_value((uint8_t)c) - a);\n"
+     "    if (err < best_err || (err == best_err && (c & 1) == 1)) {"),
     ("MX scale without E4M3's largest exponent",
      "e = (int)floor(log2(amax)) - 8;", "e = (int)floor(log2(amax));"),
     ("E2M1 exponent bias 0",

@@ -147,7 +147,7 @@ def test_e2m1_round_trip_ties_and_saturation():
         assert abs(abs(y) - min(abs(x), 6.0)) <= best + 1e-12 or abs(x) > 6
 
 
-@pytest.mark.parametrize("amax,exp", [(1.0, -2), (6.0, 0), (0.3, -4), (2.0 ** 10, 8)])
+@pytest.mark.parametrize("amax,exp", [(1.0, -2), (6.0, 0), (0.3, -4), (2.0 ** 10, 8), (5.0, 0)])
 def test_mxfp4_block_scale(amax, exp):
     x = np.zeros(32)
     x[9] = amax
@@ -155,7 +155,7 @@ def test_mxfp4_block_scale(amax, exp):
     assert exps.tolist() == [exp]
     y = oracle.mxfp4_dequantize(codes, exps)
     # amax / X lies in [4, 8): it is exact when it is a code (4 or 6), else it
-    # rounds to the nearest code or clips to 6
+    # rounds to the nearest code (5 is a tie: to 4, the even code) or clips to 6
     r = amax / 2.0 ** exp
     want = min((4.0, 6.0), key=lambda v: abs(v - r)) if r < 7 else 6.0
     assert y[9] == want * 2.0 ** exp
