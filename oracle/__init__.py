@@ -99,6 +99,10 @@ def _L():
         _lib.orc_e2m1_encode.restype = ctypes.c_uint8
         _lib.orc_mxfp4_quantize.argtypes = [i64, P, P, P]
         _lib.orc_mxfp4_dequantize.argtypes = [i64, P, P, P]
+        _lib.orc_stream_state_len.argtypes = [i32, i32, i32]
+        _lib.orc_stream_state_len.restype = i64
+        _lib.orc_stream_append.argtypes = [i32, i32, FP, i64, P, P, P, P, i32, P, P, P]
+        _lib.orc_stream_append.restype = i32
         for fn in (
             "orc_rmsnorm", "orc_rope", "orc_csa_compress", "orc_hca_compress",
             "orc_window_rows", "orc_indexer_scores", "orc_topk", "orc_attention",
@@ -321,3 +325,28 @@ def mxfp4_indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:
     qd = mxfp4_dequantize(*mxfp4_quantize(q_I))
     kd = mxfp4_dequantize(*mxfp4_quantize(k_I))
     return indexer_scores(qd, w, kd, m, q_pos=q_pos)
+
+
+# ---- (next) streaming compression for decode ---------------------------------
+
+class Stream:
+    """One sequence's compression state for decode: tokens arrive one at a
+    time; each yields its window row, and the token that completes block s
+    also yields entry s.  ``overlap`` selects CSA (two groups, the previous
+    block's group b) or HCA (one group)."""
+
+    def __init__(self, m: int, fmt: Fmt, z_cols: int, overlap: bool = True, pos0: int = 0):
+        self.m, self.fmt, self.z_cols, self.overlap, self.pos0 = m, fmt, z_cols, overlap, pos0
+        self.state = np.zeros(_L().orc_stream_state_len(m, fmt.c, z_cols))
+
+    def append(self, kv_a, z_a, kv_b=None, z_b=None):
+        kv_a, z_a = _f64(kv_a).reshape(-1), _f64(z_a).reshape(-1)
+        if self.overlap:
+            kv_b, z_b = _f64(kv_b).reshape(-1), _f64(z_b).reshape(-1)
+        win = np.empty(self.fmt.c)
+        ent = np.empty(self.fmt.c)
+        f = self.fmt._c()
+        done = _L().orc_stream_append(self.m, int(self.overlap), ctypes.byref(f), self.pos0,
+                                      _ptr(kv_a), _ptr(kv_b), _ptr(z_a), _ptr(z_b), self.z_cols,
+                                      _ptr(self.state), _ptr(win), _ptr(ent))
+        return win, (ent if done else None)

@@ -468,3 +468,68 @@ void orc_mxfp4_quantize(int64_t n, const double* x, uint8_t* codes, int32_t* exp
 void orc_mxfp4_dequantize(int64_t n, const uint8_t* codes, const int32_t* exps, double* y) {
   for (int64_t i = 0; i < n; ++i) y[i] = ldexp(orc_e2m1_value(codes[i]), exps[i / 32]);
 }
+
+/* ---- (next) streaming compression for decode ----------------------------- */
+/*
+ * Decode appends one token at a time ([P1] §3.5: the KV of an unfinished
+ * block waits in a tail buffer until the block completes).  The state of one
+ * sequence, caller-owned, for rate m and overlap (CSA) or not (HCA):
+ *   state[0]                 tokens appended so far (as a double)
+ *   rows:  cur_a[m][c], cur_b[m][c], prev_b[m][c]   (values)
+ *   logit: cur_za[m][zc], cur_zb[m][zc], prev_zb[m][zc]
+ * orc_stream_state_len() gives its length in doubles.  Each append writes the
+ * token's window row; when the token completes block s it writes entry s
+ * (pooled over the block's a rows and, for CSA with s >= 1, the previous
+ * block's b rows, then RMSNorm and RoPE at pos0 + m s) and returns 1.
+ */
+int64_t orc_stream_state_len(int32_t m, int32_t c, int32_t z_cols) {
+  return 1 + 3 * (int64_t)m * c + 3 * (int64_t)m * z_cols;
+}
+
+int32_t orc_stream_append(int32_t m, int32_t overlap, const orc_fmt* f, int64_t pos0,
+                          const double* kv_a, const double* kv_b, const double* z_a,
+                          const double* z_b, int32_t z_cols, double* state, double* win_row,
+                          double* entry) {
+  int c = f->c;
+  int64_t t = (int64_t)state[0];
+  double* cur_a = state + 1;
+  double* cur_b = cur_a + (size_t)m * c;
+  double* prev_b = cur_b + (size_t)m * c;
+  double* cur_za = prev_b + (size_t)m * c;
+  double* cur_zb = cur_za + (size_t)m * z_cols;
+  double* prev_zb = cur_zb + (size_t)m * z_cols;
+  int j = (int)(t % m);
+  memcpy(cur_a + (size_t)j * c, kv_a, sizeof(double) * (size_t)c);
+  memcpy(cur_za + (size_t)j * z_cols, z_a, sizeof(double) * (size_t)z_cols);
+  if (overlap) {
+    memcpy(cur_b + (size_t)j * c, kv_b, sizeof(double) * (size_t)c);
+    memcpy(cur_zb + (size_t)j * z_cols, z_b, sizeof(double) * (size_t)z_cols);
+  }
+  memcpy(win_row, kv_a, sizeof(double) * (size_t)c);
+  orc_norm_rope(win_row, f, (double)(pos0 + t));
+  state[0] = (double)(t + 1);
+  if (j != m - 1) return 0;
+  int64_t s = t / m;
+  const double** rows = (const double**)malloc(sizeof(double*) * (size_t)(2 * m));
+  const double** lg = (const double**)malloc(sizeof(double*) * (size_t)(2 * m));
+  int ns = 0;
+  for (int i = 0; i < m; ++i, ++ns) {
+    rows[ns] = cur_a + (size_t)i * c;
+    lg[ns] = cur_za + (size_t)i * z_cols;
+  }
+  if (overlap && s >= 1) {
+    for (int i = 0; i < m; ++i, ++ns) {
+      rows[ns] = prev_b + (size_t)i * c;
+      lg[ns] = prev_zb + (size_t)i * z_cols;
+    }
+  }
+  orc_pool(c, ns, rows, lg, z_cols, entry, NULL);
+  free(rows);
+  free(lg);
+  orc_norm_rope(entry, f, (double)(pos0 + m * s));
+  if (overlap) {   /* this block's b rows serve the next entry */
+    memcpy(prev_b, cur_b, sizeof(double) * (size_t)m * c);
+    memcpy(prev_zb, cur_zb, sizeof(double) * (size_t)m * z_cols);
+  }
+  return 1;
+}

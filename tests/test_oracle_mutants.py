@@ -2,8 +2,8 @@
 
 Each case plants one mistake in a copy of ``oracle/csa_oracle.c`` (a text
 substitution that must match the source exactly once), builds it, and runs
-``test_oracle_pins.py`` and ``test_oracle_mx.py`` against that build in a
-child process.  The planted
+``test_oracle_pins.py``, ``test_oracle_mx.py`` and ``test_oracle_stream.py``
+against that build in a child process.  The planted
 build must fail at least two pins.  The real oracle is never modified; the
 mutants live in a temporary directory.
 """
@@ -68,6 +68,13 @@ MUTANTS = [
      "    if (err < best_err || (err == best_err && (c & 1) == 1)) {"),
     ("MX scale without E4M3's largest exponent",
      "e = (int)floor(log2(amax)) - 8;", "e = (int)floor(log2(amax));"),
+    ("stream hands a block's b rows on before pooling it",
+     "  orc_pool(c, ns, rows, lg, z_cols, entry, NULL);\n  free(rows);",
+     "  if (overlap) memcpy(prev_b, cur_b, sizeof(double) * (size_t)m * c);\n"
+     "  orc_pool(c, ns, rows, lg, z_cols, entry, NULL);\n  free(rows);"),
+    ("stream entry rotated at the completing token",
+     "  orc_norm_rope(entry, f, (double)(pos0 + m * s));\n  if (overlap) {",
+     "  orc_norm_rope(entry, f, (double)(pos0 + t));\n  if (overlap) {"),
     ("E2M1 exponent bias 0",
      "ldexp(1.0 + 0.5 * (double)m, e - 1)", "ldexp(1.0 + 0.5 * (double)m, e)"),
     ("MX-FP4 scale with E4M3's largest exponent",
@@ -91,7 +98,8 @@ def _failed_pins(lib):
     env = dict(os.environ, CSA_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
     p = subprocess.run([sys.executable, "-m", "pytest",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_mx.py"), "-q", "-p",
+                        os.path.join(ROOT, "tests", "test_oracle_mx.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_stream.py"), "-q", "-p",
                         "no:cacheprovider", "--maxfail=2", "-m", "not gpu"], env=env,
                        capture_output=True, text=True, timeout=600, cwd=ROOT)
     m = re.search(r"(\d+) failed", p.stdout)
