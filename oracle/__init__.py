@@ -99,6 +99,12 @@ def _L():
         _lib.orc_e2m1_encode.restype = ctypes.c_uint8
         _lib.orc_mxfp4_quantize.argtypes = [i64, P, P, P]
         _lib.orc_mxfp4_dequantize.argtypes = [i64, P, P, P]
+        _lib.orc_bf16_round.argtypes = [f64]
+        _lib.orc_bf16_round.restype = f64
+        _lib.orc_mixed_store.argtypes = [i64, i32, i32, P, P, P, P]
+        _lib.orc_mixed_store.restype = None
+        _lib.orc_mixed_load.argtypes = [i64, i32, i32, P, P, P, P]
+        _lib.orc_mixed_load.restype = None
         _lib.orc_stream_state_len.argtypes = [i32, i32, i32]
         _lib.orc_stream_state_len.restype = i64
         _lib.orc_stream_append.argtypes = [i32, i32, FP, i64, P, P, P, P, i32, P, P, P]
@@ -350,3 +356,35 @@ class Stream:
                                       _ptr(kv_a), _ptr(kv_b), _ptr(z_a), _ptr(z_b), self.z_cols,
                                       _ptr(self.state), _ptr(win), _ptr(ent))
         return win, (ent if done else None)
+
+
+# ---- (next) mixed BF16 / FP8 storage of KV entries ----------------------------
+
+def bf16_round(x: float) -> float:
+    """Nearest BF16 value (ties to even)."""
+    return float(_L().orc_bf16_round(float(x)))
+
+
+def mixed_store(entries, rope_dims: int):
+    """Entries [n, c] -> (FP8 codes [n, c-r], MX exponents [n, (c-r)/32],
+    BF16 RoPE dims [n, r] as float64)."""
+    x = _f64(entries)
+    n, c = x.shape
+    cq = c - rope_dims
+    assert cq % 32 == 0
+    codes = np.empty((n, cq), dtype=np.uint8)
+    exps = np.empty((n, cq // 32), dtype=np.int32)
+    rope_part = np.empty((n, rope_dims))
+    _L().orc_mixed_store(n, c, rope_dims, _ptr(x), _ptr(codes), _ptr(exps), _ptr(rope_part))
+    return codes, exps, rope_part
+
+
+def mixed_load(codes, exps, rope_part) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    exps = np.ascontiguousarray(exps, dtype=np.int32)
+    rope_part = _f64(rope_part)
+    n, cq = codes.shape
+    r = rope_part.shape[1]
+    out = np.empty((n, cq + r))
+    _L().orc_mixed_load(n, cq + r, r, _ptr(codes), _ptr(exps), _ptr(rope_part), _ptr(out))
+    return out

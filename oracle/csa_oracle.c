@@ -533,3 +533,44 @@ int32_t orc_stream_append(int32_t m, int32_t overlap, const orc_fmt* f, int64_t 
   }
   return 1;
 }
+
+/* ---- (next) mixed BF16 / FP8 storage of KV entries ----------------------- */
+/*
+ * The pages store KV entries in mixed precision ([P1] §3.3, last paragraph:
+ * the RoPE dims in BF16, the rest in FP8).  Reading taken: the last r dims
+ * (RoPE) are rounded to BF16; the first c - r dims are MX-FP8 (E4M3, blocks
+ * of 32 along the entry, as orc_mxfp8_quantize).
+ */
+
+/* Nearest BF16 value to x (8 significant bits, ties to even, the exponent
+ * range of float32 with its subnormals; beyond the largest finite: inf). */
+double orc_bf16_round(double x) {
+  if (x == 0.0 || isnan(x) || isinf(x)) return x;
+  int e = (int)floor(log2(fabs(x)));
+  if (e < -126) e = -126;                 /* subnormal spacing 2^-133 */
+  double q = ldexp(1.0, e - 7);
+  double y = rint(x / q) * q;             /* rint: round half to even */
+  if (fabs(y) > ldexp(2.0 - ldexp(1.0, -7), 127)) return x > 0 ? INFINITY : -INFINITY;
+  return y;
+}
+
+/* Stores n entries of c dims (c - r a multiple of 32): codes[n][c-r],
+ * exps[n][(c-r)/32], rope[n][r] (BF16 values held as doubles); loads them
+ * back into out[n][c]. */
+void orc_mixed_store(int64_t n, int32_t c, int32_t r, const double* x, uint8_t* codes,
+                     int32_t* exps, double* rope) {
+  int cq = c - r;
+  for (int64_t i = 0; i < n; ++i) {
+    orc_mxfp8_quantize(cq, x + i * c, codes + i * cq, exps + i * (cq / 32));
+    for (int d = 0; d < r; ++d) rope[i * r + d] = orc_bf16_round(x[i * c + cq + d]);
+  }
+}
+
+void orc_mixed_load(int64_t n, int32_t c, int32_t r, const uint8_t* codes, const int32_t* exps,
+                    const double* rope, double* out) {
+  int cq = c - r;
+  for (int64_t i = 0; i < n; ++i) {
+    orc_mxfp8_dequantize(cq, codes + i * cq, exps + i * (cq / 32), out + i * c);
+    for (int d = 0; d < r; ++d) out[i * c + cq + d] = rope[i * r + d];
+  }
+}

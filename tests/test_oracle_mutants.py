@@ -2,8 +2,9 @@
 
 Each case plants one mistake in a copy of ``oracle/csa_oracle.c`` (a text
 substitution that must match the source exactly once), builds it, and runs
-``test_oracle_pins.py``, ``test_oracle_mx.py`` and ``test_oracle_stream.py``
-against that build in a child process.  The planted
+the oracle's pin suites (``test_oracle_pins.py``, ``test_oracle_mx.py``,
+``test_oracle_stream.py``, ``test_oracle_mixed.py``) against that build in a
+child process.  The planted
 build must fail at least two pins.  The real oracle is never modified; the
 mutants live in a temporary directory.
 """
@@ -75,6 +76,11 @@ MUTANTS = [
     ("stream entry rotated at the completing token",
      "  orc_norm_rope(entry, f, (double)(pos0 + m * s));\n  if (overlap) {",
      "  orc_norm_rope(entry, f, (double)(pos0 + t));\n  if (overlap) {"),
+    ("BF16 rounding by truncation",
+     "double y = rint(x / q) * q;", "double y = trunc(x / q) * q;"),
+    ("mixed storage keeps the first r dims in BF16",
+     "for (int d = 0; d < r; ++d) rope[i * r + d] = orc_bf16_round(x[i * c + cq + d]);",
+     "for (int d = 0; d < r; ++d) rope[i * r + d] = orc_bf16_round(x[i * c + d]);"),
     ("E2M1 exponent bias 0",
      "ldexp(1.0 + 0.5 * (double)m, e - 1)", "ldexp(1.0 + 0.5 * (double)m, e)"),
     ("MX-FP4 scale with E4M3's largest exponent",
@@ -99,7 +105,8 @@ def _failed_pins(lib):
     p = subprocess.run([sys.executable, "-m", "pytest",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                         os.path.join(ROOT, "tests", "test_oracle_mx.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_stream.py"), "-q", "-p",
+                        os.path.join(ROOT, "tests", "test_oracle_stream.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_mixed.py"), "-q", "-p",
                         "no:cacheprovider", "--maxfail=2", "-m", "not gpu"], env=env,
                        capture_output=True, text=True, timeout=600, cwd=ROOT)
     m = re.search(r"(\d+) failed", p.stdout)
