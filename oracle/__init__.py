@@ -388,3 +388,23 @@ def mixed_load(codes, exps, rope_part) -> np.ndarray:
     out = np.empty((n, cq + r))
     _L().orc_mixed_load(n, cq + r, r, _ptr(codes), _ptr(exps), _ptr(rope_part), _ptr(out))
     return out
+
+
+# ---- (next) grouped output projection ----------------------------------------
+
+def grouped_output_projection(o, w_group, w_out) -> np.ndarray:
+    """The attention output's grouped projection (page "DeepSeek-V4：迈向高效
+    百万 Token 上下文智能", §3.3, CSA paragraph: c n_h is large, so the heads'
+    outputs are first projected group by group to an intermediate dim d_g,
+    then concatenated and projected back to d).  Reading taken: the H heads
+    split into g consecutive groups of H/g heads.
+
+    o: [T, H, c]; w_group: [g, d_g, (H/g) c]; w_out: [d, g d_g].  Returns
+    [T, d] = w_out . concat_j(w_group[j] . concat(o[:, heads of group j]))."""
+    o, w_group, w_out = _f64(o), _f64(w_group), _f64(w_out)
+    T, H, c = o.shape
+    g, dg, gin = w_group.shape
+    assert H % g == 0 and gin == (H // g) * c and w_out.shape[1] == g * dg
+    u = o.reshape(T, g, (H // g) * c)                     # each group's heads, concatenated
+    v = np.einsum("tgi,gdi->tgd", u, w_group)            # [T, g, d_g]
+    return v.reshape(T, g * dg) @ w_out.T
