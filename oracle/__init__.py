@@ -99,6 +99,10 @@ def _L():
         _lib.orc_e2m1_encode.restype = ctypes.c_uint8
         _lib.orc_mxfp4_quantize.argtypes = [i64, P, P, P]
         _lib.orc_mxfp4_dequantize.argtypes = [i64, P, P, P]
+        _lib.orc_nvfp4_quantize.argtypes = [i64, P, P, P, P]
+        _lib.orc_nvfp4_quantize.restype = None
+        _lib.orc_nvfp4_dequantize.argtypes = [i64, P, P, f64, P]
+        _lib.orc_nvfp4_dequantize.restype = None
         _lib.orc_bf16_round.argtypes = [f64]
         _lib.orc_bf16_round.restype = f64
         _lib.orc_mixed_store.argtypes = [i64, i32, i32, P, P, P, P]
@@ -323,6 +327,34 @@ def mxfp4_dequantize(codes, exps) -> np.ndarray:
     y = np.empty(codes.shape)
     _L().orc_mxfp4_dequantize(codes.size, _ptr(codes), _ptr(exps), _ptr(y))
     return y
+
+
+def nvfp4_quantize(x):
+    """FP4 with E4M3 scales per 16 elements and one float scale for the whole
+    array: (codes uint8 [x.shape], block scales uint8 [n/16], tensor scale)."""
+    x = _f64(x)
+    assert x.size % 16 == 0
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scales = np.empty(x.size // 16, dtype=np.uint8)
+    g = ctypes.c_double(0.0)
+    _L().orc_nvfp4_quantize(x.size, _ptr(x), _ptr(codes), _ptr(scales), ctypes.byref(g))
+    return codes, scales, g.value
+
+
+def nvfp4_dequantize(codes, scales, gscale) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    y = np.empty(codes.shape)
+    _L().orc_nvfp4_dequantize(codes.size, _ptr(codes), _ptr(scales), float(gscale), _ptr(y))
+    return y
+
+
+def nvfp4_indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:
+    """Indexer scores with q_I and K_I passed through the 16-element-block FP4
+    layout (one tensor scale each); float64 products and sums."""
+    qd = nvfp4_dequantize(*nvfp4_quantize(q_I))
+    kd = nvfp4_dequantize(*nvfp4_quantize(k_I))
+    return indexer_scores(qd, w, kd, m, q_pos=q_pos)
 
 
 def mxfp4_indexer_scores(q_I, w, k_I, m: int, q_pos=None) -> np.ndarray:

@@ -574,3 +574,34 @@ void orc_mixed_load(int64_t n, int32_t c, int32_t r, const uint8_t* codes, const
     for (int d = 0; d < r; ++d) out[i * c + cq + d] = rope[i * r + d];
   }
 }
+
+/*
+ * FP4 with finer scales (the NVFP4 layout): blocks of 16 elements, each with
+ * an E4M3 scale, under one float scale per tensor g = amax / (448 * 6).  A
+ * block's scale is the E4M3 value nearest to amax_block / (6 g); its elements
+ * are the E2M1 codes nearest to v / (scale g) (an all-zero scale leaves the
+ * block at zero).
+ */
+void orc_nvfp4_quantize(int64_t n, const double* x, uint8_t* codes, uint8_t* scales,
+                        double* gscale) {
+  double amax = 0.0;
+  for (int64_t i = 0; i < n; ++i)
+    if (fabs(x[i]) > amax) amax = fabs(x[i]);
+  double g = amax > 0.0 ? amax / (448.0 * 6.0) : 1.0;
+  *gscale = g;
+  for (int64_t b = 0; b < n / 16; ++b) {
+    double bmax = 0.0;
+    for (int i = 0; i < 16; ++i)
+      if (fabs(x[b * 16 + i]) > bmax) bmax = fabs(x[b * 16 + i]);
+    uint8_t sc = orc_e4m3_encode(bmax / (6.0 * g));
+    scales[b] = sc;
+    double s = orc_e4m3_value(sc) * g;
+    for (int i = 0; i < 16; ++i) codes[b * 16 + i] = s > 0.0 ? orc_e2m1_encode(x[b * 16 + i] / s) : 0;
+  }
+}
+
+void orc_nvfp4_dequantize(int64_t n, const uint8_t* codes, const uint8_t* scales, double gscale,
+                          double* y) {
+  for (int64_t i = 0; i < n; ++i)
+    y[i] = orc_e2m1_value(codes[i]) * orc_e4m3_value(scales[i / 16]) * gscale;
+}

@@ -81,6 +81,9 @@ MUTANTS = [
     ("mixed storage keeps the first r dims in BF16",
      "for (int d = 0; d < r; ++d) rope[i * r + d] = orc_bf16_round(x[i * c + cq + d]);",
      "for (int d = 0; d < r; ++d) rope[i * r + d] = orc_bf16_round(x[i * c + d]);"),
+    ("FP4 tensor scale without the element format's maximum",
+     "double g = amax > 0.0 ? amax / (448.0 * 6.0) : 1.0;",
+     "double g = amax > 0.0 ? amax / 448.0 : 1.0;"),
     ("E2M1 exponent bias 0",
      "ldexp(1.0 + 0.5 * (double)m, e - 1)", "ldexp(1.0 + 0.5 * (double)m, e)"),
     ("MX-FP4 scale with E4M3's largest exponent",

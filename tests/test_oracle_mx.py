@@ -172,3 +172,45 @@ def test_mx_fp4_indexer_top_k_recall_on_the_workload_distribution():
     rec = [len(set(a[t][a[t] >= 0]) & set(b[t][b[t] >= 0])) / max(1, (a[t] >= 0).sum())
            for t in range(T) if (a[t] >= 0).any()]
     assert np.mean(rec) >= 0.90
+
+
+# ------------------------------------------- FP4 with 16-element E4M3 scales
+
+def test_nvfp4_tensor_and_block_scales():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal(64)
+    x[37] = 5.0 * np.abs(x).max()                 # the tensor's amax
+    codes, scales, g = oracle.nvfp4_quantize(x)
+    assert g == np.abs(x).max() / (448.0 * 6.0)
+    assert scales.shape == (4,) and oracle.e4m3_value(scales[37 // 16]) == 448.0
+    y = oracle.nvfp4_dequantize(codes, scales, g)
+    assert y[37] == x[37]                         # amax -> code 6 under scale 448
+
+
+def test_nvfp4_block_of_representable_values_is_exact():
+    # E2M1 magnitudes times 0.25 in one block, 336 in the next: the tensor
+    # scale is 336 / 2688 = 1/8, the first block's scale 1.5 / (6 / 8) = 2
+    # (an E4M3 value), so every element is exact
+    blk = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -6, -4, -3, -2, -1.5, -1, -0.5, 0]) * 0.25
+    x2 = np.concatenate([blk, np.r_[336.0, np.zeros(15)]])
+    c2, s2, g2 = oracle.nvfp4_quantize(x2)
+    assert g2 == 0.125 and oracle.e4m3_value(s2[0]) == 2.0
+    assert np.array_equal(oracle.nvfp4_dequantize(c2, s2, g2), x2)
+
+
+def test_nvfp4_zero_tensor():
+    z, zs, zg = oracle.nvfp4_quantize(np.zeros(32))
+    assert not z.any() and not zs.any() and zg == 1.0
+
+
+def test_nvfp4_indexer_top_k_recall_on_the_workload_distribution():
+    rng = np.random.default_rng(0)
+    T, HI, dI, N, m, k = 256, 64, 128, 64, 4, 16
+    q = rng.standard_normal((T, HI, dI)) / np.sqrt(dI)
+    kk = rng.standard_normal((N, dI)) / np.sqrt(dI)
+    w = rng.standard_normal((T, HI)) / 8
+    a = oracle.topk(oracle.indexer_scores(q, w, kk, m), k, m)
+    b = oracle.topk(oracle.nvfp4_indexer_scores(q, w, kk, m), k, m)
+    rec = [len(set(a[t][a[t] >= 0]) & set(b[t][b[t] >= 0])) / max(1, (a[t] >= 0).sum())
+           for t in range(T) if (a[t] >= 0).any()]
+    assert np.mean(rec) >= 0.90
