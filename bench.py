@@ -5,8 +5,12 @@ csa_prefill_8k workload (batch 1, 8192 tokens, 64 query heads, entry dim 512
 with RoPE on the last 64 dims, m = 4 -> 2048 entries, indexer 64 x 128 with
 w ~ N(0,1)/8, top-k 512, window 128, per-head sinks):
     csa_compress (entries + window rows) -> indexer_scores_topk -> sparse_mqa_attn.
-Prints one JSON line (see the keys below).  ``--impl reference`` times the
-float64 CPU oracle on a bounded sample of the same workload instead.
+Prints one JSON line (see the keys below).  Beside the headline it carries
+the HCA layer prefill step at hca_prefill_64k (hca_compress -> dense_hca_attn,
+65536 tokens, 512 entries), the two decode workloads and the compression
+kernels alone at 2^20 tokens, each with its roofline and a float64-oracle
+baseline.  ``--impl reference`` times the float64 CPU oracle on a bounded
+sample of the headline workload instead.
 
 Multi-GPU: one process per GPU (torchrun); the path has no exchange step, so
 every rank runs its own replica of the step and ``value`` sums all ranks'
@@ -63,11 +67,25 @@ def compress_bytes(w) -> float:
     return float(w.B * (4 * w.T * w.c + w.n_csa * w.c + w.T * w.c) * e)
 
 
-# DRAM bytes per attention launch at 8192 query rows: dram__bytes_read.sum +
-# dram__bytes_write.sum of the full-size launch list summarised in
-# profiles/csa_prefill_8k_launch_list.md (564.6 MB read + 489.3 MB written).
-# Refresh it whenever the attention kernel changes.
-ATTN_DRAM_BYTES_8K = 564.6e6 + 489.3e6
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch at 8192 query rows, from an ncu capture of the kernel source whose
+# SHA-256 is given.  Reported as the roofline's `traffic` only while the
+# kernel source still has that hash; otherwise null.
+ATTN_TRAFFIC = {"source": "long_context_attention_csa_b200/csrc/attn_tc.cu",
+                "sha256": None, "bytes_per_launch": None}
+
+
+def attn_traffic():
+    import hashlib
+
+    try:
+        with open(os.path.join(ROOT, ATTN_TRAFFIC["source"]), "rb") as fh:
+            h = hashlib.sha256(fh.read()).hexdigest()
+    except OSError:
+        return None, "kernel source not found"
+    if ATTN_TRAFFIC["sha256"] is None or h != ATTN_TRAFFIC["sha256"]:
+        return None, "no ncu capture of the current kernel source"
+    return ATTN_TRAFFIC["bytes_per_launch"], "ncu capture of this kernel source"
 
 
 class Clocks:
@@ -75,8 +93,7 @@ class Clocks:
 
     NVML is read from a background thread every 2 ms (the timed region of a
     default run lasts only tens of milliseconds); the device is matched to
-    torch's by UUID.  Samples are also written to gpurun_out/clocks_rank<i>.csv.
-    Only reads the GPU's state."""
+    torch's by UUID.  Only reads the GPU's state."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -87,7 +104,6 @@ class Clocks:
     def __init__(self, index: int):
         import threading
         self.samples = []
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
         self.stop_evt = threading.Event()
         self.thread = None
         try:
@@ -126,14 +142,6 @@ class Clocks:
             return None
         self.stop_evt.set()
         self.thread.join(timeout=5)
-        try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            with open(self.path, "w") as f:
-                f.write("time,sm_mhz,max_sm_mhz,event_reasons\n")
-                for t, sm, rs in self.samples:
-                    f.write(f"{t:.4f},{sm:.0f},{self.max_mhz:.0f},0x{rs:x}\n")
-        except OSError:
-            pass
         if not self.samples:
             return None
         inside = [x for x in self.samples if t0 <= x[0] <= t1]
@@ -314,6 +322,8 @@ def run_gpu(args):
     decode = {} if args.no_decode else {
         n: measure_decode(n, dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
         for n in DECODE_WORKLOADS}
+    hca = None if args.no_hca else measure_hca_prefill(
+        dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
     comp_1m = None if args.no_decode else measure_compress_1m(dev, min(K, 10), args.warmup)
 
     hbm, bf16, src = peaks()
@@ -321,6 +331,7 @@ def run_gpu(args):
     fl_attn = attn_useful_flops(w)
     fl_idx = indexer_useful_flops(w)
     achieved = fl_attn / (t_attn * 1e-3) / 1e12
+    traffic, traffic_src = attn_traffic()
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -352,10 +363,8 @@ def run_gpu(args):
             },
             "roofline": {"bound": "tensor", "kernel": "sparse_mqa_attn",
                          "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                         "frac": achieved / bf16, "traffic": ATTN_DRAM_BYTES_8K,
-                         "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of the "
-                                           "full-size ncu launch list, "
-                                           "profiles/csa_prefill_8k_launch_list.md",
+                         "frac": achieved / bf16, "traffic": traffic,
+                         "traffic_source": traffic_src,
                          "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)"
                          if src == "measured" else "fallback 1.59 PFLOP/s",
                          "algorithmic_flops_per_launch": fl_attn},
@@ -370,6 +379,8 @@ def run_gpu(args):
         }
         if decode:
             line["decode"] = decode
+        if hca:
+            line["hca_prefill_64k"] = hca
         if comp_1m:
             line["compress_1m_tokens"] = comp_1m
         if ws == 1 and not args.no_cpu_baseline:
@@ -462,6 +473,117 @@ def run_only_hca(args):
     e1.record()
     torch.cuda.synchronize()
     print(json.dumps({"only": args.only, "seq_len": w.T, "ms": e0.elapsed_time(e1) / args.steps}))
+
+
+def hca_attn_flops(w) -> float:
+    """Algorithmic FLOPs of dense_hca_attn: 4 * H * c per (query, key) pair,
+    keys = every visible entry + the window rows present."""
+    t = np.arange(w.T, dtype=np.int64)
+    vis = np.minimum((t + 1) // w.m_prime, w.n_hca)
+    pairs = vis + np.minimum(w.n_win, t + 1)
+    return float(4.0 * w.H * w.c * pairs.sum()) * w.B
+
+
+def hca_compress_bytes(w) -> float:
+    # read kv and z; write entries and window rows
+    return float(w.B * (2 * w.T * w.c + w.n_hca * w.c + w.T * w.c) * 2)
+
+
+def hca_cpu_baseline(w, inp, rows: int):
+    """The float64 oracle on a stratified sample of the HCA prefill workload:
+    compression of the whole sequence (entries and window rows), then dense
+    attention for `rows` query rows evenly spaced over the sequence (first and
+    last included).  Query tokens per second."""
+    import oracle
+
+    fmt = oracle.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
+    kv, z = inp["kv"][0].double().cpu().numpy(), inp["z"][0].double().cpu().numpy()
+    sel = np.linspace(0, w.T - 1, rows).astype(np.int64)
+    q = inp["q"][0][torch.from_numpy(sel).to(inp["q"].device)].double().cpu().numpy()
+    sink = inp["sink"].double().cpu().numpy()
+    t0 = time.perf_counter()
+    ent = oracle.hca_compress(kv, z, w.m_prime, fmt)
+    win = oracle.window_rows(kv, fmt)
+    oracle.attention(q, ent, win, fmt, w.n_win, m_dense=w.m_prime, sink=sink, q_pos=sel)
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{rows} of {w.T} query rows evenly spaced (compression of the whole "
+                      f"sequence, dense attention for those rows), float64, {dt:.1f} s"}
+
+
+def measure_hca_prefill(dev, steps: int, warmup: int, flush, ws_n: int, cpu: bool,
+                        cpu_rows: int = 256):
+    """The HCA layer prefill step at hca_prefill_64k (65536 tokens, m' = 128 ->
+    512 entries, 64 heads, entry dim 512, window 128, sinks):
+    hca_compress (entries + window rows) -> dense_hca_attn.  Tokens/s of the
+    whole step (max over ranks), each stage's time from CUDA events on the
+    launching stream, and the dense attention kernel's tensor roofline."""
+    w = wl.WORKLOADS["hca_prefill_64k"]
+    inp = wl.hca_prefill_inputs(w, dev)
+    fmt = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base)
+    entries = torch.empty((w.B, w.n_hca, w.c), dtype=w.dtype, device=dev)
+    win = torch.empty((w.B, w.T, w.c), dtype=w.dtype, device=dev)
+    out = torch.empty_like(inp["q"])
+    ws_c = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_COMPRESS, 1, w.B, w.T), dev)
+    ws_a = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_DENSE_ATTN, 1, w.B, w.T, w.H, w.c,
+                                                 w.n_hca, 0, w.n_win), dev)
+    s = torch.cuda.current_stream()
+
+    def run(ev=None):
+        if ev:
+            ev[0].record(s)
+        csa.hca_compress(inp["kv"], inp["z"], w.m_prime, fmt, entries=entries, win_out=win,
+                         ws=ws_c)
+        if ev:
+            ev[1].record(s)
+        csa.dense_hca_attn(inp["q"], entries, w.m_prime, win, fmt, w.n_win, sink=inp["sink"],
+                           out=out, ws=ws_a)
+        if ev:
+            ev[2].record(s)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    for ws in (ws_c, ws_a):
+        st, d = csa.csa_check_status(ws)
+        if st:
+            raise RuntimeError(f"hca_prefill_64k: device status {st}/{d}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()          # L2 flushed between timed steps (not timed)
+        run(evs[i])
+    torch.cuda.synchronize()
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[0].elapsed_time(e[2])]
+                    for e in evs])
+    step_ms = allmax(float(per[:, 2].mean()), ws_n)
+    t_comp, t_attn = float(per[:, 0].mean()), float(per[:, 1].mean())
+    st, d = csa.csa_check_status(ws_a)
+    if st:
+        raise RuntimeError(f"hca_prefill_64k: device status {st}/{d}")
+    hbm, bf16, src = peaks()
+    fl = hca_attn_flops(w)
+    achieved = fl / (t_attn * 1e-3) / 1e12
+    res = {
+        "value": w.B * w.T * ws_n / (step_ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
+        "config": {"workload": w.name, "batch": w.B, "seq_len": w.T, "heads": w.H,
+                   "entry_dim": w.c, "rope_dims": w.r, "m_prime": w.m_prime,
+                   "entries": w.n_hca, "n_win": w.n_win, "sink": True,
+                   "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
+        "stages_ms": {"hca_compress": t_comp, "dense_hca_attn": t_attn},
+        "stage_roofline": {"hca_compress": {
+            "bound": "hbm", "achieved_GBps": hca_compress_bytes(w) / (t_comp * 1e-3) / 1e9,
+            "peak": hbm}},
+        "roofline": {"bound": "tensor", "kernel": "dense_hca_attn", "achieved": achieved,
+                     "peak": bf16, "unit": "TFLOP/s", "frac": achieved / bf16, "traffic": None,
+                     "algorithmic_flops_per_launch": fl,
+                     "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)"
+                     if src == "measured" else "fallback 1.59 PFLOP/s"},
+    }
+    if cpu:
+        res["cpu_baseline"] = hca_cpu_baseline(w, inp, cpu_rows)
+    del inp, entries, win, out
+    torch.cuda.empty_cache()
+    return res
 
 
 DECODE_WORKLOADS = ("csa_decode_b32_128k", "decode_pair_b4_1m")
@@ -753,6 +875,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode workloads")
+    ap.add_argument("--no-hca", action="store_true", help="skip the HCA prefill workload")
     args = ap.parse_args()
     if args.only:
         run_only(args)

@@ -67,7 +67,7 @@ typedef int32_t csa_status;
 
 #define CSA_F_NO_NORM 1u   /* skip RMSNorm (test hook) */
 #define CSA_F_NO_ROPE 2u   /* skip RoPE and the output rotation (test hook) */
-#define CSA_F_PORTABLE 4u  /* use the CUDA-core kernels even where a tensor-core kernel exists */
+#define CSA_F_PORTABLE 4u  /* attention: use the CUDA-core kernel even for bf16 (cross-checks) */
 
 /* Entry format shared by all calls.  c: entry / head dim (c/vec a power of two,
  * vec = 8 for bf16, 4 for f32); rope_dims: r, even, <= c, RoPE on dims
@@ -143,6 +143,10 @@ csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, co
  *   zero-filled once before its first use (status word at offset 0).
  * Arithmetic: bf16 products with float32 accumulation (exact for small
  * integer inputs); float32 throughout for CSA_F32.
+ * Kernels: bf16 runs on the tensor cores, which need H_I = 64, d_I = 128,
+ * B <= 65535 and ceil(Tq / 4) <= 65535; other bf16 shapes return
+ * CSA_E_UNSUPPORTED.  float32 runs on CUDA cores for any H_I <= 64,
+ * d_I <= 1024.  q_I and k_I must start on a 16-byte boundary (CSA_E_ARG).
  */
 csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
                                const void* q_I, const float* w, const void* k_I, int64_t N,
@@ -154,15 +158,22 @@ csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I
  * this call: it exists for callers that cannot allocate device memory where
  * they call the indexer (an engine plug-in whose host owns all device memory
  * through its own pool, or a decode loop that must not pay for cudaMalloc and
- * its implicit synchronisation).  Same arguments and results as
+ * its implicit synchronisation).  Same arguments, checks and results as
  * indexer_scores_topk minus ws/ws_bytes.  Its scratch lives in a fixed 8 MiB
  * __device__ array inside libcsa.so that every GPU loading the library holds
- * until exit; a problem needing more (csa_workspace_bytes of the path taken
- * minus the 256-byte status word) is rejected with CSA_E_WORKSPACE.  The first
- * call on each device looks up the array's device address and caches it, so
- * make that first call before any stream capture.  All calls share the array
- * and its contents persist between calls: calls that overlap on the GPU race.
- * Kernel-side status is cleared per call and not reported.  Nothing here calls
+ * until exit.  A call is accepted iff 256 (the status word) + the scratch of
+ * the kernels it takes <= 8 MiB, else CSA_E_WORKSPACE: bf16 (tensor cores)
+ * needs 8 * B * Tq * k * n_chunks bytes when the entries span n_chunks > 1
+ * chunks of 2048 (Tq >= 4) or 4096 (Tq < 4) entries, and none otherwise;
+ * float32 (CUDA cores) needs 4 * B * Tq * N bytes.  For bf16 this equals
+ * csa_workspace_bytes(CSA_OP_INDEXER, ...) <= 8 MiB.  The first call on each
+ * device looks up the array's device address and caches it, so make that
+ * first call before any stream capture.  All calls share the array and its
+ * contents persist between calls: calls that overlap on the GPU race.
+ * Kernel-side status is cleared per call and not reported: after a device-side
+ * error (a bounded wait that ran out) the outputs are unspecified and nothing
+ * tells the caller; use indexer_scores_topk with a workspace and
+ * csa_check_status where that must be detected.  Nothing here calls
  * cudaMalloc, cudaFree or any allocating routine.
  */
 csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I,
@@ -190,7 +201,13 @@ csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int64_t Tq, int
  * The bf16 tensor-core kernel requires the stored keys to be RMS-normalised
  * (as the compression calls produce them): it uses the static logit bound
  * scale*|q^|*sqrt(c) in place of a running maximum and flags CSA_DEV_RANGE
- * when a logit goes more than 60 (natural log) beyond it.
+ * when a logit goes more than 60 (natural log) beyond it (the output is then
+ * invalid).  An index outside [-1, N) is skipped and flagged CSA_DEV_BAD_INDEX.
+ * Kernels: bf16 runs on the tensor cores, which need c = 512, H a multiple of
+ * 64, rope_dims <= 64 and (sparse) k <= 1024; other bf16 shapes return
+ * CSA_E_UNSUPPORTED unless fmt->flags has CSA_F_PORTABLE, which selects the
+ * CUDA-core kernel (float32 always runs there; it keeps an exact running
+ * maximum).
  */
 csa_status sparse_mqa_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
                            const void* q, const int64_t* q_pos, const void* entries, int64_t N,

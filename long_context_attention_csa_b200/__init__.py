@@ -28,9 +28,9 @@ CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS = 1, 2, 3
 CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX = 1, 2, 3
 
 EXPORTED = (
-    "csa_compress", "hca_compress", "indexer_scores_topk", "sparse_mqa_attn", "dense_hca_attn",
-    "csa_workspace_bytes", "csa_check_status", "csa_status_string", "csa_launch_count",
-    "csa_selftest_wait",
+    "csa_compress", "hca_compress", "indexer_scores_topk", "indexer_scores_topk_noalloc",
+    "sparse_mqa_attn", "dense_hca_attn", "csa_workspace_bytes", "csa_check_status",
+    "csa_status_string", "csa_launch_count", "csa_selftest_wait",
 )
 
 
@@ -87,6 +87,8 @@ def lib():
     L.hca_compress.argtypes = [i32, i64, i64, i32, FP, P, P, i32, i64, P, P, P, sz, P]
     L.indexer_scores_topk.argtypes = [i32, i64, i64, i32, i32, P, P, P, i64, P, i32, i32, P, P,
                                       P, sz, P]
+    L.indexer_scores_topk_noalloc.argtypes = [i32, i64, i64, i32, i32, P, P, P, i64, P, i32, i32,
+                                              P, P, P]
     L.sparse_mqa_attn.argtypes = [i32, i64, i64, i32, FP, P, P, P, i64, P, i32, P, i64, P, i32,
                                   P, f32, P, P, sz, P]
     L.dense_hca_attn.argtypes = [i32, i64, i64, i32, FP, P, P, P, i64, i32, P, i64, P, i32, P,
@@ -99,8 +101,9 @@ def lib():
     L.csa_selftest_wait.argtypes = [i64, P, sz, P]
     L.csa_launch_count.argtypes = []
     L.csa_launch_count.restype = ctypes.c_ulonglong
-    for fn in ("csa_compress", "hca_compress", "indexer_scores_topk", "sparse_mqa_attn",
-               "dense_hca_attn", "csa_check_status", "csa_selftest_wait"):
+    for fn in ("csa_compress", "hca_compress", "indexer_scores_topk",
+               "indexer_scores_topk_noalloc", "sparse_mqa_attn", "dense_hca_attn",
+               "csa_check_status", "csa_selftest_wait"):
         getattr(L, fn).restype = i32
     _lib = L
     return L

@@ -86,6 +86,60 @@ csa_status compress_common(int32_t dtype, int64_t B, int64_t T, int32_t m, bool 
 
 }  // namespace
 
+namespace csa {
+
+void note_launches(unsigned long long n) { g_launches.fetch_add(n); }
+
+csa_status indexer_prepare(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                           const void* q_I, const float* w, const void* k_I, int64_t N,
+                           const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                           float* score_out, IndexerParams* out, bool* tc) {
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
+  if (B < 0 || Tq < 0 || N < 0 || H_I <= 0 || d_I <= 0 || m < 1 || k < 1) return CSA_E_ARG;
+  if (B > 65535 || Tq > 0x7fffffffLL || N > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  if (H_I > 64 || d_I > 1024) return CSA_E_UNSUPPORTED;
+  if (B == 0 || Tq == 0) return CSA_OK;
+  if (!q_I || !w || !idx_out || (N > 0 && !k_I)) return CSA_E_ARG;
+  if (!aligned16(q_I) || (N > 0 && !aligned16(k_I))) return CSA_E_ARG;
+  IndexerParams& p = *out;
+  p.B = B;
+  p.Tq = Tq;
+  p.HI = H_I;
+  p.dI = d_I;
+  p.q_I = q_I;
+  p.w = w;
+  p.k_I = k_I;
+  p.N = N;
+  p.q_pos = q_pos;
+  p.m = m;
+  p.k = k;
+  p.idx_out = idx_out;
+  p.score_out = score_out;
+  // bf16 runs on the tensor cores only; shapes outside that kernel's envelope
+  // are rejected rather than sent to the CUDA-core kernels, which serve float32
+  *tc = dtype == CSA_BF16;
+  if (*tc && !indexer_tc_supported(p)) return CSA_E_UNSUPPORTED;
+  return CSA_OK;
+}
+
+size_t indexer_scratch(bool tc, const IndexerParams& p) {
+  return tc ? indexer_tc_scratch(p.B, p.Tq, p.N, p.k)
+            : indexer_portable_scratch(p.B, p.Tq, p.N, p.k);
+}
+
+csa_status indexer_launch(int32_t dtype, bool tc, const IndexerParams& p, cudaStream_t stream) {
+  if (tc) {
+    unsigned long long n_launch = 0;
+    cudaError_t e = launch_indexer_tc(p, stream, &n_launch);
+    note_launches(n_launch);
+    return cuda_status(e);
+  }
+  note_launches(2);
+  return cuda_status(launch_indexer_portable(dtype, p, stream));
+}
+
+}  // namespace csa
+
 extern "C" {
 
 csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const csa_fmt* fmt,
@@ -109,11 +163,9 @@ size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int
   switch (op) {
     case CSA_OP_COMPRESS:
       return kWsScratch;
-    case CSA_OP_INDEXER: {
-      size_t a = indexer_portable_scratch(B, Tq, N, k);
-      size_t b = dtype == CSA_BF16 ? indexer_tc_scratch(B, Tq, N, k) : 0;
-      return kWsScratch + (a > b ? a : b);
-    }
+    case CSA_OP_INDEXER:
+      return kWsScratch + (dtype == CSA_BF16 ? indexer_tc_scratch(B, Tq, N, k)
+                                             : indexer_portable_scratch(B, Tq, N, k));
     case CSA_OP_SPARSE_ATTN:
     case CSA_OP_DENSE_ATTN: {
       int64_t max_keys = (op == CSA_OP_SPARSE_ATTN ? (int64_t)k : N) + n_win;
@@ -129,40 +181,17 @@ csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I
                                const void* q_I, const float* w, const void* k_I, int64_t N,
                                const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
                                float* score_out, void* ws, size_t ws_bytes, void* stream) {
-  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
-  if (B < 0 || Tq < 0 || N < 0 || H_I <= 0 || d_I <= 0 || m < 1 || k < 1) return CSA_E_ARG;
-  if (B > 65535 || Tq > 0x7fffffffLL || N > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
-  if (H_I > 64 || d_I > 1024) return CSA_E_UNSUPPORTED;
-  if (B == 0 || Tq == 0) return CSA_OK;
-  if (!q_I || !w || !idx_out || (N > 0 && !k_I)) return CSA_E_ARG;
-  if (!ws) return CSA_E_WORKSPACE;
-  if (ws_bytes < csa_workspace_bytes(CSA_OP_INDEXER, dtype, B, Tq, 0, 0, N, k, 0))
-    return CSA_E_WORKSPACE;
   IndexerParams p{};
-  p.B = B;
-  p.Tq = Tq;
-  p.HI = H_I;
-  p.dI = d_I;
-  p.q_I = q_I;
-  p.w = w;
-  p.k_I = k_I;
-  p.N = N;
-  p.q_pos = q_pos;
-  p.m = m;
-  p.k = k;
-  p.idx_out = idx_out;
-  p.score_out = score_out;
+  bool tc = false;
+  csa_status st = indexer_prepare(dtype, B, Tq, H_I, d_I, q_I, w, k_I, N, q_pos, m, k, idx_out,
+                                  score_out, &p, &tc);
+  if (st != CSA_OK || B == 0 || Tq == 0) return st;
+  if (!ws) return CSA_E_WORKSPACE;
+  if (ws_bytes < kWsScratch + indexer_scratch(tc, p)) return CSA_E_WORKSPACE;
   p.status = status_word(ws);
   p.scratch = static_cast<char*>(ws) + kWsScratch;
   p.scratch_bytes = ws_bytes - kWsScratch;
-  if (dtype == CSA_BF16 && indexer_tc_supported(p)) {
-    unsigned long long n_launch = 0;
-    cudaError_t e = launch_indexer_tc(p, S(stream), &n_launch);
-    g_launches.fetch_add(n_launch);
-    return cuda_status(e);
-  }
-  g_launches.fetch_add(2);
-  return cuda_status(launch_indexer_portable(dtype, p, S(stream)));
+  return indexer_launch(dtype, tc, p, S(stream));
 }
 
 static csa_status attn_common(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const csa_fmt* fmt,
@@ -183,24 +212,29 @@ static csa_status attn_common(int32_t dtype, int64_t B, int64_t Tq, int32_t H, c
   if (!aligned16(q) || !aligned16(out) || (entries && !aligned16(entries)) ||
       (win && !aligned16(win)))
     return CSA_E_ARG;
-  if (!ws) return CSA_E_WORKSPACE;
-  const int op = sparse ? CSA_OP_SPARSE_ATTN : CSA_OP_DENSE_ATTN;
-  if (ws_bytes < csa_workspace_bytes(op, dtype, B, Tq, H, f.c, N, k, n_win)) return CSA_E_WORKSPACE;
   AttnParams p{};
   p.B = B;
   p.Tq = Tq;
   p.H = H;
   p.f = f;
   p.q = q;
-  p.q_pos = q_pos;
   p.entries = entries;
   p.N = N;
   p.sparse = sparse ? 1 : 0;
-  p.idx = idx;
   p.k = sparse ? k : 0;
-  p.m_dense = m_dense;
-  p.win = win;
   p.Tw = Tw;
+  p.out = out;
+  p.win = win;
+  // bf16 runs on the tensor cores unless CSA_F_PORTABLE asks for the CUDA-core
+  // kernel; shapes outside the tensor-core kernel's envelope are rejected
+  if (dtype == CSA_BF16 && !(f.flags & CSA_F_PORTABLE) && !attn_tc_supported(p))
+    return CSA_E_UNSUPPORTED;
+  if (!ws) return CSA_E_WORKSPACE;
+  const int op = sparse ? CSA_OP_SPARSE_ATTN : CSA_OP_DENSE_ATTN;
+  if (ws_bytes < csa_workspace_bytes(op, dtype, B, Tq, H, f.c, N, k, n_win)) return CSA_E_WORKSPACE;
+  p.q_pos = q_pos;
+  p.idx = idx;
+  p.m_dense = m_dense;
   p.win_pos0 = win_pos0;
   p.n_win = n_win;
   p.sink = sink;
@@ -209,7 +243,7 @@ static csa_status attn_common(int32_t dtype, int64_t B, int64_t Tq, int32_t H, c
   p.status = status_word(ws);
   p.scratch = static_cast<char*>(ws) + kWsScratch;
   p.scratch_bytes = ws_bytes - kWsScratch;
-  if (dtype == CSA_BF16 && attn_tc_supported(p)) {
+  if (dtype == CSA_BF16 && !(f.flags & CSA_F_PORTABLE)) {
     unsigned long long n_launch = 0;
     cudaError_t e = launch_attn_tc(p, S(stream), &n_launch);
     g_launches.fetch_add(n_launch);

@@ -1698,6 +1698,15 @@ cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t 
   return cudaGetLastError();
 }
 
+// Rows with no entry at all (N == 0): index -1 and score -inf throughout.
+__global__ void topk_padding_kernel(int64_t n, int32_t* idx, float* sc) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    idx[i] = -1;
+    if (sc) sc[i] = -INFINITY;
+  }
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -1752,8 +1761,8 @@ cudaError_t launch_persist(const IndexerParams& p, const TcIdxArgs& a, cudaStrea
 
 bool indexer_tc_supported(const IndexerParams& p) {
   auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
-  return p.HI == kHI && p.dI == kDI && p.N > 0 && p.N < (1LL << 31) &&
-         p.Tq * kHI < (1LL << 31) && p.B <= 65535 && al(p.q_I) && al(p.k_I) &&
+  return p.HI == kHI && p.dI == kDI && p.N >= 0 && p.N < (1LL << 31) &&
+         p.Tq * kHI < (1LL << 31) && p.B <= 65535 && al(p.q_I) && (p.N == 0 || al(p.k_I)) &&
          (p.Tq + 3) / 4 <= 65535;
 }
 
@@ -1768,6 +1777,13 @@ cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
                               unsigned long long* n_launch) {
   *n_launch = 0;
   if (p.B == 0 || p.Tq == 0) return cudaSuccess;
+  if (p.N == 0) {   // nothing to score: every row is padding
+    const int64_t n = p.B * p.Tq * (int64_t)p.k;
+    const int64_t blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+    topk_padding_kernel<<<(unsigned)blocks, 256, 0, stream>>>(n, p.idx_out, p.score_out);
+    *n_launch = 1;
+    return cudaGetLastError();
+  }
   const int tok = tok_for(p.Tq);
   TcIdxArgs a{};
   a.Tq = p.Tq;

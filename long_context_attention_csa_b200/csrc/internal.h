@@ -74,4 +74,18 @@ struct AttnParams {
 };
 cudaError_t launch_attn_portable(int dtype, const AttnParams& p, cudaStream_t stream);
 
+// Adds n to the library's launch counter (csa_launch_count).
+void note_launches(unsigned long long n);
+
+// Indexer entry points' shared steps: argument checks and kernel choice
+// (bf16 -> tensor cores, shapes outside that kernel -> CSA_E_UNSUPPORTED;
+// float32 -> CUDA cores), the scratch the chosen kernels need past the status
+// word, and the launch (counted).
+csa_status indexer_prepare(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                           const void* q_I, const float* w, const void* k_I, int64_t N,
+                           const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                           float* score_out, IndexerParams* out, bool* tc);
+size_t indexer_scratch(bool tc, const IndexerParams& p);
+csa_status indexer_launch(int32_t dtype, bool tc, const IndexerParams& p, cudaStream_t stream);
+
 }  // namespace csa

@@ -15,7 +15,17 @@
 // before any stream capture.  All calls share the array: calls whose
 // executions overlap on the GPU (different streams without ordering) race on
 // it.  The status word at its start is cleared by every call; device-side
-// status from this variant is not reported to the caller.
+// status from this variant is not reported to the caller, so after a device-
+// side error (a bounded wait that ran out) the outputs are unspecified and
+// nothing says so: callers who must detect that use indexer_scores_topk with a
+// workspace and csa_check_status.
+//
+// Accepted sizes: 256 bytes of status word plus the scratch of the kernels
+// the call takes must fit kNoAllocScratchBytes.  bf16 takes the tensor-core
+// kernels (H_I = 64, d_I = 128), whose scratch is 8 B x B x Tq x k x chunks
+// when the entries span more than one chunk (2048 entries for Tq >= 4, 4096
+// for single-token rows) and nothing otherwise; float32 takes the CUDA-core
+// kernels, whose scratch is the B x Tq x N float32 score matrix.
 #include <mutex>
 
 #include "common.cuh"
@@ -58,30 +68,14 @@ extern "C" csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int6
                                                   int32_t* idx_out, float* score_out,
                                                   void* stream) {
   using namespace csa;
-  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
-  if (B < 0 || Tq < 0 || N < 0 || H_I <= 0 || d_I <= 0 || m < 1 || k < 1) return CSA_E_ARG;
-  if (B > 65535 || Tq > 0x7fffffffLL || N > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
-  if (H_I > 64 || d_I > 1024) return CSA_E_UNSUPPORTED;
-  if (B == 0 || Tq == 0) return CSA_OK;
-  if (!q_I || !w || !idx_out || (N > 0 && !k_I)) return CSA_E_ARG;
-
+  // the same checks and kernel choice as indexer_scores_topk
   IndexerParams p{};
-  p.B = B;
-  p.Tq = Tq;
-  p.HI = H_I;
-  p.dI = d_I;
-  p.q_I = q_I;
-  p.w = w;
-  p.k_I = k_I;
-  p.N = N;
-  p.q_pos = q_pos;
-  p.m = m;
-  p.k = k;
-  p.idx_out = idx_out;
-  p.score_out = score_out;
-  const bool tc = dtype == CSA_BF16 && indexer_tc_supported(p);
-  const size_t need = tc ? indexer_tc_scratch(B, Tq, N, k) : indexer_portable_scratch(B, Tq, N, k);
-  if (kWsScratch + need > kNoAllocScratchBytes) return CSA_E_WORKSPACE;  // beyond the fixed array
+  bool tc = false;
+  csa_status st = indexer_prepare(dtype, B, Tq, H_I, d_I, q_I, w, k_I, N, q_pos, m, k, idx_out,
+                                  score_out, &p, &tc);
+  if (st != CSA_OK || B == 0 || Tq == 0) return st;
+  // accepted iff the status word plus the chosen kernels' scratch fit the array
+  if (kWsScratch + indexer_scratch(tc, p) > kNoAllocScratchBytes) return CSA_E_WORKSPACE;
 
   void* base = nullptr;
   if (noalloc_base(&base) != cudaSuccess) return CSA_E_CUDA;
@@ -90,12 +84,5 @@ extern "C" csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int6
   p.status = static_cast<unsigned*>(base);
   p.scratch = static_cast<unsigned char*>(base) + kWsScratch;
   p.scratch_bytes = kNoAllocScratchBytes - kWsScratch;
-  cudaError_t e;
-  if (tc) {
-    unsigned long long n = 0;
-    e = launch_indexer_tc(p, s, &n);
-  } else {
-    e = launch_indexer_portable(dtype, p, s);
-  }
-  return e == cudaSuccess ? CSA_OK : CSA_E_CUDA;
+  return indexer_launch(dtype, tc, p, s);
 }

@@ -144,3 +144,48 @@ def test_selftest_wait_rejects_bad_arguments(L):
     assert L.csa_selftest_wait(10 ** 6, ctypes.addressof(buf), 128, None) == 1   # too small
     assert L.csa_selftest_wait(10, ctypes.addressof(buf), 256, None) == 1        # limit too short
     assert L.csa_selftest_wait(10 ** 11, ctypes.addressof(buf), 256, None) == 1  # too long
+
+
+def test_bf16_shapes_outside_the_tensor_core_kernels_are_unsupported(L):
+    """bf16 indexer and attention calls run on the tensor cores only; a shape
+    that kernel does not implement is rejected (no silent CUDA-core path).
+    float32, and attention with CSA_F_PORTABLE, pass validation (they then
+    stop here at the missing workspace)."""
+    d = ctypes.c_void_p(4096)
+    mis = ctypes.c_void_p(4100)
+    # indexer: H_I = 32 or d_I = 64 in bf16 -> unsupported; the same in float32 -> workspace
+    assert L.indexer_scores_topk(1, 1, 8, 32, 128, d, d, d, 64, None, 4, 8, d, None, None, 0,
+                                 None) == 2
+    assert L.indexer_scores_topk(1, 1, 8, 64, 64, d, d, d, 64, None, 4, 8, d, None, None, 0,
+                                 None) == 2
+    assert L.indexer_scores_topk(0, 1, 8, 32, 128, d, d, d, 64, None, 4, 8, d, None, None, 0,
+                                 None) == 5
+    # the supported bf16 shape passes validation; misaligned inputs are argument errors
+    assert L.indexer_scores_topk(1, 1, 8, 64, 128, d, d, d, 64, None, 4, 8, d, None, None, 0,
+                                 None) == 5
+    assert L.indexer_scores_topk(1, 1, 8, 64, 128, mis, d, d, 64, None, 4, 8, d, None, None, 0,
+                                 None) == 1
+    # the no-workspace variant applies the same rule
+    assert L.indexer_scores_topk_noalloc(1, 1, 8, 32, 128, d, d, d, 64, None, 4, 8, d, None,
+                                         None) == 2
+    # attention: 32 heads or 48 RoPE dims are fine, 32 heads is not a multiple of 64
+    f = _fmt()
+    assert L.sparse_mqa_attn(1, 1, 4, 32, ctypes.byref(f), d, None, d, 16, d, 4, d, 8, None, 8,
+                             None, 0.0, d, None, 0, None) == 2
+    assert L.dense_hca_attn(1, 1, 4, 32, ctypes.byref(f), d, None, d, 16, 4, d, 8, None, 8,
+                            None, 0.0, d, None, 0, None) == 2
+    # c = 256 in bf16 -> unsupported; CSA_F_PORTABLE selects the CUDA-core kernel instead
+    f256 = _fmt(c=256)
+    assert L.dense_hca_attn(1, 1, 4, 64, ctypes.byref(f256), d, None, d, 16, 4, d, 8, None, 8,
+                            None, 0.0, d, None, 0, None) == 2
+    fp = _fmt(c=256, flags=4)
+    assert L.dense_hca_attn(1, 1, 4, 64, ctypes.byref(fp), d, None, d, 16, 4, d, 8, None, 8,
+                            None, 0.0, d, None, 0, None) == 5
+    # top-k beyond the tensor-core kernel's index list
+    assert L.sparse_mqa_attn(1, 1, 4, 64, ctypes.byref(f), d, None, d, 4096, d, 2048, d, 8, None,
+                             8, None, 0.0, d, None, 0, None) == 2
+    # float32 attention always takes the CUDA-core kernel
+    f64c = _fmt(c=64, r=32)
+    assert L.dense_hca_attn(0, 1, 4, 4, ctypes.byref(f64c), d, None, d, 16, 4, d, 8, None, 8,
+                            None, 0.0, d, None, 0, None) == 5
+

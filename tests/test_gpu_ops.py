@@ -132,14 +132,17 @@ def test_indexer_tiny_fp32():
     _indexer_case(wl.WORKLOADS["tiny_csa_fp32"])
 
 
-@pytest.mark.parametrize("HI,dI,T,k", [(64, 128, 700, 64), (2, 32, 300, 16), (64, 128, 1000, 256)])
-def test_indexer_integer_inputs_bit_exact(HI, dI, T, k):
+@pytest.mark.parametrize("HI,dI,T,k,dt", [(64, 128, 700, 64, torch.bfloat16),
+                                           (2, 32, 300, 16, torch.float32),
+                                           (64, 128, 1000, 256, torch.bfloat16)])
+def test_indexer_integer_inputs_bit_exact(HI, dI, T, k, dt):
     """Small-integer inputs make every product and sum exact in bf16 x bf16 ->
-    fp32: the selected sets (tie rule included) and scores must be identical."""
+    fp32 (tensor cores) and in float32 (CUDA cores): the selected sets (tie
+    rule included) and scores must be identical."""
     B, m = 1, 4
     N = T // m
-    qI = wl.randint_like_float((B, T, HI, dI), 11, -2, 3, DEV, torch.bfloat16)
-    kI = wl.randint_like_float((B, N, dI), 12, -2, 3, DEV, torch.bfloat16)
+    qI = wl.randint_like_float((B, T, HI, dI), 11, -2, 3, DEV, dt)
+    kI = wl.randint_like_float((B, N, dI), 12, -2, 3, DEV, dt)
     w = wl.randint_like_float((B, T, HI), 13, -2, 3, DEV, torch.float32)
     idx, sc = csa.indexer_scores_topk(qI, w, kI, m, k, want_scores=True)
     torch.cuda.synchronize()
@@ -463,23 +466,103 @@ def test_device_wait_timeout_is_reported_and_the_context_survives():
 
 # ----------------------------------------------------------------- whole layer
 
-@pytest.mark.parametrize("wname,T,k", [("tiny_csa_fp32", 256, 16), ("csa_prefill_8k", 512, 64)])
-def test_csa_layer_end_to_end(wname, T, k):
-    """compress -> indexer -> attention on the GPU against the oracle's own
-    chain from the same raw inputs."""
-    w = wl.scaled(wl.WORKLOADS[wname], T=T, k=k)
+def _layer_check(w, inp, ent, win, idx, out, rows):
+    """The GPU chain's entries, window rows, index sets and outputs against the
+    oracle's own chain on the same raw inputs.  A row whose GPU index set
+    differs from the oracle's (legitimately: only within the tie band, which
+    check_topk_rows enforces) has its output checked against the oracle's
+    attention over the GPU's own set, so every sampled row is checked."""
+    x = {kk: (None if v is None else f64(v[0] if v.dim() > 1 else v)) for kk, v in inp.items()}
+    ref = oracle.csa_layer(x, ofmt(w), w.m, w.k, w.n_win, rows=rows)
+    assert_close(ent[0], ref["entries"], w.dtype, "layer entries")
+    assert_close(win[0][rows], ref["win"][rows], w.dtype, "layer window rows")
+    gi = idx[0][rows].cpu().numpy()
+    check_topk_rows(gi, ref["idx"], ref["scores"], what="layer")
+    diff = np.where(~np.all(gi == ref["idx"], axis=1))[0]
+    want = ref["out"].copy()
+    if len(diff):
+        want[diff] = oracle.attention(x["q"][rows[diff]], ref["entries"], ref["win"], ofmt(w),
+                                      w.n_win, idx=gi[diff], sink=x["sink"], q_pos=rows[diff])
+    # the GPU chain stores the entries and window rows in bf16 before attention
+    # and rounds the output again: two bf16 roundings against the float64 chain
+    assert_close(out[0][rows], want, w.dtype, f"layer output ({len(diff)} rows on the GPU set)",
+                 roundings=2)
+    return len(diff)
+
+
+def _layer_run(w):
     inp = wl.csa_prefill_inputs(w, DEV)
     ent, win = csa.csa_compress(inp["kv_a"], inp["kv_b"], inp["z_a"], inp["z_b"], w.m, gfmt(w),
                                 want_win=True)
     idx = csa.indexer_scores_topk(inp["q_I"], inp["w"], inp["k_I"], w.m, w.k)
     out = csa.sparse_mqa_attn(inp["q"], ent, idx, win, gfmt(w), w.n_win, sink=inp["sink"])
     torch.cuda.synchronize()
-    ref = oracle.csa_layer({kk: (None if v is None else f64(v[0] if v.dim() > 1 else v))
-                            for kk, v in inp.items()}, ofmt(w), w.m, w.k, w.n_win)
-    gi = idx[0].cpu().numpy()
-    check_topk_rows(gi, ref["idx"], ref["scores"], what="layer")
-    same = np.all(gi == ref["idx"], axis=1)
-    assert same.mean() > 0.95
-    # the GPU chain stores the entries and window rows in bf16 before attention
-    # and rounds the output again: two bf16 roundings against the float64 chain
-    assert_close(out[0][same], ref["out"][same], w.dtype, "layer output", roundings=2)
+    return inp, ent, win, idx, out
+
+
+@pytest.mark.parametrize("wname,T,k", [("tiny_csa_fp32", 256, 16), ("csa_prefill_8k", 512, 64)])
+def test_csa_layer_end_to_end(wname, T, k):
+    """compress -> indexer -> attention on the GPU against the oracle's own
+    chain from the same raw inputs, every row."""
+    w = wl.scaled(wl.WORKLOADS[wname], T=T, k=k)
+    inp, ent, win, idx, out = _layer_run(w)
+    _layer_check(w, inp, ent, win, idx, out, np.arange(T))
+
+
+def test_csa_layer_csa_prefill_8k_sampled():
+    """The whole chain at the full csa_prefill_8k workload (8192 tokens, 2048
+    entries, top-k 512) as the benchmark runs it, checked on sampled rows."""
+    w = wl.WORKLOADS["csa_prefill_8k"]
+    inp, ent, win, idx, out = _layer_run(w)
+    _layer_check(w, inp, ent, win, idx, out, sample_rows(w.T, 40))
+
+
+# ----------------------------------------------------------------- device status
+
+def test_attention_logit_beyond_the_bound_is_flagged():
+    """Stored keys 30x larger than unit RMS (not what the compression calls
+    produce) push logits more than 60 past the tensor-core kernel's static
+    softmax bound: the kernel records CSA_DEV_RANGE in the status word.  The
+    CUDA-core kernel keeps an exact running maximum and stays correct."""
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=300, k=32)
+    inp = _attn_inputs_prefill(w)
+    inp["entries"] = (inp["entries"].float() * 30).to(torch.bfloat16)
+    ws = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_SPARSE_ATTN, 1, 1, w.T, w.H, w.c,
+                                               w.n_csa, w.k, w.n_win))
+    csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w), w.n_win,
+                        sink=inp["sink"], ws=ws)
+    assert csa.csa_check_status(ws) == (csa.CSA_E_DEVICE, csa.CSA_DEV_RANGE)
+    assert csa.csa_check_status(ws) == (csa.CSA_OK, 0)    # read and cleared
+    out = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"],
+                              gfmt(w, csa.CSA_F_PORTABLE), w.n_win, sink=inp["sink"], ws=ws)
+    assert csa.csa_check_status(ws) == (csa.CSA_OK, 0)
+    _check_attn(w, inp, out, np.arange(0, w.T, 3), dense=False, flags=csa.CSA_F_PORTABLE)
+
+
+@pytest.mark.parametrize("flags", PATHS)
+def test_attention_index_out_of_range_is_skipped_and_flagged(flags):
+    """An index in [N, allocation): the entries tensor has spare rows beyond
+    the N the call is given, so a missing guard would read allocated memory,
+    not fault.  The kernel skips the index, records CSA_DEV_BAD_INDEX, and the
+    output equals the oracle's, which skips it too."""
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=300, k=32)
+    inp = _attn_inputs_prefill(w)
+    N = w.n_csa
+    spare = wl.randn((1, N + 16, w.c), 91, DEV, dtype=torch.bfloat16)
+    spare[:, :N] = inp["entries"]
+    inp["entries"] = spare[:, :N]          # contiguous view of the first N rows
+    assert inp["entries"].is_contiguous()
+    idx = inp["idx"].clone()
+    planted = [10, 50, 100, 101]
+    for t in planted:                       # rows with fewer than k visible entries
+        v = oracle.visible(t, w.m, N)
+        assert v < w.k
+        idx[0, t, v] = N + 3
+    inp["idx"] = idx
+    ws = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_SPARSE_ATTN, 1, 1, w.T, w.H, w.c, N,
+                                               w.k, w.n_win))
+    out = csa.sparse_mqa_attn(inp["q"], inp["entries"], idx, inp["win"], gfmt(w, flags), w.n_win,
+                              sink=inp["sink"], ws=ws)
+    assert csa.csa_check_status(ws) == (csa.CSA_E_DEVICE, csa.CSA_DEV_BAD_INDEX)
+    rows = np.array(sorted(set(planted) | set(range(0, w.T, 5))))
+    _check_attn(w, inp, out, rows, dense=False, flags=flags)

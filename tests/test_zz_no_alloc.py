@@ -45,8 +45,10 @@ def test_noalloc_matches_workspace_indexer_twice(seed):
                                                   q_pos=inp["q_pos"], want_scores=True)
         idx = torch.full_like(ref_idx, -7)
         sc = torch.full_like(ref_sc, 7.0)
+        n0 = csa.csa_launch_count()
         st = _noalloc(L, inp["q_I"], inp["w"], inp["k_I"], w.m, w.k, inp["q_pos"], idx, sc)
         assert st == csa.CSA_OK
+        assert csa.csa_launch_count() - n0 == 2     # chunk scoring + candidate merge
         torch.cuda.synchronize()
         # index work is compared bit for bit; scores come from the same kernels
         assert torch.equal(idx, ref_idx)
@@ -70,3 +72,56 @@ def test_noalloc_rejects_problems_beyond_its_array():
     st = fn(csa.CSA_F32, B, Tq, HI, dI, P(q_I.data_ptr()), P(w.data_ptr()), P(k_I.data_ptr()),
             N, None, 4, 8, P(idx.data_ptr()), None, None)
     assert st == csa.CSA_E_WORKSPACE
+
+
+def _call_f32(L, B, Tq, HI, dI, N, k, q_pos, tensors):
+    q_I, w, k_I, idx, sc = tensors
+    P = ctypes.c_void_p
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return L.indexer_scores_topk_noalloc(
+        csa.CSA_F32, B, Tq, HI, dI, P(q_I.data_ptr()), P(w.data_ptr()), P(k_I.data_ptr()), N,
+        P(q_pos.data_ptr()), 4, k, P(idx.data_ptr()), P(sc.data_ptr()), stream)
+
+
+def test_noalloc_float32_at_the_limit_matches_twice():
+    """float32 takes the CUDA-core kernels, whose B*Tq*N*4-byte score matrix
+    lives in the array: 64 rows x 32767 entries need exactly 8 MiB - 256
+    bytes, the most the array holds next to its status word.  Accepted, and
+    equal bit for bit to the workspace path, on two calls in a row."""
+    L = csa.lib()
+    B, Tq, HI, dI, N, k = 1, 64, 2, 32, 32767, 8
+    assert 256 + B * Tq * N * 4 == 8 << 20
+    q_pos = torch.full((B, Tq), 4 * N - 1, dtype=torch.int64, device="cuda")
+    for call in range(2):
+        q_I = wl.randn((B, Tq, HI, dI), 200 + call, "cuda")
+        w = wl.randn((B, Tq, HI), 210 + call, "cuda")
+        k_I = wl.randn((B, N, dI), 220 + call, "cuda")
+        ref_idx, ref_sc = csa.indexer_scores_topk(q_I, w, k_I, 4, k, q_pos=q_pos,
+                                                  want_scores=True)
+        idx = torch.full_like(ref_idx, -7)
+        sc = torch.full_like(ref_sc, 7.0)
+        n0 = csa.csa_launch_count()
+        assert _call_f32(L, B, Tq, HI, dI, N, k, q_pos, (q_I, w, k_I, idx, sc)) == csa.CSA_OK
+        assert csa.csa_launch_count() - n0 == 2     # scores + top-k
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref_idx)
+        assert torch.equal(sc, ref_sc)
+
+
+def test_noalloc_float32_four_bytes_over_the_limit_is_rejected():
+    """One row over 2097089 entries needs 4 bytes more than the array holds:
+    rejected before any launch.  The tensors are allocated at full size, so
+    even a wrong size check would only read memory the call was given."""
+    L = csa.lib()
+    B, Tq, HI, dI, k = 1, 1, 2, 32, 8
+    N = ((8 << 20) - 256) // 4 + 1
+    q_pos = torch.full((B, Tq), 4 * N - 1, dtype=torch.int64, device="cuda")
+    q_I = torch.zeros((B, Tq, HI, dI), device="cuda")
+    w = torch.zeros((B, Tq, HI), device="cuda")
+    k_I = torch.zeros((B, N, dI), device="cuda")
+    idx = torch.empty((B, Tq, k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((B, Tq, k), dtype=torch.float32, device="cuda")
+    n0 = csa.csa_launch_count()
+    assert _call_f32(L, B, Tq, HI, dI, N, k, q_pos, (q_I, w, k_I, idx, sc)) == csa.CSA_E_WORKSPACE
+    assert csa.csa_launch_count() == n0
+
