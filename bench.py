@@ -322,6 +322,8 @@ def run_gpu(args):
     decode = {} if args.no_decode else {
         n: measure_decode(n, dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
         for n in DECODE_WORKLOADS}
+    proj = None if args.no_hca else measure_projection(
+        dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
     hca = None if args.no_hca else measure_hca_prefill(
         dev, K, args.warmup, flush, ws, ws == 1 and not args.no_cpu_baseline)
     comp_1m = None if args.no_decode else measure_compress_1m(dev, min(K, 10), args.warmup)
@@ -381,6 +383,8 @@ def run_gpu(args):
             line["decode"] = decode
         if hca:
             line["hca_prefill_64k"] = hca
+        if proj:
+            line["out_proj_8k"] = proj
         if comp_1m:
             line["compress_1m_tokens"] = comp_1m
         if ws == 1 and not args.no_cpu_baseline:
@@ -512,7 +516,7 @@ def hca_cpu_baseline(w, inp, rows: int):
 
 
 def measure_hca_prefill(dev, steps: int, warmup: int, flush, ws_n: int, cpu: bool,
-                        cpu_rows: int = 256):
+                        cpu_rows: int = 4096):
     """The HCA layer prefill step at hca_prefill_64k (65536 tokens, m' = 128 ->
     512 entries, 64 heads, entry dim 512, window 128, sinks):
     hca_compress (entries + window rows) -> dense_hca_attn.  Tokens/s of the
@@ -582,6 +586,68 @@ def measure_hca_prefill(dev, steps: int, warmup: int, flush, ws_n: int, cpu: boo
     if cpu:
         res["cpu_baseline"] = hca_cpu_baseline(w, inp, cpu_rows)
     del inp, entries, win, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_projection(dev, steps: int, warmup: int, flush, ws_n: int, cpu: bool,
+                       cpu_rows: int = 64):
+    """The grouped output projection of the csa_prefill_8k layer's attention
+    output (8192 rows, 64 heads x 512, g = 8 groups -> d_g = 1024, then
+    g d_g = 8192 -> d = 4096): two tcgen05 GEMMs, bf16 in and out.  Rows/s of
+    the call and its tensor roofline over 2 T (H c d_g + g d_g d) FLOPs."""
+    w = wl.WORKLOADS[WORKLOAD]
+    p = wl.PROJ
+    x = wl.projection_inputs(w, p["g"], p["d_g"], p["d"], dev)
+    y = torch.empty((w.T, p["d"]), dtype=w.dtype, device=dev)
+    ws = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_OUT_PROJ, 1, 1, w.T, 0, 0,
+                                               p["g"] * p["d_g"]), dev)
+
+    def run():
+        csa.grouped_output_projection(x["o"], x["w_group"], x["w_out"], y=y, ws=ws)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    st, d = csa.csa_check_status(ws)
+    if st:
+        raise RuntimeError(f"projection: device status {st}/{d}")
+    ms = allmax(float(np.mean([a.elapsed_time(b) for a, b in evs])), ws_n)
+    fl = 2.0 * w.T * (w.H * w.c * p["d_g"] + p["g"] * p["d_g"] * p["d"])
+    _, bf16, src = peaks()
+    achieved = fl / (ms * 1e-3) / 1e12
+    res = {"value": w.T * ws_n / (ms * 1e-3), "unit": "tokens/s", "ms": ms,
+           "config": {"workload": w.name, "rows": w.T, "heads": w.H, "head_dim": w.c, **p,
+                      "weights": "random synthetic, N(0,1)/sqrt(fan_in)",
+                      "l2": "flushed between timed calls (outside the events)"},
+           "roofline": {"bound": "tensor", "kernel": "gemm_bf16_tc_kernel (two launches)",
+                        "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                        "frac": achieved / bf16, "algorithmic_flops_per_call": fl,
+                        "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)"
+                        if src == "measured" else "fallback 1.59 PFLOP/s"}}
+    if cpu:
+        import oracle
+
+        sel = np.linspace(0, w.T - 1, cpu_rows).astype(np.int64)
+        o = x["o"][torch.from_numpy(sel).to(dev)].double().cpu().numpy()
+        wg, wo = x["w_group"].double().cpu().numpy(), x["w_out"].double().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.grouped_output_projection(o, wg, wo)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": cpu_rows / dt, "unit": "tokens/s",
+                               "cores": os.cpu_count(), "kind": "oracle",
+                               "sample": f"{cpu_rows} of {w.T} rows evenly spaced, float64 "
+                                         f"numpy matmuls, {dt:.2f} s"}
+    del x, y, ws
     torch.cuda.empty_cache()
     return res
 
@@ -821,6 +887,13 @@ def run_only(args):
         return
     if args.only.startswith("hca_"):
         return run_only_hca(args)
+    if args.only == "proj":
+        torch.cuda.set_device(0)
+        dev = torch.device("cuda", 0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        print(json.dumps({"only": "proj", **measure_projection(dev, args.steps, args.warmup,
+                                                               flush, 1, False)}))
+        return
     if args.only == "decode":
         return run_only_decode(args)
     torch.cuda.set_device(0)
@@ -861,7 +934,7 @@ def run_only(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--only", choices=["compress", "compress_stream", "indexer", "attn",
-                                       "hca_compress", "hca_attn",
+                                       "hca_compress", "hca_attn", "proj",
                                        "decode"],
                     default=None,
                     help="time one stage alone (kernel profiling)")

@@ -60,6 +60,8 @@ typedef int32_t csa_status;
 #define CSA_DEV_TIMEOUT 1u     /* a bounded mbarrier wait ran out; results invalid */
 #define CSA_DEV_RANGE 2u       /* a logit exceeded the static softmax bound (un-normalised keys) */
 #define CSA_DEV_BAD_INDEX 3u   /* an index outside [-1, N) was skipped */
+#define CSA_DEV_STREAM 4u      /* a stream state was invalid (sequence skipped) or its entry
+                                  cache full (entry dropped); detail: the sequence */
 
 /* ---- element types and flags ---------------------------------------- */
 #define CSA_F32 0   /* float32 tensors, float32 arithmetic (CUDA cores) */
@@ -86,6 +88,7 @@ typedef struct csa_fmt {
 #define CSA_OP_SPARSE_ATTN 2
 #define CSA_OP_DENSE_ATTN 3
 #define CSA_OP_COMPRESS 4
+#define CSA_OP_OUT_PROJ 5   /* Tq = T, N = g * d_g */
 
 /* ---- (1) compression ------------------------------------------------ */
 
@@ -125,6 +128,60 @@ csa_status csa_compress(int32_t dtype, int64_t B, int64_t T, int32_t m, const cs
 csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, const csa_fmt* fmt,
                         const void* kv, const void* z, int32_t z_cols, int64_t pos0, void* entries,
                         void* win_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- (1b) streaming compression for decode ----------------------------- */
+
+/*
+ * Bytes of one sequence's stream state (a multiple of 256) for
+ * csa_compress_append (overlap = 1, rate m) or hca_compress_append
+ * (overlap = 0, rate m'): a 16-byte header holding the int64 count t of tokens
+ * appended so far, then the tail buffer in the tensors' dtype -- the current
+ * block's group-a rows and logits and, for CSA, the group-b rows and logits
+ * of the current and the previous block.  Returns 0 for bad arguments.
+ */
+size_t csa_stream_state_bytes(int32_t dtype, int32_t m, int32_t overlap, int32_t c,
+                              int32_t z_cols);
+
+/*
+ * Appends one token to each of B sequences' CSA compression state, as a decode
+ * step produces them [§3.3 of the summary page: the entry of block s pools
+ * the block's group-a rows and the previous block's group-b rows under a
+ * per-channel softmax over the 2m logits; the page "DeepSeek-V4 梗概",
+ * inference-infrastructure table, row "Tail buffer": the tokens of a block
+ * that is not yet complete wait in a tail buffer].  For sequence b, with t the
+ * token count stored in its state:
+ *   - the token (kv_a[b], kv_b[b], z_a[b], z_b[b]) is stored in the tail
+ *     buffer as slot t mod m of block s = t / m;
+ *   - win_out[b] (optional) = RoPE_{pos0+t}(RMSNorm(kv_a[b])), its window row;
+ *   - when t mod m == m - 1, entry s -- exactly what csa_compress produces for
+ *     entry s of the whole sequence -- is written to entries[b, s];
+ *   - t becomes t + 1.
+ *   kv_a, kv_b: [B, c]; z_a, z_b: [B, z_cols] (dtype); state: B consecutive
+ *   states of state_stride bytes each (>= csa_stream_state_bytes, a multiple
+ *   of 16; zero-filled before a sequence's first token); entries: [B, n_cap,
+ *   c] entry cache; win_out: [B, c] or NULL.  ws: >= 256 bytes (status word).
+ * A state whose count is negative is skipped and an entry s >= n_cap is
+ * dropped, both reported as CSA_DEV_STREAM.  Sequences are independent
+ * (one CTA each): a sequence's results do not depend on the batch.
+ * Errors: CSA_E_ARG (null or misaligned pointers, m < 1, bad z_cols or a
+ * stride too small), CSA_E_UNSUPPORTED (2m > 256, c not in {64, ..., 1024} or
+ * odd), CSA_E_WORKSPACE.
+ */
+csa_status csa_compress_append(int32_t dtype, int64_t B, int32_t m, const csa_fmt* fmt,
+                               const void* kv_a, const void* kv_b, const void* z_a,
+                               const void* z_b, int32_t z_cols, int64_t pos0, void* state,
+                               size_t state_stride, void* entries, int64_t n_cap, void* win_out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * hca_compress_append: the same for an HCA layer [§3.3 of the summary page:
+ * rate m', no overlap]: entry s pools the m' rows of block s.  kv, z: [B, c] /
+ * [B, z_cols].  m' up to 4096.
+ */
+csa_status hca_compress_append(int32_t dtype, int64_t B, int32_t m_prime, const csa_fmt* fmt,
+                               const void* kv, const void* z, int32_t z_cols, int64_t pos0,
+                               void* state, size_t state_stride, void* entries, int64_t n_cap,
+                               void* win_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- (2) lightning indexer + top-k ----------------------------------- */
 
@@ -225,6 +282,31 @@ csa_status dense_hca_attn(int32_t dtype, int64_t B, int64_t Tq, int32_t H, const
                           int32_t m_prime, const void* win, int64_t Tw, const int64_t* win_pos0,
                           int32_t n_win, const float* sink, float scale, void* out, void* ws,
                           size_t ws_bytes, void* stream);
+
+/* ---- (4) grouped output projection ----------------------------------- */
+
+/*
+ * Grouped output projection of the attention output [§3.3 of the summary
+ * page, CSA paragraph: c * n_h is large, so the heads' outputs are first
+ * projected group by group to an intermediate dim d_g, then concatenated and
+ * projected back to the model dim d].  The H heads split into g consecutive
+ * groups of H/g heads (the reading taken: the pages give the map's shape,
+ * not the grouping):
+ *   v[t, j d_g + n] = sum_k o[t, j (H/g) c + k] w_group[j, n, k]   (o as [T, H c])
+ *   y[t, n]         = sum_k v[t, k] w_out[n, k]
+ *   o: [T, H, c] bf16; w_group: [g, d_g, (H/g) c] bf16; w_out: [d, g d_g] bf16;
+ *   y (out): [T, d] bf16.  v lives in the workspace as bf16 (the products
+ *   and sums of both GEMMs in float32; v and y rounded once to bf16).
+ *   ws: >= csa_workspace_bytes(CSA_OP_OUT_PROJ, CSA_BF16, 1, T, 0, 0, g d_g, 0, 0)
+ *   = 256 + 2 T g d_g bytes.
+ * Tensor cores only: bf16 with H % g == 0, (H/g) c and g d_g multiples of 64,
+ * d_g and d multiples of 32; anything else is CSA_E_UNSUPPORTED (float32
+ * included).  Errors: CSA_E_ARG, CSA_E_UNSUPPORTED, CSA_E_WORKSPACE.
+ */
+csa_status grouped_output_projection(int32_t dtype, int64_t T, int32_t H, int32_t c, int32_t g,
+                                     int32_t d_g, int32_t d, const void* o, const void* w_group,
+                                     const void* w_out, void* y, void* ws, size_t ws_bytes,
+                                     void* stream);
 
 /* ---- workspace and status --------------------------------------------- */
 

@@ -4,8 +4,9 @@ Argument marshalling only: every step of the path runs in the library's CUDA
 kernels.  PyTorch supplies device memory and streams.  The functions carry the
 names of the C entry points (include/csa.h):
 
-    csa_compress, hca_compress, indexer_scores_topk, sparse_mqa_attn,
-    dense_hca_attn, csa_workspace_bytes, csa_check_status
+    csa_compress, hca_compress, csa_compress_append, hca_compress_append,
+    indexer_scores_topk, sparse_mqa_attn, dense_hca_attn, grouped_output_projection,
+    csa_workspace_bytes, csa_check_status
 
 Importing succeeds without a GPU; calling any op without the built library or
 without a CUDA device raises ``CSAError``.  There is no CPU fallback.
@@ -24,12 +25,14 @@ LIB_PATH = os.path.join(_PKG, "libcsa.so")
 CSA_OK, CSA_E_ARG, CSA_E_UNSUPPORTED, CSA_E_CUDA, CSA_E_DEVICE, CSA_E_WORKSPACE = range(6)
 CSA_F32, CSA_BF16 = 0, 1
 CSA_F_NO_NORM, CSA_F_NO_ROPE, CSA_F_PORTABLE = 1, 2, 4
-CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS = 1, 2, 3, 4
-CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX = 1, 2, 3
+CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS, CSA_OP_OUT_PROJ = 1, 2, 3, 4, 5
+CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX, CSA_DEV_STREAM = 1, 2, 3, 4
 
 EXPORTED = (
-    "csa_compress", "hca_compress", "indexer_scores_topk", "indexer_scores_topk_noalloc",
-    "sparse_mqa_attn", "dense_hca_attn", "csa_workspace_bytes", "csa_check_status",
+    "csa_compress", "hca_compress", "csa_stream_state_bytes", "csa_compress_append",
+    "hca_compress_append", "indexer_scores_topk", "indexer_scores_topk_noalloc",
+    "sparse_mqa_attn", "dense_hca_attn", "grouped_output_projection", "csa_workspace_bytes",
+    "csa_check_status",
     "csa_status_string", "csa_launch_count", "csa_selftest_wait",
 )
 
@@ -93,6 +96,14 @@ def lib():
                                   P, f32, P, P, sz, P]
     L.dense_hca_attn.argtypes = [i32, i64, i64, i32, FP, P, P, P, i64, i32, P, i64, P, i32, P,
                                  f32, P, P, sz, P]
+    L.csa_stream_state_bytes.argtypes = [i32, i32, i32, i32, i32]
+    L.csa_stream_state_bytes.restype = sz
+    L.csa_compress_append.argtypes = [i32, i64, i32, FP, P, P, P, P, i32, i64, P, sz, P, i64, P,
+                                      P, sz, P]
+    L.hca_compress_append.argtypes = [i32, i64, i32, FP, P, P, i32, i64, P, sz, P, i64, P, P, sz,
+                                      P]
+    L.grouped_output_projection.argtypes = [i32, i64, i32, i32, i32, i32, i32, P, P, P, P, P, sz,
+                                            P]
     L.csa_workspace_bytes.argtypes = [i32, i32, i64, i64, i32, i32, i64, i32, i32]
     L.csa_workspace_bytes.restype = sz
     L.csa_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
@@ -101,9 +112,10 @@ def lib():
     L.csa_selftest_wait.argtypes = [i64, P, sz, P]
     L.csa_launch_count.argtypes = []
     L.csa_launch_count.restype = ctypes.c_ulonglong
-    for fn in ("csa_compress", "hca_compress", "indexer_scores_topk",
+    for fn in ("csa_compress", "hca_compress", "csa_compress_append", "hca_compress_append",
+               "indexer_scores_topk",
                "indexer_scores_topk_noalloc", "sparse_mqa_attn", "dense_hca_attn",
-               "csa_check_status", "csa_selftest_wait"):
+               "grouped_output_projection", "csa_check_status", "csa_selftest_wait"):
         getattr(L, fn).restype = i32
     _lib = L
     return L
@@ -203,6 +215,56 @@ def hca_compress(kv, z, m_prime: int, fmt: Fmt, pos0: int = 0, entries=None, win
     return (entries, win_out) if win_out is not None else entries
 
 
+def csa_stream_state_bytes(dtype, m: int, overlap: bool, c: int, z_cols: int) -> int:
+    dtype = dtype if isinstance(dtype, int) else (CSA_BF16 if dtype == torch.bfloat16 else CSA_F32)
+    return int(lib().csa_stream_state_bytes(dtype, m, int(bool(overlap)), c, z_cols))
+
+
+def stream_state(B: int, m: int, overlap: bool, c: int, z_cols: int, dtype, device=None):
+    """Zero-filled stream states of B sequences: a [B, stride] uint8 tensor."""
+    n = csa_stream_state_bytes(dtype, m, overlap, c, z_cols)
+    if n == 0:
+        raise CSAError(CSA_E_ARG, "csa_stream_state_bytes")
+    return torch.zeros((B, n), dtype=torch.uint8, device=device or "cuda")
+
+
+def csa_compress_append(kv_a, kv_b, z_a, z_b, m: int, fmt: Fmt, state, entries, pos0: int = 0,
+                        win_out=None, want_win=False, ws=None, stream=None):
+    """Appends one token per sequence (kv_a, kv_b: [B, c]; z_a, z_b: [B, z_cols])
+    to the CSA stream states ``state`` [B, stride]; a completed block's entry
+    goes to ``entries`` [B, n_cap, c].  Returns the window rows [B, c] when
+    asked (or given)."""
+    B, c = kv_a.shape
+    if want_win and win_out is None:
+        win_out = torch.empty_like(kv_a)
+    if ws is None:
+        ws = workspace(csa_workspace_bytes(CSA_OP_COMPRESS, _dt(kv_a), B, 1), kv_a.device)
+    f = fmt._c()
+    st = lib().csa_compress_append(_dt(kv_a), B, m, ctypes.byref(f), _p(kv_a), _p(kv_b), _p(z_a),
+                                   _p(z_b), z_a.shape[-1], pos0, _p(state), state.shape[1],
+                                   _p(entries), entries.shape[1], _p(win_out), _p(ws), ws.numel(),
+                                   _s(stream))
+    _check(st, "csa_compress_append")
+    return win_out
+
+
+def hca_compress_append(kv, z, m_prime: int, fmt: Fmt, state, entries, pos0: int = 0,
+                        win_out=None, want_win=False, ws=None, stream=None):
+    """Appends one token per sequence to the HCA stream states (see
+    csa_compress_append)."""
+    B, c = kv.shape
+    if want_win and win_out is None:
+        win_out = torch.empty_like(kv)
+    if ws is None:
+        ws = workspace(csa_workspace_bytes(CSA_OP_COMPRESS, _dt(kv), B, 1), kv.device)
+    f = fmt._c()
+    st = lib().hca_compress_append(_dt(kv), B, m_prime, ctypes.byref(f), _p(kv), _p(z),
+                                   z.shape[-1], pos0, _p(state), state.shape[1], _p(entries),
+                                   entries.shape[1], _p(win_out), _p(ws), ws.numel(), _s(stream))
+    _check(st, "hca_compress_append")
+    return win_out
+
+
 def indexer_scores_topk(q_I, w, k_I, m: int, k: int, q_pos=None, idx_out=None, score_out=None,
                         want_scores=False, ws=None, stream=None):
     """Indexer scores + causal top-k: q_I [B, Tq, H_I, d_I], w [B, Tq, H_I] fp32,
@@ -262,3 +324,20 @@ def dense_hca_attn(q, entries, m_prime: int, win, fmt: Fmt, n_win: int, sink=Non
                               _p(out), _p(ws), ws.numel(), _s(stream))
     _check(st, "dense_hca_attn")
     return out
+
+
+def grouped_output_projection(o, w_group, w_out, y=None, ws=None, stream=None):
+    """Grouped output projection: o [T, H, c], w_group [g, d_g, (H/g) c],
+    w_out [d, g d_g] -> y [T, d] (bf16)."""
+    T, H, c = o.shape
+    g, dg, _ = w_group.shape
+    d = w_out.shape[0]
+    if y is None:
+        y = torch.empty((T, d), dtype=o.dtype, device=o.device)
+    if ws is None:
+        ws = workspace(csa_workspace_bytes(CSA_OP_OUT_PROJ, _dt(o), 1, T, 0, 0, g * dg), o.device)
+    st = lib().grouped_output_projection(_dt(o), T, H, c, g, dg, d, _p(o), _p(w_group),
+                                         _p(w_out), _p(y), _p(ws), ws.numel(), _s(stream))
+    _check(st, "grouped_output_projection")
+    return y
+

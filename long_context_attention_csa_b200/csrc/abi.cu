@@ -157,12 +157,114 @@ csa_status hca_compress(int32_t dtype, int64_t B, int64_t T, int32_t m_prime, co
                          entries, win_out, ws, ws_bytes, stream);
 }
 
+size_t csa_stream_state_bytes(int32_t dtype, int32_t m, int32_t overlap, int32_t c,
+                              int32_t z_cols) {
+  if ((dtype != CSA_F32 && dtype != CSA_BF16) || m < 1 || c <= 0 || (z_cols != 1 && z_cols != c))
+    return 0;
+  return stream_state_bytes(dtype == CSA_BF16 ? 2 : 4, m, overlap ? 1 : 0, c, z_cols);
+}
+
+static csa_status append_common(int32_t dtype, int64_t B, int32_t m, bool overlap,
+                                const csa_fmt* fmt, const void* kv_a, const void* kv_b,
+                                const void* z_a, const void* z_b, int32_t z_cols, int64_t pos0,
+                                void* state, size_t state_stride, void* entries, int64_t n_cap,
+                                void* win_out, void* ws, size_t ws_bytes, void* stream) {
+  Fmt f;
+  csa_status st = check_fmt(dtype, fmt, &f);
+  if (st != CSA_OK) return st;
+  if (B < 0 || m < 1 || n_cap < 0 || B > 0x7fffffffLL) return CSA_E_ARG;
+  if (z_cols != 1 && z_cols != f.c) return CSA_E_ARG;
+  if (overlap ? (2 * m > 256) : (m > 4096)) return CSA_E_UNSUPPORTED;
+  if (f.c < 64 || f.c > 1024) return CSA_E_UNSUPPORTED;
+  if (B == 0) return CSA_OK;
+  if (!kv_a || !z_a || !state || (overlap && (!kv_b || !z_b)) || (n_cap > 0 && !entries))
+    return CSA_E_ARG;
+  if (!aligned16(kv_a) || !aligned16(z_a) || !aligned16(state) ||
+      (overlap && (!aligned16(kv_b) || !aligned16(z_b))) || (entries && !aligned16(entries)) ||
+      (win_out && !aligned16(win_out)))
+    return CSA_E_ARG;
+  const size_t need = stream_state_bytes(dtype == CSA_BF16 ? 2 : 4, m, overlap ? 1 : 0, f.c,
+                                         z_cols);
+  if (state_stride < need || (state_stride & 15)) return CSA_E_ARG;
+  if (!ws || ws_bytes < kWsScratch) return CSA_E_WORKSPACE;
+  StreamParams p{};
+  p.kv_a = kv_a;
+  p.kv_b = kv_b;
+  p.z_a = z_a;
+  p.z_b = z_b;
+  p.z_cols = z_cols;
+  p.m = m;
+  p.overlap = overlap ? 1 : 0;
+  p.f = f;
+  p.pos0 = pos0;
+  p.state = static_cast<uint8_t*>(state);
+  p.stride = state_stride;
+  p.entries = entries;
+  p.n_cap = n_cap;
+  p.win = win_out;
+  p.status = status_word(ws);
+  g_launches.fetch_add(1);
+  return cuda_status(launch_stream_append(dtype, p, B, S(stream)));
+}
+
+csa_status csa_compress_append(int32_t dtype, int64_t B, int32_t m, const csa_fmt* fmt,
+                               const void* kv_a, const void* kv_b, const void* z_a,
+                               const void* z_b, int32_t z_cols, int64_t pos0, void* state,
+                               size_t state_stride, void* entries, int64_t n_cap, void* win_out,
+                               void* ws, size_t ws_bytes, void* stream) {
+  return append_common(dtype, B, m, true, fmt, kv_a, kv_b, z_a, z_b, z_cols, pos0, state,
+                       state_stride, entries, n_cap, win_out, ws, ws_bytes, stream);
+}
+
+csa_status hca_compress_append(int32_t dtype, int64_t B, int32_t m_prime, const csa_fmt* fmt,
+                               const void* kv, const void* z, int32_t z_cols, int64_t pos0,
+                               void* state, size_t state_stride, void* entries, int64_t n_cap,
+                               void* win_out, void* ws, size_t ws_bytes, void* stream) {
+  return append_common(dtype, B, m_prime, false, fmt, kv, nullptr, z, nullptr, z_cols, pos0,
+                       state, state_stride, entries, n_cap, win_out, ws, ws_bytes, stream);
+}
+
+csa_status grouped_output_projection(int32_t dtype, int64_t T, int32_t H, int32_t c, int32_t g,
+                                     int32_t d_g, int32_t d, const void* o, const void* w_group,
+                                     const void* w_out, void* y, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
+  if (T < 0 || H <= 0 || c <= 0 || g <= 0 || d_g <= 0 || d <= 0) return CSA_E_ARG;
+  ProjParams p{};
+  p.T = T;
+  p.H = H;
+  p.c = c;
+  p.g = g;
+  p.dg = d_g;
+  p.d = d;
+  if (dtype != CSA_BF16 || !proj_supported(p)) return CSA_E_UNSUPPORTED;
+  if (T == 0) return CSA_OK;
+  if (!o || !w_group || !w_out || !y) return CSA_E_ARG;
+  if (!aligned16(o) || !aligned16(w_group) || !aligned16(w_out) || !aligned16(y))
+    return CSA_E_ARG;
+  if (!ws || ws_bytes < csa_workspace_bytes(CSA_OP_OUT_PROJ, dtype, 1, T, 0, 0,
+                                            (int64_t)g * d_g, 0, 0))
+    return CSA_E_WORKSPACE;
+  p.o = o;
+  p.w_group = w_group;
+  p.w_out = w_out;
+  p.v = static_cast<char*>(ws) + kWsScratch;
+  p.y = y;
+  p.status = status_word(ws);
+  unsigned long long n = 0;
+  cudaError_t e = launch_proj(p, S(stream), &n);
+  g_launches.fetch_add(n);
+  return cuda_status(e);
+}
+
 size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int32_t H, int32_t c,
                            int64_t N, int32_t k, int32_t n_win) {
   if (B < 0 || Tq < 0 || N < 0) return 0;
   switch (op) {
     case CSA_OP_COMPRESS:
       return kWsScratch;
+    case CSA_OP_OUT_PROJ:
+      return kWsScratch + (size_t)B * (size_t)Tq * (size_t)N * 2;
     case CSA_OP_INDEXER:
       return kWsScratch + (dtype == CSA_BF16 ? indexer_tc_scratch(B, Tq, N, k)
                                              : indexer_portable_scratch(B, Tq, N, k));

@@ -74,6 +74,39 @@ struct AttnParams {
 };
 cudaError_t launch_attn_portable(int dtype, const AttnParams& p, cudaStream_t stream);
 
+struct StreamParams {
+  const void* kv_a;   // [B, c] this call's token of each sequence (group a / HCA's group)
+  const void* kv_b;   // [B, c] group b (CSA only)
+  const void* z_a;    // [B, z_cols]
+  const void* z_b;
+  int z_cols;
+  int m;              // rate
+  int overlap;        // 1 = CSA
+  Fmt f;
+  int64_t pos0;
+  uint8_t* state;     // [B][stride] per-sequence tail buffers
+  size_t stride;
+  void* entries;      // [B, n_cap, c] entry cache
+  int64_t n_cap;
+  void* win;          // [B, c] window rows of this call's tokens, or null
+  unsigned* status;
+};
+size_t stream_state_bytes(int elem_bytes, int m, int overlap, int c, int z_cols);
+cudaError_t launch_stream_append(int dtype, StreamParams p, int64_t B, cudaStream_t stream);
+
+struct ProjParams {
+  int64_t T;
+  int H, c, g, dg, d;
+  const void* o;        // [T, H, c]
+  const void* w_group;  // [g, dg, (H/g) c]
+  const void* w_out;    // [d, g dg]
+  void* v;              // [T, g dg] intermediate
+  void* y;              // [T, d]
+  unsigned* status;
+};
+bool proj_supported(const ProjParams& p);
+cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream, unsigned long long* n_launch);
+
 // Adds n to the library's launch counter (csa_launch_count).
 void note_launches(unsigned long long n);
 

@@ -21,7 +21,13 @@ import torch
 
 # tensor ids: each tensor of a workload gets its own stream seed_base + id
 _TID = dict(kv_a=1, kv_b=2, z_a=3, z_b=4, q=5, q_I=6, k_I=7, w=8, sink=9, entries=10, win=11,
-            kv=12, z=13, idx=14, hca_entries=15, hca_win=16, hca_q=17, hca_sink=18)
+            kv=12, z=13, idx=14, hca_entries=15, hca_win=16, hca_q=17, hca_sink=18,
+            o=19, w_group=20, w_out=21)
+
+# Grouped output projection of the 64-head (V4-Flash-like) layer: model dim
+# d = 4096 (the pages' model table); g = 8 groups of 8 heads and d_g = 1024
+# are the reading taken (the pages give the map's shape, not its sizes).
+PROJ = dict(g=8, d_g=1024, d=4096)
 
 
 @dataclass(frozen=True)
@@ -205,3 +211,17 @@ def random_index_sets(counts, k: int, seed: int, device="cpu"):
     sel = torch.where(sel == big, torch.full_like(sel, -1), sel)
     out[:, :kk] = sel.to(torch.int32)
     return out.to(device)
+
+
+def projection_inputs(w: Workload, g: int, d_g: int, d: int, device="cpu"):
+    """Attention output o [T, H, c] (N(0,1), a stand-in for the attention's
+    output rows) and random synthetic projection weights scaled by
+    1/sqrt(fan_in): w_group [g, d_g, (H/g) c], w_out [d, g d_g]."""
+    T, H, c = w.T, w.H, w.c
+    kg = (H // g) * c
+    return dict(
+        o=randn((T, H, c), _seed(w, "o"), device, 1.0, w.dtype),
+        w_group=randn((g, d_g, kg), _seed(w, "w_group"), device, kg ** -0.5, w.dtype),
+        w_out=randn((d, g * d_g), _seed(w, "w_out"), device, (g * d_g) ** -0.5, w.dtype),
+    )
+

@@ -189,3 +189,53 @@ def test_bf16_shapes_outside_the_tensor_core_kernels_are_unsupported(L):
     assert L.dense_hca_attn(0, 1, 4, 4, ctypes.byref(f64c), d, None, d, 16, 4, d, 8, None, 8,
                             None, 0.0, d, None, 0, None) == 5
 
+
+
+def test_stream_append_rejects_bad_arguments(L):
+    """The streaming compression calls check their arguments before any CUDA
+    call; the state size follows the documented layout."""
+    f = _fmt()
+    d = ctypes.c_void_p(4096)
+    mis = ctypes.c_void_p(4100)
+    need = L.csa_stream_state_bytes(1, 4, 1, 512, 512)
+    assert need == ((16 + 3 * 4 * (512 + 512) * 2 + 255) // 256) * 256
+    assert L.csa_stream_state_bytes(1, 128, 0, 512, 1) == ((16 + 128 * 513 * 2 + 255) // 256) * 256
+    assert L.csa_stream_state_bytes(1, 4, 1, 512, 7) == 0
+    # stride too small / not a multiple of 16, misaligned state, bad z_cols, m too large
+    assert L.csa_compress_append(1, 2, 4, ctypes.byref(f), d, d, d, d, 512, 0, d, need - 16, d, 8,
+                                 None, d, 256, None) == 1
+    assert L.csa_compress_append(1, 2, 4, ctypes.byref(f), d, d, d, d, 512, 0, d, need + 8, d, 8,
+                                 None, d, 256, None) == 1
+    assert L.csa_compress_append(1, 2, 4, ctypes.byref(f), d, d, d, d, 512, 0, mis, need, d, 8,
+                                 None, d, 256, None) == 1
+    assert L.csa_compress_append(1, 2, 4, ctypes.byref(f), d, d, d, d, 3, 0, d, need, d, 8,
+                                 None, d, 256, None) == 1
+    assert L.csa_compress_append(1, 2, 200, ctypes.byref(f), d, d, d, d, 512, 0, d, 1 << 30, d,
+                                 8, None, d, 256, None) == 2
+    # group b missing for CSA; missing workspace; empty batch is a no-op
+    assert L.csa_compress_append(1, 2, 4, ctypes.byref(f), d, None, d, d, 512, 0, d, need, d, 8,
+                                 None, d, 256, None) == 1
+    assert L.csa_compress_append(1, 2, 4, ctypes.byref(f), d, d, d, d, 512, 0, d, need, d, 8,
+                                 None, None, 0, None) == 5
+    assert L.hca_compress_append(1, 0, 128, ctypes.byref(f), None, None, 512, 0, None, 0, None, 0,
+                                 None, None, 0, None) == 0
+
+
+def test_projection_rejects_bad_arguments(L):
+    d = ctypes.c_void_p(4096)
+    # float32, heads not divisible by groups, group width not a multiple of 64 -> unsupported
+    assert L.grouped_output_projection(0, 8, 16, 512, 4, 256, 512, d, d, d, d, d, 1 << 30,
+                                       None) == 2
+    assert L.grouped_output_projection(1, 8, 16, 512, 3, 256, 512, d, d, d, d, d, 1 << 30,
+                                       None) == 2
+    assert L.grouped_output_projection(1, 8, 1, 96, 1, 256, 512, d, d, d, d, d, 1 << 30,
+                                       None) == 2
+    # null pointer, short workspace; empty is a no-op
+    assert L.grouped_output_projection(1, 8, 16, 512, 4, 256, 512, None, d, d, d, d, 1 << 30,
+                                       None) == 1
+    need = L.csa_workspace_bytes(5, 1, 1, 8, 0, 0, 4 * 256, 0, 0)
+    assert need == 256 + 8 * 1024 * 2
+    assert L.grouped_output_projection(1, 8, 16, 512, 4, 256, 512, d, d, d, d, d, need - 1,
+                                       None) == 5
+    assert L.grouped_output_projection(1, 0, 16, 512, 4, 256, 512, None, None, None, None, None,
+                                       0, None) == 0

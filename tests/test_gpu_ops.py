@@ -268,7 +268,7 @@ def _attn_inputs_prefill(w, dense=False):
     return inp
 
 
-def _check_attn(w, inp, out, rows, dense, flags=0, q_pos=None, win_pos0=None):
+def _check_attn(w, inp, out, rows, dense, flags=0, q_pos=None, win_pos0=None, roundings=1):
     B = out.shape[0]
     for b in range(B):
         pos = rows if q_pos is None else q_pos[b].cpu().numpy()[rows]
@@ -278,7 +278,7 @@ def _check_attn(w, inp, out, rows, dense, flags=0, q_pos=None, win_pos0=None):
             w.n_win, idx=None if dense else inp["idx"][b][rows].cpu().numpy(),
             m_dense=w.m_prime if dense else 0,
             sink=None if inp["sink"] is None else f64(inp["sink"]), q_pos=pos, win_pos0=wp0)
-        assert_close(out[b][rows], ref, w.dtype, f"attention b={b}")
+        assert_close(out[b][rows], ref, w.dtype, f"attention b={b}", roundings=roundings)
 
 
 @pytest.mark.parametrize("flags", PATHS)
@@ -536,7 +536,11 @@ def test_attention_logit_beyond_the_bound_is_flagged():
     out = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"],
                               gfmt(w, csa.CSA_F_PORTABLE), w.n_win, sink=inp["sink"], ws=ws)
     assert csa.csa_check_status(ws) == (csa.CSA_OK, 0)
-    _check_attn(w, inp, out, np.arange(0, w.T, 3), dense=False, flags=csa.CSA_F_PORTABLE)
+    # logits near 100 carry float32 dot-product errors of ~1e-4 absolute, which
+    # move the weights by as much relatively: half an ulp more than the output
+    # rounding alone (measured 0.66 ulp at |out| ~ 36)
+    _check_attn(w, inp, out, np.arange(0, w.T, 3), dense=False, flags=csa.CSA_F_PORTABLE,
+                roundings=2)
 
 
 @pytest.mark.parametrize("flags", PATHS)
