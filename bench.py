@@ -708,6 +708,49 @@ class DecodeStep:
                 w.B * (n_h + w.n_win) * w.c * 2 + 2 * w.B * w.H * w.c * 2))
         self.inp = inp
 
+        # streaming compression of the step's new token (one per sequence), the
+        # states positioned at token L - 1 so the token completes a block: CSA
+        # entry L/m - 1 (and for the pair HCA entry L/m' - 1) is pooled from a
+        # filled tail buffer.  Timed beside the step, not inside it.
+        self.append = []
+        c = w.c
+
+        def state_at_end(overlap, m):
+            st = csa.stream_state(w.B, m, overlap, c, c, w.dtype, dev)
+            n = (3 if overlap else 1) * m * 2 * c
+            rows = wl.randn((w.B, n), 300 + m, dev, dtype=w.dtype)
+            st[:, 16:16 + 2 * n] = rows.view(torch.uint8).view(w.B, 2 * n)
+            st[:, :8] = torch.tensor([w.T - 1] * w.B, dtype=torch.int64).view(
+                torch.uint8).view(w.B, 8).to(dev)
+            return st
+
+        tok = [wl.randn((w.B, c), 310 + i, dev, dtype=w.dtype) for i in range(4)]
+        self.tok = tok
+        ent_c = torch.empty((w.B, w.n_csa, c), dtype=w.dtype, device=dev)
+        win_c = torch.empty((w.B, c), dtype=w.dtype, device=dev)
+        st_c = state_at_end(True, w.m)
+        ws_s = csa.workspace(256, dev)
+        self.ws.append(ws_s)
+        self.st_c = st_c
+        self.append.append(("csa_compress_append", lambda: csa.csa_compress_append(
+            tok[0], tok[1], tok[2], tok[3], w.m, fmt, st_c, ent_c, win_out=win_c, ws=ws_s),
+            st_c.shape[1] * w.B))
+        if w.kind == "decode_pair":
+            ent_h = torch.empty((w.B, w.n_hca, c), dtype=w.dtype, device=dev)
+            st_h = state_at_end(False, w.m_prime)
+            self.st_h = st_h
+            self.append.append(("hca_compress_append", lambda: csa.hca_compress_append(
+                tok[0], tok[2], w.m_prime, fmt, st_h, ent_h, win_out=win_c, ws=ws_s),
+                st_h.shape[1] * w.B))
+        self.ent_c = ent_c
+
+    def rewind(self):
+        """Puts every stream state back at token L - 1 (each append advances it)."""
+        self.st_c[:, :8] = torch.tensor([self.w.T - 1] * self.w.B, dtype=torch.int64).view(
+            torch.uint8).view(self.w.B, 8).to(self.st_c.device)
+        if hasattr(self, "st_h"):
+            self.st_h[:, :8] = self.st_c[:, :8]
+
     def run(self):
         for _, fn, _ in self.stages:
             fn()
@@ -719,17 +762,21 @@ class DecodeStep:
                 raise RuntimeError(f"{self.w.name}: device status {st}/{d}")
 
 
-def graph_ms(fn, steps: int, flush) -> float:
+def graph_ms(fn, steps: int, flush, before=None) -> float:
     """Mean device time of `fn` captured once in a CUDA graph and replayed
-    `steps` times, with the L2 flushed before each replay (outside the events),
-    as a decode server replays its step."""
+    `steps` times, with the L2 flushed (and `before` run) before each replay,
+    outside the events, as a decode server replays its step."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, capture_error_mode="thread_local"):
         fn()
+    if before:
+        before()
     g.replay()
     torch.cuda.synchronize()
     evs = []
     for _ in range(steps):
+        if before:
+            before()
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -830,6 +877,13 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
     step_ms = allmax(graph_ms(d.run, steps, flush), ws_n)
     stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.stages}
     d.check()
+    append = {}
+    for n, fn, nb in d.append:
+        # a state rewind (outside the events) before every timed append, so
+        # each one completes a block
+        ms = graph_ms(fn, steps, flush, before=d.rewind)
+        append[n] = {"ms": ms, "state_bytes_read": nb, "GBps": nb / ms / 1e6}
+    d.check()
     hbm, _, src = peaks()
     nb = decode_bytes(w)
     achieved = nb / (step_ms * 1e-3) / 1e9
@@ -841,6 +895,9 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
                    "l2": "flushed before every replay (outside the events)",
                    "timing": "whole step captured once in a CUDA graph, replayed"},
         "stages_ms": stages,
+        "stream_append": {**append, "note": "the step's new token appended to each sequence's "
+                          "compression state (completing a block: entry pooled from the tail "
+                          "buffer); latency-bound, timed beside the step"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "algorithmic_bytes_per_step": nb,
                      "peak_source": f"{src} HBM copy (MEASURED_PEAKS.json)"

@@ -179,10 +179,10 @@ static csa_status append_common(int32_t dtype, int64_t B, int32_t m, bool overla
   if (B == 0) return CSA_OK;
   if (!kv_a || !z_a || !state || (overlap && (!kv_b || !z_b)) || (n_cap > 0 && !entries))
     return CSA_E_ARG;
-  if (!aligned16(kv_a) || !aligned16(z_a) || !aligned16(state) ||
-      (overlap && (!aligned16(kv_b) || !aligned16(z_b))) || (entries && !aligned16(entries)) ||
-      (win_out && !aligned16(win_out)))
+  if (!aligned16(kv_a) || !aligned16(state) || (overlap && !aligned16(kv_b)) ||
+      (entries && !aligned16(entries)) || (win_out && !aligned16(win_out)))
     return CSA_E_ARG;
+  if (z_cols != 1 && (!aligned16(z_a) || (overlap && !aligned16(z_b)))) return CSA_E_ARG;
   const size_t need = stream_state_bytes(dtype == CSA_BF16 ? 2 : 4, m, overlap ? 1 : 0, f.c,
                                          z_cols);
   if (state_stride < need || (state_stride & 15)) return CSA_E_ARG;

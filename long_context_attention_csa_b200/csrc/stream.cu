@@ -161,34 +161,45 @@ __global__ void __launch_bounds__(1024) stream_append_kernel(StreamParams p) {
   const int G = (int)blockDim.x / np;
   const int ns = m + ((p.overlap && s >= 1) ? m : 0);
   float mx0 = -INFINITY, mx1 = -INFINITY, d0 = 0.f, d1 = 0.f, a0 = 0.f, a1 = 0.f;
-  for (int i = g; i < ns; i += G) {
-    const T* row;
-    const T* zrow;
-    if (i < m) {
-      row = ra + (size_t)i * c;
-      zrow = rza + (size_t)i * zc;
-    } else {
-      row = rb + ((size_t)(par ^ 1) * m + (i - m)) * c;
-      zrow = rzb + ((size_t)(par ^ 1) * m + (i - m)) * zc;
+  constexpr int U = 8;   // slots whose loads are in flight together
+  for (int i0 = g; i0 < ns; i0 += G * U) {
+    float v0[U], v1[U], z0[U], z1[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * G;
+      if (i < ns) {
+        const T* row;
+        const T* zrow;
+        if (i < m) {
+          row = ra + (size_t)i * c;
+          zrow = rza + (size_t)i * zc;
+        } else {
+          row = rb + ((size_t)(par ^ 1) * m + (i - m)) * c;
+          zrow = rzb + ((size_t)(par ^ 1) * m + (i - m)) * zc;
+        }
+        load2(row + ch, v0[u], v1[u]);
+        if (zc == 1) {
+          z0[u] = z1[u] = to_float(zrow[0]);
+        } else {
+          load2(zrow + ch, z0[u], z1[u]);
+        }
+      }
     }
-    float v0, v1, z0, z1;
-    load2(row + ch, v0, v1);
-    if (zc == 1) {
-      z0 = z1 = to_float(zrow[0]);
-    } else {
-      load2(zrow + ch, z0, z1);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (i0 + u * G >= ns) break;
+      // online softmax in base 2 (the running maximum never decreases)
+      const float l0 = z0[u] * kLog2e, l1 = z1[u] * kLog2e;
+      const float n0 = fmaxf(mx0, l0), n1 = fmaxf(mx1, l1);
+      const float s0 = exp2f(mx0 - n0), s1 = exp2f(mx1 - n1);
+      const float e0 = exp2f(l0 - n0), e1 = exp2f(l1 - n1);
+      d0 = d0 * s0 + e0;
+      d1 = d1 * s1 + e1;
+      a0 = a0 * s0 + e0 * v0[u];
+      a1 = a1 * s1 + e1 * v1[u];
+      mx0 = n0;
+      mx1 = n1;
     }
-    // online softmax in base 2 (the running maximum never decreases)
-    const float l0 = z0 * kLog2e, l1 = z1 * kLog2e;
-    const float n0 = fmaxf(mx0, l0), n1 = fmaxf(mx1, l1);
-    const float s0 = exp2f(mx0 - n0), s1 = exp2f(mx1 - n1);
-    const float e0 = exp2f(l0 - n0), e1 = exp2f(l1 - n1);
-    d0 = d0 * s0 + e0;
-    d1 = d1 * s1 + e1;
-    a0 = a0 * s0 + e0 * v0;
-    a1 = a1 * s1 + e1 * v1;
-    mx0 = n0;
-    mx1 = n1;
   }
   if (G > 1) {   // merge the slot groups' partial states in group order
     float* mine = part + ((size_t)g * np + pair) * 6;
