@@ -89,6 +89,7 @@ typedef struct csa_fmt {
 #define CSA_OP_DENSE_ATTN 3
 #define CSA_OP_COMPRESS 4
 #define CSA_OP_OUT_PROJ 5   /* Tq = T, N = g * d_g */
+#define CSA_OP_INDEXER_MX 6 /* indexer_scores_topk_mxfp8 */
 
 /* ---- (1) compression ------------------------------------------------ */
 
@@ -238,6 +239,44 @@ csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int64_t Tq, int
                                        const void* k_I, int64_t N, const int64_t* q_pos,
                                        int32_t m, int32_t k, int32_t* idx_out, float* score_out,
                                        void* stream);
+
+/* ---- (2b) low-precision indexer: MX-FP8 operands ------------------------ */
+
+/*
+ * The indexer's QK path in low precision [§3.3 of the summary page, last
+ * paragraph, and §3.6: the indexer's query-key product runs in FP4 (the model
+ * is trained for it) and keeps almost all of the full-precision selection].
+ * Format taken: OCP Microscaling FP8 -- E4M3 elements with one power-of-two
+ * scale per 32 consecutive elements of a 128-element row,
+ * 2^(floor(log2 amax) - 8), elements rounded to nearest (ties to even) and
+ * saturated at 448; the scale tensor is laid out for the block-scaled tensor
+ * cores: per 128 rows of a batch element a 512-byte tile whose byte
+ * 16 (r mod 32) + 4 (r div 32) + kb holds row r's block-kb exponent + 127
+ * (0 for rows past the end).
+ *   x: [B, rows, 128] (dtype CSA_BF16 or CSA_F32); codes (out): [B, rows,
+ *   128] uint8; scales (out): [B, ceil(rows / 128), 512] uint8.
+ * Used for the cached K_I (rows = N) and each step's q_I (rows = Tq H_I).
+ * Errors: CSA_E_ARG (null or misaligned pointers, negative sizes),
+ * CSA_E_UNSUPPORTED (d != 128).
+ */
+csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
+                                  const void* x, void* codes, void* scales, void* stream);
+
+/*
+ * indexer_scores_topk on MX-FP8 operands (as indexer_mxfp8_quantize writes
+ * them): I[t,s] = sum_h w[t,h] ReLU(sum_kb 2^(eq + ek) sum_{i in kb} cq_i ck_i)
+ * with the E4M3 products and their sums in float32 on block-scaled tcgen05
+ * MMAs; the causal top-k, tie rule, padding and outputs as indexer_scores_topk.
+ *   q_codes: [B, Tq, 64, 128]; q_scales: [B, ceil(64 Tq / 128), 512];
+ *   k_codes: [B, N, 128]; k_scales: [B, ceil(N / 128), 512]; the others as
+ *   indexer_scores_topk.  H_I must be 64 and d_I 128 (else CSA_E_UNSUPPORTED).
+ *   ws: >= csa_workspace_bytes(CSA_OP_INDEXER_MX, CSA_BF16, B, Tq, 0, 0, N, k, 0).
+ */
+csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                                     const void* q_codes, const void* q_scales, const float* w,
+                                     const void* k_codes, const void* k_scales, int64_t N,
+                                     const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                                     float* score_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- (3) shared-KV MQA ------------------------------------------------ */
 

@@ -25,13 +25,15 @@ LIB_PATH = os.path.join(_PKG, "libcsa.so")
 CSA_OK, CSA_E_ARG, CSA_E_UNSUPPORTED, CSA_E_CUDA, CSA_E_DEVICE, CSA_E_WORKSPACE = range(6)
 CSA_F32, CSA_BF16 = 0, 1
 CSA_F_NO_NORM, CSA_F_NO_ROPE, CSA_F_PORTABLE = 1, 2, 4
-CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS, CSA_OP_OUT_PROJ = 1, 2, 3, 4, 5
+(CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS, CSA_OP_OUT_PROJ,
+ CSA_OP_INDEXER_MX) = 1, 2, 3, 4, 5, 6
 CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX, CSA_DEV_STREAM = 1, 2, 3, 4
 
 EXPORTED = (
     "csa_compress", "hca_compress", "csa_stream_state_bytes", "csa_compress_append",
     "hca_compress_append", "indexer_scores_topk", "indexer_scores_topk_noalloc",
-    "sparse_mqa_attn", "dense_hca_attn", "grouped_output_projection", "csa_workspace_bytes",
+    "indexer_mxfp8_quantize", "indexer_scores_topk_mxfp8", "sparse_mqa_attn", "dense_hca_attn",
+    "grouped_output_projection", "csa_workspace_bytes",
     "csa_check_status",
     "csa_status_string", "csa_launch_count", "csa_selftest_wait",
 )
@@ -102,6 +104,9 @@ def lib():
                                       P, sz, P]
     L.hca_compress_append.argtypes = [i32, i64, i32, FP, P, P, i32, i64, P, sz, P, i64, P, P, sz,
                                       P]
+    L.indexer_mxfp8_quantize.argtypes = [i32, i64, i64, i32, P, P, P, P]
+    L.indexer_scores_topk_mxfp8.argtypes = [i64, i64, i32, i32, P, P, P, P, P, i64, P, i32, i32,
+                                            P, P, P, sz, P]
     L.grouped_output_projection.argtypes = [i32, i64, i32, i32, i32, i32, i32, P, P, P, P, P, sz,
                                             P]
     L.csa_workspace_bytes.argtypes = [i32, i32, i64, i64, i32, i32, i64, i32, i32]
@@ -115,7 +120,8 @@ def lib():
     for fn in ("csa_compress", "hca_compress", "csa_compress_append", "hca_compress_append",
                "indexer_scores_topk",
                "indexer_scores_topk_noalloc", "sparse_mqa_attn", "dense_hca_attn",
-               "grouped_output_projection", "csa_check_status", "csa_selftest_wait"):
+               "grouped_output_projection", "indexer_mxfp8_quantize",
+               "indexer_scores_topk_mxfp8", "csa_check_status", "csa_selftest_wait"):
         getattr(L, fn).restype = i32
     _lib = L
     return L
@@ -283,6 +289,42 @@ def indexer_scores_topk(q_I, w, k_I, m: int, k: int, q_pos=None, idx_out=None, s
                                    _p(q_pos), m, k, _p(idx_out), _p(score_out), _p(ws),
                                    ws.numel(), _s(stream))
     _check(st, "indexer_scores_topk")
+    return (idx_out, score_out) if score_out is not None else idx_out
+
+
+def indexer_mxfp8_quantize(x, codes=None, scales=None, stream=None):
+    """MX-FP8 codes and scale tiles of x [B, ..., 128] (rows = the middle dims
+    flattened): codes uint8 with x's shape, scales [B, ceil(rows/128), 512]."""
+    B, d = x.shape[0], x.shape[-1]
+    rows = x[0].numel() // d if B else 0
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, (rows + 127) // 128, 512), dtype=torch.uint8, device=x.device)
+    st = lib().indexer_mxfp8_quantize(_dt(x), B, rows, d, _p(x), _p(codes), _p(scales), _s(stream))
+    _check(st, "indexer_mxfp8_quantize")
+    return codes, scales
+
+
+def indexer_scores_topk_mxfp8(q_codes, q_scales, w, k_codes, k_scales, m: int, k: int,
+                              q_pos=None, idx_out=None, score_out=None, want_scores=False,
+                              ws=None, stream=None):
+    """indexer_scores_topk on MX-FP8 operands: q_codes [B, Tq, 64, 128] and
+    k_codes [B, N, 128] uint8 with their scale tiles."""
+    B, Tq, HI, dI = q_codes.shape
+    N = k_codes.shape[1]
+    dev = q_codes.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Tq, k), dtype=torch.int32, device=dev)
+    if want_scores and score_out is None:
+        score_out = torch.empty((B, Tq, k), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(csa_workspace_bytes(CSA_OP_INDEXER_MX, CSA_BF16, B, Tq, 0, 0, N, k), dev)
+    st = lib().indexer_scores_topk_mxfp8(B, Tq, HI, dI, _p(q_codes), _p(q_scales), _p(w),
+                                         _p(k_codes), _p(k_scales), N, _p(q_pos), m, k,
+                                         _p(idx_out), _p(score_out), _p(ws), ws.numel(),
+                                         _s(stream))
+    _check(st, "indexer_scores_topk_mxfp8")
     return (idx_out, score_out) if score_out is not None else idx_out
 
 

@@ -224,6 +224,58 @@ csa_status hca_compress_append(int32_t dtype, int64_t B, int32_t m_prime, const 
                        state, state_stride, entries, n_cap, win_out, ws, ws_bytes, stream);
 }
 
+csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
+                                  const void* x, void* codes, void* scales, void* stream) {
+  if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
+  if (B < 0 || rows < 0 || d <= 0) return CSA_E_ARG;
+  if (d != 128) return CSA_E_UNSUPPORTED;
+  if (B > 65535 || rows > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  if (B == 0 || rows == 0) return CSA_OK;
+  if (!x || !codes || !scales) return CSA_E_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return CSA_E_ARG;
+  g_launches.fetch_add(1);
+  return cuda_status(launch_mxfp8_quantize(dtype, x, codes, scales, B, rows, S(stream)));
+}
+
+csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                                     const void* q_codes, const void* q_scales, const float* w,
+                                     const void* k_codes, const void* k_scales, int64_t N,
+                                     const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                                     float* score_out, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 0 || Tq < 0 || N < 0 || H_I <= 0 || d_I <= 0 || m < 1 || k < 1) return CSA_E_ARG;
+  if (H_I != 64 || d_I != 128) return CSA_E_UNSUPPORTED;
+  if (B > 65535 || Tq > 65535 || N > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
+  if (B == 0 || Tq == 0) return CSA_OK;
+  if (!q_codes || !q_scales || !w || !idx_out || (N > 0 && (!k_codes || !k_scales)))
+    return CSA_E_ARG;
+  if (!aligned16(q_codes) || !aligned16(q_scales) ||
+      (N > 0 && (!aligned16(k_codes) || !aligned16(k_scales))))
+    return CSA_E_ARG;
+  if (!ws || ws_bytes < csa_workspace_bytes(CSA_OP_INDEXER_MX, CSA_BF16, B, Tq, 0, 0, N, k, 0))
+    return CSA_E_WORKSPACE;
+  IndexerParams p{};
+  p.B = B;
+  p.Tq = Tq;
+  p.HI = H_I;
+  p.dI = d_I;
+  p.q_I = q_codes;
+  p.w = w;
+  p.k_I = k_codes;
+  p.N = N;
+  p.q_pos = q_pos;
+  p.m = m;
+  p.k = k;
+  p.idx_out = idx_out;
+  p.score_out = score_out;
+  p.status = status_word(ws);
+  p.scratch = static_cast<char*>(ws) + kWsScratch;
+  p.scratch_bytes = ws_bytes - kWsScratch;
+  unsigned long long n = 0;
+  cudaError_t e = launch_indexer_mx(p, q_scales, k_scales, S(stream), &n);
+  g_launches.fetch_add(n);
+  return cuda_status(e);
+}
+
 csa_status grouped_output_projection(int32_t dtype, int64_t T, int32_t H, int32_t c, int32_t g,
                                      int32_t d_g, int32_t d, const void* o, const void* w_group,
                                      const void* w_out, void* y, void* ws, size_t ws_bytes,
@@ -263,6 +315,8 @@ size_t csa_workspace_bytes(int32_t op, int32_t dtype, int64_t B, int64_t Tq, int
   switch (op) {
     case CSA_OP_COMPRESS:
       return kWsScratch;
+    case CSA_OP_INDEXER_MX:
+      return kWsScratch + indexer_mx_scratch(B, Tq, N, k);
     case CSA_OP_OUT_PROJ:
       return kWsScratch + (size_t)B * (size_t)Tq * (size_t)N * 2;
     case CSA_OP_INDEXER:

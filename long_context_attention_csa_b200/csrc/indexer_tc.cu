@@ -67,14 +67,19 @@ __device__ __forceinline__ float relu_weighted_sum64(const float* wt, const uint
   return a0 + a1;
 }
 
-template <int TOK>
+// MX: the operands are MX-FP8 (one byte per element, no halves) and each
+// K_I tile and the query block bring a 512-byte scale-factor tile.
+template <int TOK, bool MX = false>
 struct Smem {
-  static constexpr int kB = TOK * kHI * kDI * 2;           // q_I block
+  static constexpr int kEl = MX ? 1 : 2;                   // bytes per operand element
+  static constexpr int kTile = kBM * kDI * kEl;            // one K_I tile
+  static constexpr int kB = TOK * kHI * kDI * kEl;         // q_I block
   static constexpr int kStages = Cfg<TOK>::kStages;
   static constexpr int kChunk = Cfg<TOK>::kChunk;
   static constexpr int off_b = 0;
   static constexpr int off_a = kB;
-  static constexpr int off_scores = off_a + kStages * kTileBytes;
+  static constexpr int off_sf = off_a + kStages * kTile;   // MX: [kStages + 1][512] scales
+  static constexpr int off_scores = off_sf + (MX ? (kStages + 1) * 512 : 0);
   static constexpr int off_w = off_scores + TOK * kChunk * 4;
   static constexpr int off_hist = off_w + TOK * kHI * 4;
   static constexpr int off_cand = off_hist + TOK * 256 * 4;   // [TOK][kBinCap] (score, index)
@@ -97,6 +102,10 @@ struct TcIdxArgs {
   float* cand_score;   // [B*Tq][n_chunks][k] when n_chunks > 1
   int32_t* cand_idx;
   unsigned* status;
+  // MX-FP8 operands: scale-factor tiles [B][tiles][512] of q_I and K_I
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  int64_t q_sf_tiles, k_sf_tiles;
 };
 
 __device__ __forceinline__ int64_t vis_count(int64_t pos, int m, int64_t N) {
@@ -833,15 +842,21 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
   if (!solo) cluster_wait();   // no CTA leaves while another may still read its shared memory
 }
 
-template <int TOK>
+template <int TOK, bool MX>
 __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k, TcIdxArgs a) {
-  using L = Smem<TOK>;
+  static_assert(!MX || TOK == 1, "MX-FP8 operands: single-token groups");
+  using L = Smem<TOK, MX>;
   constexpr int kStages = L::kStages;
   constexpr int kChunk = L::kChunk;
+  constexpr int kTile = L::kTile;
   constexpr int kN = TOK * kHI;                 // MMA N
-  constexpr uint32_t kCols = 2 * kN;            // two accumulators
+  // two accumulators; MX adds two 4-column K_I scale buffers and the query's
+  // scale tile (4 columns), rounded up to a power of two
+  constexpr uint32_t kCols = MX ? 256 : 2 * kN;
+  constexpr uint32_t kSfa = 2 * kN;
+  constexpr uint32_t kSfb = kSfa + 8;
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kN, 0, 0);
 
   extern __shared__ uint8_t smem_raw[];
@@ -902,10 +917,18 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
     if (n_tiles > 0) {   // the q_I block first: its latency overlaps the rest of the setup
       tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
-      mbar_arrive_expect_tx(bfull, L::kB);
       const int32_t qrow = (int32_t)(t0 * kHI);
-      tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
-      tma_load_3d(sB + L::kB / 2, &map_q, bfull, 64, qrow, b);
+      if constexpr (MX) {
+        // codes (128 bytes a row, one box) and the scale tile holding this token's rows
+        mbar_arrive_expect_tx(bfull, L::kB + 512);
+        tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
+        bulk_load(smem_u32(sm + L::off_sf + kStages * 512),
+                  a.q_sf + ((int64_t)b * a.q_sf_tiles + (t0 * kHI) / kBM) * 512, 512, bfull);
+      } else {
+        mbar_arrive_expect_tx(bfull, L::kB);
+        tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
+        tma_load_3d(sB + L::kB / 2, &map_q, bfull, 64, qrow, b);
+      }
     }
   }
   for (int i = threadIdx.x; i < TOK * kHI; i += blockDim.x) {
@@ -933,11 +956,18 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
           report(a.status, CSA_DEV_TIMEOUT, 1u);
           break;
         }
-        mbar_arrive_expect_tx(&full[s], kTileBytes);
-        uint8_t* dst = sA + s * kTileBytes;
         const int32_t erow = (int32_t)(e0 + (int64_t)i * kBM);
-        tma_load_3d(dst, &map_k, &full[s], 0, erow, b);
-        tma_load_3d(dst + kTileBytes / 2, &map_k, &full[s], 64, erow, b);
+        if constexpr (MX) {
+          mbar_arrive_expect_tx(&full[s], kTile + 512);
+          tma_load_3d(sA + s * kTile, &map_k, &full[s], 0, erow, b);
+          bulk_load(smem_u32(sm + L::off_sf + s * 512),
+                    a.k_sf + ((int64_t)b * a.k_sf_tiles + erow / kBM) * 512, 512, &full[s]);
+        } else {
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          uint8_t* dst = sA + s * kTileBytes;
+          tma_load_3d(dst, &map_k, &full[s], 0, erow, b);
+          tma_load_3d(dst + kTileBytes / 2, &map_k, &full[s], 64, erow, b);
+        }
         issued = i + 1;
       }
       // drain: every issued copy has landed before the CTA may exit
@@ -954,6 +984,11 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
       } else {
         const uint32_t b_base = smem_u32(sB);
         const uint32_t a_base = smem_u32(sA);
+        if constexpr (MX) {
+          // the query's scale tile into TMEM (rows 32 j + l: lane l, column j)
+          tmem_cp_32x128b_x4(tmem + kSfb,
+                             smem_desc(smem_u32(sm + L::off_sf + kStages * 512), 16, 128, 0));
+        }
         for (int i = 0; i < n_tiles; ++i) {
           const int s = i % kStages;
           const uint32_t ph = (uint32_t)(i / kStages) & 1u;
@@ -966,13 +1001,30 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
           }
           tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(buf * kN);
+          if constexpr (MX) {
+            // this tile's K_I scales into TMEM (issued before, and executed
+            // before, the MMAs below that read them)
+            const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)buf;
+            tmem_cp_32x128b_x4(sfa, smem_desc(smem_u32(sm + L::off_sf + s * 512), 16, 128, 0));
+            // a 128-row scale tile holds two tokens' 64 heads: this token's half
+            const uint32_t sfb = tmem + kSfb + 2u * (uint32_t)(t0 & 1);
 #pragma unroll
-          for (int kk = 0; kk < kDI / 16; ++kk) {
-            const uint32_t koff = (uint32_t)((kk & 3) * 32);  // 16 bf16 per K step
-            uint64_t ad = smem_desc(a_base + s * kTileBytes + (kk >> 2) * (kTileBytes / 2) + koff,
-                                    16, 1024, 2);
-            uint64_t bd = smem_desc(b_base + (kk >> 2) * (L::kB / 2) + koff, 16, 1024, 2);
-            mma_bf16_ss(d, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kDI / 32; ++kk) {   // K = 32 per MMA, one scale each
+              const uint64_t ad = smem_desc(a_base + s * kTile + kk * 32, 16, 1024, 2);
+              const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, 2);
+              mma_mxf8_ss(d, ad, bd, idesc_mxf8_e4m3(kBM, kN, kk, kk),
+                          sfa | ((uint32_t)kk << 30), sfb | ((uint32_t)kk << 30),
+                          kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kDI / 16; ++kk) {
+              const uint32_t koff = (uint32_t)((kk & 3) * 32);  // 16 bf16 per K step
+              uint64_t ad = smem_desc(a_base + s * kTileBytes + (kk >> 2) * (kTileBytes / 2) +
+                                          koff, 16, 1024, 2);
+              uint64_t bd = smem_desc(b_base + (kk >> 2) * (L::kB / 2) + koff, 16, 1024, 2);
+              mma_bf16_ss(d, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+            }
           }
           mma_commit(&empty[s]);
           mma_commit(&tfull[buf]);
@@ -1682,19 +1734,27 @@ inline int n_chunks_for(int64_t N, int tok) {
   return n < 1 ? 1 : (int)n;
 }
 
-template <int TOK>
+template <int TOK, bool MX = false>
 cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
   CUtensorMap mq, mk;
-  if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, TOK * kHI))
-    return cudaErrorInvalidValue;
-  if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64, kBM))
-    return cudaErrorInvalidValue;
-  const int smem = Smem<TOK>::bytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<TOK>,
+  if constexpr (MX) {
+    if (!make_map_u8_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, kDI, TOK * kHI))
+      return cudaErrorInvalidValue;
+    if (!make_map_u8_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, kDI, kBM))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, TOK * kHI))
+      return cudaErrorInvalidValue;
+    if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64,
+                          kBM))
+      return cudaErrorInvalidValue;
+  }
+  const int smem = Smem<TOK, MX>::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<TOK, MX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.n_chunks, (unsigned)((p.Tq + TOK - 1) / TOK), (unsigned)p.B);
-  indexer_tc_kernel<TOK><<<grid, kThreads, smem, stream>>>(mq, mk, a);
+  indexer_tc_kernel<TOK, MX><<<grid, kThreads, smem, stream>>>(mq, mk, a);
   return cudaGetLastError();
 }
 
@@ -1758,6 +1818,54 @@ cudaError_t launch_persist(const IndexerParams& p, const TcIdxArgs& a, cudaStrea
 }
 
 }  // namespace
+
+size_t indexer_mx_scratch(int64_t B, int64_t Tq, int64_t N, int k) {
+  const int nc = n_chunks_for(N, 1);
+  if (nc <= 1) return 0;
+  return (size_t)B * (size_t)Tq * (size_t)nc * (size_t)k * 8;
+}
+
+cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const void* k_sf,
+                              cudaStream_t stream, unsigned long long* n_launch) {
+  *n_launch = 0;
+  if (p.B == 0 || p.Tq == 0) return cudaSuccess;
+  if (p.N == 0) {   // nothing to score: every row is padding
+    const int64_t n = p.B * p.Tq * (int64_t)p.k;
+    const int64_t blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+    topk_padding_kernel<<<(unsigned)blocks, 256, 0, stream>>>(n, p.idx_out, p.score_out);
+    *n_launch = 1;
+    return cudaGetLastError();
+  }
+  TcIdxArgs a{};
+  a.Tq = p.Tq;
+  a.N = p.N;
+  a.m = p.m;
+  a.k = p.k;
+  a.n_chunks = n_chunks_for(p.N, 1);
+  a.w = p.w;
+  a.q_pos = p.q_pos;
+  a.idx_out = p.idx_out;
+  a.score_out = p.score_out;
+  a.status = p.status;
+  a.q_sf = static_cast<const uint8_t*>(q_sf);
+  a.k_sf = static_cast<const uint8_t*>(k_sf);
+  a.q_sf_tiles = (p.Tq * kHI + kBM - 1) / kBM;
+  a.k_sf_tiles = (p.N + kBM - 1) / kBM;
+  if (a.n_chunks > 1) {
+    const size_t n = (size_t)p.B * p.Tq * a.n_chunks * p.k;
+    if (p.scratch_bytes < n * 8) return cudaErrorInvalidValue;
+    a.cand_score = static_cast<float*>(p.scratch);
+    a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
+  }
+  cudaError_t e = launch_tok<1, true>(p, a, stream);
+  if (e != cudaSuccess) return e;
+  *n_launch = 1;
+  if (a.n_chunks > 1) {
+    e = launch_merge(a, p.B * p.Tq, stream);
+    *n_launch = 2;
+  }
+  return e;
+}
 
 bool indexer_tc_supported(const IndexerParams& p) {
   auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };

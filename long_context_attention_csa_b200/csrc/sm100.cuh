@@ -284,6 +284,44 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 A and B,
+// K-major, UE8M0 scale factors (one per 32 K elements), fp32 D.  sf_a / sf_b
+// select the byte of the scale-factor TMEM words this MMA's K block uses.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N, uint32_t sf_a,
+                                                       uint32_t sf_b) {
+  return ((sf_b & 3u) << 4)             // B scale-factor byte
+         | (0u << 7)                    // A format: E4M3
+         | (0u << 10)                   // B format: E4M3
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | (1u << 23)                   // scale format: UE8M0
+         | ((uint32_t)(M >> 4) << 24)   // M / 16
+         | ((sf_a & 3u) << 29);         // A scale-factor byte
+}
+
+// D[tmem] (+)= (A . 2^sfA)[smem] x (B . 2^sfB)[smem]^T, FP8 operands with
+// per-32-element UE8M0 scale factors read from TMEM (sfa / sfb: TMEM
+// addresses whose top two bits hold the byte the descriptor selects).
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copies 32 rows x 16 bytes from shared memory (rows contiguous: the
+// descriptor's 8-row groups 128 bytes apart, no swizzle) into TMEM lanes
+// 0..31, columns taddr .. taddr + 3, and the same into each of the other three
+// 32-lane quarters.  Issued by one thread; ordered with that thread's later
+// tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc)
+               : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(

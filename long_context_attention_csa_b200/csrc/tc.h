@@ -11,6 +11,15 @@ size_t indexer_tc_scratch(int64_t B, int64_t Tq, int64_t N, int k);
 cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
                               unsigned long long* n_launch);
 
+// The same with MX-FP8 operands (E4M3 codes, UE8M0 scale tiles; p.q_I and
+// p.k_I hold the codes), on block-scaled tcgen05 MMAs.
+size_t indexer_mx_scratch(int64_t B, int64_t Tq, int64_t N, int k);
+cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const void* k_sf,
+                              cudaStream_t stream, unsigned long long* n_launch);
+// MX-FP8 quantization of [B][rows][128] rows into codes and scale tiles.
+cudaError_t launch_mxfp8_quantize(int dtype, const void* x, void* codes, void* scales, int64_t B,
+                                  int64_t rows, cudaStream_t stream);
+
 // Shared-KV MQA (sparse and dense) on tcgen05.
 bool attn_tc_supported(const AttnParams& p);
 size_t attn_tc_scratch(int64_t B, int64_t Tq, int H, int c, int64_t max_keys);

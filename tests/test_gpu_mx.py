@@ -1,0 +1,125 @@
+"""GPU parity of the low-precision indexer path: MX-FP8 quantization of the
+indexer operands (bit for bit against the oracle's quantizer) and the indexer
+scores and top-k on block-scaled tcgen05 MMAs (bit for bit on integer inputs,
+within float32 accumulation and the tie band otherwise, against the oracle's
+indexer on the same dequantized operands)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import check_topk_rows, f64
+import long_context_attention_csa_b200 as csa
+from long_context_attention_csa_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def unpack_scales(sf, rows):
+    """[B, tiles, 512] scale tiles -> [B, rows, 4] exponents, and the bytes of
+    the padding rows of the last tile."""
+    sf = sf.cpu().numpy().astype(np.int64)
+    r = np.arange(rows)
+    pos = 16 * (r % 32) + 4 * ((r % 128) // 32)
+    out = np.empty((sf.shape[0], rows, 4), dtype=np.int64)
+    for b in range(sf.shape[0]):
+        out[b] = sf[b, r // 128][np.arange(rows)[:, None], pos[:, None] + np.arange(4)] - 127
+    pad = []
+    tiles = sf.shape[1]
+    for rr in range(rows, tiles * 128):
+        p = 16 * (rr % 32) + 4 * ((rr % 128) // 32)
+        pad.append(sf[:, tiles - 1, p:p + 4])
+    return out, (np.concatenate(pad, axis=1) if pad else np.zeros((sf.shape[0], 0)))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_mxfp8_quantize_matches_the_oracle(dtype):
+    """Codes and scale exponents equal the oracle's quantizer's, bit for bit:
+    random rows, a zero block, tiny (subnormal-scale) values, values that
+    saturate at 448, and a ragged last scale tile (300 rows)."""
+    B, rows = 2, 300
+    x = wl.randn((B, rows, 128), 501, DEV, dtype=torch.float32) * 3
+    x[0, 5, 32:64] = 0                                   # a zero block
+    x[0, 6, :32] = x[0, 6, :32] * 1e-30                  # tiny scale
+    x[1, 7, 64:96] = torch.linspace(-500, 500, 32)       # 500 / 2^(8 - 8) saturates
+    x[1, 8, :] = torch.linspace(-3, 3, 128)
+    x = x.to(dtype)
+    codes, sf = csa.indexer_mxfp8_quantize(x)
+    torch.cuda.synchronize()
+    ex, pad = unpack_scales(sf, rows)
+    assert np.all(pad == 0)
+    for b in range(B):
+        rc, re = oracle.mxfp8_quantize(f64(x[b]))
+        assert np.array_equal(codes[b].cpu().numpy(), rc), f"codes b={b}"
+        assert np.array_equal(ex[b], re), f"exponents b={b}"
+
+
+def _quantized(q_I, k_I):
+    qc, qs = csa.indexer_mxfp8_quantize(q_I)
+    kc, ks = csa.indexer_mxfp8_quantize(k_I)
+    return qc, qs, kc, ks
+
+
+@pytest.mark.parametrize("B,Tq,N,k,pos", [
+    (3, 1, 30000, 1024, "decode"),   # eight 4096-entry chunks, candidates merged
+    (1, 37, 700, 64, "prefill"),     # odd and even tokens (both halves of a scale tile)
+])
+def test_mxfp8_indexer_integer_inputs_bit_exact(B, Tq, N, k, pos):
+    """Small integers quantize exactly (scale 2^-7, codes up to 384) and every
+    product and sum is exact in float32: the selected sets (tie rule included)
+    and scores equal the oracle's on the same inputs."""
+    HI, dI, m = 64, 128, 4
+    qI = wl.randint_like_float((B, Tq, HI, dI), 511, -2, 3, DEV, torch.bfloat16)
+    kI = wl.randint_like_float((B, N, dI), 512, -2, 3, DEV, torch.bfloat16)
+    w = wl.randint_like_float((B, Tq, HI), 513, -2, 3, DEV, torch.float32)
+    if pos == "decode":
+        q_pos = torch.tensor([[m * N - 1], [m * (N // 3) + 2], [m * 200]], dtype=torch.int64)[:B]
+    else:
+        q_pos = torch.arange(Tq, dtype=torch.int64).unsqueeze(0) * 70 + 5
+    qc, qs, kc, ks = _quantized(qI, kI)
+    idx, sc = csa.indexer_scores_topk_mxfp8(qc, qs, w, kc, ks, m, k, q_pos=q_pos.to(DEV),
+                                            want_scores=True)
+    torch.cuda.synchronize()
+    for b in range(B):
+        p = q_pos[b].numpy()
+        ref_sc = oracle.mxfp8_indexer_scores(f64(qI[b]), f64(w[b]), f64(kI[b]), m, q_pos=p)
+        assert np.array_equal(ref_sc, oracle.indexer_scores(f64(qI[b]), f64(w[b]), f64(kI[b]), m,
+                                                            q_pos=p))   # quantization exact
+        ref_idx = oracle.topk(ref_sc, k, m, q_pos=p)
+        gi = idx[b].cpu().numpy()
+        assert np.array_equal(gi, ref_idx), f"b={b}"
+        v = gi >= 0
+        assert np.array_equal(sc[b].cpu().numpy().astype(np.float64)[v],
+                              np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v])
+
+
+def test_mxfp8_indexer_decode_workload():
+    """Eight rows of the csa_decode_b32_128k workload (32768 entries, top-k
+    1024) with N(0,1) operands: scores of the GPU's selection within 1e-4 of
+    the oracle's MX-FP8 scores, sets equal up to the tie band, and the MX-FP8
+    selection recalls the full-precision oracle selection at >= 95%."""
+    w = wl.scaled(wl.WORKLOADS["csa_decode_b32_128k"], B=8)
+    inp = wl.csa_decode_inputs(w, DEV)
+    qc, qs, kc, ks = _quantized(inp["q_I"], inp["k_I"])
+    idx, sc = csa.indexer_scores_topk_mxfp8(qc, qs, inp["w"], kc, ks, w.m, w.k,
+                                            q_pos=inp["q_pos"], want_scores=True)
+    torch.cuda.synchronize()
+    recall = []
+    for b in range(w.B):
+        p = inp["q_pos"][b].cpu().numpy()
+        ref_sc = oracle.mxfp8_indexer_scores(f64(inp["q_I"][b]), f64(inp["w"][b]),
+                                             f64(inp["k_I"][b]), w.m, q_pos=p)
+        ref_idx = oracle.topk(ref_sc, w.k, w.m, q_pos=p)
+        gi = idx[b].cpu().numpy()
+        check_topk_rows(gi, ref_idx, ref_sc, what=f"mx b={b}")
+        v = gi >= 0
+        gs = sc[b].cpu().numpy().astype(np.float64)[v]
+        want = np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v]
+        assert (np.abs(gs - want) / np.maximum(1.0, np.abs(want))).max() <= 1e-4
+        full = oracle.topk(oracle.indexer_scores(f64(inp["q_I"][b]), f64(inp["w"][b]),
+                                                 f64(inp["k_I"][b]), w.m, q_pos=p),
+                           w.k, w.m, q_pos=p)
+        recall.append(len(np.intersect1d(gi[v], full[full >= 0])) / max(1, (full >= 0).sum()))
+    assert np.mean(recall) >= 0.95, recall
