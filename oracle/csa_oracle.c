@@ -391,8 +391,8 @@ uint8_t orc_e4m3_encode(double x) {
       best_err = err;
     }
   }
-  if (best == 0) return 0x00;   /* +0 for both signs: the sign of zero is not kept */
-  return (uint8_t)(x < 0 ? (best | 0x80) : best);
+  /* the sign is kept, zero included: a negative value that rounds to zero is -0 */
+  return (uint8_t)(signbit(x) ? (best | 0x80) : best);
 }
 
 /* MX quantization of n elements (n a multiple of 32): codes[n], exps[n/32]
@@ -443,8 +443,7 @@ uint8_t orc_e2m1_encode(double x) {
       best_err = err;
     }
   }
-  if (best == 0) return 0;
-  return (uint8_t)(x < 0 ? (best | 8) : best);
+  return (uint8_t)(signbit(x) ? (best | 8) : best);   /* sign kept, -0 included */
 }
 
 void orc_mxfp4_quantize(int64_t n, const double* x, uint8_t* codes, int32_t* exps) {

@@ -25,9 +25,9 @@ def test_e4m3_format_values():
 
 
 def test_e4m3_round_trip_every_finite_code():
-    for c in list(range(0x00, 0x7F)) + list(range(0x81, 0xFF)):
+    for c in list(range(0x00, 0x7F)) + list(range(0x80, 0xFF)):
         assert oracle.e4m3_encode(oracle.e4m3_value(c)) == c, hex(c)
-    assert oracle.e4m3_encode(-0.0) == 0x00
+    assert oracle.e4m3_encode(-0.0) == 0x80          # the sign of zero is kept
     assert oracle.e4m3_encode(float("nan")) == 0x7F
 
 
@@ -37,7 +37,7 @@ def test_e4m3_ties_go_to_the_even_code():
         mid = (lo + hi) / 2
         want = c if c % 2 == 0 else c + 1
         assert oracle.e4m3_encode(mid) == want, hex(c)
-        assert oracle.e4m3_encode(-mid) == (want | 0x80 if want else 0x00)   # no -0 code
+        assert oracle.e4m3_encode(-mid) == (want | 0x80)   # sign kept, -0 included
 
 
 def test_e4m3_error_bound_and_monotonicity():
@@ -53,6 +53,23 @@ def test_e4m3_error_bound_and_monotonicity():
     sweep = np.linspace(-460, 460, 20001)
     codes = [oracle.e4m3_value(oracle.e4m3_encode(x)) for x in sweep]
     assert all(a <= b for a, b in zip(codes, codes[1:]))
+
+
+def test_e4m3_encode_equals_torch_float8_conversion():
+    """Against an independent implementation, torch's float32 -> float8_e4m3fn
+    conversion (IEEE rounding to nearest even, sign of zero kept), over the
+    subnormals, the normals and ties, below the first value that overflows
+    (464, halfway to the unrepresentable 480)."""
+    import torch
+
+    rng = np.random.default_rng(11)
+    xs = np.concatenate([np.linspace(-2.0 ** -5, 2.0 ** -5, 4001), rng.standard_normal(4000) * 50,
+                         [(oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) / 2 * sg
+                          for c in range(0x7E) for sg in (1, -1)], [-0.0, 0.0, 460.0, -460.0]])
+    xs = xs[np.abs(xs) < 464].astype(np.float32)
+    want = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(x)) for x in xs])
+    assert np.array_equal(got, want)
 
 
 def test_e4m3_saturates():
