@@ -744,6 +744,46 @@ class DecodeStep:
                 st_h.shape[1] * w.B))
         self.ent_c = ent_c
 
+        # the same step with the indexer on MX-FP8 operands: the cache's K_I
+        # quantized once (as the cache writer would store it), q_I every step
+        self.kc, self.ks = csa.indexer_mxfp8_quantize(inp["k_I"])
+        self.qc = torch.empty(inp["q_I"].shape, dtype=torch.uint8, device=dev)
+        self.qs = torch.empty((w.B, 1, 512), dtype=torch.uint8, device=dev)
+        ws_mx = csa.workspace(csa.csa_workspace_bytes(csa.CSA_OP_INDEXER_MX, 1, w.B, 1, 0, 0,
+                                                      w.n_csa, w.k, 0), dev)
+        self.ws.append(ws_mx)
+        self.mx_stages = [
+            ("indexer_mxfp8_quantize", lambda: csa.indexer_mxfp8_quantize(
+                inp["q_I"], self.qc, self.qs, per_token=True), w.B * w.HI * w.dI * 3),
+            ("indexer_scores_topk_mxfp8", lambda: csa.indexer_scores_topk_mxfp8(
+                self.qc, self.qs, inp["w"], self.kc, self.ks, w.m, w.k, q_pos=inp["q_pos"],
+                idx_out=self.idx, ws=ws_mx), w.B * w.n_csa * (w.dI + w.dI // 32)),
+        ] + self.stages[1:]
+
+        # the same step with the entry caches stored mixed (RoPE dims bf16,
+        # the rest MX-FP8: 592 instead of 1024 bytes an entry), written once
+        fm = csa.Fmt(c=w.c, rope_dims=w.r, rope_base=w.rope_base, flags=csa.CSA_F_MIXED)
+        self.rec = csa.csa_store_mixed(inp["entries"], fmt)
+        rb = self.rec.shape[-1]
+        self.mixed_stages = [self.stages[0], ("sparse_mqa_attn_mixed", lambda: csa.sparse_mqa_attn(
+            inp["q"], self.rec, self.idx, inp["win"], fm, w.n_win, sink=inp["sink"],
+            q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], out=self.out, ws=ws_a),
+            w.B * (min(w.k, w.n_csa) * rb + w.n_win * w.c * 2) + 2 * w.B * w.H * w.c * 2)]
+        if w.kind == "decode_pair":
+            self.rec_h = csa.csa_store_mixed(h["entries"], fmt)
+            self.mixed_stages.append(("dense_hca_attn_mixed", lambda: csa.dense_hca_attn(
+                h["q"], self.rec_h, w.m_prime, h["win"], fm, w.n_win, sink=h["sink"],
+                q_pos=h["q_pos"], win_pos0=h["win_pos0"], out=self.out_h, ws=ws_h),
+                w.B * (n_h * rb + w.n_win * w.c * 2) + 2 * w.B * w.H * w.c * 2))
+
+    def run_mixed(self):
+        for _, fn, _ in self.mixed_stages:
+            fn()
+
+    def run_mx(self):
+        for _, fn, _ in self.mx_stages:
+            fn()
+
     def rewind(self):
         """Puts every stream state back at token L - 1 (each append advances it)."""
         self.st_c[:, :8] = torch.tensor([self.w.T - 1] * self.w.B, dtype=torch.int64).view(
@@ -877,6 +917,11 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
     step_ms = allmax(graph_ms(d.run, steps, flush), ws_n)
     stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.stages}
     d.check()
+    mixed_ms = allmax(graph_ms(d.run_mixed, steps, flush), ws_n)
+    mixed_stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.mixed_stages[1:]}
+    mx_ms = allmax(graph_ms(d.run_mx, steps, flush), ws_n)
+    mx_stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.mx_stages[:2]}
+    d.check()
     append = {}
     for n, fn, nb in d.append:
         # a state rewind (outside the events) before every timed append, so
@@ -887,6 +932,9 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
     hbm, _, src = peaks()
     nb = decode_bytes(w)
     achieved = nb / (step_ms * 1e-3) / 1e9
+    # MX-FP8 indexer operands: 128 code bytes + 4 scale bytes per entry instead of 256
+    nb_mx = nb - w.B * w.n_csa * w.dI * 2 + w.B * w.n_csa * (w.dI + w.dI // 32)
+    mx_achieved = nb_mx / (mx_ms * 1e-3) / 1e9
     res = {
         "value": w.B * ws_n / (step_ms * 1e-3), "unit": "queries/s", "ms_per_step": step_ms,
         "config": {"workload": w.name, "batch": w.B, "context": w.T, "heads": w.H,
@@ -895,6 +943,19 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
                    "l2": "flushed before every replay (outside the events)",
                    "timing": "whole step captured once in a CUDA graph, replayed"},
         "stages_ms": stages,
+        "mixed_entries": {
+            "value": w.B * ws_n / (mixed_ms * 1e-3), "unit": "queries/s",
+            "ms_per_step": mixed_ms, "stages_ms": mixed_stages,
+            "stage_bytes": {n: nb_ for n, _, nb_ in d.mixed_stages[1:]},
+            "note": "the same step with the entry caches stored mixed (RoPE dims bf16, the rest "
+                    "MX-FP8 with a scale per 32 dims: 592 bytes an entry instead of 1024)"},
+        "mxfp8_indexer": {
+            "value": w.B * ws_n / (mx_ms * 1e-3), "unit": "queries/s", "ms_per_step": mx_ms,
+            "stages_ms": mx_stages,
+            "note": "the same step with q_I quantized each step and the indexer on MX-FP8 "
+                    "operands (K_I cached as E4M3 codes + UE8M0 scales per 32)",
+            "roofline": {"bound": "hbm", "achieved": mx_achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": mx_achieved / hbm, "algorithmic_bytes_per_step": nb_mx}},
         "stream_append": {**append, "note": "the step's new token appended to each sequence's "
                           "compression state (completing a block: entry pooled from the tail "
                           "buffer); latency-bound, timed beside the step"},

@@ -70,6 +70,8 @@ typedef int32_t csa_status;
 #define CSA_F_NO_NORM 1u   /* skip RMSNorm (test hook) */
 #define CSA_F_NO_ROPE 2u   /* skip RoPE and the output rotation (test hook) */
 #define CSA_F_PORTABLE 4u  /* attention: use the CUDA-core kernel even for bf16 (cross-checks) */
+#define CSA_F_MIXED 8u     /* attention: `entries` holds mixed BF16 / MX-FP8 records
+                              (csa_store_mixed) instead of dtype rows */
 
 /* Entry format shared by all calls.  c: entry / head dim (c/vec a power of two,
  * vec = 8 for bf16, 4 for f32); rope_dims: r, even, <= c, RoPE on dims
@@ -184,6 +186,27 @@ csa_status hca_compress_append(int32_t dtype, int64_t B, int32_t m_prime, const 
                                void* state, size_t state_stride, void* entries, int64_t n_cap,
                                void* win_out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- (1c) mixed BF16 / FP8 storage of compressed entries --------------- */
+
+/*
+ * Stores compressed entries in mixed precision [§3.3 of the summary page,
+ * last paragraph: the KV entries keep their RoPE dims in BF16 and store the
+ * rest in FP8].  Format taken (the page gives no block size or scale format):
+ * the c - r non-RoPE dims as MX-FP8 (E4M3 codes, one UE8M0 scale per 32 dims,
+ * 2^(floor(log2 amax) - 8), round to nearest even, saturate at 448), the r
+ * RoPE dims rounded to bf16.  One record of csa_mixed_record_bytes(c, r)
+ * bytes per entry (592 for c = 512, r = 64):
+ *   bytes [0, c-r): E4M3 codes; [c-r, c+r): bf16 RoPE dims;
+ *   [c+r, c+r+(c-r)/32): exponent + 127 per block; zeros to a multiple of 16.
+ *   entries: [B, N, c] (dtype); records (out): [B, N, record bytes].
+ * The attention calls read records in place of rows under CSA_F_MIXED.
+ * Errors: CSA_E_ARG (null or misaligned pointers, negative sizes),
+ * CSA_E_UNSUPPORTED ((c - r) not a multiple of 32, or c - r > 1024).
+ */
+size_t csa_mixed_record_bytes(int32_t c, int32_t rope_dims);
+csa_status csa_store_mixed(int32_t dtype, int64_t B, int64_t N, const csa_fmt* fmt,
+                           const void* entries, void* records, void* stream);
+
 /* ---- (2) lightning indexer + top-k ----------------------------------- */
 
 /*
@@ -255,7 +278,8 @@ csa_status indexer_scores_topk_noalloc(int32_t dtype, int64_t B, int64_t Tq, int
  * (0 for rows past the end).
  *   x: [B, rows, 128] (dtype CSA_BF16 or CSA_F32); codes (out): [B, rows,
  *   128] uint8; scales (out): [B, ceil(rows / 128), 512] uint8.
- * Used for the cached K_I (rows = N) and each step's q_I (rows = Tq H_I).
+ * Used for the cached K_I (B sequences of N rows) and each step's q_I
+ * (B Tq tokens of H_I = 64 rows: one tile per token).
  * Errors: CSA_E_ARG (null or misaligned pointers, negative sizes),
  * CSA_E_UNSUPPORTED (d != 128).
  */
@@ -267,7 +291,8 @@ csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_
  * them): I[t,s] = sum_h w[t,h] ReLU(sum_kb 2^(eq + ek) sum_{i in kb} cq_i ck_i)
  * with the E4M3 products and their sums in float32 on block-scaled tcgen05
  * MMAs; the causal top-k, tie rule, padding and outputs as indexer_scores_topk.
- *   q_codes: [B, Tq, 64, 128]; q_scales: [B, ceil(64 Tq / 128), 512];
+ *   q_codes: [B, Tq, 64, 128]; q_scales: [B, Tq, 512] (indexer_mxfp8_quantize
+ *   of q_I as B Tq batch elements of 64 rows);
  *   k_codes: [B, N, 128]; k_scales: [B, ceil(N / 128), 512]; the others as
  *   indexer_scores_topk.  H_I must be 64 and d_I 128 (else CSA_E_UNSUPPORTED).
  *   ws: >= csa_workspace_bytes(CSA_OP_INDEXER_MX, CSA_BF16, B, Tq, 0, 0, N, k, 0).
@@ -299,6 +324,10 @@ csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t
  * scale*|q^|*sqrt(c) in place of a running maximum and flags CSA_DEV_RANGE
  * when a logit goes more than 60 (natural log) beyond it (the output is then
  * invalid).  An index outside [-1, N) is skipped and flagged CSA_DEV_BAD_INDEX.
+ * With CSA_F_MIXED in fmt->flags, `entries` holds csa_store_mixed records
+ * ([B, N, csa_mixed_record_bytes(c, r)] bytes; window rows stay dtype) and
+ * the keys are the records' exact values (E4M3 x 2^e and bf16 both widen
+ * exactly); the tensor cores then need rope_dims = 64.
  * Kernels: bf16 runs on the tensor cores, which need c = 512, H a multiple of
  * 64, rope_dims <= 64 and (sparse) k <= 1024; other bf16 shapes return
  * CSA_E_UNSUPPORTED unless fmt->flags has CSA_F_PORTABLE, which selects the

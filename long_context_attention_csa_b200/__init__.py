@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libcsa.so")
 
 CSA_OK, CSA_E_ARG, CSA_E_UNSUPPORTED, CSA_E_CUDA, CSA_E_DEVICE, CSA_E_WORKSPACE = range(6)
 CSA_F32, CSA_BF16 = 0, 1
-CSA_F_NO_NORM, CSA_F_NO_ROPE, CSA_F_PORTABLE = 1, 2, 4
+CSA_F_NO_NORM, CSA_F_NO_ROPE, CSA_F_PORTABLE, CSA_F_MIXED = 1, 2, 4, 8
 (CSA_OP_INDEXER, CSA_OP_SPARSE_ATTN, CSA_OP_DENSE_ATTN, CSA_OP_COMPRESS, CSA_OP_OUT_PROJ,
  CSA_OP_INDEXER_MX) = 1, 2, 3, 4, 5, 6
 CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX, CSA_DEV_STREAM = 1, 2, 3, 4
@@ -32,7 +32,8 @@ CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX, CSA_DEV_STREAM = 1, 2, 3, 4
 EXPORTED = (
     "csa_compress", "hca_compress", "csa_stream_state_bytes", "csa_compress_append",
     "hca_compress_append", "indexer_scores_topk", "indexer_scores_topk_noalloc",
-    "indexer_mxfp8_quantize", "indexer_scores_topk_mxfp8", "sparse_mqa_attn", "dense_hca_attn",
+    "indexer_mxfp8_quantize", "indexer_scores_topk_mxfp8", "csa_mixed_record_bytes",
+    "csa_store_mixed", "sparse_mqa_attn", "dense_hca_attn",
     "grouped_output_projection", "csa_workspace_bytes",
     "csa_check_status",
     "csa_status_string", "csa_launch_count", "csa_selftest_wait",
@@ -105,6 +106,9 @@ def lib():
     L.hca_compress_append.argtypes = [i32, i64, i32, FP, P, P, i32, i64, P, sz, P, i64, P, P, sz,
                                       P]
     L.indexer_mxfp8_quantize.argtypes = [i32, i64, i64, i32, P, P, P, P]
+    L.csa_mixed_record_bytes.argtypes = [i32, i32]
+    L.csa_mixed_record_bytes.restype = sz
+    L.csa_store_mixed.argtypes = [i32, i64, i64, FP, P, P, P]
     L.indexer_scores_topk_mxfp8.argtypes = [i64, i64, i32, i32, P, P, P, P, P, i64, P, i32, i32,
                                             P, P, P, sz, P]
     L.grouped_output_projection.argtypes = [i32, i64, i32, i32, i32, i32, i32, P, P, P, P, P, sz,
@@ -120,7 +124,7 @@ def lib():
     for fn in ("csa_compress", "hca_compress", "csa_compress_append", "hca_compress_append",
                "indexer_scores_topk",
                "indexer_scores_topk_noalloc", "sparse_mqa_attn", "dense_hca_attn",
-               "grouped_output_projection", "indexer_mxfp8_quantize",
+               "grouped_output_projection", "indexer_mxfp8_quantize", "csa_store_mixed",
                "indexer_scores_topk_mxfp8", "csa_check_status", "csa_selftest_wait"):
         getattr(L, fn).restype = i32
     _lib = L
@@ -292,15 +296,37 @@ def indexer_scores_topk(q_I, w, k_I, m: int, k: int, q_pos=None, idx_out=None, s
     return (idx_out, score_out) if score_out is not None else idx_out
 
 
-def indexer_mxfp8_quantize(x, codes=None, scales=None, stream=None):
-    """MX-FP8 codes and scale tiles of x [B, ..., 128] (rows = the middle dims
-    flattened): codes uint8 with x's shape, scales [B, ceil(rows/128), 512]."""
-    B, d = x.shape[0], x.shape[-1]
-    rows = x[0].numel() // d if B else 0
+def csa_mixed_record_bytes(c: int, rope_dims: int) -> int:
+    return int(lib().csa_mixed_record_bytes(c, rope_dims))
+
+
+def csa_store_mixed(entries, fmt: Fmt, records=None, stream=None):
+    """Mixed BF16 / MX-FP8 records [B, N, record bytes] uint8 of entries
+    [B, N, c]; the attention calls read them under CSA_F_MIXED."""
+    B, N, c = entries.shape
+    rb = csa_mixed_record_bytes(c, fmt.rope_dims)
+    if records is None:
+        records = torch.empty((B, N, rb), dtype=torch.uint8, device=entries.device)
+    f = fmt._c()
+    st = lib().csa_store_mixed(_dt(entries), B, N, ctypes.byref(f), _p(entries), _p(records),
+                               _s(stream))
+    _check(st, "csa_store_mixed")
+    return records
+
+
+def indexer_mxfp8_quantize(x, codes=None, scales=None, per_token=False, stream=None):
+    """MX-FP8 codes and scale tiles of x [B, ..., 128]: codes uint8 with x's
+    shape; scales [B, ceil(rows/128), 512] with rows = the middle dims
+    flattened, or, with ``per_token`` (q_I [B, Tq, 64, 128]), one tile per
+    token: [B, Tq, 512]."""
+    d = x.shape[-1]
+    B = x.shape[0] * x.shape[1] if per_token else x.shape[0]
+    rows = x.numel() // d // B if B else 0
     if codes is None:
         codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty((B, (rows + 127) // 128, 512), dtype=torch.uint8, device=x.device)
+        shape = (x.shape[0], x.shape[1], 512) if per_token else (B, (rows + 127) // 128, 512)
+        scales = torch.empty(shape, dtype=torch.uint8, device=x.device)
     st = lib().indexer_mxfp8_quantize(_dt(x), B, rows, d, _p(x), _p(codes), _p(scales), _s(stream))
     _check(st, "indexer_mxfp8_quantize")
     return codes, scales

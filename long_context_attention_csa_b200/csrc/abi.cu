@@ -29,7 +29,8 @@ csa_status check_fmt(int32_t dtype, const csa_fmt* fmt, Fmt* out) {
   if (fmt->c <= 0 || fmt->rope_dims < 0 || fmt->rope_dims > fmt->c || (fmt->rope_dims & 1))
     return CSA_E_ARG;
   if (!(fmt->norm_eps >= 0.f) || !(fmt->rope_base > 0.f)) return CSA_E_ARG;
-  if (fmt->flags & ~(CSA_F_NO_NORM | CSA_F_NO_ROPE | CSA_F_PORTABLE)) return CSA_E_ARG;
+  if (fmt->flags & ~(CSA_F_NO_NORM | CSA_F_NO_ROPE | CSA_F_PORTABLE | CSA_F_MIXED))
+    return CSA_E_ARG;
   const int vec = dtype == CSA_BF16 ? 8 : 4;
   if (fmt->c % vec != 0 || !pow2(fmt->c / vec) || fmt->c / vec > 256) return CSA_E_UNSUPPORTED;
   out->c = fmt->c;
@@ -224,6 +225,24 @@ csa_status hca_compress_append(int32_t dtype, int64_t B, int32_t m_prime, const 
                        state, state_stride, entries, n_cap, win_out, ws, ws_bytes, stream);
 }
 
+size_t csa_mixed_record_bytes(int32_t c, int32_t rope_dims) {
+  if (c <= 0 || rope_dims < 0 || rope_dims > c || (c - rope_dims) % 32 != 0) return 0;
+  return mixed_record_bytes(c, rope_dims);
+}
+
+csa_status csa_store_mixed(int32_t dtype, int64_t B, int64_t N, const csa_fmt* fmt,
+                           const void* entries, void* records, void* stream) {
+  Fmt f;
+  csa_status st = check_fmt(dtype, fmt, &f);
+  if (st != CSA_OK) return st;
+  if (B < 0 || N < 0) return CSA_E_ARG;
+  if ((f.c - f.r) % 32 != 0 || f.c - f.r > 1024) return CSA_E_UNSUPPORTED;
+  if (B == 0 || N == 0) return CSA_OK;
+  if (!entries || !records || !aligned16(entries) || !aligned16(records)) return CSA_E_ARG;
+  g_launches.fetch_add(1);
+  return cuda_status(launch_mixed_store(dtype, entries, records, B * N, f.c, f.r, S(stream)));
+}
+
 csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
                                   const void* x, void* codes, void* scales, void* stream) {
   if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
@@ -369,6 +388,11 @@ static csa_status attn_common(int32_t dtype, int64_t B, int64_t Tq, int32_t H, c
       (win && !aligned16(win)))
     return CSA_E_ARG;
   AttnParams p{};
+  if (f.flags & CSA_F_MIXED) {
+    if ((f.c - f.r) % 32 != 0 || f.c - f.r > 1024) return CSA_E_UNSUPPORTED;
+    p.mixed = 1;
+    p.rec_bytes = (int)mixed_record_bytes(f.c, f.r);
+  }
   p.B = B;
   p.Tq = Tq;
   p.H = H;

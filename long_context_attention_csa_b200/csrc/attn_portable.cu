@@ -17,12 +17,23 @@
 // memory (rows padded to c+1 floats so that lane j reading key j is
 // conflict-free); lane j scores key j, the warp runs the online softmax, then
 // lane l accumulates output dims l, l+32, ... .
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace csa {
 
 namespace {
+
+// Element e of a mixed entry record (dims [0, c-r) as E4M3 codes with a
+// UE8M0 exponent per 32 dims, dims [c-r, c) as bf16): exact in float.
+__device__ __forceinline__ float mixed_elem(const uint8_t* rec, int e, int c, int r) {
+  const int cq = c - r;
+  if (e >= cq) return __bfloat162float(reinterpret_cast<const bf16*>(rec + cq)[e - cq]);
+  const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)rec[e], __NV_E4M3);
+  return ldexpf(__half2float(__half(h)), (int)rec[cq + 2 * r + e / 32] - 127);
+}
 
 constexpr int kHG = 8;     // heads per CTA (one warp each)
 constexpr int kKT = 32;    // keys per tile (one per lane)
@@ -63,6 +74,8 @@ __global__ void __launch_bounds__(256) attn_portable_kernel(AttnParams p) {
   const int64_t n_keys = n_ent + n_win;
 
   const T* ent = static_cast<const T*>(p.entries) + b * p.N * c;
+  // mixed records: the batch offset is added per access (records are not c wide)
+  const uint8_t* entm = p.mixed ? static_cast<const uint8_t*>(p.entries) : nullptr;
   const T* win = static_cast<const T*>(p.win) + b * p.Tw * c;
   const float scale = p.scale > 0.f ? p.scale : rsqrtf((float)c);
 
@@ -121,8 +134,13 @@ __global__ void __launch_bounds__(256) attn_portable_kernel(AttnParams p) {
       int j = idx / c, e = idx - j * c;
       int64_t off = koff[j];
       float v = 0.f;
-      if (off >= 0) v = to_float(ent[off + e]);
-      else if (off <= -2) v = to_float(win[(-2 - off) + e]);
+      if (off >= 0) {
+        v = entm ? mixed_elem(entm + (off / c) * p.rec_bytes + (int64_t)b * p.N * p.rec_bytes, e,
+                              c, p.f.r)
+                 : to_float(ent[off + e]);
+      } else if (off <= -2) {
+        v = to_float(win[(-2 - off) + e]);
+      }
       K[j * cs + e] = v;
     }
     __syncthreads();

@@ -57,6 +57,8 @@
 // size fixed by the row's own key count (at least 320 keys, at most 16
 // pieces) whose fp32 partials a combine kernel adds in a fixed order, so a
 // row's result does not depend on the batch it runs in.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc.h"
@@ -137,6 +139,8 @@ struct TcAttnArgs {
   bf16* out;
   int split, n_splits, n_hg;
   int64_t n_rows, n_items;
+  const uint8_t* ent_mixed;   // mixed BF16 / MX-FP8 entry records (mixed != 0)
+  int mixed, rec_bytes;
   float* o_part;    // [rows][n_hg][n_splits][64][512]
   float* d_part;    // [rows][n_hg][n_splits][64]
   float* mb_part;   // [rows][n_hg][64]
@@ -179,6 +183,78 @@ __device__ __forceinline__ Item decode_item(const TcAttnArgs& a, int64_t it) {
   x.jlo = jlo;
   x.n_w = jhi >= jlo ? jhi - jlo + 1 : 0;
   return x;
+}
+
+// Mixed BF16 / MX-FP8 entries: region pair h (dims 128 h .. 128 h + 127) of
+// this thread's rows of the key tile, from the entry records (E4M3 codes times
+// 2^(scale - 127) for dims below 448, bf16 for the 64 RoPE dims) or from the
+// bf16 window rows, widened exactly to bf16 and stored at the same swizzled
+// places the cp.async gather fills.  Every load of the pair is issued before
+// the first conversion; then the stores are fenced for the tensor core's
+// async-proxy reads and the thread arrives on the region pair's barrier.
+__device__ __forceinline__ void gather_mixed(const TcAttnArgs& a, uint32_t tile, int h, int pw,
+                                             int quad, int g8, int64_t key0, int64_t k_hi,
+                                             int64_t n_ent, const int32_t* list, const Item& x,
+                                             uint64_t* bar) {
+  constexpr int kCq = kC - 64;               // FP8 dims of a record
+  constexpr int kScaleOff = kCq + 2 * 64;    // scale bytes after the bf16 RoPE dims
+  uint4 raw[kGatherIters][2];
+  uint32_t sc[kGatherIters][2];              // scale byte, or 0xffffffff for a bf16 piece
+#pragma unroll
+  for (int u = 0; u < kGatherIters; ++u) {
+    const int r = 4 * (pw + kProdWarps * u) + quad;
+    const int64_t key = key0 + r;
+    const bool ok = pw + kProdWarps * u < kBK / 4 && key < k_hi;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int reg = 2 * h + rr;
+      raw[u][rr] = make_uint4(0u, 0u, 0u, 0u);
+      sc[u][rr] = 0xffffffffu;
+      if (!ok) continue;
+      if (key < n_ent) {
+        const int64_t s = a.sparse ? list[key] : key;
+        const uint8_t* rec = a.ent_mixed + (x.bidx * a.N + s) * (int64_t)a.rec_bytes;
+        if (reg < kRegions - 1) {
+          const uint2 c8 = __ldg(reinterpret_cast<const uint2*>(rec + reg * 64 + g8 * 8));
+          raw[u][rr] = make_uint4(c8.x, c8.y, 0u, 0u);
+          sc[u][rr] = rec[kScaleOff + reg * 2 + (g8 >> 2)];
+        } else {
+          raw[u][rr] = __ldg(reinterpret_cast<const uint4*>(rec + kCq + g8 * 16));
+        }
+      } else {
+        const bf16* wr = a.win + (x.bidx * a.Tw + (x.jlo - x.wp0) + (key - n_ent)) * kC;
+        raw[u][rr] = __ldg(reinterpret_cast<const uint4*>(wr + reg * 64 + g8 * 8));
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kGatherIters; ++u) {
+    if (pw + kProdWarps * u >= kBK / 4) continue;
+    const int r = 4 * (pw + kProdWarps * u) + quad;
+    const uint32_t dst = tile + (uint32_t)r * 128u + (((uint32_t)g8 ^ (uint32_t)(r & 7)) << 4);
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      uint4 v = raw[u][rr];
+      if (sc[u][rr] != 0xffffffffu) {
+        const int e = (int)sc[u][rr] - 127;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t word = q < 2 ? v.x : v.y;
+          const __nv_fp8x2_storage_t two = (__nv_fp8x2_storage_t)(word >> (16 * (q & 1)));
+          const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3)));
+          w[q] = pack_bf16x2(ldexpf(f.x, e), ldexpf(f.y, e));
+        }
+        v = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const uint32_t d = dst + (uint32_t)((2 * h + rr) * kKRegion);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d), "r"(v.x), "r"(v.y),
+                   "r"(v.z), "r"(v.w)
+                   : "memory");
+    }
+  }
+  fence_proxy_async_smem();
+  mbar_arrive(bar);
 }
 
 // Decode split size of a row with n_keys keys: at least kSplitKeys, and large
@@ -433,7 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int h = 0; h < 4; ++h) {
             wait_or_die(&bfree[4 * s + h], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
-            if (!dead) {
+            if (!dead && a.mixed) {
+              gather_mixed(a, tile, h, pw, quad, g8, k_lo + (int64_t)b * kBK, k_hi, n_ent, list,
+                           x, &kfull[4 * s + h]);
+            } else if (!dead) {
 #pragma unroll
               for (int u = 0; u < kGatherIters; ++u) {
                 if (pw + kProdWarps * u >= kBK / 4) continue;
@@ -977,6 +1056,7 @@ inline int n_splits_for(int64_t max_keys) {
 bool attn_tc_supported(const AttnParams& p) {
   auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   if (p.f.c != kC || p.H % kHG != 0 || p.f.r > 64 || (p.f.r & 1)) return false;
+  if (p.mixed && p.f.r != 64) return false;   // the bf16 part is exactly the last region
   if (p.sparse && p.k > kMaxK) return false;   // the per-item index list holds kMaxK
   if (p.B * p.Tq >= (1LL << 31)) return false;
   if (p.Tq == 1 && p.B > 65535) return false;
@@ -1006,6 +1086,9 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
   a.eps = p.f.eps;
   a.scale = p.scale;
   a.flags = p.f.flags;
+  a.mixed = p.mixed;
+  a.rec_bytes = p.rec_bytes;
+  a.ent_mixed = static_cast<const uint8_t*>(p.entries);
   a.q = static_cast<const bf16*>(p.q);
   a.q_pos = p.q_pos;
   a.entries = static_cast<const bf16*>(p.entries);

@@ -102,10 +102,11 @@ struct TcIdxArgs {
   float* cand_score;   // [B*Tq][n_chunks][k] when n_chunks > 1
   int32_t* cand_idx;
   unsigned* status;
-  // MX-FP8 operands: scale-factor tiles [B][tiles][512] of q_I and K_I
+  // MX-FP8 operands: scale-factor tiles of q_I ([B][Tq][512], one per token)
+  // and K_I ([B][ceil(N / 128)][512])
   const uint8_t* q_sf;
   const uint8_t* k_sf;
-  int64_t q_sf_tiles, k_sf_tiles;
+  int64_t k_sf_tiles;
 };
 
 __device__ __forceinline__ int64_t vis_count(int64_t pos, int m, int64_t N) {
@@ -923,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
         mbar_arrive_expect_tx(bfull, L::kB + 512);
         tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
         bulk_load(smem_u32(sm + L::off_sf + kStages * 512),
-                  a.q_sf + ((int64_t)b * a.q_sf_tiles + (t0 * kHI) / kBM) * 512, 512, bfull);
+                  a.q_sf + ((int64_t)b * a.Tq + t0) * 512, 512, bfull);
       } else {
         mbar_arrive_expect_tx(bfull, L::kB);
         tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
@@ -1006,8 +1007,7 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
             // before, the MMAs below that read them)
             const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)buf;
             tmem_cp_32x128b_x4(sfa, smem_desc(smem_u32(sm + L::off_sf + s * 512), 16, 128, 0));
-            // a 128-row scale tile holds two tokens' 64 heads: this token's half
-            const uint32_t sfb = tmem + kSfb + 2u * (uint32_t)(t0 & 1);
+            const uint32_t sfb = tmem + kSfb;   // the token's own tile: heads on rows 0..63
 #pragma unroll
             for (int kk = 0; kk < kDI / 32; ++kk) {   // K = 32 per MMA, one scale each
               const uint64_t ad = smem_desc(a_base + s * kTile + kk * 32, 16, 1024, 2);
@@ -1849,7 +1849,6 @@ cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const vo
   a.status = p.status;
   a.q_sf = static_cast<const uint8_t*>(q_sf);
   a.k_sf = static_cast<const uint8_t*>(k_sf);
-  a.q_sf_tiles = (p.Tq * kHI + kBM - 1) / kBM;
   a.k_sf_tiles = (p.N + kBM - 1) / kBM;
   if (a.n_chunks > 1) {
     const size_t n = (size_t)p.B * p.Tq * a.n_chunks * p.k;

@@ -67,6 +67,8 @@ struct AttnParams {
   int n_win;
   const float* sink;      // [H] or null
   float scale;
+  int mixed;              // entries are mixed BF16 / MX-FP8 records of rec_bytes
+  int rec_bytes;
   void* out;              // [B, Tq, H, c]
   unsigned* status;
   void* scratch;

@@ -72,7 +72,71 @@ __global__ void __launch_bounds__(256) mxfp8_quantize_kernel(const T* x, uint8_t
   if ((lane & 7) == 0) sf[sfpos] = (uint8_t)(e + 127);
 }
 
+// Mixed storage of compressed entries: one warp per entry; lane l < (c-r)/32
+// quantizes 32-element block l of the non-RoPE dims to MX-FP8 (the same rule
+// as above), every lane rounds a share of the r RoPE dims to bf16.
+template <typename T>
+__global__ void __launch_bounds__(256) mixed_store_kernel(const T* x, uint8_t* rec, int64_t n,
+                                                          int c, int r, int rec_bytes) {
+  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (e >= n) return;   // warp-uniform
+  const int cq = c - r, nblk = cq / 32;
+  const T* xe = x + e * c;
+  uint8_t* re = rec + e * rec_bytes;
+  if (lane < nblk) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = to_float(xe[32 * lane + i]);
+    float am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+    int ex = -127;
+    if (am > 0.f) {
+      ex = ilogbf(am) - 8;
+      ex = ex < -127 ? -127 : (ex > 127 ? 127 : ex);
+    }
+    uint32_t w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+          make_float2(ldexpf(v[4 * q], -ex), ldexpf(v[4 * q + 1], -ex)), __NV_SATFINITE,
+          __NV_E4M3);
+      const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(ldexpf(v[4 * q + 2], -ex), ldexpf(v[4 * q + 3], -ex)), __NV_SATFINITE,
+          __NV_E4M3);
+      w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(re + 32 * lane);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    re[cq + 2 * r + lane] = (uint8_t)(ex + 127);
+  }
+  bf16* rope = reinterpret_cast<bf16*>(re + cq);
+  for (int d = lane; d < r; d += 32) rope[d] = __float2bfloat16_rn(to_float(xe[cq + d]));
+  for (int pb = cq + 2 * r + nblk + lane; pb < rec_bytes; pb += 32) re[pb] = 0;
+}
+
 }  // namespace
+
+size_t mixed_record_bytes(int c, int r) {
+  const size_t raw = (size_t)(c - r) + 2 * (size_t)r + (size_t)(c - r) / 32;
+  return (raw + 15) & ~(size_t)15;
+}
+
+cudaError_t launch_mixed_store(int dtype, const void* x, void* rec, int64_t n, int c, int r,
+                               cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int rb = (int)mixed_record_bytes(c, r);
+  const int64_t blocks = (n * 32 + 255) / 256;
+  if (dtype == CSA_BF16)
+    mixed_store_kernel<bf16><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const bf16*>(x), static_cast<uint8_t*>(rec), n, c, r, rb);
+  else
+    mixed_store_kernel<float><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const float*>(x), static_cast<uint8_t*>(rec), n, c, r, rb);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mxfp8_quantize(int dtype, const void* x, void* codes, void* scales, int64_t B,
                                   int64_t rows, cudaStream_t stream) {

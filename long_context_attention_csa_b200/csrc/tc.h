@@ -20,6 +20,11 @@ cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const vo
 cudaError_t launch_mxfp8_quantize(int dtype, const void* x, void* codes, void* scales, int64_t B,
                                   int64_t rows, cudaStream_t stream);
 
+// Mixed BF16 / MX-FP8 entry records.
+size_t mixed_record_bytes(int c, int r);
+cudaError_t launch_mixed_store(int dtype, const void* x, void* rec, int64_t n, int c, int r,
+                               cudaStream_t stream);
+
 // Shared-KV MQA (sparse and dense) on tcgen05.
 bool attn_tc_supported(const AttnParams& p);
 size_t attn_tc_scratch(int64_t B, int64_t Tq, int H, int c, int64_t max_keys);

@@ -239,3 +239,36 @@ def test_projection_rejects_bad_arguments(L):
                                        None) == 5
     assert L.grouped_output_projection(1, 0, 16, 512, 4, 256, 512, None, None, None, None, None,
                                        0, None) == 0
+
+
+def test_mxfp8_calls_reject_bad_arguments(L):
+    d = ctypes.c_void_p(4096)
+    mis = ctypes.c_void_p(4100)
+    # quantize: rows of 64 are not the format, misaligned output, empty is a no-op
+    assert L.indexer_mxfp8_quantize(1, 1, 8, 64, d, d, d, None) == 2
+    assert L.indexer_mxfp8_quantize(1, 1, 8, 128, d, mis, d, None) == 1
+    assert L.indexer_mxfp8_quantize(1, 0, 8, 128, None, None, None, None) == 0
+    # scores: the tensor-core shape only, workspace required
+    assert L.indexer_scores_topk_mxfp8(1, 1, 32, 128, d, d, d, d, d, 64, None, 4, 8, d, None, d,
+                                       1 << 20, None) == 2
+    assert L.indexer_scores_topk_mxfp8(1, 1, 64, 128, d, d, d, d, d, 64, None, 4, 8, d, None,
+                                       None, 0, None) == 5
+    assert L.indexer_scores_topk_mxfp8(1, 1, 64, 128, d, None, d, d, d, 64, None, 4, 8, d, None,
+                                       d, 1 << 20, None) == 1
+    assert L.csa_workspace_bytes(6, 1, 32, 1, 0, 0, 32768, 1024, 0) == 256 + 32 * 8 * 1024 * 8
+
+
+def test_mixed_storage_rejects_bad_arguments(L):
+    d = ctypes.c_void_p(4096)
+    assert L.csa_mixed_record_bytes(512, 64) == 592
+    assert L.csa_mixed_record_bytes(64, 32) == 112
+    assert L.csa_mixed_record_bytes(512, 60) == 0
+    f = _fmt()
+    bad = _fmt(r=60)
+    assert L.csa_store_mixed(1, 1, 8, ctypes.byref(bad), d, d, None) == 2
+    assert L.csa_store_mixed(1, 1, 8, ctypes.byref(f), None, d, None) == 1
+    assert L.csa_store_mixed(1, 0, 8, ctypes.byref(f), None, None, None) == 0
+    # attention under CSA_F_MIXED: (c - r) must be a multiple of 32
+    fm = _fmt(r=60, flags=8)
+    assert L.dense_hca_attn(1, 1, 4, 64, ctypes.byref(fm), d, None, d, 16, 4, d, 8, None, 8,
+                            None, 0.0, d, None, 0, None) == 2

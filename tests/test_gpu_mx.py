@@ -57,7 +57,7 @@ def test_mxfp8_quantize_matches_the_oracle(dtype):
 
 
 def _quantized(q_I, k_I):
-    qc, qs = csa.indexer_mxfp8_quantize(q_I)
+    qc, qs = csa.indexer_mxfp8_quantize(q_I, per_token=True)
     kc, ks = csa.indexer_mxfp8_quantize(k_I)
     return qc, qs, kc, ks
 
