@@ -972,11 +972,15 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
 
 
 def run_only_decode(args):
-    """The decode step of --decode-workload, each stage replayed alone from a
-    CUDA graph, with its bandwidth over the bytes it must read."""
+    """The decode step of --decode-workload (--decode-batch rows, default the
+    workload's), each stage replayed alone from a CUDA graph, with its
+    bandwidth over the bytes it must read; also the MX-FP8 indexer, the
+    mixed-entry attention and the streaming compression stages."""
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = wl.WORKLOADS[args.decode_workload]
+    if args.decode_batch:
+        w = wl.scaled(w, B=args.decode_batch)
     d = DecodeStep(w, dev)
     for _ in range(args.warmup):
         d.run()
@@ -984,8 +988,11 @@ def run_only_decode(args):
     d.check()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     res = {}
-    for name, fn, nbytes in d.stages:
+    for name, fn, nbytes in d.stages + d.mx_stages[:2] + d.mixed_stages[1:]:
         ms = graph_ms(fn, args.steps, flush)
+        res[name] = {"ms": ms, "bytes": nbytes, "GBps": nbytes / ms / 1e6}
+    for name, fn, nbytes in d.append:
+        ms = graph_ms(fn, args.steps, flush, before=d.rewind)
         res[name] = {"ms": ms, "bytes": nbytes, "GBps": nbytes / ms / 1e6}
     step = graph_ms(d.run, args.steps, flush)
     d.check()
@@ -1059,6 +1066,8 @@ def main():
     ap.add_argument("--seq-len", type=int, default=0, help="tokens for --only (default 8192)")
     ap.add_argument("--decode-workload", default="csa_decode_b32_128k",
                     choices=["csa_decode_b32_128k", "decode_pair_b4_1m"], help="for --only decode")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="for --only decode: rows of the workload (a smaller case for profiles)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)

@@ -185,21 +185,21 @@ __device__ __forceinline__ Item decode_item(const TcAttnArgs& a, int64_t it) {
   return x;
 }
 
-// Mixed BF16 / MX-FP8 entries: region pair h (dims 128 h .. 128 h + 127) of
-// this thread's rows of the key tile, from the entry records (E4M3 codes times
-// 2^(scale - 127) for dims below 448, bf16 for the 64 RoPE dims) or from the
-// bf16 window rows, widened exactly to bf16 and stored at the same swizzled
-// places the cp.async gather fills.  Every load of the pair is issued before
-// the first conversion; then the stores are fenced for the tensor core's
-// async-proxy reads and the thread arrives on the region pair's barrier.
-__device__ __forceinline__ void gather_mixed(const TcAttnArgs& a, uint32_t tile, int h, int pw,
-                                             int quad, int g8, int64_t key0, int64_t k_hi,
-                                             int64_t n_ent, const int32_t* list, const Item& x,
-                                             uint64_t* bar) {
+// Mixed BF16 / MX-FP8 entries.  One 16-byte piece of a key-tile row: eight
+// E4M3 codes (x, y) with their block's scale byte (z), or eight bf16 values
+// (the RoPE dims of a record, or a window row).
+struct MixedPiece {
+  uint4 v;
+};
+
+// Loads region pair h (dims 128 h .. 128 h + 127) of this thread's rows of the
+// key tile from the entry records or the bf16 window rows.
+__device__ __forceinline__ void mixed_load(const TcAttnArgs& a, int h, int pw, int quad, int g8,
+                                           int64_t key0, int64_t k_hi, int64_t n_ent,
+                                           const int32_t* list, const Item& x,
+                                           MixedPiece (&pc)[kGatherIters][2]) {
   constexpr int kCq = kC - 64;               // FP8 dims of a record
   constexpr int kScaleOff = kCq + 2 * 64;    // scale bytes after the bf16 RoPE dims
-  uint4 raw[kGatherIters][2];
-  uint32_t sc[kGatherIters][2];              // scale byte, or 0xffffffff for a bf16 piece
 #pragma unroll
   for (int u = 0; u < kGatherIters; ++u) {
     const int r = 4 * (pw + kProdWarps * u) + quad;
@@ -208,42 +208,57 @@ __device__ __forceinline__ void gather_mixed(const TcAttnArgs& a, uint32_t tile,
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int reg = 2 * h + rr;
-      raw[u][rr] = make_uint4(0u, 0u, 0u, 0u);
-      sc[u][rr] = 0xffffffffu;
+      pc[u][rr].v = make_uint4(0u, 0u, 0u, 0u);
       if (!ok) continue;
       if (key < n_ent) {
-        const int64_t s = a.sparse ? list[key] : key;
-        const uint8_t* rec = a.ent_mixed + (x.bidx * a.N + s) * (int64_t)a.rec_bytes;
+        const int64_t e = a.sparse ? list[key] : key;
+        const uint8_t* rec = a.ent_mixed + (x.bidx * a.N + e) * (int64_t)a.rec_bytes;
         if (reg < kRegions - 1) {
           const uint2 c8 = __ldg(reinterpret_cast<const uint2*>(rec + reg * 64 + g8 * 8));
-          raw[u][rr] = make_uint4(c8.x, c8.y, 0u, 0u);
-          sc[u][rr] = rec[kScaleOff + reg * 2 + (g8 >> 2)];
+          pc[u][rr].v = make_uint4(c8.x, c8.y, (uint32_t)rec[kScaleOff + reg * 2 + (g8 >> 2)], 0u);
         } else {
-          raw[u][rr] = __ldg(reinterpret_cast<const uint4*>(rec + kCq + g8 * 16));
+          pc[u][rr].v = __ldg(reinterpret_cast<const uint4*>(rec + kCq + g8 * 16));
         }
       } else {
         const bf16* wr = a.win + (x.bidx * a.Tw + (x.jlo - x.wp0) + (key - n_ent)) * kC;
-        raw[u][rr] = __ldg(reinterpret_cast<const uint4*>(wr + reg * 64 + g8 * 8));
+        pc[u][rr].v = __ldg(reinterpret_cast<const uint4*>(wr + reg * 64 + g8 * 8));
       }
     }
   }
+}
+
+// Widens region pair h's pieces exactly to bf16 (E4M3 x 2^(scale - 127)),
+// stores them at the swizzled places the cp.async gather fills, fences them
+// for the tensor core's async-proxy reads and arrives on the pair's barrier.
+// A piece is FP8 when its row is an entry and its region is one of the first
+// seven; window rows and region 7 are bf16 as loaded; rows past the key list
+// are zeros.
+__device__ __forceinline__ void mixed_store(uint32_t tile, int h, int pw, int quad, int g8,
+                                            int64_t key0, int64_t k_hi, int64_t n_ent,
+                                            const MixedPiece (&pc)[kGatherIters][2],
+                                            uint64_t* bar) {
 #pragma unroll
   for (int u = 0; u < kGatherIters; ++u) {
     if (pw + kProdWarps * u >= kBK / 4) continue;
     const int r = 4 * (pw + kProdWarps * u) + quad;
+    const int64_t key = key0 + r;
     const uint32_t dst = tile + (uint32_t)r * 128u + (((uint32_t)g8 ^ (uint32_t)(r & 7)) << 4);
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      uint4 v = raw[u][rr];
-      if (sc[u][rr] != 0xffffffffu) {
-        const int e = (int)sc[u][rr] - 127;
+      uint4 v = pc[u][rr].v;
+      if (key >= k_hi) {
+        v = make_uint4(0u, 0u, 0u, 0u);
+      } else if (key < n_ent && 2 * h + rr < kRegions - 1) {
+        // 2^(byte - 127) as a float: the byte is the exponent field (byte 0 is
+        // the subnormal 2^-127); E4M3 x 2^k is exact in float and in bf16
+        const float sc = __uint_as_float(v.z ? (v.z << 23) : 0x00400000u);
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t word = q < 2 ? v.x : v.y;
           const __nv_fp8x2_storage_t two = (__nv_fp8x2_storage_t)(word >> (16 * (q & 1)));
           const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3)));
-          w[q] = pack_bf16x2(ldexpf(f.x, e), ldexpf(f.y, e));
+          w[q] = pack_bf16x2(f.x * sc, f.y * sc);
         }
         v = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -282,6 +297,9 @@ __device__ __forceinline__ int item_blocks(const TcAttnArgs& a, const Item& x, i
   return h > l ? (int)((h - l + kBK - 1) / kBK) : 0;
 }
 
+// MIXED: the entries are mixed BF16 / MX-FP8 records (a separate instantiation,
+// so the bf16 gather compiles exactly as without it).
+template <bool MIXED>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, TcAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -504,15 +522,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               src[u] = key < n_ent ? ent + (int64_t)(a.sparse ? list[key] : key) * kC
                                    : win + ((x.jlo - x.wp0) + (key - n_ent)) * kC;
           }
+          if constexpr (MIXED) {
+            // region pair h + 1's record loads are in flight while pair h is
+            // widened and stored (two register sets, the pair loop unrolled)
+            MixedPiece ra[kGatherIters][2], rb[kGatherIters][2];
+            const int64_t key0 = k_lo + (int64_t)b * kBK;
+            if (!dead) mixed_load(a, 0, pw, quad, g8, key0, k_hi, n_ent, list, x, ra);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              MixedPiece (&cur)[kGatherIters][2] = (h & 1) ? rb : ra;
+              MixedPiece (&nxt)[kGatherIters][2] = (h & 1) ? ra : rb;
+              if (!dead && h < 3)
+                mixed_load(a, h + 1, pw, quad, g8, key0, k_hi, n_ent, list, x, nxt);
+              wait_or_die(&bfree[4 * s + h], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
+              if (!dead)
+                mixed_store(tile, h, pw, quad, g8, key0, k_hi, n_ent, cur, &kfull[4 * s + h]);
+            }
+          } else {
           // region pair h as soon as O^T slice h of the tile's previous block
           // has read it
 #pragma unroll 1
           for (int h = 0; h < 4; ++h) {
             wait_or_die(&bfree[4 * s + h], (uint32_t)((j >> 1) & 1) ^ 1u, 21u);
-            if (!dead && a.mixed) {
-              gather_mixed(a, tile, h, pw, quad, g8, k_lo + (int64_t)b * kBK, k_hi, n_ent, list,
-                           x, &kfull[4 * s + h]);
-            } else if (!dead) {
+            if (!dead) {
 #pragma unroll
               for (int u = 0; u < kGatherIters; ++u) {
                 if (pw + kProdWarps * u >= kBK / 4) continue;
@@ -530,6 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // the barrier counts this thread's arrival once its copies land
               cp_async_arrive(&kfull[4 * s + h]);
             }
+          }
           }
         }
         if (b == 0) {
@@ -1127,9 +1160,13 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
     return cudaErrorInvalidValue;
   const int smem = SMEM_BYTES + 1024;
   cudaError_t e =
-      cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaFuncSetAttribute(a.mixed ? attn_tc_kernel<true> : attn_tc_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, a);
+  if (a.mixed)
+    attn_tc_kernel<true><<<grid, kThreads, smem, stream>>>(mq, a);
+  else
+    attn_tc_kernel<false><<<grid, kThreads, smem, stream>>>(mq, a);
   if (a.split) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -74,7 +74,8 @@ struct Smem {
   static constexpr int kEl = MX ? 1 : 2;                   // bytes per operand element
   static constexpr int kTile = kBM * kDI * kEl;            // one K_I tile
   static constexpr int kB = TOK * kHI * kDI * kEl;         // q_I block
-  static constexpr int kStages = Cfg<TOK>::kStages;
+  // MX tiles are half as large: twice the ring slots keep as many bytes in flight
+  static constexpr int kStages = MX ? 2 * Cfg<TOK>::kStages : Cfg<TOK>::kStages;
   static constexpr int kChunk = Cfg<TOK>::kChunk;
   static constexpr int off_b = 0;
   static constexpr int off_a = kB;
