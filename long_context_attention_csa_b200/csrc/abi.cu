@@ -176,7 +176,7 @@ static csa_status append_common(int32_t dtype, int64_t B, int32_t m, bool overla
   if (B < 0 || m < 1 || n_cap < 0 || B > 0x7fffffffLL) return CSA_E_ARG;
   if (z_cols != 1 && z_cols != f.c) return CSA_E_ARG;
   if (overlap ? (2 * m > 256) : (m > 4096)) return CSA_E_UNSUPPORTED;
-  if (f.c < 64 || f.c > 1024) return CSA_E_UNSUPPORTED;
+  if (f.c < 64 || f.c > 1024 || f.r > 2 * kStreamMaxPairs) return CSA_E_UNSUPPORTED;
   if (B == 0) return CSA_OK;
   if (!kv_a || !z_a || !state || (overlap && (!kv_b || !z_b)) || (n_cap > 0 && !entries))
     return CSA_E_ARG;

@@ -76,6 +76,7 @@ struct AttnParams {
 };
 cudaError_t launch_attn_portable(int dtype, const AttnParams& p, cudaStream_t stream);
 
+constexpr int kStreamMaxPairs = 64;   // RoPE pairs the streaming append takes (r <= 128)
 struct StreamParams {
   const void* kv_a;   // [B, c] this call's token of each sequence (group a / HCA's group)
   const void* kv_b;   // [B, c] group b (CSA only)
@@ -92,6 +93,7 @@ struct StreamParams {
   int64_t n_cap;
   void* win;          // [B, c] window rows of this call's tokens, or null
   unsigned* status;
+  double theta[kStreamMaxPairs];   // RoPE frequencies (set by the launcher)
 };
 size_t stream_state_bytes(int elem_bytes, int m, int overlap, int c, int z_cols);
 cudaError_t launch_stream_append(int dtype, StreamParams p, int64_t B, cudaStream_t stream);

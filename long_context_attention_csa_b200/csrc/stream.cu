@@ -83,34 +83,59 @@ __device__ __forceinline__ float cta_sum(float v, float* red) {
 // RMSNorm over the c channels held by the pair threads (others pass active =
 // false and contribute nothing), then RoPE of the pair at position pos.
 __device__ __forceinline__ void norm_rope_pair(float& x0, float& x1, bool active, int pair,
-                                               const Fmt& f, int64_t pos, float* red) {
-  if (!(f.flags & CSA_F_NO_NORM)) {
+                                               const StreamParams& p, int64_t pos, float* red) {
+  if (!(p.f.flags & CSA_F_NO_NORM)) {
     const float ss = cta_sum(active ? fmaf(x0, x0, x1 * x1) : 0.f, red);
-    const float inv = rsqrtf(ss / (float)f.c + f.eps);
+    const float inv = rsqrtf(ss / (float)p.f.c + p.f.eps);
     x0 *= inv;
     x1 *= inv;
   }
-  const int ch = 2 * pair, d0 = f.c - f.r;
-  if (active && !(f.flags & CSA_F_NO_ROPE) && ch >= d0) {
+  const int ch = 2 * pair, d0 = p.f.c - p.f.r;
+  if (active && !(p.f.flags & CSA_F_NO_ROPE) && ch >= d0) {
     float cs, sn;
-    rope_cos_sin_theta(pos, rope_theta((ch - d0) >> 1, f.r, f.base), &cs, &sn);
+    rope_cos_sin_theta(pos, p.theta[(ch - d0) >> 1], &cs, &sn);
     const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
     x0 = y0;
     x1 = y1;
   }
 }
 
+// One slot of the entry's softmax: (value pair, logit pair) of token row
+// `row` / logits `zrow` at this thread's channels.
 template <typename T>
-__global__ void __launch_bounds__(1024) stream_append_kernel(StreamParams p) {
+__device__ __forceinline__ void load_slot(const T* row, const T* zrow, int zc, int ch, float& v0,
+                                          float& v1, float& z0, float& z1) {
+  load2(row + ch, v0, v1);
+  if (zc == 1) {
+    z0 = z1 = to_float(zrow[0]);
+  } else {
+    load2(zrow + ch, z0, z1);
+  }
+}
+
+// Latency chain: the token count, then in one round every load the call
+// needs (the token's own rows; on a block's last token every other slot of
+// the entry, which earlier calls stored -- the token's own slot comes from
+// its inputs, so nothing waits for this call's stores), then the arithmetic.
+template <typename T>
+__global__ void __launch_bounds__(1024) stream_append_kernel(const StreamParams p) {
   __shared__ float red[32];
   extern __shared__ float part[];      // [G][c/2][6] partial softmax states (G > 1)
   const int c = p.f.c, m = p.m, zc = p.z_cols;
   const int np = c / 2;
   const int pair = (int)threadIdx.x % np, g = (int)threadIdx.x / np;
+  const int G = (int)blockDim.x / np;
   const int ch = 2 * pair;
   const int64_t b = blockIdx.x;
+  const T* __restrict__ ka = static_cast<const T*>(p.kv_a) + b * c;
+  const T* __restrict__ za = static_cast<const T*>(p.z_a) + b * zc;
+  const T* __restrict__ kb = p.overlap ? static_cast<const T*>(p.kv_b) + b * c : nullptr;
+  const T* __restrict__ zb = p.overlap ? static_cast<const T*>(p.z_b) + b * zc : nullptr;
+  // the token's rows (independent of the state), then the token count
+  float x0 = 0.f, x1 = 0.f, az0 = 0.f, az1 = 0.f;
+  if (g == 0) load_slot(ka, za, zc, ch, x0, x1, az0, az1);
   uint8_t* st = p.state + (size_t)b * p.stride;
-  const int64_t t = *reinterpret_cast<const int64_t*>(st);
+  const int64_t t = *reinterpret_cast<const volatile int64_t*>(st);
   if (t < 0) {   // a corrupt state: nothing of this sequence is touched
     if (threadIdx.x == 0) report(p.status, CSA_DEV_STREAM, (unsigned)b);
     return;
@@ -122,22 +147,39 @@ __global__ void __launch_bounds__(1024) stream_append_kernel(StreamParams p) {
   T* rb = ra + (size_t)m * c;
   T* rza = rb + (p.overlap ? (size_t)2 * m * c : 0);
   T* rzb = rza + (size_t)m * zc;
+  const bool closes = j == m - 1;
+  const int ns = closes ? m + ((p.overlap && s >= 1) ? m : 0) : 0;
+
+  // the entry's slots: a(s) (slot j from the inputs), then b(s - 1) for CSA
+  constexpr int U = 8;   // slots a thread holds at once
+  float v0[U], v1[U], z0[U], z1[U];
+  auto load_batch = [&](int i0) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * G;
+      if (i < ns) {
+        if (i == j)
+          load_slot(ka, za, zc, ch, v0[u], v1[u], z0[u], z1[u]);
+        else if (i < m)
+          load_slot(ra + (size_t)i * c, rza + (size_t)i * zc, zc, ch, v0[u], v1[u], z0[u], z1[u]);
+        else
+          load_slot(rb + ((size_t)(par ^ 1) * m + (i - m)) * c,
+                    rzb + ((size_t)(par ^ 1) * m + (i - m)) * zc, zc, ch, v0[u], v1[u], z0[u],
+                    z1[u]);
+      }
+    }
+  };
+  if (closes) load_batch(g);
 
   // 1. this token's rows into the tail buffer (exact copies), window row
-  const T* ka = static_cast<const T*>(p.kv_a) + b * c;
-  const T* za = static_cast<const T*>(p.z_a) + b * zc;
-  float x0 = 0.f, x1 = 0.f;
   if (g == 0) {
     copy2(ra + (size_t)j * c + ch, ka + ch);
-    load2(ka + ch, x0, x1);
     if (zc == 1) {
       if (pair == 0) rza[j] = za[0];
     } else {
       copy2(rza + (size_t)j * zc + ch, za + ch);
     }
     if (p.overlap) {
-      const T* kb = static_cast<const T*>(p.kv_b) + b * c;
-      const T* zb = static_cast<const T*>(p.z_b) + b * zc;
       copy2(rb + ((size_t)par * m + j) * c + ch, kb + ch);
       if (zc == 1) {
         if (pair == 0) rzb[par * m + j] = zb[0];
@@ -147,48 +189,22 @@ __global__ void __launch_bounds__(1024) stream_append_kernel(StreamParams p) {
     }
   }
   if (p.win != nullptr) {   // uniform: every thread takes the reduction
-    norm_rope_pair(x0, x1, g == 0, pair, p.f, p.pos0 + t, red);
+    norm_rope_pair(x0, x1, g == 0, pair, p, p.pos0 + t, red);
     if (g == 0) store2(static_cast<T*>(p.win) + b * c + ch, x0, x1);
   }
-  if (j != m - 1) {
-    __syncthreads();
+  if (!closes) {
+    __syncthreads();   // every thread has read the count
     if (threadIdx.x == 0) *reinterpret_cast<int64_t*>(st) = t + 1;
     return;
   }
 
-  // 2. the token completes block s: pool a(s) and, for CSA with s >= 1, b(s-1)
-  __syncthreads();   // the rows stored above are visible to every thread
-  const int G = (int)blockDim.x / np;
-  const int ns = m + ((p.overlap && s >= 1) ? m : 0);
+  // 2. the token completes block s: pool the slots (online softmax in base 2)
   float mx0 = -INFINITY, mx1 = -INFINITY, d0 = 0.f, d1 = 0.f, a0 = 0.f, a1 = 0.f;
-  constexpr int U = 8;   // slots whose loads are in flight together
   for (int i0 = g; i0 < ns; i0 += G * U) {
-    float v0[U], v1[U], z0[U], z1[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = i0 + u * G;
-      if (i < ns) {
-        const T* row;
-        const T* zrow;
-        if (i < m) {
-          row = ra + (size_t)i * c;
-          zrow = rza + (size_t)i * zc;
-        } else {
-          row = rb + ((size_t)(par ^ 1) * m + (i - m)) * c;
-          zrow = rzb + ((size_t)(par ^ 1) * m + (i - m)) * zc;
-        }
-        load2(row + ch, v0[u], v1[u]);
-        if (zc == 1) {
-          z0[u] = z1[u] = to_float(zrow[0]);
-        } else {
-          load2(zrow + ch, z0[u], z1[u]);
-        }
-      }
-    }
+    if (i0 != g) load_batch(i0);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (i0 + u * G >= ns) break;
-      // online softmax in base 2 (the running maximum never decreases)
       const float l0 = z0[u] * kLog2e, l1 = z1[u] * kLog2e;
       const float n0 = fmaxf(mx0, l0), n1 = fmaxf(mx1, l1);
       const float s0 = exp2f(mx0 - n0), s1 = exp2f(mx1 - n1);
@@ -226,13 +242,13 @@ __global__ void __launch_bounds__(1024) stream_append_kernel(StreamParams p) {
     }
   }
   float y0 = g == 0 ? a0 / d0 : 0.f, y1 = g == 0 ? a1 / d1 : 0.f;
-  norm_rope_pair(y0, y1, g == 0, pair, p.f, p.pos0 + (int64_t)m * s, red);
+  norm_rope_pair(y0, y1, g == 0, pair, p, p.pos0 + (int64_t)m * s, red);
   if (s < p.n_cap) {
     if (g == 0) store2(static_cast<T*>(p.entries) + ((size_t)b * p.n_cap + s) * c + ch, y0, y1);
   } else if (threadIdx.x == 0) {
     report(p.status, CSA_DEV_STREAM, (unsigned)b);   // entry cache full: entry dropped
   }
-  __syncthreads();
+  __syncthreads();   // every thread has read the count
   if (threadIdx.x == 0) *reinterpret_cast<int64_t*>(st) = t + 1;
 }
 
@@ -246,6 +262,9 @@ size_t stream_state_bytes(int elem_bytes, int m, int overlap, int c, int z_cols)
 
 cudaError_t launch_stream_append(int dtype, StreamParams p, int64_t B, cudaStream_t stream) {
   if (B == 0) return cudaSuccess;
+  if (p.f.r > 2 * kStreamMaxPairs) return cudaErrorInvalidValue;
+  for (int i = 0; i < p.f.r / 2; ++i)   // RoPE frequencies base^(-2i/r), in double
+    p.theta[i] = pow((double)p.f.base, -2.0 * (double)i / (double)p.f.r);
   const int np = p.f.c / 2;
   const int ns_max = p.overlap ? 2 * p.m : p.m;
   int G = ns_max >= 32 ? 4 : 1;
