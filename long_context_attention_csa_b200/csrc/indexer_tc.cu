@@ -847,7 +847,9 @@ struct PCfg {
   static constexpr int kTile = kBM * kDI * kEl;              // one K_I tile
   static constexpr int kB = TOK * kHI * kDI * kEl;           // q_I block
   static constexpr int kStages = TOK == 4 ? 2 : (MX ? 10 : 5);
-  static constexpr uint32_t kCols = MX ? 256 : 2 * kN;       // two accumulators (+ MX scales)
+  // TMEM accumulators: the MMAs run up to kAcc tiles ahead of the epilogue
+  static constexpr int kAcc = TOK == 4 ? 2 : 4;
+  static constexpr uint32_t kCols = MX ? 512 : kAcc * kN;    // (+ MX scales: 12 columns)
   static constexpr int off_b = 0;
   static constexpr int off_a = kB;                                   // K_I tile ring
   static constexpr int off_sf = off_a + kStages * kTile;             // MX: [kStages + 1][512]
@@ -861,10 +863,11 @@ struct PCfg {
   static constexpr int off_wcnt = off_red + TOK * kScr * 4;          // [TOK][16]
   static constexpr int off_cand = off_wcnt + TOK * kScr * 4;         // [TOK][kBinCap] pairs
   static constexpr int off_bar = off_cand + TOK * kBinCap * 8;
-  static constexpr int kBars = 2 * kStages + 12;
+  static constexpr int kBars = 2 * kStages + 2 * kAcc + 8;
   static constexpr int off_misc = off_bar + kBars * 8;
   static constexpr int bytes = off_misc + 64;
   static_assert(bytes + 1024 <= 232448, "shared memory budget");
+  static_assert(kAcc * kN + (MX ? 12 : 0) <= (int)kCols, "TMEM columns");
 };
 
 template <int TOK>
@@ -914,7 +917,8 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
   constexpr int kTile = L::kTile;
   constexpr int kG = L::kG;
   constexpr uint32_t kCols = L::kCols;
-  constexpr uint32_t kSfa = 2 * kN;      // MX: two 4-column K_I scale buffers
+  constexpr int kAcc = L::kAcc;
+  constexpr uint32_t kSfa = kAcc * kN;   // MX: two 4-column K_I scale buffers
   constexpr uint32_t kSfb = kSfa + 8;    // MX: the query's scale tile
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kN, 0, 0);
   extern __shared__ uint8_t smem_raw[];
@@ -926,9 +930,9 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::off_bar);
   uint64_t* full = bars;                   // [stages] K_I tile landed (TMA)
   uint64_t* empty = bars + kStages;        // [stages] tile consumed (MMA)
-  uint64_t* tfull = bars + 2 * kStages;    // [2] accumulator ready (MMA)
-  uint64_t* tempty = tfull + 2;            // [2] accumulator read (128 epilogue threads)
-  uint64_t* qfull = tempty + 2;            // the unit's q_I block landed (TMA)
+  uint64_t* tfull = bars + 2 * kStages;    // [kAcc] accumulator ready (MMA)
+  uint64_t* tempty = tfull + kAcc;         // [kAcc] accumulator read (128 epilogue threads)
+  uint64_t* qfull = tempty + kAcc;         // the unit's q_I block landed (TMA)
   uint64_t* qfree = qfull + 1;             // the unit's last MMA done
   uint64_t* sready = qfree + 1;            // [2] score buffer complete (128 epilogue threads)
   uint64_t* sfree = sready + 2;            // [2] score buffer consumed (the top-k warps)
@@ -942,9 +946,11 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAcc; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 128);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sready[i], 128);
       mbar_init(&sfree[i], TOK * kG);
     }
@@ -967,9 +973,11 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
   // a timed-out wait marks the thread dead (warp-uniform); dead threads skip
   // work and waits but pass every named barrier
   bool dead = false;
-  auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
+  // poll: the per-tile hand-overs poll before suspending; the per-unit ones
+  // (score buffers) suspend at once and leave the issue slots to the others
+  auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code, bool poll = false) {
     if (!dead) {
-      if (!mbar_wait(bar, parity)) {
+      if (!(poll ? mbar_wait_poll(bar, parity) : mbar_wait(bar, parity))) {
         *abort_flag = 1;
         report(a.status, CSA_DEV_TIMEOUT, code);
         dead = true;
@@ -1003,7 +1011,7 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
         ++nq;
         for (int i = 0; i < x.n_tiles; ++i, ++tile) {
           const int s = (int)(tile % kStages);
-          if (*abort_flag || !mbar_wait(&empty[s], (uint32_t)((tile / kStages) & 1) ^ 1u)) {
+          if (*abort_flag || !mbar_wait_poll(&empty[s], (uint32_t)((tile / kStages) & 1) ^ 1u)) {
             dead = true;
             break;
           }
@@ -1048,9 +1056,9 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
                              smem_desc(smem_u32(sm + L::off_sf + kStages * 512), 16, 128, 0));
         for (int i = 0; i < x.n_tiles; ++i, ++tile) {
           const int s = (int)(tile % kStages);
-          const int buf = (int)(tile & 1);
-          if (*abort_flag || !mbar_wait(&full[s], (uint32_t)((tile / kStages) & 1)) ||
-              !mbar_wait(&tempty[buf], (uint32_t)((tile >> 1) & 1) ^ 1u)) {
+          const int buf = (int)(tile % kAcc);
+          if (*abort_flag || !mbar_wait_poll(&full[s], (uint32_t)((tile / kStages) & 1)) ||
+              !mbar_wait_poll(&tempty[buf], (uint32_t)((tile / kAcc) & 1) ^ 1u)) {
             ok = false;
             break;
           }
@@ -1059,7 +1067,7 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
           const uint64_t dAs = dA + (uint64_t)((s * kTile) >> 4);
           if constexpr (MX) {
             // the tile's K_I scales into TMEM, executed before the MMAs below
-            const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)buf;
+            const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)(tile & 1);
             tmem_cp_32x128b_x4(sfa, smem_desc(smem_u32(sm + L::off_sf + s * 512), 16, 128, 0));
 #pragma unroll
             for (int kk = 0; kk < kDI / 32; ++kk)   // K = 32 per MMA, one scale each
@@ -1107,8 +1115,8 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
       named_bar(5, 128);   // weights visible
       float* sc = scores + sb * TOK * kChunk;
       for (int i = 0; i < x.n_tiles; ++i, ++tile) {
-        const int buf = (int)(tile & 1);
-        wait_or_die(&tfull[buf], (uint32_t)((tile >> 1) & 1), 4u);
+        const int buf = (int)(tile % kAcc);
+        wait_or_die(&tfull[buf], (uint32_t)((tile / kAcc) & 1), 4u, true);
         if (dead) continue;
         tc_fence_after();
         const uint32_t base = tmem_addr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kN));
