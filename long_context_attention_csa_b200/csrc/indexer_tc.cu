@@ -10,22 +10,17 @@
 // lane) and (token, head) pairs on N (TOK tokens x 64 heads), K = d_I = 128.
 // Every TMEM lane then holds all heads of one entry for TOK tokens, so the
 // epilogue sum_h w ReLU(.) is a per-thread loop with no cross-lane traffic.
-// Persistent CTAs (one per SM) walk (chunk, token group) units: four-token
-// groups for prefill rows, single tokens for decode rows.
-//   warp 0      TMA producer: the unit's q_I block, K_I tiles through a ring;
-//   warp 1      TMEM owner and single-thread MMA issuer;
-//   warps 2..5  epilogue: TMEM -> registers -> the unit's scores in shared
-//               memory (two TMEM accumulators, so tile i+1's MMAs overlap
-//               tile i's epilogue);
-//   warps 6..   top-k, on the previous unit's score buffer while the next
-//               unit streams: an exact value-binned select (radix fallback)
-//               and an ordered compaction.
-// The score matrix never reaches HBM.  When the entries span several chunks
-// (2048 entries for four-token groups, 4096 for single tokens) each unit
-// emits its chunk's top-k as candidates and a merge kernel selects the final
-// k (the union of per-chunk top-k sets contains the global top-k under the
-// same tie rule).  MX-FP8 operands (single tokens) use block-scaled MMAs
-// with the scale tiles copied into TMEM next to the accumulators.
+//   warp 0      TMA producer: q_I block once, K_I tiles through a ring;
+//   warp 1      TMEM owner and single-thread MMA issuer (8 MMAs per tile);
+//   warps 2..5  epilogue: TMEM -> registers -> scores in shared memory
+//               (two TMEM accumulators so tile i+1's MMAs overlap tile i's
+//               epilogue); afterwards one warp per token runs an exact radix
+//               select over the scores and an ordered compaction.
+// The score matrix never reaches HBM.  A CTA covers the entries of one chunk
+// (2048 for 4-token groups, 4096 for single tokens); when the entries span
+// several chunks each CTA emits its chunk's top-k as candidates and a merge
+// kernel selects the final k (the union of per-chunk top-k sets contains the
+// global top-k under the same tie rule).
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc.h"
@@ -41,9 +36,13 @@ constexpr int kBM = 128;   // entries per tile
 constexpr int kDI = 128;   // indexer dim
 constexpr int kHI = 64;    // indexer heads
 constexpr int kTileBytes = kBM * kDI * 2;     // 32 KB (two 128-byte-swizzled column halves)
+constexpr int kThreads = 192;
 constexpr int kBinCap = 64;   // largest boundary bin the value-binned top-k ranks exactly
 constexpr int kMergeCap = 2048;   // the same for the chunk-candidate merge
 
+template <int TOK> struct Cfg;
+template <> struct Cfg<4> { static constexpr int kStages = 3; static constexpr int kChunk = 2048; };
+template <> struct Cfg<1> { static constexpr int kStages = 2; static constexpr int kChunk = 4096; };
 
 // sum_h w[h] ReLU(s[h]) over 64 heads (s: two 32-column TMEM loads) with
 // packed fp32 FMAs (two heads per instruction; even and odd heads accumulate
@@ -67,6 +66,31 @@ __device__ __forceinline__ float relu_weighted_sum64(const float* wt, const uint
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
   return a0 + a1;
 }
+
+// MX: the operands are MX-FP8 (one byte per element, no halves) and each
+// K_I tile and the query block bring a 512-byte scale-factor tile.
+template <int TOK, bool MX = false>
+struct Smem {
+  static constexpr int kEl = MX ? 1 : 2;                   // bytes per operand element
+  static constexpr int kTile = kBM * kDI * kEl;            // one K_I tile
+  static constexpr int kB = TOK * kHI * kDI * kEl;         // q_I block
+  // MX tiles are half as large: twice the ring slots keep as many bytes in flight
+  static constexpr int kStages = MX ? 2 * Cfg<TOK>::kStages : Cfg<TOK>::kStages;
+  static constexpr int kChunk = Cfg<TOK>::kChunk;
+  static constexpr int off_b = 0;
+  static constexpr int off_a = kB;
+  static constexpr int off_sf = off_a + kStages * kTile;   // MX: [kStages + 1][512] scales
+  static constexpr int off_scores = off_sf + (MX ? (kStages + 1) * 512 : 0);
+  static constexpr int off_w = off_scores + TOK * kChunk * 4;
+  static constexpr int off_hist = off_w + TOK * kHI * 4;
+  static constexpr int off_cand = off_hist + TOK * 256 * 4;   // [TOK][kBinCap] (score, index)
+  static constexpr int off_red = off_cand + TOK * kBinCap * 8;  // [16] cooperative top-k
+  static constexpr int off_wcnt = off_red + 64;                 // [16]
+  static constexpr int off_bar = off_wcnt + 64;
+  static constexpr int kBars = 2 * kStages + 6;
+  static constexpr int off_misc = off_bar + kBars * 8;
+  static constexpr int bytes = off_misc + 64;
+};
 
 struct TcIdxArgs {
   int64_t Tq, N;
@@ -820,78 +844,338 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
   if (!solo) cluster_wait();   // no CTA leaves while another may still read its shared memory
 }
 
-// ---------------------------------------------------------------------------
-// Persistent form: CTAs walk (chunk, token group) units -- groups of four
-// tokens (prefill; heaviest causal groups first) or single tokens (decode) --
-// and the top-k of one unit runs on its own warps while the next unit's
-// tiles stream through the tensor core.
-//   warp 0        TMA producer: the unit's q_I block, K_I tiles through a ring
-//   warp 1        TMEM owner, single-thread MMA issuer
-//   warps 2-5     epilogue: TMEM -> sum_h w ReLU(.) -> the unit's score buffer
-//   warps 6..     top-k (block_topk), G warps per token, on the previous
-//                 unit's score buffer (two buffers alternate)
-// Four-token groups: N = 256, 2048-entry chunks, a two-slot ring, G = 2.
-// Single tokens: N = 64, 4096-entry chunks, a five-slot ring (ten half-size
-// slots for MX-FP8 operands), G = 4; one CTA per SM keeps 160 KB of K_I in
-// flight, and the top-k of a chunk overlaps the next chunk's stream.
-// ---------------------------------------------------------------------------
 template <int TOK, bool MX>
-struct PCfg {
-  static_assert(TOK == 4 || TOK == 1, "token groups of one or four");
-  static_assert(!MX || TOK == 1, "MX-FP8 operands: single tokens");
-  static constexpr int kChunk = TOK == 4 ? 2048 : 4096;
-  static constexpr int kN = TOK * kHI;                       // MMA N
-  static constexpr int kG = TOK == 4 ? 2 : 4;                // top-k warps per token
-  static constexpr int kThreads = 32 * (6 + TOK * kG);       // 448 / 320
-  static constexpr int kEl = MX ? 1 : 2;
-  static constexpr int kTile = kBM * kDI * kEl;              // one K_I tile
-  static constexpr int kB = TOK * kHI * kDI * kEl;           // q_I block
-  static constexpr int kStages = TOK == 4 ? 2 : (MX ? 10 : 5);
-  // TMEM accumulators: the MMAs run up to kAcc tiles ahead of the epilogue
-  static constexpr int kAcc = TOK == 4 ? 2 : 4;
-  static constexpr uint32_t kCols = MX ? 512 : kAcc * kN;    // (+ MX scales: 12 columns)
+__global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_k, TcIdxArgs a) {
+  static_assert(!MX || TOK == 1, "MX-FP8 operands: single-token groups");
+  using L = Smem<TOK, MX>;
+  constexpr int kStages = L::kStages;
+  constexpr int kChunk = L::kChunk;
+  constexpr int kTile = L::kTile;
+  constexpr int kN = TOK * kHI;                 // MMA N
+  // two accumulators; MX adds two 4-column K_I scale buffers and the query's
+  // scale tile (4 columns), rounded up to a power of two
+  constexpr uint32_t kCols = MX ? 256 : 2 * kN;
+  constexpr uint32_t kSfa = 2 * kN;
+  constexpr uint32_t kSfb = kSfa + 8;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kN, 0, 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sB = sm + L::off_b;
+  uint8_t* sA = sm + L::off_a;
+  float* scores = reinterpret_cast<float*>(sm + L::off_scores);
+  float* sw = reinterpret_cast<float*>(sm + L::off_w);
+  unsigned* hist = reinterpret_cast<unsigned*>(sm + L::off_hist);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::off_bar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* bfull = tempty + 2;
+  uint64_t* drain = bfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::off_misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::off_misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int group = gridDim.y - 1 - blockIdx.y;   // heaviest causal groups first
+  const int b = blockIdx.z;
+  const int64_t t0 = (int64_t)group * TOK;
+  const int64_t e0 = (int64_t)chunk * kChunk;
+
+  // visibility of the TOK tokens and the entry range this CTA scores
+  int64_t vis[TOK];
+  int64_t vmax = 0;
+#pragma unroll
+  for (int i = 0; i < TOK; ++i) {
+    int64_t t = t0 + i;
+    vis[i] = 0;
+    if (t < a.Tq) {
+      int64_t row = (int64_t)b * a.Tq + t;
+      int64_t pos = a.q_pos ? a.q_pos[row] : t;
+      vis[i] = vis_count(pos, a.m, a.N);
+    }
+    vmax = vis[i] > vmax ? vis[i] : vmax;
+  }
+  int64_t e_hi = e0 + kChunk < vmax ? e0 + kChunk : vmax;
+  const int n_tiles = e_hi > e0 ? (int)((e_hi - e0 + kBM - 1) / kBM) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    mbar_init(bfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    if (n_tiles > 0) {   // the q_I block first: its latency overlaps the rest of the setup
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      const int32_t qrow = (int32_t)(t0 * kHI);
+      if constexpr (MX) {
+        // codes (128 bytes a row, one box) and the scale tile holding this token's rows
+        mbar_arrive_expect_tx(bfull, L::kB + 512);
+        tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
+        bulk_load(smem_u32(sm + L::off_sf + kStages * 512),
+                  a.q_sf + ((int64_t)b * a.Tq + t0) * 512, 512, bfull);
+      } else {
+        mbar_arrive_expect_tx(bfull, L::kB);
+        tma_load_3d(sB, &map_q, bfull, 0, qrow, b);
+        tma_load_3d(sB + L::kB / 2, &map_q, bfull, 64, qrow, b);
+      }
+    }
+  }
+  for (int i = threadIdx.x; i < TOK * kHI; i += blockDim.x) {
+    int64_t t = t0 + i / kHI;
+    sw[i] = t < a.Tq ? a.w[((int64_t)b * a.Tq + t) * kHI + (i % kHI)] : 0.f;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (n_tiles > 0 && elect_one()) {
+      int issued = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1u)) {
+          *abort_flag = 1;
+          report(a.status, CSA_DEV_TIMEOUT, 1u);
+          break;
+        }
+        const int32_t erow = (int32_t)(e0 + (int64_t)i * kBM);
+        if constexpr (MX) {
+          mbar_arrive_expect_tx(&full[s], kTile + 512);
+          tma_load_3d(sA + s * kTile, &map_k, &full[s], 0, erow, b);
+          bulk_load(smem_u32(sm + L::off_sf + s * 512),
+                    a.k_sf + ((int64_t)b * a.k_sf_tiles + erow / kBM) * 512, 512, &full[s]);
+        } else {
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          uint8_t* dst = sA + s * kTileBytes;
+          tma_load_3d(dst, &map_k, &full[s], 0, erow, b);
+          tma_load_3d(dst + kTileBytes / 2, &map_k, &full[s], 64, erow, b);
+        }
+        issued = i + 1;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i)
+        mbar_wait(&full[i % kStages], (uint32_t)(i / kStages) & 1u);
+      mbar_wait(bfull, 0);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (n_tiles > 0 && elect_one()) {
+      if (!mbar_wait(bfull, 0)) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 2u);
+      } else {
+        const uint32_t b_base = smem_u32(sB);
+        const uint32_t a_base = smem_u32(sA);
+        if constexpr (MX) {
+          // the query's scale tile into TMEM (rows 32 j + l: lane l, column j)
+          tmem_cp_32x128b_x4(tmem + kSfb,
+                             smem_desc(smem_u32(sm + L::off_sf + kStages * 512), 16, 128, 0));
+        }
+        for (int i = 0; i < n_tiles; ++i) {
+          const int s = i % kStages;
+          const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+          const int buf = i & 1;
+          const uint32_t bph = (uint32_t)(i >> 1) & 1u;
+          if (*abort_flag || !mbar_wait(&full[s], ph) || !mbar_wait(&tempty[buf], bph ^ 1u)) {
+            *abort_flag = 1;
+            report(a.status, CSA_DEV_TIMEOUT, 3u);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(buf * kN);
+          if constexpr (MX) {
+            // this tile's K_I scales into TMEM (issued before, and executed
+            // before, the MMAs below that read them)
+            const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)buf;
+            tmem_cp_32x128b_x4(sfa, smem_desc(smem_u32(sm + L::off_sf + s * 512), 16, 128, 0));
+            const uint32_t sfb = tmem + kSfb;   // the token's own tile: heads on rows 0..63
+#pragma unroll
+            for (int kk = 0; kk < kDI / 32; ++kk) {   // K = 32 per MMA, one scale each
+              const uint64_t ad = smem_desc(a_base + s * kTile + kk * 32, 16, 1024, 2);
+              const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, 2);
+              mma_mxf8_ss(d, ad, bd, idesc_mxf8_e4m3(kBM, kN, kk, kk),
+                          sfa | ((uint32_t)kk << 30), sfb | ((uint32_t)kk << 30),
+                          kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kDI / 16; ++kk) {
+              const uint32_t koff = (uint32_t)((kk & 3) * 32);  // 16 bf16 per K step
+              uint64_t ad = smem_desc(a_base + s * kTileBytes + (kk >> 2) * (kTileBytes / 2) +
+                                          koff, 16, 1024, 2);
+              uint64_t bd = smem_desc(b_base + (kk >> 2) * (L::kB / 2) + koff, 16, 1024, 2);
+              mma_bf16_ss(d, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[buf]);
+        }
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    // ---------------- epilogue: thread <-> TMEM lane <-> entry
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int buf = i & 1;
+      const uint32_t bph = (uint32_t)(i >> 1) & 1u;
+      if (*abort_flag || !mbar_wait(&tfull[buf], bph)) {
+        *abort_flag = 1;
+        report(a.status, CSA_DEV_TIMEOUT, 4u);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = tmem_addr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kN));
+#pragma unroll
+      for (int t = 0; t < TOK; ++t) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(base + t * kHI, r0);
+        tmem_ld32(base + t * kHI + 32, r1);
+        tmem_ld_wait();
+        scores[t * kChunk + i * kBM + row] = relu_weighted_sum64(sw + t * kHI, r0, r1);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  __syncthreads();
+
+  // ---------------- top-k: one warp per token
+  if (TOK == 1 && warp >= 2 && !*abort_flag) {
+    // one token: the four epilogue warps select together (named barrier 1)
+    const int64_t tok = t0;
+    if (tok < a.Tq) {
+      const int64_t row = (int64_t)b * a.Tq + tok;
+      int64_t n64 = vis[0] - e0;
+      n64 = n64 < 0 ? 0 : (n64 > kChunk ? kChunk : n64);
+      int32_t* oi;
+      float* os;
+      if (a.n_chunks == 1) {
+        oi = a.idx_out + row * a.k;
+        os = a.score_out ? a.score_out + row * a.k : nullptr;
+      } else {
+        const int64_t c = (row * a.n_chunks + chunk) * a.k;
+        oi = a.cand_idx + c;
+        os = a.cand_score + c;
+      }
+      float* cand = reinterpret_cast<float*>(sm + L::off_cand);
+      const bool done = block_topk<4, kChunk>(
+          scores, (int)n64, a.k, e0, hist, reinterpret_cast<float*>(sm + L::off_red),
+          reinterpret_cast<unsigned*>(sm + L::off_wcnt), cand,
+          reinterpret_cast<int*>(cand + kBinCap), 1, oi, os);
+      if (!done) {
+        if (warp == 2) warp_topk(scores, (int)n64, a.k, e0, hist, oi, os);
+        named_bar(1, 128);
+      }
+    }
+  } else if (TOK > 1 && warp >= 2 && warp < 2 + TOK && !*abort_flag) {
+    const int t = warp - 2;
+    const int64_t tok = t0 + t;
+    if (tok < a.Tq) {
+      const int64_t row = (int64_t)b * a.Tq + tok;
+      int64_t n64 = vis[t] - e0;
+      n64 = n64 < 0 ? 0 : (n64 > kChunk ? kChunk : n64);
+      const int n = (int)n64;
+      int32_t* oi;
+      float* os;
+      if (a.n_chunks == 1) {
+        oi = a.idx_out + row * a.k;
+        os = a.score_out ? a.score_out + row * a.k : nullptr;
+      } else {
+        const int64_t c = (row * a.n_chunks + chunk) * a.k;
+        oi = a.cand_idx + c;
+        os = a.cand_score + c;
+      }
+      float* cand = reinterpret_cast<float*>(sm + L::off_cand) + t * 2 * kBinCap;
+      warp_topk_binned(scores + t * kChunk, n, a.k, e0, hist + t * 256, cand,
+                       reinterpret_cast<int*>(cand + kBinCap), oi, os);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Prefill form (4-token groups): persistent CTAs walk (chunk, group) units,
+// heaviest causal groups first, and the top-k of one unit runs on its own
+// warps while the next unit's tiles stream through the tensor core.
+//   warp 0        TMA producer: the unit's q_I block, K_I tiles (2-slot ring)
+//   warp 1        TMEM owner, single-thread MMA issuer (8 MMAs per tile)
+//   warps 2-5     epilogue: TMEM -> sum_h w ReLU(.) -> the unit's score buffer
+//   warps 6-13    top-k, two warps per token (block_topk), on the previous
+//                 unit's score buffer (two buffers alternate)
+// ---------------------------------------------------------------------------
+constexpr int kPTok = 4;
+constexpr int kPChunk = 2048;
+constexpr int kPN = kPTok * kHI;                  // MMA N = 256
+constexpr int kPStages = 2;
+constexpr int kPTopkWarps = 2;                    // warps per token in the top-k
+constexpr int kPThreads = 32 * (6 + kPTok * kPTopkWarps);   // 448
+
+struct PSmem {
+  static constexpr int kB = kPTok * kHI * kDI * 2;              // q_I block, 64 KB
   static constexpr int off_b = 0;
-  static constexpr int off_a = kB;                                   // K_I tile ring
-  static constexpr int off_sf = off_a + kStages * kTile;             // MX: [kStages + 1][512]
-  static constexpr int off_scores = off_sf + (MX ? (kStages + 1) * 512 : 0);  // [2][TOK][chunk]
-  static constexpr int off_w = off_scores + 2 * TOK * kChunk * 4;    // [2][TOK][64] fp32
-  static constexpr int off_hist = off_w + 2 * TOK * kHI * 4;         // [TOK][256]
-  // block_topk<G> scratch: red holds 2 G + 2 floats, wcnt G + 4 words
-  static constexpr int kScr = 16;
-  static_assert(2 * kG + 2 <= kScr && kG + 4 <= kScr, "top-k scratch");
-  static constexpr int off_red = off_hist + TOK * 256 * 4;           // [TOK][16] fp32
-  static constexpr int off_wcnt = off_red + TOK * kScr * 4;          // [TOK][16]
-  static constexpr int off_cand = off_wcnt + TOK * kScr * 4;         // [TOK][kBinCap] pairs
-  static constexpr int off_bar = off_cand + TOK * kBinCap * 8;
-  static constexpr int kBars = 2 * kStages + 2 * kAcc + 8;
+  static constexpr int off_a = kB;                               // K_I tile ring
+  static constexpr int off_scores = off_a + kPStages * kTileBytes;   // [2][4][2048] fp32
+  static constexpr int off_w = off_scores + 2 * kPTok * kPChunk * 4; // [2][4][64] fp32
+  static constexpr int off_hist = off_w + 2 * kPTok * kHI * 4;       // [4][256]
+  static constexpr int off_red = off_hist + kPTok * 256 * 4;         // [4][8] fp32
+  static constexpr int off_wcnt = off_red + kPTok * 8 * 4;           // [4][8]
+  static constexpr int off_cand = off_wcnt + kPTok * 8 * 4;          // [4][kBinCap] (score, index)
+  static constexpr int off_bar = off_cand + kPTok * kBinCap * 8;
+  static constexpr int kBars = 2 * kPStages + 12;
   static constexpr int off_misc = off_bar + kBars * 8;
   static constexpr int bytes = off_misc + 64;
-  static_assert(bytes + 1024 <= 232448, "shared memory budget");
-  static_assert(kAcc * kN + (MX ? 12 : 0) <= (int)kCols, "TMEM columns");
 };
+static_assert(PSmem::bytes + 1024 <= 232448, "shared memory budget");
 
-template <int TOK>
+
 struct PUnit {
   int64_t b, group, chunk, e0;
   int n_tiles;
-  int64_t vis[TOK];
+  int64_t vis[kPTok];
 };
 
 // Unit u: heaviest causal groups first (u = (b * n_groups + gi) * n_chunks + c,
 // group = n_groups - 1 - gi).  Every role derives it the same way.
-template <int TOK>
-__device__ __forceinline__ PUnit<TOK> punit(const TcIdxArgs& a, int64_t u, int64_t n_groups,
-                                            int chunk) {
-  PUnit<TOK> x;
+__device__ __forceinline__ PUnit punit(const TcIdxArgs& a, int64_t u, int64_t n_groups) {
+  PUnit x;
   x.chunk = u % a.n_chunks;
   const int64_t r = u / a.n_chunks;
   x.group = n_groups - 1 - r % n_groups;
   x.b = r / n_groups;
-  x.e0 = x.chunk * chunk;
+  x.e0 = x.chunk * kPChunk;
   int64_t vmax = 0;
 #pragma unroll
-  for (int i = 0; i < TOK; ++i) {
-    const int64_t t = x.group * TOK + i;
+  for (int i = 0; i < kPTok; ++i) {
+    const int64_t t = x.group * kPTok + i;
     x.vis[i] = 0;
     if (t < a.Tq) {
       const int64_t row = x.b * a.Tq + t;
@@ -900,27 +1184,18 @@ __device__ __forceinline__ PUnit<TOK> punit(const TcIdxArgs& a, int64_t u, int64
     }
     vmax = x.vis[i] > vmax ? x.vis[i] : vmax;
   }
-  const int64_t e_hi = x.e0 + chunk < vmax ? x.e0 + chunk : vmax;
+  const int64_t e_hi = x.e0 + kPChunk < vmax ? x.e0 + kPChunk : vmax;
   x.n_tiles = e_hi > x.e0 ? (int)((e_hi - x.e0 + kBM - 1) / kBM) : 0;
   return x;
 }
 
-template <int TOK, bool MX>
-__global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
+__global__ void __launch_bounds__(kPThreads, 1)
     indexer_persist_kernel(const __grid_constant__ CUtensorMap map_q,
                            const __grid_constant__ CUtensorMap map_k, TcIdxArgs a,
                            int64_t n_units, int64_t n_groups) {
-  using L = PCfg<TOK, MX>;
-  constexpr int kStages = L::kStages;
-  constexpr int kChunk = L::kChunk;
-  constexpr int kN = L::kN;
-  constexpr int kTile = L::kTile;
-  constexpr int kG = L::kG;
-  constexpr uint32_t kCols = L::kCols;
-  constexpr int kAcc = L::kAcc;
-  constexpr uint32_t kSfa = kAcc * kN;   // MX: two 4-column K_I scale buffers
-  constexpr uint32_t kSfb = kSfa + 8;    // MX: the query's scale tile
-  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kN, 0, 0);
+  using L = PSmem;
+  constexpr uint32_t kCols = 2 * kPN;   // two accumulators
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kPN, 0, 0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sB = sm + L::off_b;
@@ -928,31 +1203,29 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
   float* scores = reinterpret_cast<float*>(sm + L::off_scores);
   float* sw = reinterpret_cast<float*>(sm + L::off_w);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::off_bar);
-  uint64_t* full = bars;                   // [stages] K_I tile landed (TMA)
-  uint64_t* empty = bars + kStages;        // [stages] tile consumed (MMA)
-  uint64_t* tfull = bars + 2 * kStages;    // [kAcc] accumulator ready (MMA)
-  uint64_t* tempty = tfull + kAcc;         // [kAcc] accumulator read (128 epilogue threads)
-  uint64_t* qfull = tempty + kAcc;         // the unit's q_I block landed (TMA)
+  uint64_t* full = bars;                   // [2] K_I tile landed (TMA)
+  uint64_t* empty = bars + kPStages;       // [2] tile consumed (MMA)
+  uint64_t* tfull = bars + 2 * kPStages;   // [2] accumulator ready (MMA)
+  uint64_t* tempty = tfull + 2;            // [2] accumulator read (128 epilogue threads)
+  uint64_t* qfull = tempty + 2;            // the unit's q_I block landed (TMA)
   uint64_t* qfree = qfull + 1;             // the unit's last MMA done
   uint64_t* sready = qfree + 1;            // [2] score buffer complete (128 epilogue threads)
-  uint64_t* sfree = sready + 2;            // [2] score buffer consumed (the top-k warps)
+  uint64_t* sfree = sready + 2;            // [2] score buffer consumed (8 top-k warps)
   uint64_t* drain = sfree + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::off_misc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kPStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < kAcc; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 128);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(&sready[i], 128);
-      mbar_init(&sfree[i], TOK * kG);
+      mbar_init(&sfree[i], kPTok * kPTopkWarps);
     }
     mbar_init(qfull, 1);
     mbar_init(qfree, 1);
@@ -973,11 +1246,9 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
   // a timed-out wait marks the thread dead (warp-uniform); dead threads skip
   // work and waits but pass every named barrier
   bool dead = false;
-  // poll: the per-tile hand-overs poll before suspending; the per-unit ones
-  // (score buffers) suspend at once and leave the issue slots to the others
-  auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code, bool poll = false) {
+  auto wait_or_die = [&](uint64_t* bar, uint32_t parity, unsigned code) {
     if (!dead) {
-      if (!(poll ? mbar_wait_poll(bar, parity) : mbar_wait(bar, parity))) {
+      if (!mbar_wait(bar, parity)) {
         *abort_flag = 1;
         report(a.status, CSA_DEV_TIMEOUT, code);
         dead = true;
@@ -993,40 +1264,25 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
       int64_t tile = 0;   // tiles issued so far
       int nq = 0;         // q_I blocks loaded so far
       for (int64_t u = blockIdx.x; u < n_units && !dead; u += gridDim.x) {
-        const PUnit<TOK> x = punit<TOK>(a, u, n_groups, kChunk);
+        const PUnit x = punit(a, u, n_groups);
         if (x.n_tiles == 0) continue;
         if (nq > 0 && !mbar_wait(qfree, (uint32_t)(nq - 1) & 1u)) { dead = true; break; }
-        const int32_t qrow = (int32_t)(x.group * TOK * kHI);
-        if constexpr (MX) {
-          // codes (128 bytes a row, one box) and the token's scale tile
-          mbar_arrive_expect_tx(qfull, L::kB + 512);
-          tma_load_3d(sB, &map_q, qfull, 0, qrow, (int32_t)x.b);
-          bulk_load(smem_u32(sm + L::off_sf + kStages * 512),
-                    a.q_sf + (x.b * a.Tq + x.group) * 512, 512, qfull);
-        } else {
-          mbar_arrive_expect_tx(qfull, L::kB);
-          tma_load_3d(sB, &map_q, qfull, 0, qrow, (int32_t)x.b);
-          tma_load_3d(sB + L::kB / 2, &map_q, qfull, 64, qrow, (int32_t)x.b);
-        }
+        mbar_arrive_expect_tx(qfull, L::kB);
+        const int32_t qrow = (int32_t)(x.group * kPTok * kHI);
+        tma_load_3d(sB, &map_q, qfull, 0, qrow, (int32_t)x.b);
+        tma_load_3d(sB + L::kB / 2, &map_q, qfull, 64, qrow, (int32_t)x.b);
         ++nq;
         for (int i = 0; i < x.n_tiles; ++i, ++tile) {
-          const int s = (int)(tile % kStages);
-          if (*abort_flag || !mbar_wait_poll(&empty[s], (uint32_t)((tile / kStages) & 1) ^ 1u)) {
+          const int s = (int)(tile % kPStages);
+          if (*abort_flag || !mbar_wait(&empty[s], (uint32_t)((tile / kPStages) & 1) ^ 1u)) {
             dead = true;
             break;
           }
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          uint8_t* dst = sA + s * kTileBytes;
           const int32_t erow = (int32_t)(x.e0 + (int64_t)i * kBM);
-          if constexpr (MX) {
-            mbar_arrive_expect_tx(&full[s], kTile + 512);
-            tma_load_3d(sA + s * kTile, &map_k, &full[s], 0, erow, (int32_t)x.b);
-            bulk_load(smem_u32(sm + L::off_sf + s * 512),
-                      a.k_sf + (x.b * a.k_sf_tiles + erow / kBM) * 512, 512, &full[s]);
-          } else {
-            mbar_arrive_expect_tx(&full[s], kTile);
-            uint8_t* dst = sA + s * kTile;
-            tma_load_3d(dst, &map_k, &full[s], 0, erow, (int32_t)x.b);
-            tma_load_3d(dst + kTile / 2, &map_k, &full[s], 64, erow, (int32_t)x.b);
-          }
+          tma_load_3d(dst, &map_k, &full[s], 0, erow, (int32_t)x.b);
+          tma_load_3d(dst + kTileBytes / 2, &map_k, &full[s], 64, erow, (int32_t)x.b);
         }
       }
       if (dead) {
@@ -1034,8 +1290,8 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
         report(a.status, CSA_DEV_TIMEOUT, 1u);
       }
       // drain: the last issued copies land before the CTA may exit
-      for (int64_t t = tile - kStages > 0 ? tile - kStages : 0; t < tile; ++t)
-        mbar_wait(&full[t % kStages], (uint32_t)((t / kStages) & 1));
+      for (int64_t t = tile - kPStages > 0 ? tile - kPStages : 0; t < tile; ++t)
+        mbar_wait(&full[t % kPStages], (uint32_t)((t / kPStages) & 1));
       if (nq > 0) mbar_wait(qfull, (uint32_t)(nq - 1) & 1u);
     }
   } else if (warp == 1) {
@@ -1047,40 +1303,26 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
       int nq = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const PUnit<TOK> x = punit<TOK>(a, u, n_groups, kChunk);
+        const PUnit x = punit(a, u, n_groups);
         if (x.n_tiles == 0) continue;
         if (*abort_flag || !mbar_wait(qfull, (uint32_t)nq & 1u)) { ok = false; break; }
         ++nq;
-        if constexpr (MX)   // the query's scale tile into TMEM (rows 32 j + l: lane l, column j)
-          tmem_cp_32x128b_x4(tmem + kSfb,
-                             smem_desc(smem_u32(sm + L::off_sf + kStages * 512), 16, 128, 0));
         for (int i = 0; i < x.n_tiles; ++i, ++tile) {
-          const int s = (int)(tile % kStages);
-          const int buf = (int)(tile % kAcc);
-          if (*abort_flag || !mbar_wait_poll(&full[s], (uint32_t)((tile / kStages) & 1)) ||
-              !mbar_wait_poll(&tempty[buf], (uint32_t)((tile / kAcc) & 1) ^ 1u)) {
+          const int s = (int)(tile % kPStages);
+          const int buf = (int)(tile & 1);
+          if (*abort_flag || !mbar_wait(&full[s], (uint32_t)((tile / kPStages) & 1)) ||
+              !mbar_wait(&tempty[buf], (uint32_t)((tile >> 1) & 1) ^ 1u)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(buf * kN);
-          const uint64_t dAs = dA + (uint64_t)((s * kTile) >> 4);
-          if constexpr (MX) {
-            // the tile's K_I scales into TMEM, executed before the MMAs below
-            const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)(tile & 1);
-            tmem_cp_32x128b_x4(sfa, smem_desc(smem_u32(sm + L::off_sf + s * 512), 16, 128, 0));
+          const uint32_t d = tmem + (uint32_t)(buf * kPN);
+          const uint64_t dAs = dA + (uint64_t)((s * kTileBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kDI / 32; ++kk)   // K = 32 per MMA, one scale each
-              mma_mxf8_ss(d, dAs + (uint64_t)((kk * 32) >> 4), dB + (uint64_t)((kk * 32) >> 4),
-                          idesc_mxf8_e4m3(kBM, kN, kk, kk), sfa | ((uint32_t)kk << 30),
-                          (tmem + kSfb) | ((uint32_t)kk << 30), kk > 0 ? 1u : 0u);
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < kDI / 16; ++kk)
-              mma_bf16_ss(d, dAs + (uint64_t)(((kk >> 2) * (kTile / 2) + (kk & 3) * 32) >> 4),
-                          dB + (uint64_t)(((kk >> 2) * (L::kB / 2) + (kk & 3) * 32) >> 4), kIdesc,
-                          kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kDI / 16; ++kk)
+            mma_bf16_ss(d, dAs + (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4),
+                        dB + (uint64_t)(((kk >> 2) * (L::kB / 2) + (kk & 3) * 32) >> 4), kIdesc,
+                        kk > 0 ? 1u : 0u);
           mma_commit(&empty[s]);
           mma_commit(&tfull[buf]);
         }
@@ -1102,31 +1344,31 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
     int64_t tile = 0;
     int n = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++n) {
-      const PUnit<TOK> x = punit<TOK>(a, u, n_groups, kChunk);
+      const PUnit x = punit(a, u, n_groups);
       const int sb = n & 1;
-      float* wb = sw + sb * TOK * kHI;
+      float* wb = sw + sb * kPTok * kHI;
       // the unit's head weights (this buffer's previous unit is finished: the
       // named barrier below ran after its last tile)
-      for (int i = et; i < TOK * kHI; i += 128) {
-        const int64_t t = x.group * TOK + i / kHI;
+      for (int i = et; i < kPTok * kHI; i += 128) {
+        const int64_t t = x.group * kPTok + i / kHI;
         wb[i] = (!dead && t < a.Tq) ? a.w[(x.b * a.Tq + t) * kHI + (i % kHI)] : 0.f;
       }
       wait_or_die(&sfree[sb], (uint32_t)((n >> 1) & 1) ^ 1u, 5u);   // top-k of unit n-2 done
       named_bar(5, 128);   // weights visible
-      float* sc = scores + sb * TOK * kChunk;
+      float* sc = scores + sb * kPTok * kPChunk;
       for (int i = 0; i < x.n_tiles; ++i, ++tile) {
-        const int buf = (int)(tile % kAcc);
-        wait_or_die(&tfull[buf], (uint32_t)((tile / kAcc) & 1), 4u, true);
+        const int buf = (int)(tile & 1);
+        wait_or_die(&tfull[buf], (uint32_t)((tile >> 1) & 1), 4u);
         if (dead) continue;
         tc_fence_after();
-        const uint32_t base = tmem_addr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kN));
+        const uint32_t base = tmem_addr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kPN));
 #pragma unroll
-        for (int t = 0; t < TOK; ++t) {
+        for (int t = 0; t < kPTok; ++t) {
           uint32_t r0[32], r1[32];
           tmem_ld32(base + t * kHI, r0);
           tmem_ld32(base + t * kHI + 32, r1);
           tmem_ld_wait();
-          sc[t * kChunk + i * kBM + row] = relu_weighted_sum64(wb + t * kHI, r0, r1);
+          sc[t * kPChunk + i * kBM + row] = relu_weighted_sum64(wb + t * kHI, r0, r1);
         }
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
@@ -1135,24 +1377,24 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
       if (!dead) mbar_arrive(&sready[sb]);
     }
   } else {
-    // ---------------- top-k: G warps per token
+    // ---------------- top-k: two warps per token
     const int tw = warp - 6;
-    const int t = tw / kG;
-    const bool lead = tw % kG == 0;
+    const int t = tw / kPTopkWarps;
+    const bool lead = tw % kPTopkWarps == 0;
     unsigned* hist = reinterpret_cast<unsigned*>(sm + L::off_hist) + t * 256;
-    float* red = reinterpret_cast<float*>(sm + L::off_red) + t * L::kScr;
-    unsigned* wcnt = reinterpret_cast<unsigned*>(sm + L::off_wcnt) + t * L::kScr;
+    float* red = reinterpret_cast<float*>(sm + L::off_red) + t * 8;
+    unsigned* wcnt = reinterpret_cast<unsigned*>(sm + L::off_wcnt) + t * 8;
     float* cand = reinterpret_cast<float*>(sm + L::off_cand) + t * 2 * kBinCap;
     int n = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++n) {
-      const PUnit<TOK> x = punit<TOK>(a, u, n_groups, kChunk);
+      const PUnit x = punit(a, u, n_groups);
       const int sb = n & 1;
       wait_or_die(&sready[sb], (uint32_t)(n >> 1) & 1u, 6u);
-      const int64_t tok = x.group * TOK + t;
+      const int64_t tok = x.group * kPTok + t;
       if (tok < a.Tq) {
         const int64_t row = x.b * a.Tq + tok;
         int64_t n64 = x.vis[t] - x.e0;
-        n64 = n64 < 0 ? 0 : (n64 > kChunk ? kChunk : n64);
+        n64 = n64 < 0 ? 0 : (n64 > kPChunk ? kPChunk : n64);
         int32_t* oi;
         float* os;
         if (a.n_chunks == 1) {
@@ -1163,16 +1405,16 @@ __global__ void __launch_bounds__(PCfg<TOK, MX>::kThreads, 1)
           oi = a.cand_idx + c;
           os = a.cand_score + c;
         }
-        const float* sc = scores + (sb * TOK + t) * kChunk;
-        // the token's warps run the same barrier sequence even after a
+        const float* sc = scores + (sb * kPTok + t) * kPChunk;
+        // both warps of the token run the same barrier sequence even after a
         // timed-out wait (the selection then reads stale scores; the status
         // word already holds the error)
-        const bool done = block_topk<kG, kChunk>(
+        const bool done = block_topk<kPTopkWarps, kPChunk>(
             sc, (int)n64, a.k, x.e0, hist, red, wcnt, cand,
             reinterpret_cast<int*>(cand + kBinCap), 1 + t, oi, os);
         if (!done) {
           if (lead) warp_topk(sc, (int)n64, a.k, x.e0, hist, oi, os);
-          named_bar(1 + t, 32 * kG);
+          named_bar(1 + t, 32 * kPTopkWarps);
         }
       }
       if (lane == 0 && !dead) mbar_arrive(&sfree[sb]);
@@ -1486,13 +1728,35 @@ __global__ void __launch_bounds__(kMThreads)
 }
 
 inline int tok_for(int64_t Tq) { return Tq >= 4 ? 4 : 1; }
-inline int chunk_for(int tok) {
-  return tok == 4 ? PCfg<4, false>::kChunk : PCfg<1, false>::kChunk;
-}
+inline int chunk_for(int tok) { return tok == 4 ? Cfg<4>::kChunk : Cfg<1>::kChunk; }
 inline int n_chunks_for(int64_t N, int tok) {
   int64_t c = chunk_for(tok);
   int64_t n = (N + c - 1) / c;
   return n < 1 ? 1 : (int)n;
+}
+
+template <int TOK, bool MX = false>
+cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
+  CUtensorMap mq, mk;
+  if constexpr (MX) {
+    if (!make_map_u8_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, kDI, TOK * kHI))
+      return cudaErrorInvalidValue;
+    if (!make_map_u8_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, kDI, kBM))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, TOK * kHI))
+      return cudaErrorInvalidValue;
+    if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64,
+                          kBM))
+      return cudaErrorInvalidValue;
+  }
+  const int smem = Smem<TOK, MX>::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<TOK, MX>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)a.n_chunks, (unsigned)((p.Tq + TOK - 1) / TOK), (unsigned)p.B);
+  indexer_tc_kernel<TOK, MX><<<grid, kThreads, smem, stream>>>(mq, mk, a);
+  return cudaGetLastError();
 }
 
 // Rows with no entry at all (N == 0): index -1 and score -inf throughout.
@@ -1536,32 +1800,21 @@ cudaError_t launch_merge(const TcIdxArgs& a, int64_t rows, cudaStream_t stream) 
   return cudaLaunchKernelEx(&cfg, indexer_merge_cluster_kernel, a);
 }
 
-template <int TOK, bool MX>
 cudaError_t launch_persist(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
-  using L = PCfg<TOK, MX>;
   CUtensorMap mq, mk;
-  if constexpr (MX) {
-    if (!make_map_u8_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, kDI, TOK * kHI))
-      return cudaErrorInvalidValue;
-    if (!make_map_u8_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, kDI, kBM))
-      return cudaErrorInvalidValue;
-  } else {
-    if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, TOK * kHI))
-      return cudaErrorInvalidValue;
-    if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64,
-                          kBM))
-      return cudaErrorInvalidValue;
-  }
-  const int smem = L::bytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_persist_kernel<TOK, MX>,
+  if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, kPTok * kHI))
+    return cudaErrorInvalidValue;
+  if (!make_map_bf16_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, 64, kBM))
+    return cudaErrorInvalidValue;
+  const int smem = PSmem::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_persist_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int64_t n_groups = (p.Tq + TOK - 1) / TOK;
+  const int64_t n_groups = (p.Tq + kPTok - 1) / kPTok;
   const int64_t n_units = p.B * n_groups * a.n_chunks;
   const int64_t sms = sm_count();
   const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);
-  indexer_persist_kernel<TOK, MX><<<grid, L::kThreads, smem, stream>>>(mq, mk, a, n_units,
-                                                                         n_groups);
+  indexer_persist_kernel<<<grid, kPThreads, smem, stream>>>(mq, mk, a, n_units, n_groups);
   return cudaGetLastError();
 }
 
@@ -1604,7 +1857,7 @@ cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const vo
     a.cand_score = static_cast<float*>(p.scratch);
     a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
   }
-  cudaError_t e = launch_persist<1, true>(p, a, stream);
+  cudaError_t e = launch_tok<1, true>(p, a, stream);
   if (e != cudaSuccess) return e;
   *n_launch = 1;
   if (a.n_chunks > 1) {
@@ -1657,8 +1910,7 @@ cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
     a.cand_score = static_cast<float*>(p.scratch);
     a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
   }
-  cudaError_t e = tok == 4 ? launch_persist<4, false>(p, a, stream)
-                           : launch_persist<1, false>(p, a, stream);
+  cudaError_t e = tok == 4 ? launch_persist(p, a, stream) : launch_tok<1>(p, a, stream);
   if (e != cudaSuccess) return e;
   *n_launch = 1;
   if (a.n_chunks > 1) {

@@ -105,29 +105,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
-// Non-blocking test of the phase of `parity` (never suspends the thread).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// mbar_wait for short, frequent hand-overs: polls without suspending (the
-// phase is seen as soon as it completes) and falls back to the suspending
-// wait after `spin` polls; gives up after `limit_ns` like mbar_wait.
-__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, int spin = 2048,
-                                               uint64_t limit_ns = 2000000000ull) {
-  for (int i = 0; i < spin; ++i)
-    if (mbar_test_wait(bar, parity)) return true;
-  return mbar_wait(bar, parity, limit_ns);
-}
-
 // ---- TMA --------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
