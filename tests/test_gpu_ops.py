@@ -570,3 +570,26 @@ def test_attention_index_out_of_range_is_skipped_and_flagged(flags):
     assert csa.csa_check_status(ws) == (csa.CSA_E_DEVICE, csa.CSA_DEV_BAD_INDEX)
     rows = np.array(sorted(set(planted) | set(range(0, w.T, 5))))
     _check_attn(w, inp, out, rows, dense=False, flags=flags)
+
+
+def test_prefill_row_agrees_with_the_decode_query_at_its_position():
+    """A prefill row t and the same query run as a decode step (one query at
+    position t, its key list split into pieces whose float32 partials are
+    added in a fixed order) differ only by the float32 summation order: at
+    most one bf16 ulp of the larger value, element by element, over rows
+    spanning the first blocks, the window's reach and the sequence's end."""
+    w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=700, k=128)
+    inp = _attn_inputs_prefill(w)
+    pre = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w), w.n_win,
+                              sink=inp["sink"])
+    torch.cuda.synchronize()
+    for t in (0, 3, 127, 128, 400, 699):
+        pos = torch.tensor([[t]], dtype=torch.int64, device=DEV)
+        dec = csa.sparse_mqa_attn(inp["q"][:, t:t + 1].contiguous(), inp["entries"],
+                                  inp["idx"][:, t:t + 1].contiguous(), inp["win"], gfmt(w),
+                                  w.n_win, sink=inp["sink"], q_pos=pos)
+        torch.cuda.synchronize()
+        a, b = f64(pre[0, t]), f64(dec[0, 0])
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.maximum(np.abs(a), np.abs(b)),
+                                                   np.finfo(np.float32).tiny))) - 7)
+        assert np.all(np.abs(a - b) <= ulp), f"row {t}: {np.abs(a - b).max()}"
