@@ -303,6 +303,26 @@ csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t
                                      const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
                                      float* score_out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * The same low-precision path with FP4, the precision the pages name for the
+ * indexer ([§3.3 last paragraph and §3.6 of the summary page]).  Format taken:
+ * OCP MX-FP4 -- E2M1 elements (magnitudes 0, 0.5, ..., 6) with one UE8M0
+ * scale per 32 elements, 2^(floor(log2 amax) - 2), rounded to nearest (ties
+ * to even) and saturated at 6, packed two to a byte (the even element in the
+ * low nibble): codes [B, rows, 64] uint8; the scale tiles exactly as for
+ * MX-FP8.  indexer_scores_topk_mxfp4 takes q_codes [B, Tq, 64, 64] and
+ * k_codes [B, N, 64] (with their scale tiles) and runs block-scaled
+ * kind::mxf4 MMAs (K = 64, two scales each); everything else as
+ * indexer_scores_topk_mxfp8 (same workspace).
+ */
+csa_status indexer_mxfp4_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
+                                  const void* x, void* codes, void* scales, void* stream);
+csa_status indexer_scores_topk_mxfp4(int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                                     const void* q_codes, const void* q_scales, const float* w,
+                                     const void* k_codes, const void* k_scales, int64_t N,
+                                     const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                                     float* score_out, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- (3) shared-KV MQA ------------------------------------------------ */
 
 /*

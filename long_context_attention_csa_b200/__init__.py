@@ -32,7 +32,8 @@ CSA_DEV_TIMEOUT, CSA_DEV_RANGE, CSA_DEV_BAD_INDEX, CSA_DEV_STREAM = 1, 2, 3, 4
 EXPORTED = (
     "csa_compress", "hca_compress", "csa_stream_state_bytes", "csa_compress_append",
     "hca_compress_append", "indexer_scores_topk", "indexer_scores_topk_noalloc",
-    "indexer_mxfp8_quantize", "indexer_scores_topk_mxfp8", "csa_mixed_record_bytes",
+    "indexer_mxfp8_quantize", "indexer_scores_topk_mxfp8", "indexer_mxfp4_quantize",
+    "indexer_scores_topk_mxfp4", "csa_mixed_record_bytes",
     "csa_store_mixed", "sparse_mqa_attn", "dense_hca_attn",
     "grouped_output_projection", "csa_workspace_bytes",
     "csa_check_status",
@@ -106,6 +107,9 @@ def lib():
     L.hca_compress_append.argtypes = [i32, i64, i32, FP, P, P, i32, i64, P, sz, P, i64, P, P, sz,
                                       P]
     L.indexer_mxfp8_quantize.argtypes = [i32, i64, i64, i32, P, P, P, P]
+    L.indexer_mxfp4_quantize.argtypes = [i32, i64, i64, i32, P, P, P, P]
+    L.indexer_scores_topk_mxfp4.argtypes = [i64, i64, i32, i32, P, P, P, P, P, i64, P, i32, i32,
+                                            P, P, P, sz, P]
     L.csa_mixed_record_bytes.argtypes = [i32, i32]
     L.csa_mixed_record_bytes.restype = sz
     L.csa_store_mixed.argtypes = [i32, i64, i64, FP, P, P, P]
@@ -125,6 +129,7 @@ def lib():
                "indexer_scores_topk",
                "indexer_scores_topk_noalloc", "sparse_mqa_attn", "dense_hca_attn",
                "grouped_output_projection", "indexer_mxfp8_quantize", "csa_store_mixed",
+               "indexer_mxfp4_quantize", "indexer_scores_topk_mxfp4",
                "indexer_scores_topk_mxfp8", "csa_check_status", "csa_selftest_wait"):
         getattr(L, fn).restype = i32
     _lib = L
@@ -314,30 +319,40 @@ def csa_store_mixed(entries, fmt: Fmt, records=None, stream=None):
     return records
 
 
-def indexer_mxfp8_quantize(x, codes=None, scales=None, per_token=False, stream=None):
-    """MX-FP8 codes and scale tiles of x [B, ..., 128]: codes uint8 with x's
-    shape; scales [B, ceil(rows/128), 512] with rows = the middle dims
-    flattened, or, with ``per_token`` (q_I [B, Tq, 64, 128]), one tile per
-    token: [B, Tq, 512]."""
+def indexer_mxfp8_quantize(x, codes=None, scales=None, per_token=False, stream=None, fp4=False):
+    """MX-FP8 (or, with ``fp4``, packed MX-FP4) codes and scale tiles of x
+    [B, ..., 128]: codes uint8 with x's shape (the last dim 64 for FP4);
+    scales [B, ceil(rows/128), 512] with rows = the middle dims flattened, or,
+    with ``per_token`` (q_I [B, Tq, 64, 128]), one tile per token: [B, Tq, 512]."""
     d = x.shape[-1]
     B = x.shape[0] * x.shape[1] if per_token else x.shape[0]
     rows = x.numel() // d // B if B else 0
     if codes is None:
-        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+        shape = tuple(x.shape[:-1]) + ((d // 2,) if fp4 else (d,))
+        codes = torch.empty(shape, dtype=torch.uint8, device=x.device)
     if scales is None:
         shape = (x.shape[0], x.shape[1], 512) if per_token else (B, (rows + 127) // 128, 512)
         scales = torch.empty(shape, dtype=torch.uint8, device=x.device)
-    st = lib().indexer_mxfp8_quantize(_dt(x), B, rows, d, _p(x), _p(codes), _p(scales), _s(stream))
-    _check(st, "indexer_mxfp8_quantize")
+    fn = lib().indexer_mxfp4_quantize if fp4 else lib().indexer_mxfp8_quantize
+    st = fn(_dt(x), B, rows, d, _p(x), _p(codes), _p(scales), _s(stream))
+    _check(st, "indexer_mxfp4_quantize" if fp4 else "indexer_mxfp8_quantize")
     return codes, scales
+
+
+def indexer_mxfp4_quantize(x, codes=None, scales=None, per_token=False, stream=None):
+    """Packed MX-FP4 codes [..., 64] and scale tiles of x [B, ..., 128]."""
+    return indexer_mxfp8_quantize(x, codes, scales, per_token, stream, fp4=True)
 
 
 def indexer_scores_topk_mxfp8(q_codes, q_scales, w, k_codes, k_scales, m: int, k: int,
                               q_pos=None, idx_out=None, score_out=None, want_scores=False,
                               ws=None, stream=None):
     """indexer_scores_topk on MX-FP8 operands: q_codes [B, Tq, 64, 128] and
-    k_codes [B, N, 128] uint8 with their scale tiles."""
+    k_codes [B, N, 128] uint8 with their scale tiles; packed MX-FP4 codes
+    (last dim 64) take the FP4 kernel."""
     B, Tq, HI, dI = q_codes.shape
+    fp4 = dI == 64
+    dI = 128
     N = k_codes.shape[1]
     dev = q_codes.device
     if idx_out is None:
@@ -346,7 +361,8 @@ def indexer_scores_topk_mxfp8(q_codes, q_scales, w, k_codes, k_scales, m: int, k
         score_out = torch.empty((B, Tq, k), dtype=torch.float32, device=dev)
     if ws is None:
         ws = workspace(csa_workspace_bytes(CSA_OP_INDEXER_MX, CSA_BF16, B, Tq, 0, 0, N, k), dev)
-    st = lib().indexer_scores_topk_mxfp8(B, Tq, HI, dI, _p(q_codes), _p(q_scales), _p(w),
+    fn = lib().indexer_scores_topk_mxfp4 if fp4 else lib().indexer_scores_topk_mxfp8
+    st = fn(B, Tq, HI, dI, _p(q_codes), _p(q_scales), _p(w),
                                          _p(k_codes), _p(k_scales), N, _p(q_pos), m, k,
                                          _p(idx_out), _p(score_out), _p(ws), ws.numel(),
                                          _s(stream))

@@ -243,8 +243,8 @@ csa_status csa_store_mixed(int32_t dtype, int64_t B, int64_t N, const csa_fmt* f
   return cuda_status(launch_mixed_store(dtype, entries, records, B * N, f.c, f.r, S(stream)));
 }
 
-csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
-                                  const void* x, void* codes, void* scales, void* stream) {
+static csa_status mx_quantize(int fmt, int32_t dtype, int64_t B, int64_t rows, int32_t d,
+                              const void* x, void* codes, void* scales, void* stream) {
   if (dtype != CSA_F32 && dtype != CSA_BF16) return CSA_E_ARG;
   if (B < 0 || rows < 0 || d <= 0) return CSA_E_ARG;
   if (d != 128) return CSA_E_UNSUPPORTED;
@@ -253,14 +253,25 @@ csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_
   if (!x || !codes || !scales) return CSA_E_ARG;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return CSA_E_ARG;
   g_launches.fetch_add(1);
-  return cuda_status(launch_mxfp8_quantize(dtype, x, codes, scales, B, rows, S(stream)));
+  return cuda_status(fmt == 2 ? launch_mxfp4_quantize(dtype, x, codes, scales, B, rows, S(stream))
+                              : launch_mxfp8_quantize(dtype, x, codes, scales, B, rows, S(stream)));
 }
 
-csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
-                                     const void* q_codes, const void* q_scales, const float* w,
-                                     const void* k_codes, const void* k_scales, int64_t N,
-                                     const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
-                                     float* score_out, void* ws, size_t ws_bytes, void* stream) {
+csa_status indexer_mxfp8_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
+                                  const void* x, void* codes, void* scales, void* stream) {
+  return mx_quantize(1, dtype, B, rows, d, x, codes, scales, stream);
+}
+
+csa_status indexer_mxfp4_quantize(int32_t dtype, int64_t B, int64_t rows, int32_t d,
+                                  const void* x, void* codes, void* scales, void* stream) {
+  return mx_quantize(2, dtype, B, rows, d, x, codes, scales, stream);
+}
+
+static csa_status scores_mx(int fmt, int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                            const void* q_codes, const void* q_scales, const float* w,
+                            const void* k_codes, const void* k_scales, int64_t N,
+                            const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                            float* score_out, void* ws, size_t ws_bytes, void* stream) {
   if (B < 0 || Tq < 0 || N < 0 || H_I <= 0 || d_I <= 0 || m < 1 || k < 1) return CSA_E_ARG;
   if (H_I != 64 || d_I != 128) return CSA_E_UNSUPPORTED;
   if (B > 65535 || Tq > 65535 || N > 0x7fffffffLL) return CSA_E_UNSUPPORTED;
@@ -290,9 +301,27 @@ csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t
   p.scratch = static_cast<char*>(ws) + kWsScratch;
   p.scratch_bytes = ws_bytes - kWsScratch;
   unsigned long long n = 0;
-  cudaError_t e = launch_indexer_mx(p, q_scales, k_scales, S(stream), &n);
+  cudaError_t e = launch_indexer_mx(p, fmt, q_scales, k_scales, S(stream), &n);
   g_launches.fetch_add(n);
   return cuda_status(e);
+}
+
+csa_status indexer_scores_topk_mxfp8(int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                                     const void* q_codes, const void* q_scales, const float* w,
+                                     const void* k_codes, const void* k_scales, int64_t N,
+                                     const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                                     float* score_out, void* ws, size_t ws_bytes, void* stream) {
+  return scores_mx(1, B, Tq, H_I, d_I, q_codes, q_scales, w, k_codes, k_scales, N, q_pos, m, k,
+                   idx_out, score_out, ws, ws_bytes, stream);
+}
+
+csa_status indexer_scores_topk_mxfp4(int64_t B, int64_t Tq, int32_t H_I, int32_t d_I,
+                                     const void* q_codes, const void* q_scales, const float* w,
+                                     const void* k_codes, const void* k_scales, int64_t N,
+                                     const int64_t* q_pos, int32_t m, int32_t k, int32_t* idx_out,
+                                     float* score_out, void* ws, size_t ws_bytes, void* stream) {
+  return scores_mx(2, B, Tq, H_I, d_I, q_codes, q_scales, w, k_codes, k_scales, N, q_pos, m, k,
+                   idx_out, score_out, ws, ws_bytes, stream);
 }
 
 csa_status grouped_output_projection(int32_t dtype, int64_t T, int32_t H, int32_t c, int32_t g,

@@ -67,15 +67,18 @@ __device__ __forceinline__ float relu_weighted_sum64(const float* wt, const uint
   return a0 + a1;
 }
 
-// MX: the operands are MX-FP8 (one byte per element, no halves) and each
-// K_I tile and the query block bring a 512-byte scale-factor tile.
-template <int TOK, bool MX = false>
+// Operand formats: bf16 (FMT 0, rows of 256 bytes in two 128-byte swizzled
+// halves), MX-FP8 (FMT 1, 128-byte rows) and MX-FP4 (FMT 2, packed, 64-byte
+// rows, 64-byte swizzle); each MX K_I tile and the query block bring a
+// 512-byte scale-factor tile.
+template <int TOK, int FMT = 0>
 struct Smem {
-  static constexpr int kEl = MX ? 1 : 2;                   // bytes per operand element
-  static constexpr int kTile = kBM * kDI * kEl;            // one K_I tile
-  static constexpr int kB = TOK * kHI * kDI * kEl;         // q_I block
-  // MX tiles are half as large: twice the ring slots keep as many bytes in flight
-  static constexpr int kStages = MX ? 2 * Cfg<TOK>::kStages : Cfg<TOK>::kStages;
+  static constexpr bool MX = FMT != 0;
+  static constexpr int kRowB = FMT == 0 ? kDI * 2 : (FMT == 1 ? kDI : kDI / 2);
+  static constexpr int kTile = kBM * kRowB;                // one K_I tile
+  static constexpr int kB = TOK * kHI * kRowB;             // q_I block
+  // smaller tiles: more ring slots keep as many bytes in flight
+  static constexpr int kStages = Cfg<TOK>::kStages * (256 / kRowB);
   static constexpr int kChunk = Cfg<TOK>::kChunk;
   static constexpr int off_b = 0;
   static constexpr int off_a = kB;
@@ -844,12 +847,13 @@ __device__ void cluster_topk_emit(const float (&v)[R], const int32_t (&id)[R], i
   if (!solo) cluster_wait();   // no CTA leaves while another may still read its shared memory
 }
 
-template <int TOK, bool MX>
+template <int TOK, int FMT>
 __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k, TcIdxArgs a) {
-  static_assert(!MX || TOK == 1, "MX-FP8 operands: single-token groups");
-  using L = Smem<TOK, MX>;
+  constexpr bool MX = FMT != 0;
+  static_assert(!MX || TOK == 1, "MX operands: single-token groups");
+  using L = Smem<TOK, FMT>;
   constexpr int kStages = L::kStages;
   constexpr int kChunk = L::kChunk;
   constexpr int kTile = L::kTile;
@@ -1009,13 +1013,26 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
             const uint32_t sfa = tmem + kSfa + 4u * (uint32_t)buf;
             tmem_cp_32x128b_x4(sfa, smem_desc(smem_u32(sm + L::off_sf + s * 512), 16, 128, 0));
             const uint32_t sfb = tmem + kSfb;   // the token's own tile: heads on rows 0..63
+            if constexpr (FMT == 1) {
 #pragma unroll
-            for (int kk = 0; kk < kDI / 32; ++kk) {   // K = 32 per MMA, one scale each
-              const uint64_t ad = smem_desc(a_base + s * kTile + kk * 32, 16, 1024, 2);
-              const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, 2);
-              mma_mxf8_ss(d, ad, bd, idesc_mxf8_e4m3(kBM, kN, kk, kk),
-                          sfa | ((uint32_t)kk << 30), sfb | ((uint32_t)kk << 30),
-                          kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < kDI / 32; ++kk) {   // K = 32 per MMA, one scale each
+                const uint64_t ad = smem_desc(a_base + s * kTile + kk * 32, 16, 1024, 2);
+                const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, 2);
+                mma_mxf8_ss(d, ad, bd, idesc_mxf8_e4m3(kBM, kN, kk, kk),
+                            sfa | ((uint32_t)kk << 30), sfb | ((uint32_t)kk << 30),
+                            kk > 0 ? 1u : 0u);
+              }
+            } else {
+              // K = 64 per MMA (32 bytes of the 64-byte row), two scales each:
+              // bytes 2 kk and 2 kk + 1 of the scale words
+#pragma unroll
+              for (int kk = 0; kk < kDI / 64; ++kk) {
+                const uint64_t ad = smem_desc(a_base + s * kTile + kk * 32, 16, 512, 4);
+                const uint64_t bd = smem_desc(b_base + kk * 32, 16, 512, 4);
+                mma_mxf4_ss(d, ad, bd, idesc_mxf4_e2m1(kBM, kN, 2 * kk, 2 * kk),
+                            sfa | ((uint32_t)(2 * kk) << 30), sfb | ((uint32_t)(2 * kk) << 30),
+                            kk > 0 ? 1u : 0u);
+              }
             }
           } else {
 #pragma unroll
@@ -1735,13 +1752,16 @@ inline int n_chunks_for(int64_t N, int tok) {
   return n < 1 ? 1 : (int)n;
 }
 
-template <int TOK, bool MX = false>
+template <int TOK, int FMT = 0>
 cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t stream) {
   CUtensorMap mq, mk;
-  if constexpr (MX) {
-    if (!make_map_u8_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, kDI, TOK * kHI))
+  if constexpr (FMT != 0) {
+    constexpr uint32_t rb = Smem<TOK, FMT>::kRowB;
+    const CUtensorMapSwizzle swz = FMT == 1 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!make_map_u8_3d(&mq, p.q_I, rb, (uint64_t)p.Tq * kHI, (uint64_t)p.B, rb, TOK * kHI, swz))
       return cudaErrorInvalidValue;
-    if (!make_map_u8_3d(&mk, p.k_I, kDI, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, kDI, kBM))
+    if (!make_map_u8_3d(&mk, p.k_I, rb, (uint64_t)(p.N > 0 ? p.N : 1), (uint64_t)p.B, rb, kBM,
+                        swz))
       return cudaErrorInvalidValue;
   } else {
     if (!make_map_bf16_3d(&mq, p.q_I, kDI, (uint64_t)p.Tq * kHI, (uint64_t)p.B, 64, TOK * kHI))
@@ -1750,12 +1770,12 @@ cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t 
                           kBM))
       return cudaErrorInvalidValue;
   }
-  const int smem = Smem<TOK, MX>::bytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<TOK, MX>,
+  const int smem = Smem<TOK, FMT>::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<TOK, FMT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.n_chunks, (unsigned)((p.Tq + TOK - 1) / TOK), (unsigned)p.B);
-  indexer_tc_kernel<TOK, MX><<<grid, kThreads, smem, stream>>>(mq, mk, a);
+  indexer_tc_kernel<TOK, FMT><<<grid, kThreads, smem, stream>>>(mq, mk, a);
   return cudaGetLastError();
 }
 
@@ -1826,8 +1846,9 @@ size_t indexer_mx_scratch(int64_t B, int64_t Tq, int64_t N, int k) {
   return (size_t)B * (size_t)Tq * (size_t)nc * (size_t)k * 8;
 }
 
-cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const void* k_sf,
-                              cudaStream_t stream, unsigned long long* n_launch) {
+cudaError_t launch_indexer_mx(const IndexerParams& p, int fmt, const void* q_sf,
+                              const void* k_sf, cudaStream_t stream,
+                              unsigned long long* n_launch) {
   *n_launch = 0;
   if (p.B == 0 || p.Tq == 0) return cudaSuccess;
   if (p.N == 0) {   // nothing to score: every row is padding
@@ -1857,7 +1878,7 @@ cudaError_t launch_indexer_mx(const IndexerParams& p, const void* q_sf, const vo
     a.cand_score = static_cast<float*>(p.scratch);
     a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
   }
-  cudaError_t e = launch_tok<1, true>(p, a, stream);
+  cudaError_t e = fmt == 2 ? launch_tok<1, 2>(p, a, stream) : launch_tok<1, 1>(p, a, stream);
   if (e != cudaSuccess) return e;
   *n_launch = 1;
   if (a.n_chunks > 1) {

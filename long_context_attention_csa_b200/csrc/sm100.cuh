@@ -312,6 +312,35 @@ __device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// Instruction descriptor of kind::mxf4 with block scaling: E2M1 A and B
+// (packed, two per byte), K-major, UE8M0 scale factors (one per 32 K
+// elements, two per K = 64 MMA), fp32 D.  sf_a / sf_b select the first of
+// the two scale bytes this MMA uses (0 or 2).
+__host__ __device__ constexpr uint32_t idesc_mxf4_e2m1(int M, int N, uint32_t sf_a,
+                                                       uint32_t sf_b) {
+  return ((sf_b & 3u) << 4)             // B scale-factor byte
+         | (1u << 7)                    // A format: E2M1
+         | (1u << 10)                   // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | (1u << 23)                   // scale format: UE8M0
+         | ((uint32_t)(M >> 4) << 24)   // M / 16
+         | ((sf_a & 3u) << 29);         // A scale-factor byte
+}
+
+// D[tmem] (+)= block-scaled E2M1 A x E2M1 B^T (K = 64 per MMA, a UE8M0 scale
+// per 32 elements from TMEM).
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa),
+      "r"(sfb)
+      : "memory");
+}
+
 // Copies 32 rows x 16 bytes from shared memory (rows contiguous: the
 // descriptor's 8-row groups 128 bytes apart, no swizzle) into TMEM lanes
 // 0..31, columns taddr .. taddr + 3, and the same into each of the other three

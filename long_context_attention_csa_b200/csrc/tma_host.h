@@ -46,10 +46,11 @@ inline bool make_map_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, ui
 }
 
 // 3-D 8-bit tensor [d2][d1][d0] (d0 innermost, contiguous, a multiple of 16),
-// box {b0, b1, 1} with b0 <= 128 bytes, 128-byte swizzle, out-of-range
-// elements read as 0.
+// box {b0, b1, 1} with b0 bytes equal to the swizzle span (128 by default, or
+// 64), out-of-range elements read as 0.
 inline bool make_map_u8_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
-                           uint64_t d2, uint32_t b0, uint32_t b1) {
+                           uint64_t d2, uint32_t b0, uint32_t b1,
+                           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {d0, d1, d2};
@@ -57,7 +58,7 @@ inline bool make_map_u8_3d(CUtensorMap* map, const void* base, uint64_t d0, uint
   cuuint32_t box[3] = {b0, b1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -272,3 +272,14 @@ def test_mixed_storage_rejects_bad_arguments(L):
     fm = _fmt(r=60, flags=8)
     assert L.dense_hca_attn(1, 1, 4, 64, ctypes.byref(fm), d, None, d, 16, 4, d, 8, None, 8,
                             None, 0.0, d, None, 0, None) == 2
+
+
+def test_mxfp4_calls_reject_bad_arguments(L):
+    d = ctypes.c_void_p(4096)
+    assert L.indexer_mxfp4_quantize(1, 1, 8, 64, d, d, d, None) == 2
+    assert L.indexer_mxfp4_quantize(1, 0, 8, 128, None, None, None, None) == 0
+    assert L.indexer_scores_topk_mxfp4(1, 1, 32, 128, d, d, d, d, d, 64, None, 4, 8, d, None, d,
+                                       1 << 20, None) == 2
+    assert L.indexer_scores_topk_mxfp4(1, 1, 64, 128, d, d, d, d, d, 64, None, 4, 8, d, None,
+                                       None, 0, None) == 5
+

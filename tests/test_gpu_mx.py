@@ -123,3 +123,100 @@ def test_mxfp8_indexer_decode_workload():
                            w.k, w.m, q_pos=p)
         recall.append(len(np.intersect1d(gi[v], full[full >= 0])) / max(1, (full >= 0).sum()))
     assert np.mean(recall) >= 0.95, recall
+
+
+# ----------------------------------------------------------------- MX-FP4
+
+def unpack_fp4(codes):
+    """Packed [..., 64] bytes -> [..., 128] 4-bit codes (even element in the
+    low nibble)."""
+    c = codes.cpu().numpy()
+    out = np.empty(c.shape[:-1] + (c.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = c & 0xF
+    out[..., 1::2] = c >> 4
+    return out
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_mxfp4_quantize_matches_the_oracle(dtype):
+    """Packed E2M1 codes and scale exponents equal the oracle's MX-FP4
+    quantizer's, bit for bit (random rows, a zero block, tiny values, values
+    that saturate at 6, a ragged last tile)."""
+    B, rows = 2, 300
+    x = wl.randn((B, rows, 128), 521, DEV, dtype=torch.float32) * 3
+    x[0, 5, 32:64] = 0
+    x[0, 6, :32] = x[0, 6, :32] * 1e-30
+    x[1, 7, 64:96] = torch.linspace(-7, 7, 32)
+    x[1, 8, :] = torch.linspace(-3, 3, 128)
+    x = x.to(dtype)
+    codes, sf = csa.indexer_mxfp4_quantize(x)
+    torch.cuda.synchronize()
+    assert codes.shape == (B, rows, 64)
+    ex, pad = unpack_scales(sf, rows)
+    assert np.all(pad == 0)
+    got = unpack_fp4(codes)
+    for b in range(B):
+        rc, re = oracle.mxfp4_quantize(f64(x[b]))
+        assert np.array_equal(got[b], rc), f"codes b={b}"
+        assert np.array_equal(ex[b], re), f"exponents b={b}"
+
+
+@pytest.mark.parametrize("B,Tq,N,k", [(3, 1, 30000, 1024), (1, 37, 700, 64)])
+def test_mxfp4_indexer_integer_inputs_bit_exact(B, Tq, N, k):
+    """Integers in [-2, 2] quantize exactly to E2M1 (scale 2^-1: codes up to 4)
+    and every product and sum is exact in float32: sets and scores equal the
+    oracle's."""
+    HI, dI, m = 64, 128, 4
+    qI = wl.randint_like_float((B, Tq, HI, dI), 531, -2, 3, DEV, torch.bfloat16)
+    kI = wl.randint_like_float((B, N, dI), 532, -2, 3, DEV, torch.bfloat16)
+    w = wl.randint_like_float((B, Tq, HI), 533, -2, 3, DEV, torch.float32)
+    if Tq == 1:
+        q_pos = torch.tensor([[m * N - 1], [m * (N // 3) + 2], [m * 200]], dtype=torch.int64)[:B]
+    else:
+        q_pos = torch.arange(Tq, dtype=torch.int64).unsqueeze(0) * 70 + 5
+    qc, qs = csa.indexer_mxfp4_quantize(qI, per_token=True)
+    kc, ks = csa.indexer_mxfp4_quantize(kI)
+    idx, sc = csa.indexer_scores_topk_mxfp8(qc, qs, w, kc, ks, m, k, q_pos=q_pos.to(DEV),
+                                            want_scores=True)
+    torch.cuda.synchronize()
+    for b in range(B):
+        p = q_pos[b].numpy()
+        ref_sc = oracle.mxfp4_indexer_scores(f64(qI[b]), f64(w[b]), f64(kI[b]), m, q_pos=p)
+        assert np.array_equal(ref_sc, oracle.indexer_scores(f64(qI[b]), f64(w[b]), f64(kI[b]), m,
+                                                            q_pos=p))
+        ref_idx = oracle.topk(ref_sc, k, m, q_pos=p)
+        gi = idx[b].cpu().numpy()
+        assert np.array_equal(gi, ref_idx), f"b={b}"
+        v = gi >= 0
+        assert np.array_equal(sc[b].cpu().numpy().astype(np.float64)[v],
+                              np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v])
+
+
+def test_mxfp4_indexer_decode_workload():
+    """Eight rows of the csa_decode_b32_128k workload with N(0,1) operands in
+    MX-FP4: scores within 1e-4 of the oracle's MX-FP4 scores, sets equal up
+    to the tie band, and recall of the full-precision selection >= 90%."""
+    w = wl.scaled(wl.WORKLOADS["csa_decode_b32_128k"], B=8)
+    inp = wl.csa_decode_inputs(w, DEV)
+    qc, qs = csa.indexer_mxfp4_quantize(inp["q_I"], per_token=True)
+    kc, ks = csa.indexer_mxfp4_quantize(inp["k_I"])
+    idx, sc = csa.indexer_scores_topk_mxfp8(qc, qs, inp["w"], kc, ks, w.m, w.k,
+                                            q_pos=inp["q_pos"], want_scores=True)
+    torch.cuda.synchronize()
+    recall = []
+    for b in range(w.B):
+        p = inp["q_pos"][b].cpu().numpy()
+        ref_sc = oracle.mxfp4_indexer_scores(f64(inp["q_I"][b]), f64(inp["w"][b]),
+                                             f64(inp["k_I"][b]), w.m, q_pos=p)
+        ref_idx = oracle.topk(ref_sc, w.k, w.m, q_pos=p)
+        gi = idx[b].cpu().numpy()
+        check_topk_rows(gi, ref_idx, ref_sc, what=f"mx4 b={b}")
+        v = gi >= 0
+        gs = sc[b].cpu().numpy().astype(np.float64)[v]
+        want = np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v]
+        assert (np.abs(gs - want) / np.maximum(1.0, np.abs(want))).max() <= 1e-4
+        full = oracle.topk(oracle.indexer_scores(f64(inp["q_I"][b]), f64(inp["w"][b]),
+                                                 f64(inp["k_I"][b]), w.m, q_pos=p),
+                           w.k, w.m, q_pos=p)
+        recall.append(len(np.intersect1d(gi[v], full[full >= 0])) / max(1, (full >= 0).sum()))
+    assert np.mean(recall) >= 0.90, recall
