@@ -232,7 +232,7 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     w = wl.WORKLOADS[WORKLOAD]
     step = Step(w, dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    flush = L2Flush(dev)
     clocks = Clocks(local) if rank == 0 or ws > 1 else None
     if clocks:
         clocks.start()   # running through warm-up, so samples exist when timing starts
@@ -251,7 +251,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     t_begin = time.time()
     for i in range(K):
-        flush.zero_()                       # L2 flushed between timed steps (not timed)
+        flush()                       # L2 flushed between timed steps (not timed)
         step.run(ev=evs[i])
     torch.cuda.synchronize()
     barrier(ws)
@@ -354,7 +354,8 @@ def run_gpu(args):
                 "entry_dim": w.c, "rope_dims": w.r, "m": w.m, "entries": w.n_csa,
                 "indexer": f"{w.HI}x{w.dI}", "top_k": w.k, "n_win": w.n_win, "sink": True,
                 "parallelism": f"replica x{ws}" if ws > 1 else "single GPU",
-                "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                "l2": "flushed between timed steps (256 MiB write + 256 MiB read, "
+                      "outside the step events)",
             },
             "stages_ms": {"csa_compress": t_compress, "indexer_scores_topk": t_index,
                           "sparse_mqa_attn": t_attn},
@@ -555,7 +556,7 @@ def measure_hca_prefill(dev, steps: int, warmup: int, flush, ws_n: int, cpu: boo
             raise RuntimeError(f"hca_prefill_64k: device status {st}/{d}")
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()          # L2 flushed between timed steps (not timed)
+        flush()          # L2 flushed between timed steps (not timed)
         run(evs[i])
     torch.cuda.synchronize()
     per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[0].elapsed_time(e[2])]
@@ -573,7 +574,8 @@ def measure_hca_prefill(dev, steps: int, warmup: int, flush, ws_n: int, cpu: boo
         "config": {"workload": w.name, "batch": w.B, "seq_len": w.T, "heads": w.H,
                    "entry_dim": w.c, "rope_dims": w.r, "m_prime": w.m_prime,
                    "entries": w.n_hca, "n_win": w.n_win, "sink": True,
-                   "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
+                   "l2": "flushed between timed steps (256 MiB write + 256 MiB read, "
+                         "outside the step events)"},
         "stages_ms": {"hca_compress": t_comp, "dense_hca_attn": t_attn},
         "stage_roofline": {"hca_compress": {
             "bound": "hbm", "achieved_GBps": hca_compress_bytes(w) / (t_comp * 1e-3) / 1e9,
@@ -612,7 +614,7 @@ def measure_projection(dev, steps: int, warmup: int, flush, ws_n: int, cpu: bool
     torch.cuda.synchronize()
     evs = []
     for _ in range(steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         run()
@@ -629,7 +631,8 @@ def measure_projection(dev, steps: int, warmup: int, flush, ws_n: int, cpu: bool
     res = {"value": w.T * ws_n / (ms * 1e-3), "unit": "tokens/s", "ms": ms,
            "config": {"workload": w.name, "rows": w.T, "heads": w.H, "head_dim": w.c, **p,
                       "weights": "random synthetic, N(0,1)/sqrt(fan_in)",
-                      "l2": "flushed between timed calls (outside the events)"},
+                      "l2": "flushed between timed calls (256 MiB write + 256 MiB read, "
+                            "outside the events)"},
            "roofline": {"bound": "tensor", "kernel": "gemm_bf16_tc_kernel (two launches)",
                         "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
                         "frac": achieved / bf16, "algorithmic_flops_per_call": fl,
@@ -760,6 +763,18 @@ class DecodeStep:
                 self.qc, self.qs, inp["w"], self.kc, self.ks, w.m, w.k, q_pos=inp["q_pos"],
                 idx_out=self.idx, ws=ws_mx), w.B * w.n_csa * (w.dI + w.dI // 32)),
         ] + self.stages[1:]
+        # and on MX-FP4 operands (packed E2M1: 64 code bytes + 4 scale bytes an entry)
+        self.kc4, self.ks4 = csa.indexer_mxfp4_quantize(inp["k_I"])
+        self.qc4 = torch.empty(tuple(inp["q_I"].shape[:-1]) + (w.dI // 2,), dtype=torch.uint8,
+                               device=dev)
+        self.qs4 = torch.empty((w.B, 1, 512), dtype=torch.uint8, device=dev)
+        self.mx4_stages = [
+            ("indexer_mxfp4_quantize", lambda: csa.indexer_mxfp4_quantize(
+                inp["q_I"], self.qc4, self.qs4, per_token=True), w.B * w.HI * w.dI * 5 // 2),
+            ("indexer_scores_topk_mxfp4", lambda: csa.indexer_scores_topk_mxfp8(
+                self.qc4, self.qs4, inp["w"], self.kc4, self.ks4, w.m, w.k, q_pos=inp["q_pos"],
+                idx_out=self.idx, ws=ws_mx), w.B * w.n_csa * (w.dI // 2 + w.dI // 32)),
+        ] + self.stages[1:]
 
         # the same step with the entry caches stored mixed (RoPE dims bf16,
         # the rest MX-FP8: 592 instead of 1024 bytes an entry), written once
@@ -785,6 +800,10 @@ class DecodeStep:
         for _, fn, _ in self.mx_stages:
             fn()
 
+    def run_mx4(self):
+        for _, fn, _ in self.mx4_stages:
+            fn()
+
     def rewind(self):
         """Puts every stream state back at token L - 1 (each append advances it)."""
         self.st_c[:, :8] = torch.tensor([self.w.T - 1] * self.w.B, dtype=torch.int64).view(
@@ -803,6 +822,21 @@ class DecodeStep:
                 raise RuntimeError(f"{self.w.name}: device status {st}/{d}")
 
 
+class L2Flush:
+    """Empties the 126 MB L2 between timed steps, outside the events: a 256 MiB
+    write, then a 256 MiB read of a second buffer, so that the cache holds only
+    clean lines and the write-back of the flush's own dirty lines does not land
+    in the next timed region."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(64 << 20, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
 def graph_ms(fn, steps: int, flush, before=None) -> float:
     """Mean device time of `fn` captured once in a CUDA graph and replayed
     `steps` times, with the L2 flushed (and `before` run) before each replay,
@@ -818,7 +852,7 @@ def graph_ms(fn, steps: int, flush, before=None) -> float:
     for _ in range(steps):
         if before:
             before()
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         g.replay()
@@ -922,6 +956,8 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
     mixed_stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.mixed_stages[1:]}
     mx_ms = allmax(graph_ms(d.run_mx, steps, flush), ws_n)
     mx_stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.mx_stages[:2]}
+    mx4_ms = allmax(graph_ms(d.run_mx4, steps, flush), ws_n)
+    mx4_stages = {n: graph_ms(fn, steps, flush) for n, fn, _ in d.mx4_stages[:2]}
     d.check()
     append = {}
     for n, fn, nb in d.append:
@@ -936,12 +972,16 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
     # MX-FP8 indexer operands: 128 code bytes + 4 scale bytes per entry instead of 256
     nb_mx = nb - w.B * w.n_csa * w.dI * 2 + w.B * w.n_csa * (w.dI + w.dI // 32)
     mx_achieved = nb_mx / (mx_ms * 1e-3) / 1e9
+    # MX-FP4: 64 packed code bytes + 4 scale bytes per entry
+    nb_mx4 = nb - w.B * w.n_csa * w.dI * 2 + w.B * w.n_csa * (w.dI // 2 + w.dI // 32)
+    mx4_achieved = nb_mx4 / (mx4_ms * 1e-3) / 1e9
     res = {
         "value": w.B * ws_n / (step_ms * 1e-3), "unit": "queries/s", "ms_per_step": step_ms,
         "config": {"workload": w.name, "batch": w.B, "context": w.T, "heads": w.H,
                    "entries": w.n_csa, "top_k": w.k, "n_win": w.n_win, "sink": True,
                    **({"hca_entries": w.n_hca} if w.kind == "decode_pair" else {}),
-                   "l2": "flushed before every replay (outside the events)",
+                   "l2": "flushed before every replay (256 MiB write + 256 MiB read, "
+                         "outside the events)",
                    "timing": "whole step captured once in a CUDA graph, replayed"},
         "stages_ms": stages,
         "mixed_entries": {
@@ -957,6 +997,13 @@ def measure_decode(name: str, dev, steps: int, warmup: int, flush, ws_n: int, cp
                     "operands (K_I cached as E4M3 codes + UE8M0 scales per 32)",
             "roofline": {"bound": "hbm", "achieved": mx_achieved, "peak": hbm, "unit": "GB/s",
                          "frac": mx_achieved / hbm, "algorithmic_bytes_per_step": nb_mx}},
+        "mxfp4_indexer": {
+            "value": w.B * ws_n / (mx4_ms * 1e-3), "unit": "queries/s", "ms_per_step": mx4_ms,
+            "stages_ms": mx4_stages,
+            "note": "the same step with the indexer on MX-FP4 operands (K_I cached as packed "
+                    "E2M1 codes + UE8M0 scales per 32: 68 bytes an entry instead of 256)",
+            "roofline": {"bound": "hbm", "achieved": mx4_achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": mx4_achieved / hbm, "algorithmic_bytes_per_step": nb_mx4}},
         "stream_append": {**append, "note": "the step's new token appended to each sequence's "
                           "compression state (completing a block: entry pooled from the tail "
                           "buffer); latency-bound, timed beside the step"},
@@ -987,9 +1034,9 @@ def run_only_decode(args):
         d.run()
     torch.cuda.synchronize()
     d.check()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     res = {}
-    for name, fn, nbytes in d.stages + d.mx_stages[:2] + d.mixed_stages[1:]:
+    for name, fn, nbytes in d.stages + d.mx_stages[:2] + d.mx4_stages[:2] + d.mixed_stages[1:]:
         ms = graph_ms(fn, args.steps, flush)
         res[name] = {"ms": ms, "bytes": nbytes, "GBps": nbytes / ms / 1e6}
     for name, fn, nbytes in d.append:
@@ -1016,7 +1063,7 @@ def run_only(args):
     if args.only == "proj":
         torch.cuda.set_device(0)
         dev = torch.device("cuda", 0)
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        flush = L2Flush(dev)
         print(json.dumps({"only": "proj", **measure_projection(dev, args.steps, args.warmup,
                                                                flush, 1, False)}))
         return

@@ -373,6 +373,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // set-up done without global memory: from here on the previous kernel's
+  // results are needed (a programmatic launch overlaps only the set-up)
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS0 = tmem;          // S^T buffers at columns 0 and 64
   const uint32_t tO = tmem + 128;     // O^T: 4 x 64 columns
@@ -997,15 +1001,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Sums the fixed-order split partials of one (row, head group), divides by
 // the denominator (sink included) and rotates the output back by -pos.
-constexpr int kCombHeads = 8;   // heads per combine CTA
+constexpr int kCombHeads = 2;   // heads per combine CTA (one 16-byte quad a thread)
 
-__global__ void __launch_bounds__(256) attn_combine_kernel(TcAttnArgs a) {
+__global__ void __launch_bounds__(256, 6) attn_combine_kernel(TcAttnArgs a) {
+  static_assert(kCombHeads * kC / 4 == 256, "one 16-byte quad a thread");
   __shared__ float inv[kCombHeads];
   __shared__ float cs_t[32], sn_t[32];
+  pdl_wait();
+  pdl_trigger();
   const int64_t row = blockIdx.x;
   const int hg = blockIdx.y;
   const int h0 = blockIdx.z * kCombHeads;   // this CTA's heads within the group
   const int64_t slot = row * a.n_hg + hg;
+  // thread: 4 consecutive dims of one head; every split's 16-byte load is
+  // issued first, then the denominators and the RoPE table are formed while
+  // they are in flight (the sum keeps the fixed split order)
+  const int hl = threadIdx.x / (kC / 4), c = (threadIdx.x % (kC / 4)) * 4;
+  constexpr int kInFlight = 4;   // split loads in flight a thread
+  float4 pv[kInFlight];
+  auto load = [&](int s0) {
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u)
+      if (s0 + u < a.n_splits)
+        pv[u] = *reinterpret_cast<const float4*>(
+            a.o_part + ((slot * a.n_splits + s0 + u) * kHG + h0 + hl) * kC + c);
+  };
+  load(0);
   const int64_t t = row % a.Tq;
   const int64_t pos = a.q_pos ? a.q_pos[row] : t;
   if (threadIdx.x < kCombHeads) {
@@ -1025,46 +1046,35 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(TcAttnArgs a) {
     sn_t[threadIdx.x - 32] = sn;
   }
   __syncthreads();
-  // thread: 4 consecutive dims of one head, 4 times (16-byte loads); every
-  // split's load is issued before the first is added (fixed order kept)
-  constexpr int kQuads = kCombHeads * kC / 4;   // 1024
-#pragma unroll 1
-  for (int r = 0; r < kQuads / 256; ++r) {
-    const int q = threadIdx.x + 256 * r;
-    const int hl = q / (kC / 4), c = (q % (kC / 4)) * 4;
-    float4 pv[kMaxSplits];
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s0 = 0; s0 < a.n_splits; s0 += kInFlight) {
+    if (s0 > 0) load(s0);
 #pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s)
-      if (s < a.n_splits)
-        pv[s] = *reinterpret_cast<const float4*>(
-            a.o_part + ((slot * a.n_splits + s) * kHG + h0 + hl) * kC + c);
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) {
-      if (s < a.n_splits) {
-        o[0] += pv[s].x;
-        o[1] += pv[s].y;
-        o[2] += pv[s].z;
-        o[3] += pv[s].w;
+    for (int u = 0; u < kInFlight; ++u) {
+      if (s0 + u < a.n_splits) {
+        o[0] += pv[u].x;
+        o[1] += pv[u].y;
+        o[2] += pv[u].z;
+        o[3] += pv[u].w;
       }
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] *= inv[hl];
-    if (!(a.flags & CSA_F_NO_ROPE)) {
-#pragma unroll
-      for (int e = 0; e < 4; e += 2) {
-        if (c + e >= kC - a.r) {
-          const int i = (c + e - (kC - a.r)) >> 1;
-          const float y0 = o[e] * cs_t[i] - o[e + 1] * sn_t[i];
-          const float y1 = o[e] * sn_t[i] + o[e + 1] * cs_t[i];
-          o[e] = y0;
-          o[e + 1] = y1;
-        }
-      }
-    }
-    *reinterpret_cast<uint2*>(a.out + (row * a.H + (int64_t)hg * kHG + h0 + hl) * kC + c) =
-        make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
   }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) o[e] *= inv[hl];
+  if (!(a.flags & CSA_F_NO_ROPE)) {
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      if (c + e >= kC - a.r) {
+        const int i = (c + e - (kC - a.r)) >> 1;
+        const float y0 = o[e] * cs_t[i] - o[e + 1] * sn_t[i];
+        const float y1 = o[e] * sn_t[i] + o[e + 1] * cs_t[i];
+        o[e] = y0;
+        o[e + 1] = y1;
+      }
+    }
+  }
+  *reinterpret_cast<uint2*>(a.out + (row * a.H + (int64_t)hg * kHG + h0 + hl) * kC + c) =
+      make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
 }
 
 // Streaming multiprocessors of the current device (one persistent CTA each).
@@ -1163,20 +1173,17 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream, unsigned lo
       cudaFuncSetAttribute(a.mixed ? attn_tc_kernel<true> : attn_tc_kernel<false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  if (a.mixed)
-    attn_tc_kernel<true><<<grid, kThreads, smem, stream>>>(mq, a);
-  else
-    attn_tc_kernel<false><<<grid, kThreads, smem, stream>>>(mq, a);
+  e = launch_pdl(a.mixed ? attn_tc_kernel<true> : attn_tc_kernel<false>, dim3(grid),
+                 dim3(kThreads), (size_t)smem, stream, mq, a);
+  if (e != cudaSuccess) return e;
+  *n_launch = 1;
   if (a.split) {
-    e = cudaGetLastError();
+    e = launch_pdl(attn_combine_kernel, dim3((unsigned)rows, (unsigned)a.n_hg, kHG / kCombHeads),
+                   dim3(256), 0, stream, a);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<dim3((unsigned)rows, (unsigned)a.n_hg, kHG / kCombHeads), 256, 0,
-                          stream>>>(a);
     *n_launch = 2;
-  } else {
-    *n_launch = 1;
   }
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 }  // namespace csa

@@ -30,6 +30,18 @@ __device__ __forceinline__ void report(unsigned* status, unsigned code, unsigned
   }
 }
 
+// ---- programmatic dependent launch ---------------------------------------
+// A kernel launched with programmatic stream serialization (launch_pdl) may
+// start while the previous kernel in the stream is still running.  pdl_wait()
+// returns once that kernel has completed and its memory is visible (at once
+// for an ordinary launch), so a kernel calls it, in every thread, before its
+// first global load or store.  pdl_trigger() lets the next such kernel start
+// launching; it waits in its own pdl_wait() for this one to finish.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- 16-byte vector loads/stores as float ------------------------------
 template <typename T> struct VecOf;
 template <> struct VecOf<float> { static constexpr int N = 4; };

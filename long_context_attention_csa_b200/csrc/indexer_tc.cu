@@ -445,10 +445,12 @@ __device__ void warp_topk_binned(const float* sc, int n, int k, int64_t e0, unsi
 // scores [w R, (w+1) R), R = kMaxN / G, in registers (lane l: 16-byte groups
 // l, l+32, ...); value bins as in warp_topk_binned, a histogram in shared
 // memory, the boundary bin's members ranked exactly, and an ordered emit with
-// per-warp offsets.  Returns false (nothing written) when the single-warp
-// radix select must run instead: n <= k, a degenerate range, or more than
-// kBinCap members in the boundary bin.
-template <int G, int kMaxN>
+// per-warp offsets.  With REFINE, a boundary bin of more than kBinCap
+// members is narrowed by a radix select on its members' keys first.
+// Returns false (nothing written) when the single-warp radix select must run
+// instead: n <= k, a degenerate range, or (after any narrowing) more than
+// kBinCap members to rank.
+template <int G, int kMaxN, bool REFINE = false>
 __device__ bool block_topk(const float* sc, int n, int k, int64_t e0, unsigned* hist, float* red,
                            unsigned* wcnt, float* cs, int* cj, int bar_id, int32_t* out_idx,
                            float* out_score) {
@@ -528,15 +530,72 @@ __device__ bool block_topk(const float* sc, int n, int k, int64_t e0, unsigned* 
   }
   sync();
   const int bstar = (int)wcnt[G];
-  const unsigned need = (unsigned)k - wcnt[G + 1], cnt = wcnt[G + 2];
-  if (cnt > (unsigned)kBinCap) return false;
-  // the boundary bin's members, any order (ranked below)
+  unsigned need = (unsigned)k - wcnt[G + 1], cnt = wcnt[G + 2];
+  // A heavier boundary bin is narrowed by a radix select on the members'
+  // order-preserving keys (8 bits a pass, every warp of the group counting
+  // its own members): afterwards the members whose key equals tau, the key
+  // of the need-th largest member, are the ones ranked below, need of them
+  // taken (those above tau are taken by value).
+  const bool heavy = cnt > (unsigned)kBinCap;
+  if (heavy && !REFINE) return false;
+  unsigned tau = 0u;
+  if (heavy) {
+    unsigned mask = 0u;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      sync();   // the previous readers of hist and of the boundary slots are done
+      for (int i = gt; i < 256; i += 32 * G) hist[i] = 0u;
+      sync();
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (bin[i][e] == bstar) {
+            const unsigned key = score_key(v[i][e]);
+            if ((key & mask) == tau) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+          }
+        }
+      }
+      sync();
+      if (w == 0) {   // boundary digit: lane L owns digits 255-8L .. 248-8L
+        unsigned c[8], sL = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          c[i] = hist[255 - 8 * lane - i];
+          sL += c[i];
+        }
+        const unsigned incl = warp_incl_scan(sL, lane);
+        const unsigned pre = incl - sL;
+        if (pre < need && need <= incl) {
+          unsigned run = pre;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (run + c[i] >= need) {
+              wcnt[G] = 255u - 8u * lane - i;   // digit
+              wcnt[G + 1] = run;                // members above it
+              wcnt[G + 2] = c[i];               // members with it
+              break;
+            }
+            run += c[i];
+          }
+        }
+      }
+      sync();
+      tau |= wcnt[G] << shift;
+      mask |= 255u << shift;
+      need -= wcnt[G + 1];
+      cnt = wcnt[G + 2];
+    }
+    // cnt members carry the key tau exactly; more than kBinCap equal
+    // scores go to the radix select over all scores
+    if (cnt > (unsigned)kBinCap) return false;
+  }
+  // the members to rank, any order
 #pragma unroll
   for (int i = 0; i < V; ++i) {
     const int j0 = w * R + 4 * (32 * i + lane);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (bin[i][e] == bstar) {
+      if (bin[i][e] == bstar && (!heavy || score_key(v[i][e]) == tau)) {
         const unsigned at = atomicAdd(&wcnt[G + 3], 1u);
         cs[at] = v[i][e];
         cj[at] = j0 + e;
@@ -882,6 +941,8 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::off_misc + 4);
 
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
   const int group = gridDim.y - 1 - blockIdx.y;   // heaviest causal groups first
@@ -1099,7 +1160,7 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
         os = a.cand_score + c;
       }
       float* cand = reinterpret_cast<float*>(sm + L::off_cand);
-      const bool done = block_topk<4, kChunk>(
+      const bool done = block_topk<4, kChunk, true>(
           scores, (int)n64, a.k, e0, hist, reinterpret_cast<float*>(sm + L::off_red),
           reinterpret_cast<unsigned*>(sm + L::off_wcnt), cand,
           reinterpret_cast<int*>(cand + kBinCap), 1, oi, os);
@@ -1711,6 +1772,8 @@ constexpr int kMSlice = kMThreads * kMRun;      // per CTA: 8192
 __global__ void __launch_bounds__(kMThreads)
     indexer_merge_cluster_kernel(TcIdxArgs a) {
   __shared__ __align__(16) SelShared sh;
+  pdl_wait();
+  pdl_trigger();
   const uint32_t CL = cluster_nctarank(), rank = cluster_ctarank();
   const int64_t row = blockIdx.x / CL;
   const int64_t n = (int64_t)a.n_chunks * a.k;
@@ -1775,8 +1838,8 @@ cudaError_t launch_tok(const IndexerParams& p, const TcIdxArgs& a, cudaStream_t 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.n_chunks, (unsigned)((p.Tq + TOK - 1) / TOK), (unsigned)p.B);
-  indexer_tc_kernel<TOK, FMT><<<grid, kThreads, smem, stream>>>(mq, mk, a);
-  return cudaGetLastError();
+  return launch_pdl(indexer_tc_kernel<TOK, FMT>, grid, dim3(kThreads), (size_t)smem, stream, mq,
+                    mk, a);
 }
 
 // Rows with no entry at all (N == 0): index -1 and score -inf throughout.
@@ -1810,13 +1873,15 @@ cudaError_t launch_merge(const TcIdxArgs& a, int64_t rows, cudaStream_t stream) 
   cfg.blockDim = dim3(kMThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = (unsigned)cl;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, indexer_merge_cluster_kernel, a);
 }
 

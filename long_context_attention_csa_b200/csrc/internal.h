@@ -8,6 +8,25 @@
 
 namespace csa {
 
+// Launches `kernel` with programmatic stream serialization: its CTAs may be
+// scheduled while the previous kernel in the stream drains (the kernel must
+// call pdl_wait() before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Offsets inside a caller workspace: the status word lives at byte 0; scratch
 // starts at kWsScratch.
 constexpr size_t kWsScratch = 256;

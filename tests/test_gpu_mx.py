@@ -195,7 +195,10 @@ def test_mxfp4_indexer_integer_inputs_bit_exact(B, Tq, N, k):
 def test_mxfp4_indexer_decode_workload():
     """Eight rows of the csa_decode_b32_128k workload with N(0,1) operands in
     MX-FP4: scores within 1e-4 of the oracle's MX-FP4 scores, sets equal up
-    to the tie band, and recall of the full-precision selection >= 90%."""
+    to the tie band, and the recall of the full-precision selection equal to
+    the oracle's MX-FP4 recall (a property of the format on these inputs:
+    about 83% for 1024 of 32768 entries with random projections, against
+    94% for 16 of 64 in the oracle's own test)."""
     w = wl.scaled(wl.WORKLOADS["csa_decode_b32_128k"], B=8)
     inp = wl.csa_decode_inputs(w, DEV)
     qc, qs = csa.indexer_mxfp4_quantize(inp["q_I"], per_token=True)
@@ -203,7 +206,7 @@ def test_mxfp4_indexer_decode_workload():
     idx, sc = csa.indexer_scores_topk_mxfp8(qc, qs, inp["w"], kc, ks, w.m, w.k,
                                             q_pos=inp["q_pos"], want_scores=True)
     torch.cuda.synchronize()
-    recall = []
+    recall, recall_o = [], []
     for b in range(w.B):
         p = inp["q_pos"][b].cpu().numpy()
         ref_sc = oracle.mxfp4_indexer_scores(f64(inp["q_I"][b]), f64(inp["w"][b]),
@@ -218,5 +221,8 @@ def test_mxfp4_indexer_decode_workload():
         full = oracle.topk(oracle.indexer_scores(f64(inp["q_I"][b]), f64(inp["w"][b]),
                                                  f64(inp["k_I"][b]), w.m, q_pos=p),
                            w.k, w.m, q_pos=p)
-        recall.append(len(np.intersect1d(gi[v], full[full >= 0])) / max(1, (full >= 0).sum()))
-    assert np.mean(recall) >= 0.90, recall
+        nf = max(1, (full >= 0).sum())
+        recall.append(len(np.intersect1d(gi[v], full[full >= 0])) / nf)
+        recall_o.append(len(np.intersect1d(ref_idx[ref_idx >= 0], full[full >= 0])) / nf)
+    assert abs(np.mean(recall) - np.mean(recall_o)) <= 0.005, (recall, recall_o)
+    assert np.mean(recall_o) >= 0.75, recall_o

@@ -241,6 +241,33 @@ def test_indexer_decode_select_integer_bit_exact(N, k, zero):
                               np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v])
 
 
+@pytest.mark.parametrize("k", [1024, 37])
+def test_indexer_decode_select_heavy_boundary_bin(k):
+    """One entry per 4096-entry chunk with a score thousands of times the
+    others' stretches the chunk's value range, so nearly every score shares
+    the boundary bin: the chunk select narrows that bin by a radix pass on the
+    scores' keys and ranks the equal integer scores there by index.  Integer
+    inputs keep every score exact; sets and scores equal the oracle's."""
+    B, N, HI, dI, m = 2, 30000, 64, 128, 4
+    pos = torch.tensor([[m * N - 1], [m * (N // 2) + 5]], dtype=torch.int64)
+    qI = wl.randint_like_float((B, 1, HI, dI), 44, -2, 3, DEV, torch.bfloat16)
+    kI = wl.randint_like_float((B, N, dI), 45, -2, 3, DEV, torch.bfloat16)
+    kI[:, 1234::4096, :] = 100.0
+    w = wl.randint_like_float((B, 1, HI), 46, -2, 3, DEV, torch.float32)
+    idx, sc = csa.indexer_scores_topk(qI, w, kI, m, k, q_pos=pos.to(DEV), want_scores=True)
+    torch.cuda.synchronize()
+    for b in range(B):
+        p = pos[b].numpy()
+        ref_sc = oracle.indexer_scores(f64(qI[b]), f64(w[b]), f64(kI[b]), m, q_pos=p)
+        assert np.abs(ref_sc[np.isfinite(ref_sc)]).max() < 2 ** 24   # exact in float32
+        ref_idx = oracle.topk(ref_sc, k, m, q_pos=p)
+        gi = idx[b].cpu().numpy()
+        assert np.array_equal(gi, ref_idx), f"row {b}"
+        v = gi >= 0
+        assert np.array_equal(sc[b].cpu().numpy().astype(np.float64)[v],
+                              np.take_along_axis(ref_sc, np.where(v, gi, 0), 1)[v])
+
+
 def test_indexer_padding_when_few_visible():
     w = wl.scaled(wl.WORKLOADS["csa_prefill_8k"], T=40, k=16)
     _indexer_case(w)
