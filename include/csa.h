@@ -244,9 +244,11 @@ csa_status indexer_scores_topk(int32_t dtype, int64_t B, int64_t Tq, int32_t H_I
  * __device__ array inside libcsa.so that every GPU loading the library holds
  * until exit.  A call is accepted iff 256 (the status word) + the scratch of
  * the kernels it takes <= 8 MiB, else CSA_E_WORKSPACE: bf16 (tensor cores)
- * needs 8 * B * Tq * k * n_chunks bytes when the entries span n_chunks > 1
- * chunks of 2048 (Tq >= 4) or 4096 (Tq < 4) entries, and none otherwise;
- * float32 (CUDA cores) needs 4 * B * Tq * N bytes.  For bf16 this equals
+ * needs, when the entries span n_chunks > 1 chunks of 2048 (Tq >= 4) or 4096
+ * (Tq < 4) entries, 4 * B * Tq * 4096 * n_chunks bytes for Tq < 4 and
+ * n_chunks <= 16 (the raw score rows) and 8 * B * Tq * k * n_chunks bytes
+ * otherwise (the chunks' candidates), and none for one chunk; float32 (CUDA
+ * cores) needs 4 * B * Tq * N bytes.  For bf16 this equals
  * csa_workspace_bytes(CSA_OP_INDEXER, ...) <= 8 MiB.  The first call on each
  * device looks up the array's device address and caches it, so make that
  * first call before any stream capture.  All calls share the array and its

@@ -160,18 +160,26 @@ struct Item {
   int64_t bidx, pos, wp0, jlo, n_w;
 };
 
+// (query row, head group) of item `it`, from the launch arguments alone.
+__device__ __forceinline__ void item_row_hg(const TcAttnArgs& a, int64_t it, int64_t* row,
+                                            int64_t* hg) {
+  if (a.split) {
+    const int64_t rest = it / a.n_splits;
+    *hg = rest % a.n_hg;
+    *row = rest / a.n_hg;
+  } else {
+    *hg = it % a.n_hg;
+    *row = a.n_rows - 1 - it / a.n_hg;   // late (heavier) rows first
+  }
+}
+
 __device__ __forceinline__ Item decode_item(const TcAttnArgs& a, int64_t it) {
   Item x;
-  if (a.split) {
-    x.split = (int)(it % a.n_splits);
-    const int64_t rest = it / a.n_splits;
-    x.hg = (int)(rest % a.n_hg);
-    x.row = rest / a.n_hg;
-  } else {
-    x.split = 0;
-    x.hg = (int)(it % a.n_hg);
-    x.row = a.n_rows - 1 - it / a.n_hg;   // late (heavier) rows first
-  }
+  int64_t row, hg;
+  item_row_hg(a, it, &row, &hg);
+  x.row = row;
+  x.hg = (int)hg;
+  x.split = a.split ? (int)(it % a.n_splits) : 0;
   x.bidx = x.row / a.Tq;
   const int64_t t = x.row % a.Tq;
   x.pos = a.q_pos ? a.q_pos[x.row] : t;
@@ -370,11 +378,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0 && (int64_t)blockIdx.x < a.n_items) {
+    // the first item's q rows into L2 while the previous kernel may still
+    // run: a prefetch reads nothing into this CTA (L2 stays coherent with
+    // that kernel's writes) and its address needs only the launch arguments
+    int64_t row, hg;
+    item_row_hg(a, blockIdx.x, &row, &hg);
+    const bf16* q0 = a.q + (row * a.H + hg * kHG) * kC;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(q0), "r"(kHG * kC * 2)
+                 : "memory");
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // set-up done without global memory: from here on the previous kernel's
-  // results are needed (a programmatic launch overlaps only the set-up)
+  // set-up done without a global load or store: from here on the previous
+  // kernel's results are needed (a programmatic launch overlaps only the
+  // set-up and the prefetch)
   pdl_wait();
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
@@ -479,6 +498,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0;
     int64_t cur_ent = 0;
     if ((int64_t)blockIdx.x < a.n_items) {
+      if (ptid == 0) {
+        // the first item's raw q rows, before anything else: their load
+        // overlaps the item's position reads and index compaction
+        int64_t row, hg;
+        item_row_hg(a, blockIdx.x, &row, &hg);
+        mbar_arrive_expect_tx(qraw, kRegions * kQRegion);
+        for (int r = 0; r < kRegions; ++r)
+          tma_load_3d(sQ + r * kQRegion, &map_q, qraw, r * 64, (int32_t)(hg * kHG), (int32_t)row);
+      }
       const Item y = decode_item(a, blockIdx.x);
       load_idx(y.row);
       cur_ent = compact(y, 0);
@@ -499,8 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
       }
       // the previous item's last S^T is done with Q: the raw q rows by TMA
+      // (the first item's were issued before its compaction)
       if (n > 0) wait_or_die(qfree, (uint32_t)(n - 1) & 1u, 20u);
-      if (!dead && ptid == 0) {
+      if (!dead && ptid == 0 && n > 0) {
         mbar_arrive_expect_tx(qraw, kRegions * kQRegion);
         for (int r = 0; r < kRegions; ++r)
           tma_load_3d(sQ + r * kQRegion, &map_q, qraw, r * 64, x.hg * kHG, (int32_t)x.row);

@@ -103,8 +103,12 @@ struct TcIdxArgs {
   const int64_t* q_pos;
   int32_t* idx_out;
   float* score_out;
-  float* cand_score;   // [B*Tq][n_chunks][k] when n_chunks > 1
+  float* cand_score;   // [B*Tq][n_chunks][k] when n_chunks > 1 ([B*Tq][n_chunks][kChunk] direct)
   int32_t* cand_idx;
+  // single-token rows whose whole score row fits one merge cluster: the chunk
+  // kernel writes its raw scores (no chunk top-k) and the merge selects
+  // among all of them (entry j of a row is a candidate iff j < its visible count)
+  int direct;
   unsigned* status;
   // MX-FP8 operands: scale-factor tiles of q_I ([B][Tq][512], one per token)
   // and K_I ([B][ceil(N / 128)][512])
@@ -1132,7 +1136,11 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
         tmem_ld32(base + t * kHI, r0);
         tmem_ld32(base + t * kHI + 32, r1);
         tmem_ld_wait();
-        scores[t * kChunk + i * kBM + row] = relu_weighted_sum64(sw + t * kHI, r0, r1);
+        const float sc = relu_weighted_sum64(sw + t * kHI, r0, r1);
+        if (TOK == 1 && a.direct)
+          a.cand_score[(((int64_t)b * a.Tq + t0) * a.n_chunks + chunk) * kChunk + i * kBM + row] = sc;
+        else
+          scores[t * kChunk + i * kBM + row] = sc;
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
@@ -1141,8 +1149,9 @@ __global__ void __launch_bounds__(kThreads, TOK == 1 ? 2 : 1)
 
   __syncthreads();
 
-  // ---------------- top-k: one warp per token
-  if (TOK == 1 && warp >= 2 && !*abort_flag) {
+  // ---------------- top-k: one warp per token (none when the merge selects
+  // from the raw scores)
+  if (TOK == 1 && warp >= 2 && !*abort_flag && !a.direct) {
     // one token: the four epilogue warps select together (named barrier 1)
     const int64_t tok = t0;
     if (tok < a.Tq) {
@@ -1776,13 +1785,25 @@ __global__ void __launch_bounds__(kMThreads)
   pdl_trigger();
   const uint32_t CL = cluster_nctarank(), rank = cluster_ctarank();
   const int64_t row = blockIdx.x / CL;
-  const int64_t n = (int64_t)a.n_chunks * a.k;
+  const int64_t n = (int64_t)a.n_chunks * (a.direct ? Cfg<1>::kChunk : a.k);
   const float* cs = a.cand_score + row * n;
   const int32_t* ci = a.cand_idx + row * n;
   const int64_t j0 = (int64_t)rank * kMSlice + (int64_t)threadIdx.x * kMRun;
   float v[kMRun];
   int32_t id[kMRun];
-  if ((n & 3) == 0) {   // 16-byte aligned rows: j0 and n are multiples of 4
+  if (a.direct) {   // raw scores in entry order: entry j is a candidate iff visible
+    const int64_t pos = a.q_pos ? a.q_pos[row] : row % a.Tq;
+    const int64_t vis = vis_count(pos, a.m, a.N);
+#pragma unroll
+    for (int q = 0; q < kMRun / 4; ++q) {
+      const int64_t j = j0 + 4 * q;
+      float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < vis) s4 = *reinterpret_cast<const float4*>(cs + j);
+      v[4 * q] = s4.x; v[4 * q + 1] = s4.y; v[4 * q + 2] = s4.z; v[4 * q + 3] = s4.w;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) id[4 * q + e] = j + e < vis ? (int32_t)(j + e) : -1;
+    }
+  } else if ((n & 3) == 0) {   // 16-byte aligned rows: j0 and n are multiples of 4
 #pragma unroll
     for (int q = 0; q < kMRun / 4; ++q) {
       const int64_t j = j0 + 4 * q;
@@ -1809,6 +1830,17 @@ __global__ void __launch_bounds__(kMThreads)
 
 inline int tok_for(int64_t Tq) { return Tq >= 4 ? 4 : 1; }
 inline int chunk_for(int tok) { return tok == 4 ? Cfg<4>::kChunk : Cfg<1>::kChunk; }
+// Direct selection (no chunk top-k) for single-token rows of 2 to 16 chunks:
+// the merge's cluster then holds the whole score row.
+inline bool direct_for(int tok, int nc) {
+  return tok == 1 && nc > 1 && (int64_t)nc * Cfg<1>::kChunk <= (int64_t)kSelMaxCluster * kMSlice;
+}
+// Scratch of the candidate lists (or, direct, of the raw score rows).
+inline size_t cand_bytes(int64_t B, int64_t Tq, int nc, int k, bool direct) {
+  if (nc <= 1) return 0;
+  return direct ? (size_t)B * (size_t)Tq * (size_t)nc * (size_t)Cfg<1>::kChunk * 4
+                : (size_t)B * (size_t)Tq * (size_t)nc * (size_t)k * 8;
+}
 inline int n_chunks_for(int64_t N, int tok) {
   int64_t c = chunk_for(tok);
   int64_t n = (N + c - 1) / c;
@@ -1862,7 +1894,7 @@ int sm_count() {
 // The candidate merge: the cluster kernel when one row's candidates fit a
 // cluster of at most kSelMaxCluster CTAs, else one CTA per row.
 cudaError_t launch_merge(const TcIdxArgs& a, int64_t rows, cudaStream_t stream) {
-  const int64_t n = (int64_t)a.n_chunks * a.k;
+  const int64_t n = (int64_t)a.n_chunks * (a.direct ? Cfg<1>::kChunk : a.k);
   const int64_t cl = (n + kMSlice - 1) / kMSlice;
   if (cl > kSelMaxCluster || rows * cl > (int64_t)0x7fffffff) {
     indexer_merge_kernel<<<(unsigned)rows, 1024, 0, stream>>>(a);
@@ -1907,8 +1939,7 @@ cudaError_t launch_persist(const IndexerParams& p, const TcIdxArgs& a, cudaStrea
 
 size_t indexer_mx_scratch(int64_t B, int64_t Tq, int64_t N, int k) {
   const int nc = n_chunks_for(N, 1);
-  if (nc <= 1) return 0;
-  return (size_t)B * (size_t)Tq * (size_t)nc * (size_t)k * 8;
+  return cand_bytes(B, Tq, nc, k, direct_for(1, nc));
 }
 
 cudaError_t launch_indexer_mx(const IndexerParams& p, int fmt, const void* q_sf,
@@ -1937,11 +1968,13 @@ cudaError_t launch_indexer_mx(const IndexerParams& p, int fmt, const void* q_sf,
   a.q_sf = static_cast<const uint8_t*>(q_sf);
   a.k_sf = static_cast<const uint8_t*>(k_sf);
   a.k_sf_tiles = (p.N + kBM - 1) / kBM;
+  a.direct = direct_for(1, a.n_chunks) ? 1 : 0;
   if (a.n_chunks > 1) {
+    if (p.scratch_bytes < cand_bytes(p.B, p.Tq, a.n_chunks, p.k, a.direct))
+      return cudaErrorInvalidValue;
     const size_t n = (size_t)p.B * p.Tq * a.n_chunks * p.k;
-    if (p.scratch_bytes < n * 8) return cudaErrorInvalidValue;
     a.cand_score = static_cast<float*>(p.scratch);
-    a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
+    a.cand_idx = a.direct ? nullptr : reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
   }
   cudaError_t e = fmt == 2 ? launch_tok<1, 2>(p, a, stream) : launch_tok<1, 1>(p, a, stream);
   if (e != cudaSuccess) return e;
@@ -1963,8 +1996,7 @@ bool indexer_tc_supported(const IndexerParams& p) {
 size_t indexer_tc_scratch(int64_t B, int64_t Tq, int64_t N, int k) {
   const int tok = tok_for(Tq);
   const int nc = n_chunks_for(N, tok);
-  if (nc <= 1) return 0;
-  return (size_t)B * (size_t)Tq * (size_t)nc * (size_t)k * 8;
+  return cand_bytes(B, Tq, nc, k, direct_for(tok, nc));
 }
 
 cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
@@ -1990,11 +2022,13 @@ cudaError_t launch_indexer_tc(const IndexerParams& p, cudaStream_t stream,
   a.idx_out = p.idx_out;
   a.score_out = p.score_out;
   a.status = p.status;
+  a.direct = direct_for(tok, a.n_chunks) ? 1 : 0;
   if (a.n_chunks > 1) {
+    if (p.scratch_bytes < cand_bytes(p.B, p.Tq, a.n_chunks, p.k, a.direct))
+      return cudaErrorInvalidValue;
     const size_t n = (size_t)p.B * p.Tq * a.n_chunks * p.k;
-    if (p.scratch_bytes < n * 8) return cudaErrorInvalidValue;
     a.cand_score = static_cast<float*>(p.scratch);
-    a.cand_idx = reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
+    a.cand_idx = a.direct ? nullptr : reinterpret_cast<int32_t*>(static_cast<float*>(p.scratch) + n);
   }
   cudaError_t e = tok == 4 ? launch_persist(p, a, stream) : launch_tok<1>(p, a, stream);
   if (e != cudaSuccess) return e;

@@ -255,7 +255,8 @@ def test_mxfp8_calls_reject_bad_arguments(L):
                                        None, 0, None) == 5
     assert L.indexer_scores_topk_mxfp8(1, 1, 64, 128, d, None, d, d, d, 64, None, 4, 8, d, None,
                                        d, 1 << 20, None) == 1
-    assert L.csa_workspace_bytes(6, 1, 32, 1, 0, 0, 32768, 1024, 0) == 256 + 32 * 8 * 1024 * 8
+    # eight 4096-entry chunks a row: the raw score rows (one merge cluster holds a row)
+    assert L.csa_workspace_bytes(6, 1, 32, 1, 0, 0, 32768, 1024, 0) == 256 + 32 * 8 * 4096 * 4
 
 
 def test_mixed_storage_rejects_bad_arguments(L):
