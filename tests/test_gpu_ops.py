@@ -405,6 +405,27 @@ def test_decode_batch_invariance():
     assert torch.equal(again, full)
 
 
+def test_decode_rows_equal_when_ctas_take_several_items():
+    """A batch with more split items than SMs (160 here) has persistent CTAs
+    that take two items each; the split boundaries and the combine's order
+    depend on a row's own key count only, so its rows are bitwise equal to
+    the same rows in a batch of 4 (one item per CTA) and match the oracle."""
+    w = wl.scaled(wl.WORKLOADS["csa_decode_b32_128k"], B=40)   # 160 split items > 148
+    inp = wl.csa_decode_inputs(w, DEV)
+    inp["idx"] = _decode_idx(w, inp, 6)
+    args = dict(sink=inp["sink"])
+    full = csa.sparse_mqa_attn(inp["q"], inp["entries"], inp["idx"], inp["win"], gfmt(w), w.n_win,
+                               q_pos=inp["q_pos"], win_pos0=inp["win_pos0"], **args)
+    part = slice(8, 12)   # 16 split items: one cluster of 4 per row
+    sub = {k: (v if k == "sink" else v[part].contiguous()) for k, v in inp.items()}
+    few = csa.sparse_mqa_attn(sub["q"], sub["entries"], sub["idx"], sub["win"], gfmt(w), w.n_win,
+                              q_pos=sub["q_pos"], win_pos0=sub["win_pos0"], **args)
+    torch.cuda.synchronize()
+    assert torch.equal(few, full[part])
+    _check_attn(w, sub, few, np.arange(1), dense=False, q_pos=sub["q_pos"],
+                win_pos0=sub["win_pos0"].cpu().numpy())
+
+
 def test_decode_mixed_contexts_and_invariance():
     """Decode rows of very different context lengths in one batch (the split
     size follows each row's own key count, so short rows leave splits empty
