@@ -623,8 +623,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int64_t k_lo, k_hi;
         const int nb = item_blocks(a, x, nent[n & 1], &k_lo, &k_hi);
         mbar_arrive(&ifree[n & 1]);
-        if (*abort_flag || !mbar_wait(qload, (uint32_t)n & 1u)) { ok = false; break; }
+        // the raw q rows suffice for Q regions 0-5; region 7's RoPE dims are
+        // rotated in place by the softmax warps (qload) before region pair 3
+        if (*abort_flag || !mbar_wait(qraw, (uint32_t)n & 1u)) { ok = false; break; }
         tc_fence_after();
+        if (nb == 0 && (*abort_flag || !mbar_wait(qload, (uint32_t)n & 1u))) { ok = false; break; }
         for (int b = 0; b < nb; ++b) {
           const int64_t j = gblk + b;
           const int s = (int)(j & 1);
@@ -637,6 +640,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // each region pair as soon as its gather landed
 #pragma unroll 1
           for (int h = 0; h < 4 && ok; ++h) {
+            if (b == 0 && h == 3 && (*abort_flag || !mbar_wait(qload, (uint32_t)n & 1u))) {
+              ok = false;
+              break;
+            }
             if (*abort_flag || !mbar_wait(&kfull[4 * s + h], (uint32_t)(j >> 1) & 1u)) {
               ok = false;
               break;
