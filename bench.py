@@ -72,8 +72,8 @@ def compress_bytes(w) -> float:
 # SHA-256 is given.  Reported as the roofline's `traffic` only while the
 # kernel source still has that hash; otherwise null.
 ATTN_TRAFFIC = {"source": "long_context_attention_csa_b200/csrc/attn_tc.cu",
-                "sha256": "6b324bedeaff5fc8035ca10361b7bfd238a5f9b14676a5b27a88480288555a2d",
-                "bytes_per_launch": 565.23e6 + 492.98e6}
+                "sha256": "71432149def5493f370ffca271d31a7bb5e7127d10eacd89d6c86f35604781b0",
+                "bytes_per_launch": 564.28e6 + 492.45e6}
 
 
 def attn_traffic():
