@@ -61,6 +61,29 @@ def test_workspace_sizes(L):
     assert L.csa_workspace_bytes(99, 1, 1, 1, 1, 1, 1, 1, 1) == 0
 
 
+def test_indexer_workspace_follows_the_selection_scheme(L):
+    """bf16 indexer scratch: none for one chunk; for single-token rows of 2 to
+    16 chunks of 4096 the raw score rows (the merge selects among them);
+    beyond, and for multi-token rows (chunks of 2048), the chunks' top-k
+    candidates (score and index)."""
+    from long_context_attention_csa_b200 import CSA_OP_INDEXER, CSA_OP_INDEXER_MX
+
+    def ws(B, Tq, N, k, op=CSA_OP_INDEXER):
+        return L.csa_workspace_bytes(op, 1, B, Tq, 0, 0, N, k, 0) - 256
+
+    assert ws(3, 1, 4096, 1024) == 0
+    assert ws(3, 1, 4097, 1024) == 3 * 2 * 4096 * 4
+    assert ws(2, 1, 16 * 4096, 1024) == 2 * 16 * 4096 * 4
+    assert ws(2, 1, 16 * 4096 + 1, 1024) == 2 * 17 * 1024 * 8
+    assert ws(1, 3, 30000, 512) == 3 * 8 * 4096 * 4
+    assert ws(1, 4, 30000, 512) == 4 * 15 * 512 * 8      # 2048-entry chunks, candidates
+    assert ws(1, 8, 2048, 512) == 0
+    # the MX-FP8 / MX-FP4 calls take single-token units at any Tq
+    assert ws(3, 1, 4097, 1024, CSA_OP_INDEXER_MX) == 3 * 2 * 4096 * 4
+    assert ws(2, 1, 16 * 4096 + 1, 1024, CSA_OP_INDEXER_MX) == 2 * 17 * 1024 * 8
+    assert ws(1, 5, 30000, 64, CSA_OP_INDEXER_MX) == 5 * 8 * 4096 * 4
+
+
 def _fmt(c=512, r=64, flags=0):
     from long_context_attention_csa_b200 import Fmt
 
